@@ -1,0 +1,148 @@
+/*
+ * mlstm.h -- C ABI of libmlstm, the mLSTM matrix-memory cell on NVIDIA B200 (sm_100a).
+ *
+ * The cell (per batch element b and head h, token t = 1..S):
+ *
+ *   log f_t = logsigmoid(f~_t)
+ *   m_t     = max(log f_t + m_{t-1}, i~_t)                  stabilizer
+ *   f'_t    = exp(log f_t + m_{t-1} - m_t),  i'_t = exp(i~_t - m_t)
+ *   C_t     = f'_t C_{t-1} + i'_t k_t v_t^T                 C stored [DHQK][DHV]
+ *   n_t     = f'_t n_{t-1} + i'_t k_t
+ *   h_t     = o_t * (C_t^T qh_t) / max(|n_t . qh_t|, exp(-m_t)),  qh_t = q_t / sqrt(DHQK)
+ *
+ * Sources: "xLSTM Guide: Extended LSTM Architecture & Matrix Memory" -- sections
+ * "The Stabilizer State: Preventing Numerical Overflow" (m_t and the stabilized
+ * exponential gates), "mLSTM: Matrix Key-Value Memory and Covariance Updates" /
+ * "Recurrent Formulation (Inference Mode)" (C_t, n_t, h_t), "The Dual
+ * Formulation" (the parallel form over a causal decay matrix) and "Exploit
+ * Chunkwise Hardware Kernels for Production Training" (chunks of 64 or 128
+ * tokens: dense products inside a chunk, a scan across chunks).  The forget
+ * gate is the sigmoid gate in log space; q carries the 1/sqrt(DHQK) factor, so
+ * C and n hold raw k; the floor exp(-m_t) is the guide's floor of 1 on the
+ * unstabilized states.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned by the caller, contiguous,
+ *    row-major, 16-byte aligned.  The library allocates no memory and keeps no
+ *    state between calls.
+ *  - Layouts: q, k [B][NH][S][DHQK]; v, ogate, h [B][NH][S][DHV];
+ *    igate, fgate [B][NH][S] (float32 pre-activations i~, f~);
+ *    C [B][NH][DHQK][DHV], n [B][NH][DHQK], m [B][NH] (float32).
+ *  - q, k, v, ogate and h have the element type `dt`; gates and states are
+ *    always float32.  ogate holds the already-activated output gate (for
+ *    example sigmoid(o~)); NULL means o = 1.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is enqueued asynchronously; nothing synchronizes.
+ *  - Arguments are checked on the host before anything is enqueued; a bad
+ *    argument returns an error status and launches nothing.  A failed launch
+ *    returns MLSTM_ERR_CUDA.  No call throws or aborts.
+ */
+#ifndef MLSTM_H
+#define MLSTM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mlstm_status {
+    MLSTM_OK = 0,
+    MLSTM_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, misaligned pointer */
+    MLSTM_ERR_UNSUPPORTED = 2,  /* valid but unsupported shape / chunk / dtype */
+    MLSTM_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than mlstm_fwd_workspace_size() */
+    MLSTM_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+    MLSTM_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see mlstm_fwd_status) */
+} mlstm_status;
+
+typedef enum mlstm_dtype {
+    MLSTM_F32 = 0,
+    MLSTM_BF16 = 1
+} mlstm_dtype;
+
+/*
+ * Bytes of device workspace mlstm_fwd needs for these arguments (0 when the
+ * arguments are unsupported).  The workspace holds the gate preprocessing
+ * (cumulative log forget gates, stabilizers) and the chunk-boundary states.
+ */
+size_t mlstm_fwd_workspace_size(int B, int NH, int S, int DHQK, int DHV, int chunk,
+                                mlstm_dtype dt);
+
+/*
+ * Chunkwise parallel forward pass from the zero state (C = 0, n = 0, m = 0)
+ * over S tokens.  Writes h_out and, where the pointers are non-NULL, the final
+ * state C_final, n_final, m_final.  Mathematically the result equals the
+ * recurrence above token by token; `chunk` (16, 32, 64 or 128) is the length
+ * of the blocks inside which the causal decay matrix is used.  S may be any
+ * value >= 0 (a last, shorter chunk is allowed; S == 0 writes the zero state).
+ * Supported: DHQK and DHV multiples of 8 in [8, 512].
+ *
+ * The source defining the operation: the guide's "Recurrent Formulation
+ * (Inference Mode)" (what is computed) and "The Dual Formulation" with
+ * "Exploit Chunkwise Hardware Kernels for Production Training" (how).
+ *
+ * workspace: device memory of at least mlstm_fwd_workspace_size() bytes,
+ * 256-byte aligned, owned by the caller, used until the enqueued work ends.
+ * Two calls in flight must not share a workspace.
+ */
+mlstm_status mlstm_fwd(const void *q, const void *k, const void *v,
+                       const float *igate, const float *fgate, const void *ogate,
+                       mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                       void *h_out, float *C_final, float *n_final, float *m_final,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * mlstm_fwd with per-phase timing: identical work and results, and in addition
+ * records CUDA events (cudaEvent_t passed as void*, created by the caller) on
+ * `stream`: events[p] just before phase p and events[MLSTM_FWD_PHASES] after
+ * the last one.  Phases, in order: 0 gate preprocessing, 1 chunk or segment
+ * state contributions, 2 scan of the states across chunks or segments,
+ * 3 outputs (and, on the tensor-core path, the in-segment state walk).  A
+ * phase that launches nothing on a given path has two events back to back.
+ */
+#define MLSTM_FWD_PHASES 4
+mlstm_status mlstm_fwd_profiled(const void *q, const void *k, const void *v,
+                                const float *igate, const float *fgate, const void *ogate,
+                                mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                                void *h_out, float *C_final, float *n_final, float *m_final,
+                                void *workspace, size_t workspace_bytes, void *stream,
+                                void *const *events);
+
+/*
+ * Number of kernels one mlstm_fwd call with these arguments launches (0 when
+ * the arguments are unsupported or there is nothing to compute).
+ */
+int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
+
+/*
+ * Reports whether the last mlstm_fwd that used `workspace` ran to completion:
+ * synchronizes `stream`, reads the status word kept in the workspace and
+ * returns MLSTM_OK or MLSTM_ERR_TIMEOUT (a bounded device-side wait gave up;
+ * the outputs of that call are then undefined).
+ */
+mlstm_status mlstm_fwd_status(const void *workspace, void *stream);
+
+/*
+ * One recurrent decode step for every (b, h): reads the state (C, n, m),
+ * applies one token and writes the new state back IN PLACE, plus h_out
+ * [B][NH][DHV].  Token inputs: q, k [B][NH][DHQK] and v, ogate [B][NH][DHV]
+ * in `dt`; igate, fgate [B][NH] float32.  Supported: DHQK multiple of 8 in
+ * [8, 512], DHV multiple of 4 in [4, 1024].
+ *
+ * The source defining the operation: the guide's "Recurrent Formulation
+ * (Inference Mode)", applied once.
+ */
+mlstm_status mlstm_step(float *C, float *n, float *m,
+                        const void *q, const void *k, const void *v,
+                        const float *igate, const float *fgate, const void *ogate,
+                        mlstm_dtype dt, int B, int NH, int DHQK, int DHV,
+                        void *h_out, void *stream);
+
+/* Static English text for a status code. */
+const char *mlstm_status_string(mlstm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLSTM_H */

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/mlstm.h declares, and rejects bad arguments before touching the GPU."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from xlstm_mlstm_cell_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    names = []
+    for fname in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fname.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fname)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(mlstm_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "mlstm_fwd" in names and "mlstm_step" in names
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in binding.SIGNATURES, "binding lacks " + name
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = lib.mlstm_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.mlstm_status_string(0) == b"ok"
+
+
+def test_workspace_size(lib):
+    ws = lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 512, 64, binding.MLSTM_BF16)
+    assert ws > 0 and ws % 256 == 0
+    assert lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 512, 48, binding.MLSTM_BF16) == 0   # chunk
+    assert lib.mlstm_fwd_workspace_size(1, 8, 8192, 12, 512, 64, binding.MLSTM_BF16) == 0    # DHQK % 8
+    assert lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 1024, 64, binding.MLSTM_BF16) == 0  # DHV > 512
+    assert lib.mlstm_fwd_workspace_size(-1, 8, 8192, 256, 512, 64, binding.MLSTM_BF16) == 0
+    assert lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 512, 64, 7) == 0                    # dtype
+    assert lib.mlstm_fwd_workspace_size(1, 8, 0, 256, 512, 64, binding.MLSTM_BF16) > 0
+
+
+FAKE = 1 << 20   # a 16-byte-aligned non-NULL address that is never dereferenced
+
+
+def fwd_args(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, ig=FAKE, fg=FAKE, og=None, dt=binding.MLSTM_BF16, B=1, NH=2, S=128,
+             DHQK=64, DHV=64, chunk=64, h=FAKE, C=None, n=None, m=None, ws=FAKE, wsb=1 << 40, stream=None)
+    a.update(over)
+    return a
+
+
+def call_fwd(lib, a):
+    return lib.mlstm_fwd(a["q"], a["k"], a["v"], a["ig"], a["fg"], a["og"], a["dt"], a["B"], a["NH"], a["S"],
+                         a["DHQK"], a["DHV"], a["chunk"], a["h"], a["C"], a["n"], a["m"], a["ws"], a["wsb"],
+                         a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(ig=None), 1), (dict(fg=None), 1),
+    (dict(h=None), 1), (dict(q=FAKE + 4), 1), (dict(og=FAKE + 8), 1), (dict(C=FAKE + 2), 1),
+    (dict(B=-1), 1), (dict(S=-5), 1), (dict(dt=3), 2), (dict(chunk=48), 2), (dict(chunk=256), 2),
+    (dict(DHQK=12), 2), (dict(DHV=520), 2), (dict(DHQK=0), 2),
+    (dict(ws=None), 3), (dict(wsb=100), 3), (dict(ws=FAKE + 16), 1),
+])
+def test_fwd_rejects_bad_arguments(lib, over, expect):
+    assert call_fwd(lib, fwd_args(**over)) == expect
+
+
+def step_args(**over):
+    a = dict(C=FAKE, n=FAKE, m=FAKE, q=FAKE, k=FAKE, v=FAKE, ig=FAKE, fg=FAKE, og=None, dt=binding.MLSTM_BF16,
+             B=2, NH=2, DHQK=64, DHV=64, h=FAKE, stream=None)
+    a.update(over)
+    return a
+
+
+def call_step(lib, a):
+    return lib.mlstm_step(a["C"], a["n"], a["m"], a["q"], a["k"], a["v"], a["ig"], a["fg"], a["og"], a["dt"],
+                          a["B"], a["NH"], a["DHQK"], a["DHV"], a["h"], a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(C=None), 1), (dict(n=None), 1), (dict(m=None), 1), (dict(q=None), 1), (dict(h=None), 1),
+    (dict(C=FAKE + 4), 1), (dict(og=FAKE + 4), 1), (dict(B=-2), 1), (dict(dt=9), 2),
+    (dict(DHQK=10), 2), (dict(DHV=2), 2), (dict(DHV=2048), 2), (dict(DHQK=1024), 2),
+])
+def test_step_rejects_bad_arguments(lib, over, expect):
+    assert call_step(lib, step_args(**over)) == expect
+
+
+def test_empty_batch_is_a_no_op(lib):
+    # B * NH == 0 enqueues nothing for the step and returns before any launch
+    assert call_step(lib, step_args(B=0, C=None, n=None, m=None)) == 0
+
+
+def test_fwd_status_rejects_null(lib):
+    assert lib.mlstm_fwd_status(None, None) == 1

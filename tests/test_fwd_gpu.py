@@ -1,0 +1,142 @@
+"""GPU parity of mlstm_fwd against the fp64 oracle, called through the C ABI.
+
+Small and medium shapes compare every output element (h, C, n, m) with the
+oracle; they span several chunks and state tiles and end in a ragged chunk.
+The full-size workloads compare whole tensors where the oracle finishes in
+seconds and, for the 131072-token workload, sampled heads and value columns
+(column j of h and C depends only on column j of v and o, and heads are
+independent: both are pinned on the oracle), plus h at 1024 seeded positions.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import TOL, assert_close, rel_l2
+from xlstm_mlstm_cell_b200 import binding
+from xlstm_mlstm_cell_b200.workloads import WORKLOADS, make_custom, make_fwd_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(inputs, chunk):
+    q, k, v, i, f, o = (None if x is None else x.cuda() for x in inputs)
+    h, C, n, m = binding.fwd(q, k, v, i, f, o, chunk=chunk)
+    torch.cuda.synchronize()
+    return h.cpu(), C.cpu(), n.cpu(), m.cpu()
+
+
+def check_against_oracle(inputs, chunk, tol, nthreads=0):
+    h, C, n, m = run_gpu(inputs, chunk)
+    hr, Cr, nr, mr = oracle.mlstm_fwd(*inputs, nthreads=nthreads)
+    errs = {
+        "h": assert_close("h", h, hr, tol),
+        "C": assert_close("C", C, Cr, tol),
+        "n": assert_close("n", n, nr, tol),
+        "m": assert_close("m", m, mr, tol),
+    }
+    return errs
+
+
+def test_fwd_f32_small_workload(cuda_lib):
+    w = WORKLOADS["fwd_f32_small"]
+    check_against_oracle(make_fwd_inputs(w), w.chunk, TOL["f32"])
+
+
+SMALL = [
+    # B, NH, S, DHQK, DHV, chunk, dtype
+    (1, 2, 100, 16, 16, 16, "f32"),
+    (2, 3, 200, 32, 48, 32, "f32"),
+    (1, 1, 1, 8, 8, 16, "f32"),
+    (1, 2, 257, 64, 40, 64, "f32"),
+    (1, 2, 256, 64, 64, 64, "bf16"),
+    (1, 2, 300, 128, 128, 64, "bf16"),
+    (2, 2, 520, 256, 256, 128, "bf16"),
+    (1, 2, 384, 256, 512, 128, "bf16"),
+    (1, 2, 200, 64, 128, 32, "bf16"),
+    (1, 1, 130, 256, 512, 64, "bf16"),
+]
+
+
+@pytest.mark.parametrize("B,NH,S,DHQK,DHV,chunk,dt", SMALL)
+def test_fwd_small_shapes(cuda_lib, B, NH, S, DHQK, DHV, chunk, dt):
+    inputs = make_custom(B, NH, S, DHQK, DHV, dt, seed=S * 7 + DHQK, ig=(-1.0, 2.0), fg=(3.0, 1.5))
+    check_against_oracle(inputs, chunk, TOL[dt])
+
+
+@pytest.mark.parametrize("ig,fg", [((0.0, 8.0), (3.0, 1.0)), ((0.0, 1.0), (-4.0, 1.0)),
+                                   ((0.0, 1.0), (10.0, 1.0)), ((-10.0, 1.0), (2.0, 1.0))])
+@pytest.mark.parametrize("dt,DHQK,DHV,chunk", [("f32", 32, 32, 32), ("bf16", 128, 256, 64),
+                                               ("bf16", 256, 256, 128)])
+def test_fwd_adversarial_gates(cuda_lib, ig, fg, dt, DHQK, DHV, chunk):
+    inputs = make_custom(1, 2, 3 * chunk + 5, DHQK, DHV, dt, seed=11, ig=ig, fg=fg)
+    check_against_oracle(inputs, chunk, TOL[dt])
+
+
+def test_fwd_no_output_gate(cuda_lib):
+    inputs = make_custom(1, 2, 192, 128, 128, "bf16", seed=5, ogate=False)
+    check_against_oracle(inputs, 64, TOL["bf16"])
+
+
+def test_fwd_empty_sequence(cuda_lib):
+    inputs = make_custom(2, 2, 0, 64, 64, "bf16", seed=1)
+    h, C, n, m = run_gpu(inputs, 64)
+    assert h.shape == (2, 2, 0, 64)
+    assert not C.any() and not n.any() and not m.any()
+
+
+@pytest.mark.parametrize("dt,DHQK,DHV", [("f32", 32, 32), ("bf16", 256, 256)])
+def test_fwd_chunk_size_independent(cuda_lib, dt, DHQK, DHV):
+    inputs = make_custom(1, 2, 512, DHQK, DHV, dt, seed=3, ig=(-1.0, 2.0), fg=(4.0, 1.0))
+    ref = run_gpu(inputs, 128)
+    for chunk in (16, 32, 64):
+        out = run_gpu(inputs, chunk)
+        for name, x, r in zip("hCnm", out, ref):
+            assert rel_l2(x, r) <= TOL[dt], (chunk, name)
+
+
+@pytest.mark.parametrize("dt,DHQK,DHV,chunk", [("f32", 16, 16, 16), ("bf16", 256, 512, 64)])
+def test_fwd_then_step_equals_longer_fwd(cuda_lib, dt, DHQK, DHV, chunk):
+    S = 4 * chunk + 3
+    q, k, v, i, f, o = make_custom(1, 2, S + 1, DHQK, DHV, dt, seed=21, ig=(-1.0, 2.0), fg=(4.0, 1.0))
+    cut = lambda x, a, b: x[:, :, a:b].contiguous().cuda()
+    h1, C1, n1, m1 = binding.fwd(cut(q, 0, S), cut(k, 0, S), cut(v, 0, S), cut(i, 0, S), cut(f, 0, S),
+                                 cut(o, 0, S), chunk=chunk)
+    hs = binding.step(C1, n1, m1, q[:, :, S].contiguous().cuda(), k[:, :, S].contiguous().cuda(),
+                      v[:, :, S].contiguous().cuda(), i[:, :, S].contiguous().cuda(),
+                      f[:, :, S].contiguous().cuda(), o[:, :, S].contiguous().cuda())
+    h2, C2, n2, m2 = binding.fwd(q.cuda(), k.cuda(), v.cuda(), i.cuda(), f.cuda(), o.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    tol = TOL[dt]
+    assert rel_l2(hs.cpu(), h2[:, :, S].cpu()) <= tol
+    assert rel_l2(C1.cpu(), C2.cpu()) <= tol and rel_l2(n1.cpu(), n2.cpu()) <= tol
+    assert rel_l2(m1.cpu(), m2.cpu()) <= tol
+
+
+@pytest.mark.parametrize("name", ["fwd_bf16_d256", "fwd_bf16_7b"])
+def test_fwd_full_workload(cuda_lib, name):
+    """Whole-tensor parity at the workload's full size (the oracle takes seconds here)."""
+    w = WORKLOADS[name]
+    check_against_oracle(make_fwd_inputs(w), w.chunk, TOL[w.dtype])
+
+
+def test_fwd_long_context_sampled(cuda_lib):
+    """131072 tokens: sampled heads x value columns in full, plus h at 1024 seeded positions."""
+    w = WORKLOADS["fwd_bf16_long"]
+    q, k, v, i, f, o = make_fwd_inputs(w)
+    h, C, n, m = run_gpu((q, k, v, i, f, o), w.chunk)
+    rng = np.random.default_rng(4242)
+    heads = [0, 5]
+    cols = np.sort(rng.choice(w.DHV, size=16, replace=False))
+    tol = TOL[w.dtype]
+    for hd in heads:
+        sl = lambda x: x[:, hd:hd + 1]
+        hr, Cr, nr, mr = oracle.run(sl(q), sl(k), sl(v)[..., cols], sl(i), sl(f), sl(o)[..., cols])
+        assert_close("h[head %d]" % hd, h[:, hd:hd + 1][..., cols], hr, tol)
+        assert_close("C[head %d]" % hd, C[:, hd:hd + 1][..., cols], Cr, tol)
+        assert_close("n[head %d]" % hd, n[:, hd:hd + 1], nr, tol)
+        assert_close("m[head %d]" % hd, m[:, hd:hd + 1], mr, tol)
+        pos = np.sort(rng.choice(w.S, size=1024 // len(heads), replace=False))
+        assert_close("h[head %d, 512 positions]" % hd, h[0, hd][pos][:, cols], hr[0, 0][pos], tol)

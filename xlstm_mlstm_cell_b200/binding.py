@@ -1,0 +1,157 @@
+"""Thin ctypes binding of libmlstm (argument marshalling only).
+
+The functions take torch tensors that already live on the GPU, pass their
+device pointers, sizes and the current CUDA stream to the C ABI declared in
+``include/mlstm.h``, and raise ``MlstmError`` on a non-zero status.  Every step
+of the computation runs in the library's CUDA kernels; there is no other code
+path.  If the library cannot be loaded the import of the functions fails
+loudly (``load()`` raises).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmlstm.so")
+
+MLSTM_F32, MLSTM_BF16 = 0, 1
+STATUS = {0: "MLSTM_OK", 1: "MLSTM_ERR_INVALID_ARG", 2: "MLSTM_ERR_UNSUPPORTED", 3: "MLSTM_ERR_WORKSPACE",
+          4: "MLSTM_ERR_CUDA", 5: "MLSTM_ERR_TIMEOUT"}
+
+# Every symbol include/mlstm.h declares, with its ctypes signature.
+_vp, _fp, _i, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "mlstm_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "mlstm_fwd": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp, _vp, _sz,
+                       _vp]),
+    "mlstm_fwd_profiled": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp,
+                                _vp, _sz, _vp, ctypes.POINTER(ctypes.c_void_p)]),
+    "mlstm_fwd_status": (_i, [_vp, _vp]),
+    "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
+    "mlstm_step": (_i, [_fp, _fp, _fp, _vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "mlstm_status_string": (ctypes.c_char_p, [_i]),
+}
+
+_lib = None
+
+
+class MlstmError(RuntimeError):
+    def __init__(self, fn: str, status: int, lib=None):
+        text = lib.mlstm_status_string(status).decode() if lib is not None else ""
+        super().__init__("%s returned %s (%s)" % (fn, STATUS.get(status, status), text))
+        self.status = status
+
+
+def load(path: str | None = None):
+    """Loads libmlstm.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError("libmlstm.so not found at %s; build it with `python -m xlstm_mlstm_cell_b200.build`" % p)
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MLSTM_F32
+    if t.dtype == torch.bfloat16:
+        return MLSTM_BF16
+    raise TypeError("q, k, v must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, status):
+    if status != 0:
+        raise MlstmError(fn, status, _lib)
+
+
+def workspace_size(B, NH, S, DHQK, DHV, chunk, dtype) -> int:
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().mlstm_fwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dt))
+
+
+def fwd_kernel_launches(B, NH, S, DHQK, DHV, chunk, dtype) -> int:
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().mlstm_fwd_kernel_launches(B, NH, S, DHQK, DHV, chunk, dt))
+
+
+def alloc_workspace(B, NH, S, DHQK, DHV, chunk, dtype, device="cuda") -> torch.Tensor:
+    n = workspace_size(B, NH, S, DHQK, DHV, chunk, dtype)
+    if n == 0:
+        raise MlstmError("mlstm_fwd_workspace_size", 2)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+FWD_PHASES = 4
+PHASE_NAMES = ("gate_prep", "state_contributions", "state_scan", "outputs")
+
+
+def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=None, n_final=None,
+        m_final=None, workspace=None, return_state: bool = True, stream=None, events=None):
+    """mlstm_fwd on device tensors; returns ``(h, C, n, m)`` (states None unless requested).
+
+    With ``events`` (FWD_PHASES + 1 ``torch.cuda.Event(enable_timing=True)``) the call goes
+    through mlstm_fwd_profiled, which records them around its phases on the stream.
+    """
+    lib = load()
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    dt = _dt(q)
+    if h_out is None:
+        h_out = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=q.device)
+    if return_state:
+        if C_final is None:
+            C_final = torch.empty((B, NH, DHQK, DHV), dtype=torch.float32, device=q.device)
+        if n_final is None:
+            n_final = torch.empty((B, NH, DHQK), dtype=torch.float32, device=q.device)
+        if m_final is None:
+            m_final = torch.empty((B, NH), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, NH, S, DHQK, DHV, chunk, q.dtype, q.device)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate), dt, B, NH, S, DHQK, DHV, chunk,
+            _ptr(h_out), _ptr(C_final), _ptr(n_final), _ptr(m_final), _ptr(workspace), workspace.numel(),
+            _stream(stream))
+    if events is None:
+        _check("mlstm_fwd", lib.mlstm_fwd(*args))
+    else:
+        assert len(events) == FWD_PHASES + 1
+        arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[e.cuda_event for e in events])
+        _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
+    return h_out, C_final, n_final, m_final
+
+
+def fwd_status(workspace, stream=None) -> int:
+    return int(load().mlstm_fwd_status(_ptr(workspace), _stream(stream)))
+
+
+def step(C, n, m, q, k, v, igate, fgate, ogate=None, h_out=None, stream=None):
+    """mlstm_step on device tensors; the state (C, n, m) is updated in place; returns h."""
+    lib = load()
+    B, NH, DHQK = q.shape
+    DHV = v.shape[-1]
+    if h_out is None:
+        h_out = torch.empty((B, NH, DHV), dtype=q.dtype, device=q.device)
+    st = lib.mlstm_step(_ptr(C), _ptr(n), _ptr(m), _ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate),
+                        _ptr(ogate), _dt(q), B, NH, DHQK, DHV, _ptr(h_out), _stream(stream))
+    _check("mlstm_step", st)
+    return h_out

@@ -1,0 +1,54 @@
+// common.cuh -- small device helpers shared by the libmlstm kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define MLSTM_DEVINL __device__ __forceinline__
+
+namespace mlstm {
+
+// Element loads/stores for the two supported element types of q, k, v, o and h.
+MLSTM_DEVINL float to_f32(float x) { return x; }
+MLSTM_DEVINL float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> MLSTM_DEVINL T from_f32(float x);
+template <> MLSTM_DEVINL float from_f32<float>(float x) { return x; }
+template <> MLSTM_DEVINL __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Four consecutive elements as float (16-byte aligned for float, 8 for bf16).
+MLSTM_DEVINL float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+MLSTM_DEVINL float4 load4(const __nv_bfloat16 *p)
+{
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+MLSTM_DEVINL void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+MLSTM_DEVINL void store4(__nv_bfloat16 *p, float4 v)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+
+// logsigmoid(x) = -log(1 + exp(-x)) without overflow, through CUDA's own expf/log1pf.
+MLSTM_DEVINL float log_sigmoid(float x)
+{
+    return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
+}
+
+MLSTM_DEVINL float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+}  // namespace mlstm

@@ -1,0 +1,278 @@
+// fwd_simt.cu -- chunkwise forward pass on CUDA cores in fp32 (no tensor cores).
+//
+// This path serves float32 inputs (where bf16 tensor-core operands cannot meet
+// an fp32 error budget) and the shapes the tensor-core path does not take
+// (small head dimensions, chunks of 16 or 32).  It computes the same chunkwise
+// decomposition as the tensor-core path, with every product in fp32 FMAs:
+//
+// Carry ("inter-chunk states via a scan", xLSTM Guide, "Exploit Chunkwise
+// Hardware Kernels for Production Training"), per chunk c with the gate
+// preprocessing a, g, m of gate_prep.cu:
+//   w_s     = exp(g_c - a_s + i~_s - m_{c+1})              (<= 1)
+//   C_{c+1} = exp(g_c + m_c - m_{c+1}) C_c + sum_s w_s k_s v_s^T
+//   n_{c+1} = exp(g_c + m_c - m_{c+1}) n_c + sum_s w_s k_s
+//
+// Output (the causal decay matrix of "The Dual Formulation", restricted to a
+// chunk, plus the state of the chunk start), for token tau of chunk c:
+//   D_{tau,s} = exp(a_tau - a_s + i~_s - m_tau)  for s <= tau, else 0     (<= 1)
+//   sc_tau    = exp(a_tau + m_c - m_tau)                                  (<= 1)
+//   num_tau   = sc_tau C_c^T qh_tau + sum_s D_{tau,s} (qh_tau . k_s) v_s
+//   den_tau   = sc_tau n_c . qh_tau + sum_s D_{tau,s} (qh_tau . k_s)
+//   h_tau     = o_tau * num_tau / max(|den_tau|, exp(-m_tau))
+// In exact arithmetic this equals the token-by-token recurrence.
+#include "common.cuh"
+#include "mlstm_internal.h"
+
+namespace mlstm {
+
+constexpr int ST = 32;   // state tile edge (rows of C and columns of C / h)
+
+// ---------------------------------------------------------------- carry
+// grid (BH, ceil(DHQK/32), ceil(DHV/32)), 256 threads; a thread owns 4 rows x 1 column
+// of a 32 x 32 tile of C.  Walks all chunks of its head in order, storing the
+// state at every chunk start (CS) and the final state.
+template <typename T>
+__global__ void __launch_bounds__(256)
+carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ igate,
+                  const float *__restrict__ A, const float *__restrict__ G, const float *__restrict__ MC,
+                  int S, int L, int NC, int DHQK, int DHV,
+                  float *__restrict__ CS, float *__restrict__ NS,
+                  float *__restrict__ C_final, float *__restrict__ n_final, float *__restrict__ m_final)
+{
+    extern __shared__ float sm[];
+    float *ks = sm;                    // [L][ST]
+    float *vs = ks + L * ST;           // [L][ST]
+    float *ws = vs + L * ST;           // [L]
+    const int bh = blockIdx.x, i0 = blockIdx.y * ST, j0 = blockIdx.z * ST;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // column, row group
+    const int j = j0 + tx;
+    const bool do_n = blockIdx.z == 0 && ty == 0;              // warp 0 of dv tile 0 keeps n
+    const T *kb = k + (size_t)bh * S * DHQK;
+    const T *vb = v + (size_t)bh * S * DHV;
+    const float *igb = igate + (size_t)bh * S;
+    const float *Ab = A + (size_t)bh * S;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    float nn = 0.f;
+
+    for (int ch = 0; ch < NC; ++ch) {
+        const int t0 = ch * L, len = min(L, S - t0);
+        // state at the chunk start
+        float *cs = CS + ((size_t)bh * NC + ch) * DHQK * DHV;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = i0 + ty * 4 + r;
+            if (i < DHQK && j < DHV) cs[(size_t)i * DHV + j] = c[r];
+        }
+        if (do_n && i0 + tx < DHQK) NS[((size_t)bh * NC + ch) * DHQK + i0 + tx] = nn;
+
+        const float mc = MC[(size_t)bh * (NC + 1) + ch], mn = MC[(size_t)bh * (NC + 1) + ch + 1];
+        const float g = G[(size_t)bh * NC + ch];
+        const float decay = expf(g + mc - mn);
+        __syncthreads();
+        for (int e = threadIdx.x; e < len * ST; e += blockDim.x) {
+            const int s = e / ST, x = e % ST;
+            ks[e] = (i0 + x < DHQK) ? to_f32(kb[(size_t)(t0 + s) * DHQK + i0 + x]) : 0.f;
+            vs[e] = (j0 + x < DHV) ? to_f32(vb[(size_t)(t0 + s) * DHV + j0 + x]) : 0.f;
+        }
+        for (int s = threadIdx.x; s < len; s += blockDim.x)
+            ws[s] = expf(g - Ab[t0 + s] + igb[t0 + s] - mn);
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 4; ++r) c[r] *= decay;
+        nn *= decay;
+        for (int s = 0; s < len; ++s) {
+            const float wv = ws[s] * vs[s * ST + tx];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) c[r] = fmaf(ks[s * ST + ty * 4 + r], wv, c[r]);
+            if (do_n) nn = fmaf(ws[s], ks[s * ST + tx], nn);
+        }
+    }
+    if (C_final) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = i0 + ty * 4 + r;
+            if (i < DHQK && j < DHV) C_final[((size_t)bh * DHQK + i) * DHV + j] = c[r];
+        }
+    }
+    if (n_final && do_n && i0 + tx < DHQK) n_final[(size_t)bh * DHQK + i0 + tx] = nn;
+    if (m_final && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+        m_final[bh] = MC[(size_t)bh * (NC + 1) + NC];
+}
+
+// ---------------------------------------------------------------- output
+// grid (BH, NC, ceil(DHV/32)), 256 threads.  Shared: P [L][L+1], q/k slices
+// [L][33], v tile [L][33], C slice [32][33], per-row scalars.
+template <typename T>
+__global__ void __launch_bounds__(256)
+output_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                   const float *__restrict__ igate, const T *__restrict__ ogate,
+                   const float *__restrict__ A, const float *__restrict__ Mtok, const float *__restrict__ MC,
+                   const float *__restrict__ CS, const float *__restrict__ NS,
+                   int S, int L, int NC, int DHQK, int DHV, T *__restrict__ h)
+{
+    extern __shared__ float sm[];
+    const int LP = L + 1;
+    float *P = sm;                       // [L][L+1]
+    float *qs = P + L * LP;              // [L][33]
+    float *ks2 = qs + L * 33;            // [L][33]   (k slice, later the v tile)
+    float *cs = ks2 + L * 33;            // [32][33]
+    float *ar = cs + 32 * 33;            // [L] a
+    float *mr = ar + L;                  // [L] m
+    float *ir = mr + L;                  // [L] i~
+    float *sc = ir + L;                  // [L] sc
+    float *den = sc + L;                 // [L]
+
+    const int bh = blockIdx.x, ch = blockIdx.y, j0 = blockIdx.z * ST;
+    const int t0 = ch * L, len = min(L, S - t0);
+    const int tid = threadIdx.x;
+    const float scale = rsqrtf((float)DHQK);
+    const T *qb = q + ((size_t)bh * S + t0) * DHQK;
+    const T *kb = k + ((size_t)bh * S + t0) * DHQK;
+    const T *vb = v + ((size_t)bh * S + t0) * DHV;
+    const float mc = MC[(size_t)bh * (NC + 1) + ch];
+
+    for (int t = tid; t < L; t += blockDim.x) {
+        const bool ok = t < len;
+        ar[t] = ok ? A[(size_t)bh * S + t0 + t] : 0.f;
+        mr[t] = ok ? Mtok[(size_t)bh * S + t0 + t] : 0.f;
+        ir[t] = ok ? igate[(size_t)bh * S + t0 + t] : -INFINITY;
+        sc[t] = ok ? expf(ar[t] + mc - mr[t]) : 0.f;
+    }
+    for (int e = tid; e < L * LP; e += blockDim.x) P[e] = 0.f;
+    __syncthreads();
+
+    // S = qh K^T over DHQK slices of 32
+    for (int d0 = 0; d0 < DHQK; d0 += 32) {
+        for (int e = tid; e < L * 32; e += blockDim.x) {
+            const int t = e / 32, x = e % 32;
+            const bool ok = t < len && d0 + x < DHQK;
+            qs[t * 33 + x] = ok ? to_f32(qb[(size_t)t * DHQK + d0 + x]) * scale : 0.f;
+            ks2[t * 33 + x] = ok ? to_f32(kb[(size_t)t * DHQK + d0 + x]) : 0.f;
+        }
+        __syncthreads();
+        for (int e = tid; e < L * L; e += blockDim.x) {
+            const int t = e / L, s = e % L;
+            if (s <= t) {
+                float acc = P[t * LP + s];
+#pragma unroll 8
+                for (int x = 0; x < 32; ++x) acc = fmaf(qs[t * 33 + x], ks2[s * 33 + x], acc);
+                P[t * LP + s] = acc;
+            }
+        }
+        __syncthreads();
+    }
+    // P = S * D, row sums
+    for (int e = tid; e < L * L; e += blockDim.x) {
+        const int t = e / L, s = e % L;
+        if (s <= t && t < len) P[t * LP + s] *= expf(ar[t] - ar[s] + ir[s] - mr[t]);
+        else P[t * LP + s] = 0.f;
+    }
+    __syncthreads();
+    for (int t = tid; t < L; t += blockDim.x) {
+        float r = 0.f;
+        for (int s = 0; s <= t; ++s) r += P[t * LP + s];
+        // inter-chunk normalizer term sc * n_c . qh
+        float dn = 0.f;
+        if (t < len) {
+            const float *nc = NS + ((size_t)bh * NC + ch) * DHQK;
+            for (int d = 0; d < DHQK; ++d) dn = fmaf(nc[d], to_f32(qb[(size_t)t * DHQK + d]), dn);
+            dn *= scale * sc[t];
+        }
+        den[t] = r + dn;
+    }
+    __syncthreads();
+
+    // num = sc * qh C_c + P V over the 32 columns of this tile.  Thread layout:
+    // column x = tid % 32, rows t = tid / 32 + 8 r.
+    const int x = tid & 31, ty = tid >> 5;
+    const int RPT = (L + 7) / 8;     // rows per thread (L <= 128 -> <= 16)
+    float acc[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+    const float *Cc = CS + ((size_t)bh * NC + ch) * DHQK * DHV;
+    for (int d0 = 0; d0 < DHQK; d0 += 32) {
+        for (int e = tid; e < L * 32; e += blockDim.x) {
+            const int t = e / 32, xx = e % 32;
+            const bool ok = t < len && d0 + xx < DHQK;
+            qs[t * 33 + xx] = ok ? to_f32(qb[(size_t)t * DHQK + d0 + xx]) * scale : 0.f;
+        }
+        for (int e = tid; e < 32 * 32; e += blockDim.x) {
+            const int d = e / 32, xx = e % 32;
+            cs[d * 33 + xx] = (d0 + d < DHQK && j0 + xx < DHV) ? Cc[(size_t)(d0 + d) * DHV + j0 + xx] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int t = ty + 8 * r;
+            if (r < RPT && t < L) {
+                float a2 = 0.f;
+#pragma unroll 8
+                for (int d = 0; d < 32; ++d) a2 = fmaf(qs[t * 33 + d], cs[d * 33 + x], a2);
+                acc[r] = fmaf(sc[t], a2, acc[r]);
+            }
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < L * 32; e += blockDim.x) {
+        const int s = e / 32, xx = e % 32;
+        ks2[s * 33 + xx] = (s < len && j0 + xx < DHV) ? to_f32(vb[(size_t)s * DHV + j0 + xx]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const int t = ty + 8 * r;
+        if (r < RPT && t < L) {
+            float a2 = 0.f;
+            for (int s = 0; s <= t; ++s) a2 = fmaf(P[t * LP + s], ks2[s * 33 + x], a2);
+            acc[r] += a2;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const int t = ty + 8 * r;
+        if (r < RPT && t < len && j0 + x < DHV) {
+            const size_t off = ((size_t)bh * S + t0 + t) * DHV + j0 + x;
+            const float o = ogate ? to_f32(ogate[off]) : 1.f;
+            h[off] = from_f32<T>(o * acc[r] / fmaxf(fabsf(den[t]), expf(-mr[t])));
+        }
+    }
+}
+
+template <typename T>
+static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark)
+{
+    const int L = a.chunk;
+    dim3 g1(a.BH, (a.DHQK + ST - 1) / ST, (a.DHV + ST - 1) / ST);
+    const size_t sm1 = sizeof(float) * (2 * (size_t)L * ST + L);
+    carry_simt_kernel<T><<<g1, 256, sm1, a.stream>>>((const T *)a.k, (const T *)a.v, a.igate, w.A, w.G, w.MC,
+                                                     a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS, a.C_final,
+                                                     a.n_final, a.m_final);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if ((e = mark(2)) != cudaSuccess) return e;   // the chunk scan is fused into the carry walk
+    if ((e = mark(3)) != cudaSuccess) return e;
+    dim3 g2(a.BH, w.NC, (a.DHV + ST - 1) / ST);
+    const size_t sm2 = sizeof(float) * ((size_t)L * (L + 1) + 2 * (size_t)L * 33 + 32 * 33 + 5 * (size_t)L);
+    static int smem_set = 0;   // opt in once per process (keeps the launch path capturable)
+    if (sm2 > 48 * 1024 && (int)sm2 > smem_set) {
+        e = cudaFuncSetAttribute(output_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+        if (e != cudaSuccess) return e;
+        smem_set = (int)sm2;
+    }
+    output_simt_kernel<T><<<g2, 256, sm2, a.stream>>>((const T *)a.q, (const T *)a.k, (const T *)a.v, a.igate,
+                                                      (const T *)a.ogate, w.A, w.M, w.MC, w.CS, w.NS, a.S, L,
+                                                      w.NC, a.DHQK, a.DHV, (T *)a.h);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark)
+{
+    return a.bf16 ? launch_fwd_simt_t<__nv_bfloat16>(a, w, mark) : launch_fwd_simt_t<float>(a, w, mark);
+}
+
+size_t simt_state_bytes(int BH, int NC, int DHQK, int DHV)
+{
+    return sizeof(float) * ((size_t)BH * NC * DHQK * DHV + (size_t)BH * NC * DHQK);
+}
+
+}  // namespace mlstm

@@ -1,0 +1,194 @@
+// mlstm_api.cu -- the C ABI of libmlstm: argument checks, workspace layout, dispatch.
+//
+// Every entry point checks its arguments on the host before it enqueues
+// anything, returns a status code and never throws.  Kernels are enqueued on
+// the caller's stream; nothing here synchronizes except mlstm_fwd_status.
+#include "mlstm.h"
+#include "mlstm_internal.h"
+
+#include <stdint.h>
+
+using namespace mlstm;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool dims_ok_fwd(int DHQK, int DHV)
+{
+    return DHQK >= 8 && DHQK <= 512 && DHQK % 8 == 0 && DHV >= 8 && DHV <= 512 && DHV % 8 == 0;
+}
+
+bool chunk_ok(int chunk) { return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128; }
+
+// Lays out the workspace (base may be NULL to size it).  Returns the bytes used.
+size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, FwdWorkspace *w)
+{
+    FwdWorkspace tmp;
+    if (!w) w = &tmp;
+    const int NC = (S + chunk - 1) / chunk;
+    w->NC = NC;
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char * {
+        char *p = base ? base + off : nullptr;
+        off = align_up(off + bytes, 256);
+        return p;
+    };
+    w->status = reinterpret_cast<uint32_t *>(take(sizeof(uint32_t)));
+    w->A = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * S));
+    w->M = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * S));
+    w->G = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC));
+    w->Bc = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC));
+    w->MC = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * (NC + 1)));
+    w->CS = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC * DHQK * DHV));
+    w->NS = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC * DHQK));
+    w->NSEG = 0;
+    w->R = 0;
+    w->SA = w->SG = w->SB = w->SM = w->DC = w->DN = w->SC = w->SN = nullptr;
+    return off;
+}
+
+mlstm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" const char *mlstm_status_string(mlstm_status s)
+{
+    switch (s) {
+    case MLSTM_OK: return "ok";
+    case MLSTM_ERR_INVALID_ARG: return "invalid argument (NULL pointer, negative size or misaligned pointer)";
+    case MLSTM_ERR_UNSUPPORTED: return "unsupported shape, chunk or dtype";
+    case MLSTM_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLSTM_ERR_CUDA: return "CUDA launch or runtime error";
+    case MLSTM_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    }
+    return "unknown status";
+}
+
+extern "C" size_t mlstm_fwd_workspace_size(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if (B < 0 || NH < 0 || S < 0 || (dt != MLSTM_F32 && dt != MLSTM_BF16)) return 0;
+    if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return 0;
+    return plan_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, nullptr);
+}
+
+extern "C" int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if (mlstm_fwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dt) == 0) return 0;
+    if (B == 0 || NH == 0 || S == 0) return 0;
+    return 3;   // gate preprocessing, carry walk, outputs
+}
+
+namespace {
+
+mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
+                      const void *ogate, mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                      void *h_out, float *C_final, float *n_final, float *m_final, void *workspace,
+                      size_t workspace_bytes, void *stream, void *const *events)
+{
+    if (B < 0 || NH < 0 || S < 0) return MLSTM_ERR_INVALID_ARG;
+    if (dt != MLSTM_F32 && dt != MLSTM_BF16) return MLSTM_ERR_UNSUPPORTED;
+    if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return MLSTM_ERR_UNSUPPORTED;
+    if ((long long)B * NH > (1LL << 30) || (long long)S * DHV > (1LL << 40)) return MLSTM_ERR_UNSUPPORTED;
+    const int BH = B * NH;
+    const bool has_tokens = BH > 0 && S > 0;
+    if (has_tokens) {
+        if (!q || !k || !v || !igate || !fgate || !h_out) return MLSTM_ERR_INVALID_ARG;
+        const void *ptrs[] = {q, k, v, igate, fgate, h_out};
+        for (const void *p : ptrs)
+            if (!aligned16(p)) return MLSTM_ERR_INVALID_ARG;
+        if (ogate && !aligned16(ogate)) return MLSTM_ERR_INVALID_ARG;
+    }
+    if ((C_final && !aligned16(C_final)) || (n_final && !aligned16(n_final)) || (m_final && !aligned16(m_final)))
+        return MLSTM_ERR_INVALID_ARG;
+    const size_t need = plan_workspace(nullptr, BH, S, DHQK, DHV, chunk, nullptr);
+    if (!workspace || workspace_bytes < need) return MLSTM_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLSTM_ERR_INVALID_ARG;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    FwdWorkspace w;
+    plan_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, &w);
+    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+    if (BH == 0) return MLSTM_OK;
+    if (S == 0) {   // the zero state
+        if (C_final) e = cudaMemsetAsync(C_final, 0, sizeof(float) * (size_t)BH * DHQK * DHV, st);
+        if (e == cudaSuccess && n_final) e = cudaMemsetAsync(n_final, 0, sizeof(float) * (size_t)BH * DHQK, st);
+        if (e == cudaSuccess && m_final) e = cudaMemsetAsync(m_final, 0, sizeof(float) * (size_t)BH, st);
+        return cuda_status(e);
+    }
+
+    PhaseMark mark;
+    mark.events = events;
+    mark.stream = st;
+    if (mark(0) != cudaSuccess) return MLSTM_ERR_CUDA;
+    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, st};
+    e = launch_gate_prep(gp);
+    if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+    if (mark(1) != cudaSuccess) return MLSTM_ERR_CUDA;
+    FwdArgs fa{q, k, v, ogate, igate, fgate, h_out, C_final, n_final, m_final, BH, S, DHQK, DHV, chunk,
+               dt == MLSTM_BF16, st};
+    e = launch_fwd_simt(fa, w, mark);
+    if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+    return cuda_status(mark(MLSTM_FWD_PHASES));
+}
+
+}  // namespace
+
+extern "C" {
+
+mlstm_status mlstm_fwd(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
+                       const void *ogate, mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                       void *h_out, float *C_final, float *n_final, float *m_final, void *workspace,
+                       size_t workspace_bytes, void *stream)
+{
+    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, h_out, C_final, n_final,
+                    m_final, workspace, workspace_bytes, stream, nullptr);
+}
+
+mlstm_status mlstm_fwd_profiled(const void *q, const void *k, const void *v, const float *igate,
+                                const float *fgate, const void *ogate, mlstm_dtype dt, int B, int NH, int S,
+                                int DHQK, int DHV, int chunk, void *h_out, float *C_final, float *n_final,
+                                float *m_final, void *workspace, size_t workspace_bytes, void *stream,
+                                void *const *events)
+{
+    if (!events) return MLSTM_ERR_INVALID_ARG;
+    for (int p = 0; p <= MLSTM_FWD_PHASES; ++p)
+        if (!events[p]) return MLSTM_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, h_out, C_final, n_final,
+                    m_final, workspace, workspace_bytes, stream, events);
+}
+
+mlstm_status mlstm_fwd_status(const void *workspace, void *stream)
+{
+    if (!workspace) return MLSTM_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MLSTM_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
+    return word == 0 ? MLSTM_OK : MLSTM_ERR_TIMEOUT;
+}
+
+mlstm_status mlstm_step(float *C, float *n, float *m, const void *q, const void *k, const void *v,
+                        const float *igate, const float *fgate, const void *ogate, mlstm_dtype dt, int B, int NH,
+                        int DHQK, int DHV, void *h_out, void *stream)
+{
+    if (B < 0 || NH < 0) return MLSTM_ERR_INVALID_ARG;
+    if (dt != MLSTM_F32 && dt != MLSTM_BF16) return MLSTM_ERR_UNSUPPORTED;
+    if (DHQK < 8 || DHQK > 512 || DHQK % 8 || DHV < 4 || DHV > 1024 || DHV % 4) return MLSTM_ERR_UNSUPPORTED;
+    if ((long long)B * NH > (1LL << 30)) return MLSTM_ERR_UNSUPPORTED;
+    const int BH = B * NH;
+    if (BH == 0) return MLSTM_OK;
+    if (!C || !n || !m || !q || !k || !v || !igate || !fgate || !h_out) return MLSTM_ERR_INVALID_ARG;
+    const void *ptrs[] = {C, n, m, q, k, v, igate, fgate, h_out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MLSTM_ERR_INVALID_ARG;
+    if (ogate && !aligned16(ogate)) return MLSTM_ERR_INVALID_ARG;
+    StepArgs a{C, n, m, q, k, v, ogate, igate, fgate, h_out, BH, DHQK, DHV, dt == MLSTM_BF16,
+               reinterpret_cast<cudaStream_t>(stream)};
+    return cuda_status(launch_step(a));
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// step.cu -- the recurrent decode step of the mLSTM cell (one token, state in place).
+//
+// "xLSTM Guide: Extended LSTM Architecture & Matrix Memory", "Recurrent
+// Formulation (Inference Mode)" applied once per (batch, head):
+//   m' = max(log f + m, i~),  f' = exp(log f + m - m'),  i' = exp(i~ - m')
+//   C' = f' C + i' k v^T,     n' = f' n + i' k
+//   h  = o * (C'^T qh) / max(|n' . qh|, exp(-m')),  qh = q / sqrt(DHQK)
+//
+// The step is bound by HBM: every byte of the fp32 state C is read once and
+// written once, and nothing else is of comparable size.  One CTA owns one head.
+// Its threads form RG row groups of DHV/4 threads; a thread owns four
+// consecutive columns of C (one 16-byte vector) and walks the rows i = g,
+// g + RG, ... so that each iteration the CTA streams RG whole rows, contiguous
+// in memory.  The column sums of h stay in the thread; the row groups are
+// combined through shared memory at the end.  n' . qh is a block reduction.
+// C is loaded and stored with the streaming (evict-first) cache hint since it
+// is touched once per step.
+#include "common.cuh"
+#include "mlstm_internal.h"
+
+namespace mlstm {
+
+template <typename T, int UNROLL>
+__global__ void __launch_bounds__(512, 2)
+step_kernel(float *__restrict__ C, float *__restrict__ n, float *__restrict__ m,
+            const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+            const float *__restrict__ igate, const float *__restrict__ fgate,
+            const T *__restrict__ ogate, int DHQK, int DHV, int RG, T *__restrict__ h)
+{
+    extern __shared__ float smem[];
+    float *qs = smem;                 // [DHQK] qh
+    float *ks = qs + DHQK;            // [DHQK] k
+    float *part = ks + DHQK;          // [RG][DHV] partial column sums
+    __shared__ float red[32];
+
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int nthr = blockDim.x;
+    const int tx = tid % (DHV / 4);   // column group
+    const int g = tid / (DHV / 4);    // row group
+
+    const float lf = log_sigmoid(fgate[bh]);
+    const float it = igate[bh];
+    const float m_old = m[bh];
+    const float m_new = fmaxf(lf + m_old, it);
+    const float fp = expf(lf + m_old - m_new);
+    const float ip = expf(it - m_new);
+    const float scale = rsqrtf((float)DHQK);
+
+    const T *qb = q + (size_t)bh * DHQK;
+    const T *kb = k + (size_t)bh * DHQK;
+    float *nb = n + (size_t)bh * DHQK;
+    float den = 0.f;
+    for (int i = tid; i < DHQK; i += nthr) {
+        const float qi = to_f32(qb[i]) * scale;
+        const float ki = to_f32(kb[i]);
+        const float ni = fp * nb[i] + ip * ki;
+        nb[i] = ni;
+        qs[i] = qi;
+        ks[i] = ki;
+        den += ni * qi;
+    }
+    den = warp_sum(den);
+    if ((tid & 31) == 0) red[tid >> 5] = den;
+    __syncthreads();
+    if (tid < 32) {
+        float x = tid < (nthr + 31) / 32 ? red[tid] : 0.f;
+        x = warp_sum(x);
+        if (tid == 0) red[0] = x;
+    }
+
+    const int j = tx * 4;
+    const float4 v4 = load4(v + (size_t)bh * DHV + j);
+    const float4 iv = make_float4(ip * v4.x, ip * v4.y, ip * v4.z, ip * v4.w);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float *Cb = C + (size_t)bh * DHQK * DHV + j;
+
+    int i = g;
+    for (; i + (UNROLL - 1) * RG < DHQK; i += UNROLL * RG) {
+        float4 c[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+            c[u] = __ldcs(reinterpret_cast<const float4 *>(Cb + (size_t)(i + u * RG) * DHV));
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const float kk = ks[i + u * RG], qq = qs[i + u * RG];
+            c[u].x = fmaf(fp, c[u].x, kk * iv.x);
+            c[u].y = fmaf(fp, c[u].y, kk * iv.y);
+            c[u].z = fmaf(fp, c[u].z, kk * iv.z);
+            c[u].w = fmaf(fp, c[u].w, kk * iv.w);
+            __stcs(reinterpret_cast<float4 *>(Cb + (size_t)(i + u * RG) * DHV), c[u]);
+            acc.x = fmaf(qq, c[u].x, acc.x);
+            acc.y = fmaf(qq, c[u].y, acc.y);
+            acc.z = fmaf(qq, c[u].z, acc.z);
+            acc.w = fmaf(qq, c[u].w, acc.w);
+        }
+    }
+    for (; i < DHQK; i += RG) {
+        float4 c = __ldcs(reinterpret_cast<const float4 *>(Cb + (size_t)i * DHV));
+        const float kk = ks[i], qq = qs[i];
+        c.x = fmaf(fp, c.x, kk * iv.x);
+        c.y = fmaf(fp, c.y, kk * iv.y);
+        c.z = fmaf(fp, c.z, kk * iv.z);
+        c.w = fmaf(fp, c.w, kk * iv.w);
+        __stcs(reinterpret_cast<float4 *>(Cb + (size_t)i * DHV), c);
+        acc.x = fmaf(qq, c.x, acc.x);
+        acc.y = fmaf(qq, c.y, acc.y);
+        acc.z = fmaf(qq, c.z, acc.z);
+        acc.w = fmaf(qq, c.w, acc.w);
+    }
+    *reinterpret_cast<float4 *>(part + (size_t)g * DHV + j) = acc;
+    __syncthreads();
+    if (g == 0) {
+        for (int r = 1; r < RG; ++r) {
+            const float4 p = *reinterpret_cast<const float4 *>(part + (size_t)r * DHV + j);
+            acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+        }
+        const float inv = 1.f / fmaxf(fabsf(red[0]), expf(-m_new));
+        float4 o4 = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (ogate) o4 = load4(ogate + (size_t)bh * DHV + j);
+        store4(h + (size_t)bh * DHV + j,
+               make_float4(o4.x * acc.x * inv, o4.y * acc.y * inv, o4.z * acc.z * inv, o4.w * acc.w * inv));
+        if (tid == 0) m[bh] = m_new;
+    }
+}
+
+template <typename T>
+static cudaError_t launch_step_t(const StepArgs &a)
+{
+    const int tx = a.DHV / 4;
+    int RG = 512 / tx;
+    if (RG < 1) RG = 1;
+    if (RG > a.DHQK) RG = a.DHQK;
+    const int threads = tx * RG;
+    const size_t smem = sizeof(float) * (2 * (size_t)a.DHQK + (size_t)RG * a.DHV);
+    step_kernel<T, 8><<<a.BH, threads, smem, a.stream>>>(
+        a.C, a.n, a.m, (const T *)a.q, (const T *)a.k, (const T *)a.v, a.igate, a.fgate,
+        (const T *)a.ogate, a.DHQK, a.DHV, RG, (T *)a.h);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_step(const StepArgs &a)
+{
+    return a.bf16 ? launch_step_t<__nv_bfloat16>(a) : launch_step_t<float>(a);
+}
+
+}  // namespace mlstm
