@@ -181,6 +181,23 @@ def set_bytes(s):
     return sum(t.numel() * t.element_size() for t in s.values() if t is not None)
 
 
+# ---------------------------------------------------------------- multi-rank host logic
+
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time: an all-reduce MAX when a process group is up, else ``ms``."""
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_step_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return world * units_per_step_per_rank * steps / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------- our arm
 
 class Runner:
@@ -284,11 +301,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     tw1 = time.time()
     barrier()
-    ms = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms], device=device, dtype=torch.float64)
-    if dist:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), device)
 
     # ---- per-phase timing (eager, the same K steps, events on the launching stream)
     nph = binding.FWD_PHASES
@@ -327,15 +340,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     te1 = time.time()
     clocks.stop()
-    e2e_ms = e0.elapsed_time(e1)
-    t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-    if dist:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
 
     tokens_per_step = w.B * (w.S + 1)
-    value = world * tokens_per_step * args.steps / (ms_max / 1e3)
-    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, ms_max)
+    e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
     fw = fwd_work(w, "")
@@ -410,7 +419,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 def path_is_tensor(w: Workload) -> bool:
-    return False   # the chunkwise path in use computes on CUDA cores
+    """True when the library takes its tensor-core path for this workload (4 launches)."""
+    return binding.fwd_kernel_launches(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 4
 
 
 def extras(device, peaks):

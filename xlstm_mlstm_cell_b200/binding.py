@@ -135,6 +135,9 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
         _check("mlstm_fwd", lib.mlstm_fwd(*args))
     else:
         assert len(events) == FWD_PHASES + 1
+        for e in events:            # torch creates the CUDA event lazily, on its first record
+            if not e.cuda_event:
+                e.record()
         arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[e.cuda_event for e in events])
         _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
     return h_out, C_final, n_final, m_final

@@ -51,4 +51,23 @@ MLSTM_DEVINL float warp_sum(float x)
     return x;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), so that
+// launches stay free of attribute calls after the first one.
+inline cudaError_t ensure_dynamic_smem(const void *kernel, int bytes)
+{
+    struct Entry { const void *fn; int dev; int bytes; };
+    static Entry reg[128];
+    static int used = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    for (int i = 0; i < used; ++i)
+        if (reg[i].fn == kernel && reg[i].dev == dev && reg[i].bytes >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < used; ++i)
+        if (reg[i].fn == kernel && reg[i].dev == dev) { reg[i].bytes = bytes; return cudaSuccess; }
+    if (used < 128) reg[used++] = Entry{kernel, dev, bytes};
+    return cudaSuccess;
+}
+
 }  // namespace mlstm

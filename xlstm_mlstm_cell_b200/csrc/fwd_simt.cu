@@ -253,12 +253,8 @@ static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, co
     if ((e = mark(3)) != cudaSuccess) return e;
     dim3 g2(a.BH, w.NC, (a.DHV + ST - 1) / ST);
     const size_t sm2 = sizeof(float) * ((size_t)L * (L + 1) + 2 * (size_t)L * 33 + 32 * 33 + 5 * (size_t)L);
-    static int smem_set = 0;   // opt in once per process (keeps the launch path capturable)
-    if (sm2 > 48 * 1024 && (int)sm2 > smem_set) {
-        e = cudaFuncSetAttribute(output_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-        if (e != cudaSuccess) return e;
-        smem_set = (int)sm2;
-    }
+    if (sm2 > 48 * 1024 && (e = ensure_dynamic_smem((const void *)output_simt_kernel<T>, (int)sm2)) != cudaSuccess)
+        return e;
     output_simt_kernel<T><<<g2, 256, sm2, a.stream>>>((const T *)a.q, (const T *)a.k, (const T *)a.v, a.igate,
                                                       (const T *)a.ogate, w.A, w.M, w.MC, w.CS, w.NS, a.S, L,
                                                       w.NC, a.DHQK, a.DHV, (T *)a.h);

@@ -1,0 +1,837 @@
+// fwd_tc.cu -- chunkwise forward pass on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// Inputs q, k, v, o are bf16; gates, states and accumulation are fp32.  The
+// sequence of every (batch, head) is cut into chunks of L tokens, and the chunks
+// into NSEG segments of R chunks.  Three kernels follow the gate preprocessing:
+//
+// 1. segsum (tensor cores): for every segment, its contribution to the state,
+//      dC_s^T = V_s^T diag(w) K_s,  dn_s = K_s^T w,
+//      w_t = exp(G_s - A_t + i~_t - b_s) <= 1
+//    where A_t is the segment-local cumulative log decay, G_s its total and
+//    (G_s, b_s) the max-plus map of the segment (the composition of its chunk
+//    maps).  One long-K GEMM per (segment, value tile); K rows are scaled by w
+//    in shared memory between the TMA load and the MMA.
+// 2. seg_scan (CUDA cores): the state at every segment start by an in-place
+//    exclusive scan over segments,
+//      C_{s+1} = exp(G_s + M_s - M_{s+1}) C_s + exp(b_s - M_{s+1}) dC_s,
+//    and the final state.  This is the scan across chunks of the xLSTM Guide's
+//    "Exploit Chunkwise Hardware Kernels for Production Training", taken per
+//    segment.
+// 3. walk (tensor cores): one CTA per (segment, 128-wide value tile) starts from
+//    the segment's state, kept in TMEM in fp32, and walks its chunks in order.
+//    Per chunk, with the per-token stabilizer m and chunk-local cumulative log
+//    decay a of the gate preprocessing:
+//      S   = Q K^T                                      (tcgen05, fp32 in TMEM)
+//      P   = S * D * d^-1/2,  D_ts = exp(a_t - a_s + i~_s - m_t), s <= t      (<= 1)
+//      H^T = Cb^T Q'^T + V^T P'^T                       (tcgen05; Cb^T read from TMEM)
+//      h_t = o_t * r_t H_t / max(|rowsum(P)_t + sc_t q_t . n|, exp(-m_t))
+//      C^T += V^T K',  n += sum_s W_s k_s               (state for the next chunk)
+//    with sc_t = exp(a_t + m_c - m_t) / sqrt(d) = r_t 2^e_t (r_t in [1, 2)),
+//    Q' = diag(2^(e_t + kc)) Q and Cb = C_c 2^-kc in fp16 (kc a power-of-two range
+//    scale per chunk; q is bf16, so Q' is exact), P' = diag(1/r) P in bf16 and
+//    K' = diag(W) K in bf16.  The causal decay matrix D and the inter-chunk term
+//    are those of the guide's "The Dual Formulation" restricted to a chunk.
+//    The normalizer and the inter-chunk part of the denominator are computed in
+//    fp32 from the unrounded q and k: rounding them dominated the error through
+//    cancellation in the denominator, and the fp16 inter-chunk product keeps
+//    inputs with one dominant token (huge input gates) within the error budget.
+//
+//    The state in TMEM is kept in a lazily rescaled frame: TMEM holds
+//    X = Cbar exp(-rho) (Cbar the unstabilized state), the chunk decay is folded
+//    into rho instead of rescaling TMEM, and new tokens enter with weight
+//    W_s = exp(i~_s - a_s - rho) <= exp(THRESH).  TMEM is rescaled only when that
+//    bound would be exceeded.  Cb is always the stabilized C_c = X exp(rho - m_c).
+#include "common.cuh"
+#include "mlstm_internal.h"
+#include "tc_common.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace mlstm {
+namespace tcfwd {
+
+using namespace tc;
+
+constexpr int DVT = 128;         // value columns per CTA (TMEM lanes of the state)
+constexpr int TB = 64;           // tokens per pipeline stage in segsum
+constexpr int SS_STAGES = 4;
+constexpr float THRESH = 20.f;   // log of the largest weight before TMEM is rescaled
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct Params {
+    int S, L, NC, R, NSEG, DK, DV, BH;
+    const float *A, *Mtok, *ig, *MC, *G, *GP, *SGb;
+    float *DC, *DN;
+    const __nv_bfloat16 *o;
+    __nv_bfloat16 *h;
+    uint32_t *status;
+};
+
+// ---------------------------------------------------------------- segsum
+
+template <int DK>
+struct SegSmem {
+    static constexpr uint32_t K_BYTES = DK * TB * 2;
+    static constexpr uint32_t V_BYTES = DVT * TB * 2;
+    static constexpr uint32_t STAGE = K_BYTES + V_BYTES;
+    static constexpr uint32_t BAR_OFF = STAGE * SS_STAGES;
+    static constexpr uint32_t TOTAL = BAR_OFF + 128 + TB * 4 + 1024;   // + barriers, weights, alignment slack
+};
+
+template <int DK>
+__global__ void __launch_bounds__(192, 1)
+segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Params p)
+{
+    using SM = SegSmem<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
+    uint64_t *scaled = full + SS_STAGES;
+    uint64_t *empty = scaled + SS_STAGES;
+    uint64_t *acc_full = empty + SS_STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint32_t *abort_flag = tmem_slot + 1;
+    float *wst = reinterpret_cast<float *>(smem + SM::BAR_OFF + 128);   // [TB] weights of the stage
+
+    const int tile = blockIdx.x, seg = blockIdx.y, bh = blockIdx.z;
+    const int j0 = tile * DVT;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_begin = seg * p.R * p.L;
+    const int t_end = min(t_begin + p.R * p.L, p.S);
+    const int nstage = (t_end - t_begin + TB - 1) / TB;
+    WaitCtx wc{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < SS_STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&scaled[i], 4);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_k);
+        tma_prefetch(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {   // TMA producer
+            int issued = 0;
+            for (int it = 0; it < nstage; ++it) {
+                const int st = it % SS_STAGES;
+                const uint32_t ph = (uint32_t)(it / SS_STAGES) & 1u;
+                if (it >= SS_STAGES && !mbar_wait(&empty[st], ph ^ 1u, wc)) break;
+                ++issued;
+                uint8_t *kb = smem + st * SM::STAGE;
+                uint8_t *vb = kb + SM::K_BYTES;
+                const int t0 = t_begin + it * TB;
+                mbar_arrive_expect_tx(&full[st], SM::STAGE);
+                for (int b = 0; b < DK / 64; ++b) tma_load_3d(kb + b * TB * 128, &tm_k, b * 64, t0, bh, &full[st]);
+                for (int b = 0; b < DVT / 64; ++b)
+                    tma_load_3d(vb + b * TB * 128, &tm_v, j0 + b * 64, t0, bh, &full[st]);
+            }
+            for (int it = issued > SS_STAGES ? issued - SS_STAGES : 0; it < issued; ++it)   // drain
+                mbar_wait_drain(&full[it % SS_STAGES], (uint32_t)(it / SS_STAGES) & 1u);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // MMA issuer: dC^T (DVT x DK) += V^T (DVT x TB) * K' (TB x DK)
+            constexpr uint32_t IDESC = idesc_bf16(DVT, DK, 1, 1);
+            int it = 0;
+            for (; it < nstage; ++it) {
+                const int st = it % SS_STAGES;
+                const uint32_t ph = (uint32_t)(it / SS_STAGES) & 1u;
+                if (!mbar_wait(&scaled[st], ph, wc)) break;
+                tc_fence_after();
+                const uint32_t kb = smem_u32(smem + st * SM::STAGE);
+                const uint32_t vb = kb + SM::K_BYTES;
+#pragma unroll
+                for (int k = 0; k < TB / 16; ++k) {
+                    const uint64_t a = smem_desc(vb + k * 2048, TB * 128, 1024);
+                    const uint64_t b = smem_desc(kb + k * 2048, TB * 128, 1024);
+                    mma_ss(tmem, a, b, IDESC, (it > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[st]);
+            }
+            mma_commit(acc_full);
+            mbar_wait_drain(acc_full, 0);
+        }
+    } else {
+        // scalers (warps 2..5): K rows *= w, then (tile 0) dn += column sums of K'
+        const int ct = threadIdx.x - 64;                 // 0..127
+        const float Gs = p.SGb[((size_t)bh * p.NSEG + seg) * 2 + 0];
+        const float bs = p.SGb[((size_t)bh * p.NSEG + seg) * 2 + 1];
+        const float *Ab = p.A + (size_t)bh * p.S;
+        const float *igb = p.ig + (size_t)bh * p.S;
+        const float *GPb = p.GP + (size_t)bh * p.NC;
+        float n0 = 0.f, n1 = 0.f;
+        bool ok = true;
+        for (int it = 0; it < nstage; ++it) {
+            const int st = it % SS_STAGES;
+            const uint32_t ph = (uint32_t)(it / SS_STAGES) & 1u;
+            if (!mbar_wait(&full[st], ph, wc)) { ok = false; break; }
+            uint8_t *kb = smem + st * SM::STAGE;
+            const int r = ct & (TB - 1);                 // row of the stage
+            const int t = t_begin + it * TB + r;
+            float w = 0.f;
+            if (t < t_end) w = expf(Gs - GPb[t / p.L] - Ab[t] + igb[t] - bs);
+            if (tile == 0) {
+                // dn += sum_r w_r k_r from the unrounded bf16 k, in fp32, before K is scaled
+                if (ct < TB) wst[ct] = w;
+                named_sync(1, 128);
+                for (int rr = 0; rr < TB; ++rr) {
+                    const float wr = wst[rr];
+                    if (ct < DK)
+                        n0 += wr * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kb + sw128_offset(rr, ct, TB)));
+                    if (DK > 128)
+                        n1 += wr * __bfloat162float(
+                                       *reinterpret_cast<const __nv_bfloat16 *>(kb + sw128_offset(rr, ct + 128, TB)));
+                }
+                named_sync(1, 128);
+            }
+            // each thread scales half of its row: chunks [half * DK/16, (half+1) * DK/16)
+            const int half = ct / TB;
+            constexpr int CPR = DK / 8;                  // 16-byte chunks per row
+            for (int j = half * (CPR / 2); j < (half + 1) * (CPR / 2); ++j) {
+                uint4 *ptr = reinterpret_cast<uint4 *>(kb + sw128_chunk(r, j, TB));
+                uint4 u = *ptr;
+                float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z), f3 = unpack_bf16(u.w);
+                u.x = pack_bf16(f0.x * w, f0.y * w);
+                u.y = pack_bf16(f1.x * w, f1.y * w);
+                u.z = pack_bf16(f2.x * w, f2.y * w);
+                u.w = pack_bf16(f3.x * w, f3.y * w);
+                *ptr = u;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&scaled[st]);
+        }
+        // epilogue: TMEM (lane = value column, columns = DK) -> workspace, quad layout [DK/4][DV][4]
+        if (ok && mbar_wait(acc_full, 0, wc)) {
+            tc_fence_after();
+            const int q = warp & 3;
+            const int j = q * 32 + lane;
+            float *dst = p.DC + ((size_t)bh * p.NSEG + seg) * (size_t)DK * p.DV;
+            for (int c0 = 0; c0 < DK; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem_addr(tmem, q * 32, c0), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float4 v4 = make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                            __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+                    *reinterpret_cast<float4 *>(dst + ((size_t)((c0 >> 2) + u) * p.DV + j0 + j) * 4) = v4;
+                }
+            }
+            if (tile == 0) {
+                float *dn = p.DN + ((size_t)bh * p.NSEG + seg) * DK;
+                if (ct < DK) dn[ct] = n0;
+                if (DK > 128 && ct + 128 < DK) dn[ct + 128] = n1;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------- scan over segments
+
+__global__ void __launch_bounds__(256)
+seg_scan_kernel(Params p, float *__restrict__ C_final, float *__restrict__ n_final, float *__restrict__ m_final)
+{
+    const int bh = blockIdx.y;
+    const int nquad = p.DK * p.DV / 4;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;    // quad index: (i4, j) = (e / DV, e % DV)
+    const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
+    const float *SG = p.SGb + (size_t)bh * p.NSEG * 2;
+    if (e < nquad) {
+        float4 C = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < p.NSEG; ++s) {
+            float4 *slot = reinterpret_cast<float4 *>(p.DC + ((size_t)bh * p.NSEG + s) * (size_t)p.DK * p.DV) + e;
+            const float4 d = *slot;
+            *slot = C;
+            const float Ms = MCb[s * p.R], Mn = MCb[min((s + 1) * p.R, p.NC)];
+            const float gam = expf(SG[2 * s] + Ms - Mn), bet = expf(SG[2 * s + 1] - Mn);
+            C.x = gam * C.x + bet * d.x;
+            C.y = gam * C.y + bet * d.y;
+            C.z = gam * C.z + bet * d.z;
+            C.w = gam * C.w + bet * d.w;
+        }
+        if (C_final) {
+            const int i4 = e / p.DV, j = e % p.DV;
+            float *cf = C_final + (size_t)bh * p.DK * p.DV;
+            cf[(size_t)(4 * i4 + 0) * p.DV + j] = C.x;
+            cf[(size_t)(4 * i4 + 1) * p.DV + j] = C.y;
+            cf[(size_t)(4 * i4 + 2) * p.DV + j] = C.z;
+            cf[(size_t)(4 * i4 + 3) * p.DV + j] = C.w;
+        }
+    }
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < p.DK; i += blockDim.x) {
+            float n = 0.f;
+            for (int s = 0; s < p.NSEG; ++s) {
+                float *slot = p.DN + ((size_t)bh * p.NSEG + s) * p.DK + i;
+                const float d = *slot;
+                *slot = n;
+                const float Ms = MCb[s * p.R], Mn = MCb[min((s + 1) * p.R, p.NC)];
+                n = expf(SG[2 * s] + Ms - Mn) * n + expf(SG[2 * s + 1] - Mn) * d;
+            }
+            if (n_final) n_final[(size_t)bh * p.DK + i] = n;
+        }
+        if (m_final && threadIdx.x == 0) m_final[bh] = MCb[p.NC];
+    }
+}
+
+// ---------------------------------------------------------------- walk
+
+template <int DK, int L>
+struct WalkSmem {
+    static constexpr uint32_t Q_OFF = 0;
+    static constexpr uint32_t K_OFF = Q_OFF + DK * L * 2;
+    static constexpr uint32_t V_OFF = K_OFF + DK * L * 2;
+    static constexpr uint32_t P_OFF = V_OFF + DVT * L * 2;
+    static constexpr uint32_t F_OFF = P_OFF + L * L * 2;          // float arrays
+    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [2][L]; dint [4][L]; inv, ivalid, qexp, rrow [L];
+    // nX [DK]; red [16]
+    static constexpr uint32_t NF = L * 15 + DK + 16;
+    static constexpr uint32_t BAR_OFF = F_OFF + NF * 4;
+    static constexpr uint32_t TOTAL = BAR_OFF + 16 * 8 + 16 + 1024;
+    static constexpr uint32_t C_COL = 0, CB_COL = DK, HS_COL = DK + DK / 2;
+};
+
+template <int DK, int L>
+__global__ void __launch_bounds__(320, 1)
+walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const __grid_constant__ CUtensorMap tm_v, Params p)
+{
+    using SM = WalkSmem<DK, L>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *Qs = smem + SM::Q_OFF;
+    uint8_t *Ks = smem + SM::K_OFF;
+    uint8_t *Vs = smem + SM::V_OFF;
+    uint8_t *Ps = smem + SM::P_OFF;
+    float *F = reinterpret_cast<float *>(smem + SM::F_OFF);
+    float *arow = F, *mrow = F + L, *icol = F + 2 * L, *srow = F + 3 * L, *wcol = F + 4 * L;
+    float *rs = F + 5 * L, *dint = F + 7 * L, *inv = F + 11 * L, *ivalid = F + 12 * L;
+    float *qexp = F + 13 * L, *rrow = F + 14 * L, *nX = F + 15 * L, *red = nX + DK;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
+    uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *h_full = bars + 4;
+    uint64_t *c_upd = bars + 5, *q_empty = bars + 6, *k_empty = bars + 7, *v_empty = bars + 8, *ep1 = bars + 9;
+    uint64_t *hs_free = bars + 10, *drain = bars + 11;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    uint32_t *abort_flag = tmem_slot + 1;
+
+    const int tile = blockIdx.x, seg = blockIdx.y, bh = blockIdx.z;
+    const int j0 = tile * DVT;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c_begin = seg * p.R;
+    const int nck = min(p.R, p.NC - c_begin);
+    WaitCtx wc{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(k_full, 1);
+        mbar_init(v_full, 1);
+        mbar_init(s_full, 1);
+        mbar_init(h_full, 1);
+        mbar_init(c_upd, 1);
+        mbar_init(q_empty, 1);
+        mbar_init(k_empty, 1);
+        mbar_init(v_empty, 1);
+        mbar_init(ep1, 8);
+        mbar_init(hs_free, 8);
+        mbar_init(drain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_q);
+        tma_prefetch(&tm_k);
+        tma_prefetch(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {   // TMA producer: Q, K (all DK) and the V tile of every chunk
+            int nq = 0, nk = 0, nv = 0;
+            for (int i = 0; i < nck; ++i) {
+                const int t0 = (c_begin + i) * L;
+                const uint32_t pp = (uint32_t)(i - 1) & 1u;
+                if (i > 0 && !mbar_wait(q_empty, pp, wc)) break;
+                mbar_arrive_expect_tx(q_full, DK * L * 2);
+                for (int b = 0; b < DK / 64; ++b) tma_load_3d(Qs + b * L * 128, &tm_q, b * 64, t0, bh, q_full);
+                ++nq;
+                if (i > 0 && !mbar_wait(k_empty, pp, wc)) break;
+                mbar_arrive_expect_tx(k_full, DK * L * 2);
+                for (int b = 0; b < DK / 64; ++b) tma_load_3d(Ks + b * L * 128, &tm_k, b * 64, t0, bh, k_full);
+                ++nk;
+                if (i > 0 && !mbar_wait(v_empty, pp, wc)) break;
+                mbar_arrive_expect_tx(v_full, DVT * L * 2);
+                for (int b = 0; b < DVT / 64; ++b)
+                    tma_load_3d(Vs + b * L * 128, &tm_v, j0 + b * 64, t0, bh, v_full);
+                ++nv;
+            }
+            // drain: the last load issued into each buffer has landed
+            if (nq > 0) mbar_wait_drain(q_full, (uint32_t)(nq - 1) & 1u);
+            if (nk > 0) mbar_wait_drain(k_full, (uint32_t)(nk - 1) & 1u);
+            if (nv > 0) mbar_wait_drain(v_full, (uint32_t)(nv - 1) & 1u);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // MMA issuer
+            constexpr uint32_t ID_S = idesc_bf16(L, L, 0, 0);       // S  = Q K^T
+            constexpr uint32_t ID_HC = idesc_f16(DVT, L, 0, 0);     // H^T = Cb^T Q'^T   (fp16, A in TMEM)
+            constexpr uint32_t ID_HP = idesc_bf16(DVT, L, 1, 0);    // H^T += V^T P^T
+            constexpr uint32_t ID_C = idesc_bf16(DVT, DK, 1, 1);    // C^T += V^T K'
+            const uint32_t qa = smem_u32(Qs), ka = smem_u32(Ks), va = smem_u32(Vs), pa = smem_u32(Ps);
+            const uint32_t hs = tmem + SM::HS_COL;
+            for (int i = 0; i < nck; ++i) {
+                const uint32_t ph = (uint32_t)i & 1u;
+                if (!mbar_wait(q_full, ph, wc)) break;
+                if (!mbar_wait(k_full, ph, wc)) break;
+                if (i > 0 && !mbar_wait(hs_free, ph ^ 1u, wc)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = (k >> 2) * L * 128 + (k & 3) * 32;
+                    mma_ss(hs, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), ID_S, k > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full);
+                if (!mbar_wait(ep1, ph, wc)) break;
+                if (!mbar_wait(v_full, ph, wc)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = (k >> 2) * L * 128 + (k & 3) * 32;
+                    mma_ts(hs, tmem + SM::CB_COL + k * 8, smem_desc(qa + off, 16, 1024), ID_HC, k > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int k = 0; k < L / 16; ++k) {
+                    const uint32_t poff = (k >> 2) * L * 128 + (k & 3) * 32;
+                    mma_ss(hs, smem_desc(va + k * 2048, L * 128, 1024), smem_desc(pa + poff, 16, 1024), ID_HP, 1u);
+                }
+                mma_commit(h_full);
+                mma_commit(q_empty);
+                if (i < nck - 1) {
+#pragma unroll
+                    for (int k = 0; k < L / 16; ++k)
+                        mma_ss(tmem + SM::C_COL, smem_desc(va + k * 2048, L * 128, 1024),
+                               smem_desc(ka + k * 2048, L * 128, 1024), ID_C, 1u);
+                    mma_commit(c_upd);
+                }
+                mma_commit(k_empty);
+                mma_commit(v_empty);
+            }
+            mma_commit(drain);           // every MMA of this CTA has completed
+            mbar_wait_drain(drain, 0);
+        }
+    } else {
+        // compute warps 2..9: two per TMEM lane quadrant
+        const int ct = threadIdx.x - 64;          // 0..255
+        const int q = warp & 3;                   // TMEM lane quadrant
+        const int hf = (warp - 2) >> 2;           // which half of the columns
+        const float scale = rsqrtf((float)DK);
+        const float *Ab = p.A + (size_t)bh * p.S;
+        const float *Mb = p.Mtok + (size_t)bh * p.S;
+        const float *igb = p.ig + (size_t)bh * p.S;
+        const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
+        const float *Gb = p.G + (size_t)bh * p.NC;
+
+        // the segment's start state -> TMEM (C^T, lane = value column) and shared (n)
+        {
+            const float *src = p.DC + ((size_t)bh * p.NSEG + seg) * (size_t)DK * p.DV;
+            const int j = q * 32 + lane;
+            for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
+                uint32_t r[32];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(src + ((size_t)((c0 >> 2) + u) * p.DV + j0 + j) * 4);
+                    r[4 * u] = __float_as_uint(v4.x);
+                    r[4 * u + 1] = __float_as_uint(v4.y);
+                    r[4 * u + 2] = __float_as_uint(v4.z);
+                    r[4 * u + 3] = __float_as_uint(v4.w);
+                }
+                tmem_st32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+            }
+            tmem_wait_st();
+            for (int i = ct; i < DK; i += 256) nX[i] = p.DN[((size_t)bh * p.NSEG + seg) * DK + i];
+        }
+        float rho = MCb[c_begin];
+        bool ok = true;
+
+        for (int i = 0; i < nck && ok; ++i) {
+            const int c = c_begin + i;
+            const int t0 = c * L;
+            const int len = min(L, p.S - t0);
+            const uint32_t ph = (uint32_t)i & 1u;
+            const float mc = MCb[c], mn = MCb[c + 1], g = Gb[c];
+            const bool last = (i == nck - 1);
+            const bool rescale = !last && (mn - (rho + g) > THRESH);
+            const float rho_new = rescale ? (mn - g) : rho;
+            const float alpha = expf(rho - mc);
+            const float beta = expf(rho - rho_new);
+
+            named_sync(1, 256);   // previous chunk's readers of the per-row arrays are done
+            if (ct < L) {
+                const int t = t0 + ct;
+                if (ct < len) {
+                    const float a = Ab[t], m = Mb[t], it = igb[t];
+                    arow[ct] = (a - m) * LOG2E;
+                    mrow[ct] = m;
+                    icol[ct] = (it - a) * LOG2E;
+                    const float sc = expf(a + mc - m) * scale;
+                    srow[ct] = sc;
+                    int ex = 0;
+                    const float fr = frexpf(sc, &ex);            // sc = fr 2^ex, fr in [0.5, 1)
+                    qexp[ct] = sc > 0.f ? (float)(ex - 1) : -1000.f;
+                    rrow[ct] = sc > 0.f ? 2.f * fr : 1.f;
+                    wcol[ct] = last ? 0.f : expf(it - a - rho_new);
+                    ivalid[ct] = 1.f;
+                } else {
+                    arow[ct] = 0.f;
+                    mrow[ct] = 0.f;
+                    icol[ct] = -INFINITY;
+                    srow[ct] = 0.f;
+                    qexp[ct] = -1000.f;
+                    rrow[ct] = 1.f;
+                    wcol[ct] = 0.f;
+                    ivalid[ct] = 0.f;
+                }
+            }
+            named_sync(1, 256);
+
+            // (b) Cb = fp16(C_c 2^-kc) into TMEM, kc from max |C_c| over the tile; rescale the
+            //     fp32 state when the frame moves
+            if (i > 0 && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
+            tc_fence_after();
+            float cmax = 0.f;
+            for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) cmax = fmaxf(cmax, fabsf(__uint_as_float(r[u])));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+            if (lane == 0) red[ct >> 5] = cmax;
+            named_sync(1, 256);
+            cmax = red[0];
+#pragma unroll
+            for (int w8 = 1; w8 < 8; ++w8) cmax = fmaxf(cmax, red[w8]);
+            cmax *= alpha;
+            int kc = 0;
+            if (cmax > 0.f) {
+                int ex = 0;
+                frexpf(cmax, &ex);                       // cmax < 2^ex
+                kc = min(max(ex - 8, -120), 14);         // |Cb| < 2^8
+            }
+            const float cbs = ldexpf(alpha, -kc);
+            for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    pk[u] = pack_f16(__uint_as_float(r[2 * u]) * cbs, __uint_as_float(r[2 * u + 1]) * cbs);
+                tmem_st16(tmem_addr(tmem, q * 32, SM::CB_COL + c0 / 2), pk);
+                if (rescale) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
+                    tmem_st32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                }
+            }
+            tmem_wait_st();
+
+            // (c) S -> P (bf16, shared, K-major swizzled), row sums
+            if (!mbar_wait(s_full, ph, wc)) { ok = false; break; }
+            tc_fence_after();
+            if (L == 128) {
+                const int tau = q * 32 + lane;
+                float sum = 0.f;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int s0 = hf * 64 + u * 32;
+                    uint32_t r[32];
+                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                    tmem_wait_ld();
+                    const float at = arow[tau];
+                    const float ri = 1.f / rrow[tau];
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float v2[2];
+#pragma unroll
+                        for (int z = 0; z < 2; ++z) {
+                            const int sg = s0 + 2 * e + z;
+                            float d = 0.f;
+                            if (sg <= tau) d = exp2f(at + icol[sg]);
+                            v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
+                            sum += v2[z];
+                        }
+                        pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int jc = (s0 >> 3) + e;          // 16-byte chunk index within the row
+                        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jc, L)) =
+                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                }
+                rs[hf * L + tau] = sum;
+            } else {   // L == 64: M = 64 accumulator, rows 16q..16q+15 in lanes 0..15 of quadrant q
+                const int tau = q * 16 + (lane & 15);
+                const int s0 = hf * 32;
+                uint32_t r[32];
+                tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    float sum = 0.f;
+                    const float at = arow[tau];
+                    const float ri = 1.f / rrow[tau];
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float v2[2];
+#pragma unroll
+                        for (int z = 0; z < 2; ++z) {
+                            const int sg = s0 + 2 * e + z;
+                            float d = 0.f;
+                            if (sg <= tau) d = exp2f(at + icol[sg]);
+                            v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
+                            sum += v2[z];
+                        }
+                        pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int jc = (s0 >> 3) + e;
+                        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jc, L)) =
+                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                    rs[hf * L + tau] = sum;
+                }
+            }
+
+            named_sync(1, 256);
+
+            // (e1) inter-chunk denominator alpha * sc_t * (q_t . nX) from the unscaled bf16 q, in fp32
+            {
+                constexpr int PARTS = 256 / L;
+                const int row = ct % L, part = ct / L;
+                constexpr int SPAN = DK / PARTS;
+                float acc = 0.f;
+                for (int d = part * SPAN; d < (part + 1) * SPAN; d += 8) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(Qs + sw128_chunk(row, d >> 3, L));
+                    const float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z),
+                                 f3 = unpack_bf16(u.w);
+                    acc += f0.x * nX[d] + f0.y * nX[d + 1] + f1.x * nX[d + 2] + f1.y * nX[d + 3] +
+                           f2.x * nX[d + 4] + f2.y * nX[d + 5] + f3.x * nX[d + 6] + f3.y * nX[d + 7];
+                }
+                dint[part * L + row] = acc * alpha * srow[row];
+            }
+            named_sync(1, 256);
+            // (e2) normalizer for the next chunk from the unscaled bf16 k and fp32 weights;
+            //      1 / denominator of this chunk
+            if (!last) {
+                for (int d = ct; d < DK; d += 256) {
+                    float acc = nX[d] * beta;
+                    for (int s = 0; s < len; ++s)
+                        acc += wcol[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Ks + sw128_offset(s, d, L)));
+                    nX[d] = acc;
+                }
+            }
+            if (ct < L) {
+                constexpr int PARTS = 256 / L;
+                float den = rs[ct] + rs[L + ct];
+#pragma unroll
+                for (int pp = 0; pp < PARTS; ++pp) den += dint[pp * L + ct];
+                inv[ct] = rrow[ct] / fmaxf(fabsf(den), expf(-mrow[ct]));
+            }
+            named_sync(1, 256);
+
+            // (d) Q' = diag(2^(e + kc)) Q in fp16 (exact) and K' = diag(W) K in bf16, in place
+            for (int e = ct; e < L * (DK / 8); e += 256) {
+                const int row = e % L, jc = e / L;
+                uint4 *pq = reinterpret_cast<uint4 *>(Qs + sw128_chunk(row, jc, L));
+                uint4 *pkk = reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, jc, L));
+                const int qe = (int)qexp[row] + kc;
+                const float sk = wcol[row];
+                uint4 u = *pq;
+                float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z), f3 = unpack_bf16(u.w);
+                *pq = make_uint4(pack_f16(ldexpf(f0.x, qe), ldexpf(f0.y, qe)),
+                                 pack_f16(ldexpf(f1.x, qe), ldexpf(f1.y, qe)),
+                                 pack_f16(ldexpf(f2.x, qe), ldexpf(f2.y, qe)),
+                                 pack_f16(ldexpf(f3.x, qe), ldexpf(f3.y, qe)));
+                u = *pkk;
+                f0 = unpack_bf16(u.x); f1 = unpack_bf16(u.y); f2 = unpack_bf16(u.z); f3 = unpack_bf16(u.w);
+                *pkk = make_uint4(pack_bf16(f0.x * sk, f0.y * sk), pack_bf16(f1.x * sk, f1.y * sk),
+                                  pack_bf16(f2.x * sk, f2.y * sk), pack_bf16(f3.x * sk, f3.y * sk));
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_sync(1, 256);
+            if (lane == 0) mbar_arrive(ep1);
+
+            // (g) outputs: H^T (lane = value column j, columns = tokens)
+            if (!mbar_wait(h_full, ph, wc)) { ok = false; break; }
+            tc_fence_after();
+            {
+                const int j = q * 32 + lane;
+                const size_t rowbase = ((size_t)bh * p.S + t0) * p.DV + j0 + j;
+#pragma unroll
+                for (int u = 0; u < L / 64; ++u) {
+                    const int tb = hf * (L / 2) + u * 32;
+                    uint32_t r[32];
+                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + tb), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int tau = tb + e;
+                        if (tau < len) {
+                            const size_t off = rowbase + (size_t)tau * p.DV;
+                            const float o = p.o ? __bfloat162float(p.o[off]) : 1.f;
+                            p.h[off] = __float2bfloat16_rn(o * __uint_as_float(r[e]) * inv[tau]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hs_free);
+            rho = rho_new + g;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [BH][S][D] bf16 tensor, boxes of 64 columns x rows tokens x 1 head, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int D, int S, int BH, int rows)
+{
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int DK, int L>
+cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark)
+{
+    Params p;
+    p.S = a.S; p.L = L; p.NC = w.NC; p.R = w.R; p.NSEG = w.NSEG; p.DK = DK; p.DV = a.DHV; p.BH = a.BH;
+    p.A = w.A; p.Mtok = w.M; p.ig = a.igate; p.MC = w.MC; p.G = w.G; p.GP = w.GP; p.SGb = w.SGb;
+    p.DC = w.DC; p.DN = w.DN;
+    p.o = static_cast<const __nv_bfloat16 *>(a.ogate);
+    p.h = static_cast<__nv_bfloat16 *>(a.h);
+    p.status = w.status;
+
+    CUtensorMap mq, mk, mv, mk64, mv64;
+    if (!make_map(&mq, a.q, DK, a.S, a.BH, L) || !make_map(&mk, a.k, DK, a.S, a.BH, L) ||
+        !make_map(&mv, a.v, a.DHV, a.S, a.BH, L) || !make_map(&mk64, a.k, DK, a.S, a.BH, TB) ||
+        !make_map(&mv64, a.v, a.DHV, a.S, a.BH, TB))
+        return cudaErrorInvalidValue;
+    const int ntile = a.DHV / DVT;
+    cudaError_t e;
+
+    if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK>, SegSmem<DK>::TOTAL)) != cudaSuccess) return e;
+    segsum_kernel<DK><<<dim3(ntile, w.NSEG, a.BH), 192, SegSmem<DK>::TOTAL, a.stream>>>(mk64, mv64, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = mark(2)) != cudaSuccess) return e;
+
+    const int nquad = DK * a.DHV / 4;
+    seg_scan_kernel<<<dim3((nquad + 255) / 256, a.BH), 256, 0, a.stream>>>(p, a.C_final, a.n_final, a.m_final);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = mark(3)) != cudaSuccess) return e;
+
+    using WS = WalkSmem<DK, L>;
+    if ((e = ensure_dynamic_smem((const void *)walk_kernel<DK, L>, WS::TOTAL)) != cudaSuccess) return e;
+    walk_kernel<DK, L><<<dim3(ntile, w.NSEG, a.BH), 320, WS::TOTAL, a.stream>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace tcfwd
+
+bool tc_path_supported(bool bf16, int DHQK, int DHV, int chunk)
+{
+    return bf16 && (DHQK == 64 || DHQK == 128 || DHQK == 256) && DHV % tcfwd::DVT == 0 &&
+           (chunk == 64 || chunk == 128);
+}
+
+// Segments per head: balances whole waves of one CTA per SM (148 SMs) against
+// the number of chunks each CTA walks.
+int tc_num_segments(int BH, int DHV, int NC)
+{
+    const int ntile = DHV / tcfwd::DVT;
+    const long long ctas_per_seg = (long long)BH * ntile;
+    long long best_cost = -1;
+    int best = 1;
+    for (int nseg = 1; nseg <= NC; ++nseg) {
+        const int R = (NC + nseg - 1) / nseg;
+        const int ns = (NC + R - 1) / R;
+        if (ns != nseg) continue;
+        const long long rounds = (ctas_per_seg * ns + 147) / 148;
+        const long long cost = rounds * (R + 1) * 100 + ns;     // +1: a chunk's worth of start-up per CTA
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = ns;
+        }
+    }
+    return best;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark)
+{
+    using namespace tcfwd;
+    if (a.DHQK == 256 && a.chunk == 128) return launch_dk_l<256, 128>(a, w, mark);
+    if (a.DHQK == 256 && a.chunk == 64) return launch_dk_l<256, 64>(a, w, mark);
+    if (a.DHQK == 128 && a.chunk == 128) return launch_dk_l<128, 128>(a, w, mark);
+    if (a.DHQK == 128 && a.chunk == 64) return launch_dk_l<128, 64>(a, w, mark);
+    if (a.DHQK == 64 && a.chunk == 128) return launch_dk_l<64, 128>(a, w, mark);
+    if (a.DHQK == 64 && a.chunk == 64) return launch_dk_l<64, 64>(a, w, mark);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mlstm

@@ -26,7 +26,8 @@ namespace mlstm {
 __global__ void __launch_bounds__(1024)
 gate_prep_kernel(const float *__restrict__ igate, const float *__restrict__ fgate, int S, int L, int NC,
                  float *__restrict__ A, float *__restrict__ Mtok, float *__restrict__ G,
-                 float *__restrict__ Bc, float *__restrict__ MC)
+                 float *__restrict__ Bc, float *__restrict__ MC, int R, int NSEG,
+                 float *__restrict__ GP, float *__restrict__ SGb)
 {
     const int bh = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
@@ -75,6 +76,21 @@ gate_prep_kernel(const float *__restrict__ igate, const float *__restrict__ fgat
     }
     __syncthreads();
 
+    // Phase 1b (segments of R chunks): in-segment prefix of the chunk decays and the
+    // segment map, the composition of its chunk maps.
+    for (int sg = threadIdx.x; sg < NSEG; sg += blockDim.x) {
+        float ga = 0.f, gb = -INFINITY;
+        const int c1 = min((sg + 1) * R, NC);
+        for (int c = sg * R; c < c1; ++c) {
+            GP[(size_t)bh * NC + c] = ga;
+            const float g = g_out[c];
+            ga += g;
+            gb = fmaxf(gb + g, b_out[c]);
+        }
+        SGb[((size_t)bh * NSEG + sg) * 2 + 0] = ga;
+        SGb[((size_t)bh * NSEG + sg) * 2 + 1] = gb;
+    }
+
     // Phase 2: max-plus scan of the chunk maps m -> max(m + g_c, b_c), m_0 = 0.
     if (warp == 0) {
         const int per = (NC + 31) / 32;
@@ -119,7 +135,7 @@ gate_prep_kernel(const float *__restrict__ igate, const float *__restrict__ fgat
 cudaError_t launch_gate_prep(const GatePrepArgs &a)
 {
     gate_prep_kernel<<<a.BH, 1024, 0, a.stream>>>(a.igate, a.fgate, a.S, a.L, a.NC, a.A, a.M, a.G, a.Bc,
-                                                  a.MC);
+                                                  a.MC, a.R, a.NSEG, a.GP, a.SGb);
     return cudaGetLastError();
 }
 

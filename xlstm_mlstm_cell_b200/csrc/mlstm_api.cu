@@ -24,7 +24,7 @@ bool dims_ok_fwd(int DHQK, int DHV)
 bool chunk_ok(int chunk) { return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128; }
 
 // Lays out the workspace (base may be NULL to size it).  Returns the bytes used.
-size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, FwdWorkspace *w)
+size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, bool bf16, FwdWorkspace *w)
 {
     FwdWorkspace tmp;
     if (!w) w = &tmp;
@@ -42,11 +42,22 @@ size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, F
     w->G = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC));
     w->Bc = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC));
     w->MC = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * (NC + 1)));
-    w->CS = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC * DHQK * DHV));
-    w->NS = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC * DHQK));
+    w->tc = tc_path_supported(bf16, DHQK, DHV, chunk) && S > 0;
+    w->CS = w->NS = w->GP = w->SGb = w->DC = w->DN = nullptr;
     w->NSEG = 0;
     w->R = 0;
-    w->SA = w->SG = w->SB = w->SM = w->DC = w->DN = w->SC = w->SN = nullptr;
+    if (w->tc) {
+        const int nseg = tc_num_segments(BH, DHV, NC);
+        w->R = (NC + nseg - 1) / nseg;
+        w->NSEG = (NC + w->R - 1) / w->R;
+        w->GP = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC));
+        w->SGb = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * w->NSEG * 2));
+        w->DC = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * w->NSEG * DHQK * DHV));
+        w->DN = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * w->NSEG * DHQK));
+    } else {
+        w->CS = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC * DHQK * DHV));
+        w->NS = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * NC * DHQK));
+    }
     return off;
 }
 
@@ -71,14 +82,15 @@ extern "C" size_t mlstm_fwd_workspace_size(int B, int NH, int S, int DHQK, int D
 {
     if (B < 0 || NH < 0 || S < 0 || (dt != MLSTM_F32 && dt != MLSTM_BF16)) return 0;
     if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return 0;
-    return plan_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, nullptr);
+    return plan_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, dt == MLSTM_BF16, nullptr);
 }
 
 extern "C" int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt)
 {
     if (mlstm_fwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dt) == 0) return 0;
     if (B == 0 || NH == 0 || S == 0) return 0;
-    return 3;   // gate preprocessing, carry walk, outputs
+    // gate preprocessing + (segment sums, segment scan, walk) or (carry walk, outputs)
+    return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 4 : 3;
 }
 
 namespace {
@@ -103,13 +115,14 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     }
     if ((C_final && !aligned16(C_final)) || (n_final && !aligned16(n_final)) || (m_final && !aligned16(m_final)))
         return MLSTM_ERR_INVALID_ARG;
-    const size_t need = plan_workspace(nullptr, BH, S, DHQK, DHV, chunk, nullptr);
+    const bool bf16 = dt == MLSTM_BF16;
+    const size_t need = plan_workspace(nullptr, BH, S, DHQK, DHV, chunk, bf16, nullptr);
     if (!workspace || workspace_bytes < need) return MLSTM_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLSTM_ERR_INVALID_ARG;
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     FwdWorkspace w;
-    plan_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, &w);
+    plan_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, bf16, &w);
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     if (BH == 0) return MLSTM_OK;
@@ -124,13 +137,13 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     mark.events = events;
     mark.stream = st;
     if (mark(0) != cudaSuccess) return MLSTM_ERR_CUDA;
-    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, st};
+    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, w.R, w.NSEG, w.GP, w.SGb, st};
     e = launch_gate_prep(gp);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     if (mark(1) != cudaSuccess) return MLSTM_ERR_CUDA;
     FwdArgs fa{q, k, v, ogate, igate, fgate, h_out, C_final, n_final, m_final, BH, S, DHQK, DHV, chunk,
                dt == MLSTM_BF16, st};
-    e = launch_fwd_simt(fa, w, mark);
+    e = w.tc ? launch_fwd_tc(fa, w, mark) : launch_fwd_simt(fa, w, mark);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     return cuda_status(mark(MLSTM_FWD_PHASES));
 }

@@ -21,6 +21,8 @@ struct GatePrepArgs {
     const float *igate, *fgate;
     int BH, S, L, NC;
     float *A, *M, *G, *Bc, *MC;
+    int R, NSEG;             // segments of R chunks (tensor-core path; NSEG = 0 otherwise)
+    float *GP, *SGb;         // [BH][NC] in-segment prefix of chunk decays, [BH][NSEG][2] segment maps
     cudaStream_t stream;
 };
 
@@ -43,13 +45,12 @@ struct FwdWorkspace {
     float *MC;             // [BH][NC+1] stabilizer at chunk starts (last = final m)
     float *CS, *NS;        // SIMT path: state at every chunk start
     // tensor-core path
-    int NSEG, R;           // segments and chunks per segment
-    float *SA, *SG, *SB;   // [BH][NSEG] segment log decay, max-plus offset (tensor-core path)
-    float *SM;             // [BH][NSEG+1] stabilizer at segment starts
-    float *DC;             // [BH][NSEG][DHQK][DHV] segment contributions (fp32)
-    float *DN;             // [BH][NSEG][DHQK]
-    float *SC;             // [BH][NSEG][DHQK][DHV] state at segment starts (fp32)
-    float *SN;             // [BH][NSEG][DHQK]
+    bool tc;               // the tensor-core path is used
+    int NSEG, R;           // segments per head and chunks per segment
+    float *GP;             // [BH][NC] sum of the decays of the earlier chunks of the same segment
+    float *SGb;            // [BH][NSEG][2] segment max-plus map (total log decay G, offset b)
+    float *DC;             // [BH][NSEG][DHQK/4][DHV][4] segment contributions, then segment start states
+    float *DN;             // [BH][NSEG][DHQK] same for the normalizer
 };
 
 // Records the caller's phase events (mlstm_fwd_profiled); a no-op without events.
@@ -66,5 +67,8 @@ cudaError_t launch_step(const StepArgs &a);
 cudaError_t launch_gate_prep(const GatePrepArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark);
 size_t simt_state_bytes(int BH, int NC, int DHQK, int DHV);
+bool tc_path_supported(bool bf16, int DHQK, int DHV, int chunk);
+int tc_num_segments(int BH, int DHV, int NC);
+cudaError_t launch_fwd_tc(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark);
 
 }  // namespace mlstm
