@@ -138,6 +138,40 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
                         mlstm_dtype dt, int B, int NH, int DHQK, int DHV,
                         void *h_out, void *stream);
 
+/*
+ * mlstm_fwd for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this entry point; it exists for callers that may not call
+ * cudaMalloc or any allocating routine: code running inside a host framework
+ * that owns all device memory and hands out no scratch space (plugin and
+ * extension interfaces), and latency-critical paths where an allocation's
+ * implicit device synchronization is not acceptable.
+ *
+ * Same arguments, results and conventions as mlstm_fwd, without the workspace:
+ * the scratch memory comes from one device array of MLSTM_FWD_NOALLOC_MAX_BYTES
+ * built into the library.  That array exists on every GPU that loads the
+ * library and stays allocated until the process exits.  This entry point
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
+ *
+ * - Its first call on a device looks up the array's device address on that
+ *   device (cudaGetSymbolAddress); make that first call before any stream
+ *   capture.
+ * - Shapes whose mlstm_fwd_workspace_size() exceeds MLSTM_FWD_NOALLOC_MAX_BYTES
+ *   are rejected with MLSTM_ERR_WORKSPACE before anything is enqueued;
+ *   unsupported shapes return MLSTM_ERR_UNSUPPORTED as with mlstm_fwd.
+ * - Every call on a device shares the one array, and it keeps the contents of
+ *   the last call (each call clears the part that must start at zero).  Calls
+ *   whose work overlaps on the GPU (other streams, other host threads) race on
+ *   the array: serialize them.
+ * - The status word of mlstm_fwd_status lives in the shared array and is not
+ *   reachable through this entry point.
+ */
+#define MLSTM_FWD_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+mlstm_status mlstm_fwd_noalloc(const void *q, const void *k, const void *v,
+                               const float *igate, const float *fgate, const void *ogate,
+                               mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                               void *h_out, float *C_final, float *n_final, float *m_final,
+                               void *stream);
+
 /* Static English text for a status code. */
 const char *mlstm_status_string(mlstm_status s);
 

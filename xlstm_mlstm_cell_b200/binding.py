@@ -30,6 +30,8 @@ SIGNATURES = {
     "mlstm_fwd_profiled": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp,
                                 _vp, _sz, _vp, ctypes.POINTER(ctypes.c_void_p)]),
     "mlstm_fwd_status": (_i, [_vp, _vp]),
+    "mlstm_fwd_noalloc": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp,
+                               _vp]),
     "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_step": (_i, [_fp, _fp, _fp, _vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "mlstm_status_string": (ctypes.c_char_p, [_i]),
@@ -140,6 +142,34 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
                 e.record()
         arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[e.cuda_event for e in events])
         _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
+    return h_out, C_final, n_final, m_final
+
+
+NOALLOC_MAX_BYTES = 32 * 1024 * 1024
+
+
+def fwd_noalloc(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=None, n_final=None,
+                m_final=None, stream=None):
+    """mlstm_fwd_noalloc: the forward pass with the library's built-in scratch array.
+
+    For callers that may not allocate device memory for a workspace (the outputs are still
+    the caller's).  Returns ``(h, C, n, m)``.
+    """
+    lib = load()
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    if h_out is None:
+        h_out = torch.empty((B, NH, S, DHV), dtype=q.dtype, device=q.device)
+    if C_final is None:
+        C_final = torch.empty((B, NH, DHQK, DHV), dtype=torch.float32, device=q.device)
+    if n_final is None:
+        n_final = torch.empty((B, NH, DHQK), dtype=torch.float32, device=q.device)
+    if m_final is None:
+        m_final = torch.empty((B, NH), dtype=torch.float32, device=q.device)
+    st = lib.mlstm_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate), _dt(q), B, NH,
+                               S, DHQK, DHV, chunk, _ptr(h_out), _ptr(C_final), _ptr(n_final), _ptr(m_final),
+                               _stream(stream))
+    _check("mlstm_fwd_noalloc", st)
     return h_out, C_final, n_final, m_final
 
 
