@@ -58,6 +58,20 @@ constexpr int SS_STAGES = 4;
 constexpr float THRESH = 20.f;   // log of the largest weight before TMEM is rescaled
 constexpr float LOG2E = 1.4426950408889634f;
 
+// Optional timeline trace of the walk (build with -DMLSTM_WALK_TRACE): clock64 stamps of
+// the three roles of tile 0, head 0, per segment and chunk.  Off in normal builds.
+#ifdef MLSTM_WALK_TRACE
+constexpr int TR_SLOTS = 24, TR_CHUNKS = 256, TR_SEGS = 64;
+__device__ long long g_walk_trace[TR_SEGS * TR_CHUNKS * TR_SLOTS];
+#define WALK_TRACE(slot)                                                                                   \
+    do {                                                                                                   \
+        if (tile == 0 && bh == 0 && seg < TR_SEGS && i < TR_CHUNKS)                                        \
+            g_walk_trace[((size_t)seg * TR_CHUNKS + i) * TR_SLOTS + (slot)] = clock64();                   \
+    } while (0)
+#else
+#define WALK_TRACE(slot) do { } while (0)
+#endif
+
 struct Params {
     int S, L, NC, R, NSEG, DK, DV, BH;
     const float *A, *Mtok, *ig, *MC, *G, *GP, *SGb;
@@ -302,9 +316,9 @@ struct WalkSmem {
     static constexpr uint32_t V_OFF = K_OFF + DK * L * 2;
     static constexpr uint32_t P_OFF = V_OFF + DVT * L * 2;
     static constexpr uint32_t F_OFF = P_OFF + L * L * 2;          // float arrays
-    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [2][L]; dint [4][L]; inv, ivalid, qexp, rrow [L];
-    // nX [DK]; red [16]
-    static constexpr uint32_t NF = L * 15 + DK + 16;
+    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [2][L]; dint, inv, qexp, rrow [L]; nX [DK];
+    // red [16]; npart [2048] (n partial sums of the row pass)
+    static constexpr uint32_t NF = L * 11 + DK + 16 + 2048;
     static constexpr uint32_t BAR_OFF = F_OFF + NF * 4;
     static constexpr uint32_t TOTAL = BAR_OFF + 16 * 8 + 16 + 1024;
     static constexpr uint32_t C_COL = 0, CB_COL = DK, HS_COL = DK + DK / 2;
@@ -324,8 +338,8 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint8_t *Ps = smem + SM::P_OFF;
     float *F = reinterpret_cast<float *>(smem + SM::F_OFF);
     float *arow = F, *mrow = F + L, *icol = F + 2 * L, *srow = F + 3 * L, *wcol = F + 4 * L;
-    float *rs = F + 5 * L, *dint = F + 7 * L, *inv = F + 11 * L, *ivalid = F + 12 * L;
-    float *qexp = F + 13 * L, *rrow = F + 14 * L, *nX = F + 15 * L, *red = nX + DK;
+    float *rs = F + 5 * L, *dint = F + 7 * L, *inv = F + 8 * L;
+    float *qexp = F + 9 * L, *rrow = F + 10 * L, *nX = F + 11 * L, *red = nX + DK, *npart = red + 16;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
     uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *h_full = bars + 4;
     uint64_t *c_upd = bars + 5, *q_empty = bars + 6, *k_empty = bars + 7, *v_empty = bars + 8, *ep1 = bars + 9;
@@ -375,14 +389,17 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int t0 = (c_begin + i) * L;
                 const uint32_t pp = (uint32_t)(i - 1) & 1u;
                 if (i > 0 && !mbar_wait(q_empty, pp, wc)) break;
+                WALK_TRACE(0);
                 mbar_arrive_expect_tx(q_full, DK * L * 2);
                 for (int b = 0; b < DK / 64; ++b) tma_load_3d(Qs + b * L * 128, &tm_q, b * 64, t0, bh, q_full);
                 ++nq;
                 if (i > 0 && !mbar_wait(k_empty, pp, wc)) break;
+                WALK_TRACE(1);
                 mbar_arrive_expect_tx(k_full, DK * L * 2);
                 for (int b = 0; b < DK / 64; ++b) tma_load_3d(Ks + b * L * 128, &tm_k, b * 64, t0, bh, k_full);
                 ++nk;
                 if (i > 0 && !mbar_wait(v_empty, pp, wc)) break;
+                WALK_TRACE(2);
                 mbar_arrive_expect_tx(v_full, DVT * L * 2);
                 for (int b = 0; b < DVT / 64; ++b)
                     tma_load_3d(Vs + b * L * 128, &tm_v, j0 + b * 64, t0, bh, v_full);
@@ -404,8 +421,11 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             for (int i = 0; i < nck; ++i) {
                 const uint32_t ph = (uint32_t)i & 1u;
                 if (!mbar_wait(q_full, ph, wc)) break;
+                WALK_TRACE(3);
                 if (!mbar_wait(k_full, ph, wc)) break;
+                WALK_TRACE(4);
                 if (i > 0 && !mbar_wait(hs_free, ph ^ 1u, wc)) break;
+                WALK_TRACE(5);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k) {
@@ -414,7 +434,9 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
                 mma_commit(s_full);
                 if (!mbar_wait(ep1, ph, wc)) break;
+                WALK_TRACE(6);
                 if (!mbar_wait(v_full, ph, wc)) break;
+                WALK_TRACE(7);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k) {
@@ -428,6 +450,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
                 mma_commit(h_full);
                 mma_commit(q_empty);
+                WALK_TRACE(8);
                 if (i < nck - 1) {
 #pragma unroll
                     for (int k = 0; k < L / 16; ++k)
@@ -444,6 +467,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     } else {
         // compute warps 2..9: two per TMEM lane quadrant
         const int ct = threadIdx.x - 64;          // 0..255
+        const int cw = ct >> 5;                   // compute warp 0..7
         const int q = warp & 3;                   // TMEM lane quadrant
         const int hf = (warp - 2) >> 2;           // which half of the columns
         const float scale = rsqrtf((float)DK);
@@ -452,6 +476,10 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float *igb = p.ig + (size_t)bh * p.S;
         const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
         const float *Gb = p.G + (size_t)bh * p.NC;
+        // row pass mapping: a warp takes RPW rows at a time, one 16-byte chunk (8 columns) per lane
+        constexpr int CPR = DK / 8;               // chunks per row
+        constexpr int RPW = 32 / CPR;             // rows per warp step
+        const int rsub = lane / CPR, jc = lane % CPR;
 
         // the segment's start state -> TMEM (C^T, lane = value column) and shared (n)
         {
@@ -475,12 +503,34 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         float rho = MCb[c_begin];
         bool ok = true;
 
+        // gate values of the next chunk, loaded one chunk ahead
+        float pa = 0.f, pm = 0.f, pi = 0.f;
+        float pmc = MCb[c_begin], pmn = MCb[c_begin + 1], pg = Gb[c_begin];
+        if (ct < L && c_begin * L + ct < p.S) {
+            const int t = c_begin * L + ct;
+            pa = Ab[t];
+            pm = Mb[t];
+            pi = igb[t];
+        }
+
         for (int i = 0; i < nck && ok; ++i) {
             const int c = c_begin + i;
             const int t0 = c * L;
             const int len = min(L, p.S - t0);
             const uint32_t ph = (uint32_t)i & 1u;
-            const float mc = MCb[c], mn = MCb[c + 1], g = Gb[c];
+            const float mc = pmc, mn = pmn, g = pg;
+            const float ca = pa, cm = pm, ci = pi;
+            if (i + 1 < nck) {                    // prefetch the next chunk's gate values
+                pmc = MCb[c + 1];
+                pmn = MCb[c + 2];
+                pg = Gb[c + 1];
+                const int t = t0 + L + ct;
+                if (ct < L && t < p.S) {
+                    pa = Ab[t];
+                    pm = Mb[t];
+                    pi = igb[t];
+                }
+            }
             const bool last = (i == nck - 1);
             const bool rescale = !last && (mn - (rho + g) > THRESH);
             const float rho_new = rescale ? (mn - g) : rho;
@@ -488,21 +538,19 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float beta = expf(rho - rho_new);
 
             named_sync(1, 256);   // previous chunk's readers of the per-row arrays are done
+            if (ct == 0) WALK_TRACE(10);
             if (ct < L) {
-                const int t = t0 + ct;
                 if (ct < len) {
-                    const float a = Ab[t], m = Mb[t], it = igb[t];
-                    arow[ct] = (a - m) * LOG2E;
-                    mrow[ct] = m;
-                    icol[ct] = (it - a) * LOG2E;
-                    const float sc = expf(a + mc - m) * scale;
+                    arow[ct] = (ca - cm) * LOG2E;
+                    mrow[ct] = cm;
+                    icol[ct] = (ci - ca) * LOG2E;
+                    const float sc = expf(ca + mc - cm) * scale;
                     srow[ct] = sc;
                     int ex = 0;
                     const float fr = frexpf(sc, &ex);            // sc = fr 2^ex, fr in [0.5, 1)
                     qexp[ct] = sc > 0.f ? (float)(ex - 1) : -1000.f;
                     rrow[ct] = sc > 0.f ? 2.f * fr : 1.f;
-                    wcol[ct] = last ? 0.f : expf(it - a - rho_new);
-                    ivalid[ct] = 1.f;
+                    wcol[ct] = last ? 0.f : expf(ci - ca - rho_new);
                 } else {
                     arow[ct] = 0.f;
                     mrow[ct] = 0.f;
@@ -511,14 +559,15 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     qexp[ct] = -1000.f;
                     rrow[ct] = 1.f;
                     wcol[ct] = 0.f;
-                    ivalid[ct] = 0.f;
                 }
             }
             named_sync(1, 256);
 
             // (b) Cb = fp16(C_c 2^-kc) into TMEM, kc from max |C_c| over the tile; rescale the
             //     fp32 state when the frame moves
+            if (ct == 0) WALK_TRACE(11);
             if (i > 0 && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
+            if (ct == 0) WALK_TRACE(12);
             tc_fence_after();
             float cmax = 0.f;
             for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
@@ -561,7 +610,9 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tmem_wait_st();
 
             // (c) S -> P (bf16, shared, K-major swizzled), row sums
+            if (ct == 0) WALK_TRACE(13);
             if (!mbar_wait(s_full, ph, wc)) { ok = false; break; }
+            if (ct == 0) WALK_TRACE(14);
             tc_fence_after();
             if (L == 128) {
                 const int tau = q * 32 + lane;
@@ -630,68 +681,68 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
 
-            named_sync(1, 256);
-
-            // (e1) inter-chunk denominator alpha * sc_t * (q_t . nX) from the unscaled bf16 q, in fp32
+            if (ct == 0) WALK_TRACE(15);
+            // (d) one pass over the rows of Q and K (a warp per row, a 16-byte chunk per lane):
+            //     den_inter = alpha sc (q . nX) from the unscaled bf16 q (fp32, warp reduction),
+            //     Q' = 2^(e + kc) q in fp16 (exact), n partial sums W k from the unscaled k (fp32),
+            //     K' = W k in bf16.  Both tiles are rewritten in place as MMA operands.
             {
-                constexpr int PARTS = 256 / L;
-                const int row = ct % L, part = ct / L;
-                constexpr int SPAN = DK / PARTS;
-                float acc = 0.f;
-                for (int d = part * SPAN; d < (part + 1) * SPAN; d += 8) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(Qs + sw128_chunk(row, d >> 3, L));
-                    const float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z),
-                                 f3 = unpack_bf16(u.w);
-                    acc += f0.x * nX[d] + f0.y * nX[d + 1] + f1.x * nX[d + 2] + f1.y * nX[d + 3] +
-                           f2.x * nX[d + 4] + f2.y * nX[d + 5] + f3.x * nX[d + 6] + f3.y * nX[d + 7];
+                float nacc[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) nacc[z] = 0.f;
+                float nx[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) nx[z] = nX[jc * 8 + z];
+                for (int row = cw * RPW + rsub; row < L; row += 8 * RPW) {
+                    uint4 *pq = reinterpret_cast<uint4 *>(Qs + sw128_chunk(row, jc, L));
+                    uint4 *pkk = reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, jc, L));
+                    uint4 u = *pq;
+                    float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z), f3 = unpack_bf16(u.w);
+                    float dot = f0.x * nx[0] + f0.y * nx[1] + f1.x * nx[2] + f1.y * nx[3] + f2.x * nx[4] +
+                                f2.y * nx[5] + f3.x * nx[6] + f3.y * nx[7];
+#pragma unroll
+                    for (int o = CPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                    if (jc == 0) dint[row] = dot * alpha * srow[row];
+                    const int qe = (int)qexp[row] + kc;
+                    const float s2 = qe >= -126 ? __int_as_float((qe + 127) << 23) : 0.f;
+                    *pq = make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
+                                     pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
+                    const float w = wcol[row];
+                    u = *pkk;
+                    f0 = unpack_bf16(u.x); f1 = unpack_bf16(u.y); f2 = unpack_bf16(u.z); f3 = unpack_bf16(u.w);
+                    nacc[0] += w * f0.x; nacc[1] += w * f0.y; nacc[2] += w * f1.x; nacc[3] += w * f1.y;
+                    nacc[4] += w * f2.x; nacc[5] += w * f2.y; nacc[6] += w * f3.x; nacc[7] += w * f3.y;
+                    *pkk = make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
+                                      pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
                 }
-                dint[part * L + row] = acc * alpha * srow[row];
+                float *np = npart + (size_t)(cw * RPW + rsub) * DK + jc * 8;
+#pragma unroll
+                for (int z = 0; z < 8; ++z) np[z] = nacc[z];
             }
+            if (ct == 0) WALK_TRACE(16);
             named_sync(1, 256);
-            // (e2) normalizer for the next chunk from the unscaled bf16 k and fp32 weights;
-            //      1 / denominator of this chunk
+            // normalizer for the next chunk; 1 / denominator (times r) of this chunk
             if (!last) {
                 for (int d = ct; d < DK; d += 256) {
                     float acc = nX[d] * beta;
-                    for (int s = 0; s < len; ++s)
-                        acc += wcol[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Ks + sw128_offset(s, d, L)));
+#pragma unroll 8
+                    for (int pr = 0; pr < 8 * RPW; ++pr) acc += npart[pr * DK + d];
                     nX[d] = acc;
                 }
             }
             if (ct < L) {
-                constexpr int PARTS = 256 / L;
-                float den = rs[ct] + rs[L + ct];
-#pragma unroll
-                for (int pp = 0; pp < PARTS; ++pp) den += dint[pp * L + ct];
+                const float den = rs[ct] + rs[L + ct] + dint[ct];
                 inv[ct] = rrow[ct] / fmaxf(fabsf(den), expf(-mrow[ct]));
-            }
-            named_sync(1, 256);
-
-            // (d) Q' = diag(2^(e + kc)) Q in fp16 (exact) and K' = diag(W) K in bf16, in place
-            for (int e = ct; e < L * (DK / 8); e += 256) {
-                const int row = e % L, jc = e / L;
-                uint4 *pq = reinterpret_cast<uint4 *>(Qs + sw128_chunk(row, jc, L));
-                uint4 *pkk = reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, jc, L));
-                const int qe = (int)qexp[row] + kc;
-                const float sk = wcol[row];
-                uint4 u = *pq;
-                float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z), f3 = unpack_bf16(u.w);
-                *pq = make_uint4(pack_f16(ldexpf(f0.x, qe), ldexpf(f0.y, qe)),
-                                 pack_f16(ldexpf(f1.x, qe), ldexpf(f1.y, qe)),
-                                 pack_f16(ldexpf(f2.x, qe), ldexpf(f2.y, qe)),
-                                 pack_f16(ldexpf(f3.x, qe), ldexpf(f3.y, qe)));
-                u = *pkk;
-                f0 = unpack_bf16(u.x); f1 = unpack_bf16(u.y); f2 = unpack_bf16(u.z); f3 = unpack_bf16(u.w);
-                *pkk = make_uint4(pack_bf16(f0.x * sk, f0.y * sk), pack_bf16(f1.x * sk, f1.y * sk),
-                                  pack_bf16(f2.x * sk, f2.y * sk), pack_bf16(f3.x * sk, f3.y * sk));
             }
             fence_proxy_async();
             tc_fence_before();
             named_sync(1, 256);
             if (lane == 0) mbar_arrive(ep1);
+            if (ct == 0) WALK_TRACE(17);
 
             // (g) outputs: H^T (lane = value column j, columns = tokens)
             if (!mbar_wait(h_full, ph, wc)) { ok = false; break; }
+            if (ct == 0) WALK_TRACE(18);
             tc_fence_after();
             {
                 const int j = q * 32 + lane;
@@ -716,6 +767,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(hs_free);
+            if (ct == 0) WALK_TRACE(19);
             rho = rho_new + g;
         }
     }
@@ -793,6 +845,13 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
 }
 
 }  // namespace tcfwd
+
+#ifdef MLSTM_WALK_TRACE
+extern "C" int mlstm_walk_trace_copy(void *dst, size_t bytes)
+{
+    return (int)cudaMemcpyFromSymbol(dst, tcfwd::g_walk_trace, bytes);
+}
+#endif
 
 bool tc_path_supported(bool bf16, int DHQK, int DHV, int chunk)
 {
