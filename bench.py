@@ -58,29 +58,49 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 
-def fwd_work(w: Workload, path: str):
+def tc_num_segments(BH: int, DHV: int, NC: int) -> int:
+    """Segments per head of the tensor-core path (mirrors the library's planner)."""
+    ctas_per_seg = BH * (DHV // 128)
+    best, best_cost = 1, None
+    for nseg in range(1, min(NC, 256) + 1):
+        R = -(-NC // nseg)
+        ns = -(-NC // R)
+        if ns != nseg:
+            continue
+        rounds = -(-(ctas_per_seg * ns) // 148)
+        cost = rounds * (R + 1) * 100 + ns
+        if best_cost is None or cost < best_cost:
+            best, best_cost = ns, cost
+    return best
+
+
+def fwd_work(w: Workload, tensor_path: bool):
     """Algorithmic bytes and flops of one mlstm_fwd, total and per phase.
 
     Bytes count every input read once and every output written once; flops
     count the causal half of the intra-chunk products (masked work excluded).
     Per token and head: 4 dk dv (state contribution and inter-chunk read-out)
-    + (L + 1)(dk + dv) (intra-chunk) + 4 dk.
+    + (L + 1)(dk + dv) (intra-chunk) + 4 dk.  Per phase, the state traffic is
+    the path's own: per-segment states on the tensor-core path, per-chunk
+    states on the CUDA-core path.
     """
     e = 4 if w.dtype == "f32" else 2
     tok = w.B * w.NH * w.S
     dk, dv, L = w.DHQK, w.DHV, w.chunk
     heads = w.B * w.NH
     NC = math.ceil(w.S / L)
+    nstate = tc_num_segments(heads, dv, NC) if tensor_path else NC
+    state = heads * nstate * 4 * (dk * dv + dk)
     in_bytes = tok * (e * (2 * dk + dv) + (e * dv if w.ogate else 0) + 8)
     out_bytes = tok * e * dv + heads * 4 * (dk * dv + dk + 1)
     flops_tok = 4 * dk * dv + (L + 1) * (dk + dv) + 4 * dk
     phases = {
         "gate_prep": {"bytes": tok * 16 + heads * NC * 16, "flops": tok * 10},
-        "state_contributions": {"bytes": tok * (e * (dk + dv) + 12) + heads * NC * 4 * (dk * dv + dk),
-                                "flops": tok * 2 * dk * (dv + 1)},
-        "outputs": {"bytes": tok * (e * (2 * dk + dv) + (e * dv if w.ogate else 0) + e * dv + 12)
-                             + heads * NC * 4 * (dk * dv + dk),
-                    "flops": tok * (2 * dk * dv + (L + 1) * (dk + dv) + 2 * dk)},
+        "state_contributions": {"bytes": tok * (e * (dk + dv) + 12) + state, "flops": tok * 2 * dk * (dv + 1)},
+        "state_scan": {"bytes": 2 * state, "flops": heads * nstate * 3 * (dk * dv + dk)},
+        "outputs": {"bytes": tok * (e * (2 * dk + dv) + (e * dv if w.ogate else 0) + e * dv + 12) + state,
+                    "flops": tok * (2 * dk * dv + (L + 1) * (dk + dv) + 2 * dk)
+                    + (tok * 2 * dk * dv if tensor_path else 0)},
     }
     return {"bytes": in_bytes + out_bytes, "flops": tok * flops_tok, "phases": phases}
 
@@ -347,7 +367,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
-    fw = fwd_work(w, "")
+    fw = fwd_work(w, path_is_tensor(w))
     sw = step_work(w.B, w.NH, w.DHQK, w.DHV, 4 if w.dtype == "f32" else 2, w.ogate)
     works = dict(fw["phases"])
     works["decode_step"] = sw
@@ -419,8 +439,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 def path_is_tensor(w: Workload) -> bool:
-    """True when the library takes its tensor-core path for this workload (4 launches)."""
-    return binding.fwd_kernel_launches(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 4
+    """True when the library takes its tensor-core path for this workload (5 launches)."""
+    return binding.fwd_kernel_launches(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 5
 
 
 def extras(device, peaks):
@@ -444,10 +464,16 @@ def extras(device, peaks):
         e1.record()
         torch.cuda.synchronize()
         t = e0.elapsed_time(e1) / reps / 1e3
-        fw = fwd_work(w, "")
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(binding.FWD_PHASES + 1)]
+        binding.fwd(s["q"], s["k"], s["v"], s["i"], s["f"], s["o"], chunk=w.chunk, h_out=run.h, C_final=run.C,
+                    n_final=run.n, m_final=run.m, workspace=run.ws, events=ev)
+        torch.cuda.synchronize()
+        phases = {nm: round(ev[p].elapsed_time(ev[p + 1]) * 1e3, 1) for p, nm in enumerate(binding.PHASE_NAMES)}
+        fw = fwd_work(w, path_is_tensor(w))
         res[name] = {"ms": t * 1e3, "tokens_per_s": w.B * w.S / t, "tflops": fw["flops"] / t / 1e12,
                      "frac_tc_peak": fw["flops"] / t / 1e12 / tc, "hbm_gbs": fw["bytes"] / t / 1e9,
-                     "frac_roofline": max(fw["flops"] / (tc * 1e12), fw["bytes"] / (bw * 1e9)) / t}
+                     "frac_roofline": max(fw["flops"] / (tc * 1e12), fw["bytes"] / (bw * 1e9)) / t,
+                     "phases_us": phases}
         del s, run
         torch.cuda.empty_cache()
     w = WORKLOADS["step_bf16"]
@@ -542,7 +568,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="fwd_bf16_d256", choices=[k for k in WORKLOADS if k.startswith("fwd_")])

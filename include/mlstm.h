@@ -92,6 +92,25 @@ mlstm_status mlstm_fwd(const void *q, const void *k, const void *v,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Forward pass that starts from a given state instead of the zero state: the
+ * chunked prefill / resume form of the recurrence (the constant-size state is
+ * the whole memory of the sequence so far, "Inference VRAM and Throughput
+ * Scaling" and "Deploy xLSTM for Continuous Streaming" of the xLSTM guide).
+ * Same arguments as mlstm_fwd plus the initial state C0 [B][NH][DHQK][DHV],
+ * n0 [B][NH][DHQK], m0 [B][NH] (float32, device, 16-byte aligned): all three,
+ * or all NULL for the zero state.  Running S1 tokens and then S2 more from the
+ * returned state equals one pass over S1 + S2 tokens.  The final state may
+ * alias the initial one (C_final == C0 and so on) to update it in place.
+ * S == 0 copies the initial state to the final-state outputs.
+ */
+mlstm_status mlstm_fwd_state(const void *q, const void *k, const void *v,
+                             const float *igate, const float *fgate, const void *ogate,
+                             mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                             const float *C0, const float *n0, const float *m0,
+                             void *h_out, float *C_final, float *n_final, float *m_final,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * mlstm_fwd with per-phase timing: identical work and results, and in addition
  * records CUDA events (cudaEvent_t passed as void*, created by the caller) on
  * `stream`: events[p] just before phase p and events[MLSTM_FWD_PHASES] after

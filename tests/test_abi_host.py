@@ -108,5 +108,17 @@ def test_empty_batch_is_a_no_op(lib):
     assert call_step(lib, step_args(B=0, C=None, n=None, m=None)) == 0
 
 
+def test_fwd_state_needs_the_whole_state(lib):
+    a = fwd_args()
+    st = lib.mlstm_fwd_state(a["q"], a["k"], a["v"], a["ig"], a["fg"], a["og"], a["dt"], a["B"], a["NH"], a["S"],
+                             a["DHQK"], a["DHV"], a["chunk"], FAKE, None, FAKE, a["h"], None, None, None, a["ws"],
+                             a["wsb"], None)
+    assert st == 1
+    st = lib.mlstm_fwd_state(a["q"], a["k"], a["v"], a["ig"], a["fg"], a["og"], a["dt"], a["B"], a["NH"], a["S"],
+                             a["DHQK"], a["DHV"], a["chunk"], FAKE + 4, FAKE, FAKE, a["h"], None, None, None, a["ws"],
+                             a["wsb"], None)
+    assert st == 1
+
+
 def test_fwd_status_rejects_null(lib):
     assert lib.mlstm_fwd_status(None, None) == 1

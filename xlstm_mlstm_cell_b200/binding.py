@@ -27,6 +27,8 @@ SIGNATURES = {
     "mlstm_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_fwd": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp, _vp, _sz,
                        _vp]),
+    "mlstm_fwd_state": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _fp, _fp,
+                             _fp, _vp, _sz, _vp]),
     "mlstm_fwd_profiled": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp,
                                 _vp, _sz, _vp, ctypes.POINTER(ctypes.c_void_p)]),
     "mlstm_fwd_status": (_i, [_vp, _vp]),
@@ -109,9 +111,10 @@ PHASE_NAMES = ("gate_prep", "state_contributions", "state_scan", "outputs")
 
 
 def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=None, n_final=None,
-        m_final=None, workspace=None, return_state: bool = True, stream=None, events=None):
+        m_final=None, workspace=None, return_state: bool = True, stream=None, events=None, state=None):
     """mlstm_fwd on device tensors; returns ``(h, C, n, m)`` (states None unless requested).
 
+    ``state=(C0, n0, m0)`` starts from that state (mlstm_fwd_state) instead of the zero state.
     With ``events`` (FWD_PHASES + 1 ``torch.cuda.Event(enable_timing=True)``) the call goes
     through mlstm_fwd_profiled, which records them around its phases on the stream.
     """
@@ -133,7 +136,12 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate), dt, B, NH, S, DHQK, DHV, chunk,
             _ptr(h_out), _ptr(C_final), _ptr(n_final), _ptr(m_final), _ptr(workspace), workspace.numel(),
             _stream(stream))
-    if events is None:
+    if state is not None:
+        assert events is None
+        C0, n0, m0 = state
+        sargs = args[:13] + (_ptr(C0), _ptr(n0), _ptr(m0)) + args[13:]
+        _check("mlstm_fwd_state", lib.mlstm_fwd_state(*sargs))
+    elif events is None:
         _check("mlstm_fwd", lib.mlstm_fwd(*args))
     else:
         assert len(events) == FWD_PHASES + 1

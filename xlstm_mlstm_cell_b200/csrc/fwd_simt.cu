@@ -37,7 +37,7 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
                   const float *__restrict__ A, const float *__restrict__ G, const float *__restrict__ MC,
                   int S, int L, int NC, int DHQK, int DHV,
                   float *__restrict__ CS, float *__restrict__ NS,
-                  float *__restrict__ C_final, float *__restrict__ n_final, float *__restrict__ m_final)
+                  float *C_final, float *n_final, float *__restrict__ m_final, const float *C0, const float *n0)
 {
     extern __shared__ float sm[];
     float *ks = sm;                    // [L][ST]
@@ -51,8 +51,18 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
     const T *vb = v + (size_t)bh * S * DHV;
     const float *igb = igate + (size_t)bh * S;
     const float *Ab = A + (size_t)bh * S;
+    // initial state (zero when C0 is NULL); C_final may alias C0: every element is read here,
+    // by the thread that writes it at the end
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     float nn = 0.f;
+    if (C0) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int i = i0 + ty * 4 + r;
+            if (i < DHQK && j < DHV) c[r] = C0[((size_t)bh * DHQK + i) * DHV + j];
+        }
+    }
+    if (n0 && do_n && i0 + tx < DHQK) nn = n0[(size_t)bh * DHQK + i0 + tx];
 
     for (int ch = 0; ch < NC; ++ch) {
         const int t0 = ch * L, len = min(L, S - t0);
@@ -134,7 +144,7 @@ output_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
     for (int t = tid; t < L; t += blockDim.x) {
         const bool ok = t < len;
         ar[t] = ok ? A[(size_t)bh * S + t0 + t] : 0.f;
-        mr[t] = ok ? Mtok[(size_t)bh * S + t0 + t] : 0.f;
+        mr[t] = ok ? ar[t] + fmaxf(mc, Mtok[(size_t)bh * S + t0 + t]) : 0.f;   // m = a + max(m_c, p)
         ir[t] = ok ? igate[(size_t)bh * S + t0 + t] : -INFINITY;
         sc[t] = ok ? expf(ar[t] + mc - mr[t]) : 0.f;
     }
@@ -246,7 +256,7 @@ static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, co
     const size_t sm1 = sizeof(float) * (2 * (size_t)L * ST + L);
     carry_simt_kernel<T><<<g1, 256, sm1, a.stream>>>((const T *)a.k, (const T *)a.v, a.igate, w.A, w.G, w.MC,
                                                      a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS, a.C_final,
-                                                     a.n_final, a.m_final);
+                                                     a.n_final, a.m_final, a.C0, a.n0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;   // the chunk scan is fused into the carry walk

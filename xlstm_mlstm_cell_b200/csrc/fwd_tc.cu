@@ -178,54 +178,85 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             mbar_wait_drain(acc_full, 0);
         }
     } else {
-        // scalers (warps 2..5): K rows *= w, then (tile 0) dn += column sums of K'
+        // scalers (warps 2..5): K rows *= w in place; tile 0 also sums dn = sum_t w_t k_t in fp32 from
+        // the unrounded bf16 k.  A warp takes RPW rows at a time, one 16-byte chunk per lane.
         const int ct = threadIdx.x - 64;                 // 0..127
+        const int sw = ct >> 5;                          // scaler warp 0..3
+        constexpr int CPR = DK / 8;                      // 16-byte chunks per row
+        constexpr int RPW = 32 / CPR;                    // rows per warp step
+        constexpr int RSTEP = 4 * RPW;
+        constexpr int NB = 4;                            // rows in flight per iteration
+        static_assert(TB % (RSTEP * NB) == 0, "segsum row pass unroll");
+        const int rsub = lane / CPR, jc = lane % CPR;
         const float Gs = p.SGb[((size_t)bh * p.NSEG + seg) * 2 + 0];
         const float bs = p.SGb[((size_t)bh * p.NSEG + seg) * 2 + 1];
         const float *Ab = p.A + (size_t)bh * p.S;
         const float *igb = p.ig + (size_t)bh * p.S;
         const float *GPb = p.GP + (size_t)bh * p.NC;
-        float n0 = 0.f, n1 = 0.f;
+        float nacc[8];
+#pragma unroll
+        for (int z = 0; z < 8; ++z) nacc[z] = 0.f;
         bool ok = true;
+        // this thread's token weight of the next stage, loaded one stage ahead (threads 0..TB-1)
+        float pa = 0.f, pi = 0.f, pgp = 0.f;
+        if (ct < TB && t_begin + ct < t_end) {
+            pa = Ab[t_begin + ct];
+            pi = igb[t_begin + ct];
+            pgp = GPb[(t_begin + ct) / p.L];
+        }
         for (int it = 0; it < nstage; ++it) {
             const int st = it % SS_STAGES;
             const uint32_t ph = (uint32_t)(it / SS_STAGES) & 1u;
+            const int t = t_begin + it * TB + ct;
+            const float ca = pa, ci = pi, cgp = pgp;
+            if (ct < TB && t + TB < t_end) {             // prefetch the next stage's gate values
+                pa = Ab[t + TB];
+                pi = igb[t + TB];
+                pgp = GPb[(t + TB) / p.L];
+            }
+            named_sync(1, 128);                          // the previous stage's readers of wst are done
+            if (ct < TB) wst[ct] = (t < t_end) ? expf(Gs - cgp - ca + ci - bs) : 0.f;
+            named_sync(1, 128);
             if (!mbar_wait(&full[st], ph, wc)) { ok = false; break; }
             uint8_t *kb = smem + st * SM::STAGE;
-            const int r = ct & (TB - 1);                 // row of the stage
-            const int t = t_begin + it * TB + r;
-            float w = 0.f;
-            if (t < t_end) w = expf(Gs - GPb[t / p.L] - Ab[t] + igb[t] - bs);
-            if (tile == 0) {
-                // dn += sum_r w_r k_r from the unrounded bf16 k, in fp32, before K is scaled
-                if (ct < TB) wst[ct] = w;
-                named_sync(1, 128);
-                for (int rr = 0; rr < TB; ++rr) {
-                    const float wr = wst[rr];
-                    if (ct < DK)
-                        n0 += wr * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kb + sw128_offset(rr, ct, TB)));
-                    if (DK > 128)
-                        n1 += wr * __bfloat162float(
-                                       *reinterpret_cast<const __nv_bfloat16 *>(kb + sw128_offset(rr, ct + 128, TB)));
+            for (int row0 = sw * RPW + rsub; row0 < TB; row0 += RSTEP * NB) {
+                uint4 uk[NB];
+#pragma unroll
+                for (int b2 = 0; b2 < NB; ++b2)
+                    uk[b2] = *reinterpret_cast<const uint4 *>(kb + sw128_chunk(row0 + b2 * RSTEP, jc, TB));
+#pragma unroll
+                for (int b2 = 0; b2 < NB; ++b2) {
+                    const int row = row0 + b2 * RSTEP;
+                    const float w = wst[row];
+                    const float2 f0 = unpack_bf16(uk[b2].x), f1 = unpack_bf16(uk[b2].y), f2 = unpack_bf16(uk[b2].z),
+                                 f3 = unpack_bf16(uk[b2].w);
+                    if (tile == 0) {
+                        nacc[0] += w * f0.x; nacc[1] += w * f0.y; nacc[2] += w * f1.x; nacc[3] += w * f1.y;
+                        nacc[4] += w * f2.x; nacc[5] += w * f2.y; nacc[6] += w * f3.x; nacc[7] += w * f3.y;
+                    }
+                    *reinterpret_cast<uint4 *>(kb + sw128_chunk(row, jc, TB)) =
+                        make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
+                                   pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
                 }
-                named_sync(1, 128);
-            }
-            // each thread scales half of its row: chunks [half * DK/16, (half+1) * DK/16)
-            const int half = ct / TB;
-            constexpr int CPR = DK / 8;                  // 16-byte chunks per row
-            for (int j = half * (CPR / 2); j < (half + 1) * (CPR / 2); ++j) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(kb + sw128_chunk(r, j, TB));
-                uint4 u = *ptr;
-                float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z), f3 = unpack_bf16(u.w);
-                u.x = pack_bf16(f0.x * w, f0.y * w);
-                u.y = pack_bf16(f1.x * w, f1.y * w);
-                u.z = pack_bf16(f2.x * w, f2.y * w);
-                u.w = pack_bf16(f3.x * w, f3.y * w);
-                *ptr = u;
             }
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&scaled[st]);
+        }
+        if (tile == 0) {    // reduce the n partial sums of the scaler warps (and lanes sharing a chunk)
+            float *npart = reinterpret_cast<float *>(smem);      // stage buffers are idle once acc_full fires
+            if (ok && mbar_wait(acc_full, 0, wc)) {
+#pragma unroll
+                for (int z = 0; z < 8; ++z) npart[(sw * RPW + rsub) * DK + jc * 8 + z] = nacc[z];
+            }
+            named_sync(1, 128);
+            if (ok) {
+                for (int d = ct; d < DK; d += 128) {
+                    float acc = 0.f;
+                    for (int pr = 0; pr < 4 * RPW; ++pr) acc += npart[pr * DK + d];
+                    p.DN[((size_t)bh * p.NSEG + seg) * DK + d] = acc;
+                }
+            }
         }
         // epilogue: TMEM (lane = value column, columns = DK) -> workspace, quad layout [DK/4][DV][4]
         if (ok && mbar_wait(acc_full, 0, wc)) {
@@ -244,11 +275,6 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     *reinterpret_cast<float4 *>(dst + ((size_t)((c0 >> 2) + u) * p.DV + j0 + j) * 4) = v4;
                 }
             }
-            if (tile == 0) {
-                float *dn = p.DN + ((size_t)bh * p.NSEG + seg) * DK;
-                if (ct < DK) dn[ct] = n0;
-                if (DK > 128 && ct + 128 < DK) dn[ct + 128] = n1;
-            }
         }
     }
     tc_fence_before();
@@ -261,26 +287,53 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
 // ---------------------------------------------------------------- scan over segments
 
+constexpr int SCAN_MAX_SEG = 256;   // segments per head handled by seg_scan_kernel's shared tables
+
 __global__ void __launch_bounds__(256)
-seg_scan_kernel(Params p, float *__restrict__ C_final, float *__restrict__ n_final, float *__restrict__ m_final)
+seg_scan_kernel(Params p, float *C_final, float *n_final, float *__restrict__ m_final, const float *C0,
+                const float *n0)
 {
+    __shared__ float gam[SCAN_MAX_SEG], bet[SCAN_MAX_SEG];
     const int bh = blockIdx.y;
     const int nquad = p.DK * p.DV / 4;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;    // quad index: (i4, j) = (e / DV, e % DV)
     const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
     const float *SG = p.SGb + (size_t)bh * p.NSEG * 2;
+    // decay of the running state and weight of the segment's contribution, per segment
+    for (int s = threadIdx.x; s < p.NSEG; s += blockDim.x) {
+        const float Ms = MCb[s * p.R], Mn = MCb[min((s + 1) * p.R, p.NC)];
+        gam[s] = expf(SG[2 * s] + Ms - Mn);
+        bet[s] = expf(SG[2 * s + 1] - Mn);
+    }
+    __syncthreads();
     if (e < nquad) {
+        float4 *__restrict__ slot0 = reinterpret_cast<float4 *>(p.DC + (size_t)bh * p.NSEG * p.DK * p.DV) + e;
+        const size_t stride = (size_t)p.DK * p.DV / 4;
         float4 C = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < p.NSEG; ++s) {
-            float4 *slot = reinterpret_cast<float4 *>(p.DC + ((size_t)bh * p.NSEG + s) * (size_t)p.DK * p.DV) + e;
-            const float4 d = *slot;
-            *slot = C;
-            const float Ms = MCb[s * p.R], Mn = MCb[min((s + 1) * p.R, p.NC)];
-            const float gam = expf(SG[2 * s] + Ms - Mn), bet = expf(SG[2 * s + 1] - Mn);
-            C.x = gam * C.x + bet * d.x;
-            C.y = gam * C.y + bet * d.y;
-            C.z = gam * C.z + bet * d.z;
-            C.w = gam * C.w + bet * d.w;
+        if (C0) {   // initial state (user layout); C_final may alias C0: each element is read before written
+            const int i4 = e / p.DV, j = e % p.DV;
+            const float *c0 = C0 + (size_t)bh * p.DK * p.DV;
+            C = make_float4(c0[(size_t)(4 * i4 + 0) * p.DV + j], c0[(size_t)(4 * i4 + 1) * p.DV + j],
+                            c0[(size_t)(4 * i4 + 2) * p.DV + j], c0[(size_t)(4 * i4 + 3) * p.DV + j]);
+        }
+        constexpr int BATCH = 8;                       // contributions loaded ahead of the stores
+        for (int s0 = 0; s0 < p.NSEG; s0 += BATCH) {
+            float4 d[BATCH];
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u)
+                if (s0 + u < p.NSEG) d[u] = __ldcs(slot0 + (s0 + u) * stride);
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int s = s0 + u;
+                if (s < p.NSEG) {
+                    slot0[s * stride] = C;
+                    const float ga = gam[s], be = bet[s];
+                    C.x = ga * C.x + be * d[u].x;
+                    C.y = ga * C.y + be * d[u].y;
+                    C.z = ga * C.z + be * d[u].z;
+                    C.w = ga * C.w + be * d[u].w;
+                }
+            }
         }
         if (C_final) {
             const int i4 = e / p.DV, j = e % p.DV;
@@ -293,13 +346,12 @@ seg_scan_kernel(Params p, float *__restrict__ C_final, float *__restrict__ n_fin
     }
     if (blockIdx.x == 0) {
         for (int i = threadIdx.x; i < p.DK; i += blockDim.x) {
-            float n = 0.f;
+            float n = n0 ? n0[(size_t)bh * p.DK + i] : 0.f;
             for (int s = 0; s < p.NSEG; ++s) {
                 float *slot = p.DN + ((size_t)bh * p.NSEG + s) * p.DK + i;
                 const float d = *slot;
                 *slot = n;
-                const float Ms = MCb[s * p.R], Mn = MCb[min((s + 1) * p.R, p.NC)];
-                n = expf(SG[2 * s] + Ms - Mn) * n + expf(SG[2 * s + 1] - Mn) * d;
+                n = gam[s] * n + bet[s] * d;
             }
             if (n_final) n_final[(size_t)bh * p.DK + i] = n;
         }
@@ -315,7 +367,9 @@ struct WalkSmem {
     static constexpr uint32_t K_OFF = Q_OFF + DK * L * 2;
     static constexpr uint32_t V_OFF = K_OFF + DK * L * 2;
     static constexpr uint32_t P_OFF = V_OFF + DVT * L * 2;
-    static constexpr uint32_t F_OFF = P_OFF + L * L * 2;          // float arrays
+    // transpose staging of the output epilogue (8 warps x 4 KB): the P tile when it is 32 KB
+    static constexpr uint32_t T_OFF = (L * L * 2 >= 32768) ? P_OFF : P_OFF + L * L * 2;
+    static constexpr uint32_t F_OFF = T_OFF == P_OFF ? P_OFF + L * L * 2 : T_OFF + 32768;   // float arrays
     // float arrays: arow, mrow, icol, srow, wcol [L]; rs [2][L]; dint, inv, qexp, rrow [L]; nX [DK];
     // red [16]; npart [2048] (n partial sums of the row pass)
     static constexpr uint32_t NF = L * 11 + DK + 16 + 2048;
@@ -336,6 +390,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint8_t *Ks = smem + SM::K_OFF;
     uint8_t *Vs = smem + SM::V_OFF;
     uint8_t *Ps = smem + SM::P_OFF;
+    uint8_t *Ts = smem + SM::T_OFF;
     float *F = reinterpret_cast<float *>(smem + SM::F_OFF);
     float *arow = F, *mrow = F + L, *icol = F + 2 * L, *srow = F + 3 * L, *wcol = F + 4 * L;
     float *rs = F + 5 * L, *dint = F + 7 * L, *inv = F + 8 * L;
@@ -343,7 +398,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
     uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *h_full = bars + 4;
     uint64_t *c_upd = bars + 5, *q_empty = bars + 6, *k_empty = bars + 7, *v_empty = bars + 8, *ep1 = bars + 9;
-    uint64_t *hs_free = bars + 10, *drain = bars + 11;
+    uint64_t *hs_free = bars + 10, *drain = bars + 11, *kready = bars + 12;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
     uint32_t *abort_flag = tmem_slot + 1;
 
@@ -367,6 +422,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(ep1, 8);
         mbar_init(hs_free, 8);
         mbar_init(drain, 1);
+        mbar_init(kready, 8);
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch(&tm_q);
@@ -452,6 +508,9 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 mma_commit(q_empty);
                 WALK_TRACE(8);
                 if (i < nck - 1) {
+                    if (!mbar_wait(kready, ph, wc)) break;
+                    WALK_TRACE(9);
+                    tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < L / 16; ++k)
                         mma_ss(tmem + SM::C_COL, smem_desc(va + k * 2048, L * 128, 1024),
@@ -472,7 +531,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int hf = (warp - 2) >> 2;           // which half of the columns
         const float scale = rsqrtf((float)DK);
         const float *Ab = p.A + (size_t)bh * p.S;
-        const float *Mb = p.Mtok + (size_t)bh * p.S;
+        const float *Mb = p.Mtok + (size_t)bh * p.S;   // chunk-local prefix maxima p
         const float *igb = p.ig + (size_t)bh * p.S;
         const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
         const float *Gb = p.G + (size_t)bh * p.NC;
@@ -537,14 +596,23 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float alpha = expf(rho - mc);
             const float beta = expf(rho - rho_new);
 
+            if (p.o) {   // bring this thread's output-gate rows of the epilogue into L2 early
+#pragma unroll
+                for (int u = 0; u < L / 64; ++u) {
+                    const int tau = hf * (L / 2) + u * 32 + lane;
+                    if (tau < len)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32));
+                }
+            }
             named_sync(1, 256);   // previous chunk's readers of the per-row arrays are done
             if (ct == 0) WALK_TRACE(10);
             if (ct < L) {
                 if (ct < len) {
-                    arow[ct] = (ca - cm) * LOG2E;
-                    mrow[ct] = cm;
+                    const float mt = ca + fmaxf(mc, cm);   // per-token stabilizer from the prefix maximum p
+                    arow[ct] = (ca - mt) * LOG2E;
+                    mrow[ct] = mt;
                     icol[ct] = (ci - ca) * LOG2E;
-                    const float sc = expf(ca + mc - cm) * scale;
+                    const float sc = expf(ca + mc - mt) * scale;
                     srow[ct] = sc;
                     int ex = 0;
                     const float fr = frexpf(sc, &ex);            // sc = fr 2^ex, fr in [0.5, 1)
@@ -620,24 +688,30 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int s0 = hf * 64 + u * 32;
-                    uint32_t r[32];
-                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
-                    tmem_wait_ld();
-                    const float at = arow[tau];
-                    const float ri = 1.f / rrow[tau];
                     uint32_t pk[16];
+                    if (s0 > q * 32) {                 // whole 32 x 32 block above the diagonal: zeros
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float v2[2];
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else {
+                        uint32_t r[32];
+                        tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                        tmem_wait_ld();
+                        const float at = arow[tau];
+                        const float ri = 1.f / rrow[tau];
+                        const bool diag = (s0 == q * 32);
 #pragma unroll
-                        for (int z = 0; z < 2; ++z) {
-                            const int sg = s0 + 2 * e + z;
-                            float d = 0.f;
-                            if (sg <= tau) d = exp2f(at + icol[sg]);
-                            v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
-                            sum += v2[z];
+                        for (int e = 0; e < 16; ++e) {
+                            float v2[2];
+#pragma unroll
+                            for (int z = 0; z < 2; ++z) {
+                                const int sg = s0 + 2 * e + z;
+                                float d = exp2f(at + icol[sg]);
+                                if (diag && sg > tau) d = 0.f;
+                                v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
+                                sum += v2[z];
+                            }
+                            pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
                         }
-                        pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
                     }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -650,9 +724,13 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             } else {   // L == 64: M = 64 accumulator, rows 16q..16q+15 in lanes 0..15 of quadrant q
                 const int tau = q * 16 + (lane & 15);
                 const int s0 = hf * 32;
+                const bool above = s0 > q * 16 + 15;   // the whole 16 x 32 block is masked
+                const bool below = s0 + 31 < q * 16;   // the whole block is causal
                 uint32_t r[32];
-                tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
-                tmem_wait_ld();
+                if (!above) {
+                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                    tmem_wait_ld();
+                }
                 if (lane < 16) {
                     float sum = 0.f;
                     const float at = arow[tau];
@@ -665,8 +743,11 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         for (int z = 0; z < 2; ++z) {
                             const int sg = s0 + 2 * e + z;
                             float d = 0.f;
-                            if (sg <= tau) d = exp2f(at + icol[sg]);
-                            v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
+                            if (!above) {
+                                d = exp2f(at + icol[sg]);
+                                if (!below && sg > tau) d = 0.f;
+                            }
+                            v2[z] = above ? 0.f : __uint_as_float(r[2 * e + z]) * d * scale;
                             sum += v2[z];
                         }
                         pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
@@ -682,44 +763,84 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
 
             if (ct == 0) WALK_TRACE(15);
-            // (d) one pass over the rows of Q and K (a warp per row, a 16-byte chunk per lane):
-            //     den_inter = alpha sc (q . nX) from the unscaled bf16 q (fp32, warp reduction),
-            //     Q' = 2^(e + kc) q in fp16 (exact), n partial sums W k from the unscaled k (fp32),
-            //     K' = W k in bf16.  Both tiles are rewritten in place as MMA operands.
+            constexpr int RSTEP = 8 * RPW;            // row stride of a warp in the row passes
+            constexpr int NB = (L / RSTEP) < 4 ? (L / RSTEP) : 4;   // rows in flight per iteration
+            static_assert(L % (RSTEP * NB) == 0, "row pass unroll");
+            // (d) Q row pass (a warp per row, a 16-byte chunk per lane): den_inter = alpha sc (q . nX)
+            //     from the unscaled bf16 q (fp32, warp reduction), then Q' = 2^(e + kc) q in fp16 (exact),
+            //     in place as the MMA operand
             {
-                float nacc[8];
-#pragma unroll
-                for (int z = 0; z < 8; ++z) nacc[z] = 0.f;
                 float nx[8];
 #pragma unroll
                 for (int z = 0; z < 8; ++z) nx[z] = nX[jc * 8 + z];
-                for (int row = cw * RPW + rsub; row < L; row += 8 * RPW) {
-                    uint4 *pq = reinterpret_cast<uint4 *>(Qs + sw128_chunk(row, jc, L));
-                    uint4 *pkk = reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, jc, L));
-                    uint4 u = *pq;
-                    float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z), f3 = unpack_bf16(u.w);
-                    float dot = f0.x * nx[0] + f0.y * nx[1] + f1.x * nx[2] + f1.y * nx[3] + f2.x * nx[4] +
-                                f2.y * nx[5] + f3.x * nx[6] + f3.y * nx[7];
+                for (int row0 = cw * RPW + rsub; row0 < L; row0 += RSTEP * NB) {
+                    uint4 uq[NB];
 #pragma unroll
-                    for (int o = CPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                    if (jc == 0) dint[row] = dot * alpha * srow[row];
-                    const int qe = (int)qexp[row] + kc;
-                    const float s2 = qe >= -126 ? __int_as_float((qe + 127) << 23) : 0.f;
-                    *pq = make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
-                                     pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
-                    const float w = wcol[row];
-                    u = *pkk;
-                    f0 = unpack_bf16(u.x); f1 = unpack_bf16(u.y); f2 = unpack_bf16(u.z); f3 = unpack_bf16(u.w);
-                    nacc[0] += w * f0.x; nacc[1] += w * f0.y; nacc[2] += w * f1.x; nacc[3] += w * f1.y;
-                    nacc[4] += w * f2.x; nacc[5] += w * f2.y; nacc[6] += w * f3.x; nacc[7] += w * f3.y;
-                    *pkk = make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
-                                      pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
+                    for (int b = 0; b < NB; ++b)
+                        uq[b] = *reinterpret_cast<const uint4 *>(Qs + sw128_chunk(row0 + b * RSTEP, jc, L));
+                    float dot[NB];
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const float2 f0 = unpack_bf16(uq[b].x), f1 = unpack_bf16(uq[b].y), f2 = unpack_bf16(uq[b].z),
+                                     f3 = unpack_bf16(uq[b].w);
+                        dot[b] = f0.x * nx[0] + f0.y * nx[1] + f1.x * nx[2] + f1.y * nx[3] + f2.x * nx[4] +
+                                 f2.y * nx[5] + f3.x * nx[6] + f3.y * nx[7];
+                    }
+#pragma unroll
+                    for (int o = CPR / 2; o > 0; o >>= 1)
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) dot[b] += __shfl_xor_sync(0xffffffffu, dot[b], o);
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const int row = row0 + b * RSTEP;
+                        if (jc == 0) dint[row] = dot[b] * alpha * srow[row];
+                        const int qe = (int)qexp[row] + kc;
+                        const float s2 = qe >= -126 ? __int_as_float((qe + 127) << 23) : 0.f;
+                        const float2 f0 = unpack_bf16(uq[b].x), f1 = unpack_bf16(uq[b].y), f2 = unpack_bf16(uq[b].z),
+                                     f3 = unpack_bf16(uq[b].w);
+                        *reinterpret_cast<uint4 *>(Qs + sw128_chunk(row, jc, L)) =
+                            make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
+                                       pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
+                    }
                 }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_sync(1, 256);
+            if (lane == 0) mbar_arrive(ep1);         // P, Q' and Cb are ready: the output MMA can start
+            if (ct == 0) WALK_TRACE(16);
+
+            // (e) while the output MMA runs: K row pass, n partial sums W k from the unscaled bf16 k
+            //     (fp32) and K' = W k in bf16 in place, the operand of the state update
+            if (!last) {
+                float nacc[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) nacc[z] = 0.f;
+                for (int row0 = cw * RPW + rsub; row0 < L; row0 += RSTEP * NB) {
+                    uint4 uk[NB];
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        uk[b] = *reinterpret_cast<const uint4 *>(Ks + sw128_chunk(row0 + b * RSTEP, jc, L));
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const int row = row0 + b * RSTEP;
+                        const float w = wcol[row];
+                        const float2 f0 = unpack_bf16(uk[b].x), f1 = unpack_bf16(uk[b].y), f2 = unpack_bf16(uk[b].z),
+                                     f3 = unpack_bf16(uk[b].w);
+                        nacc[0] += w * f0.x; nacc[1] += w * f0.y; nacc[2] += w * f1.x; nacc[3] += w * f1.y;
+                        nacc[4] += w * f2.x; nacc[5] += w * f2.y; nacc[6] += w * f3.x; nacc[7] += w * f3.y;
+                        *reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, jc, L)) =
+                            make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
+                                       pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
+                    }
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(kready);  // K' is ready: the state update can start
                 float *np = npart + (size_t)(cw * RPW + rsub) * DK + jc * 8;
 #pragma unroll
                 for (int z = 0; z < 8; ++z) np[z] = nacc[z];
             }
-            if (ct == 0) WALK_TRACE(16);
             named_sync(1, 256);
             // normalizer for the next chunk; 1 / denominator (times r) of this chunk
             if (!last) {
@@ -734,10 +855,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float den = rs[ct] + rs[L + ct] + dint[ct];
                 inv[ct] = rrow[ct] / fmaxf(fabsf(den), expf(-mrow[ct]));
             }
-            fence_proxy_async();
-            tc_fence_before();
             named_sync(1, 256);
-            if (lane == 0) mbar_arrive(ep1);
             if (ct == 0) WALK_TRACE(17);
 
             // (g) outputs: H^T (lane = value column j, columns = tokens)
@@ -745,21 +863,61 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (ct == 0) WALK_TRACE(18);
             tc_fence_after();
             {
-                const int j = q * 32 + lane;
-                const size_t rowbase = ((size_t)bh * p.S + t0) * p.DV + j0 + j;
+                // each warp owns value columns [32q, 32q + 32) and tokens [hf L/2, (hf+1) L/2); per block of
+                // 32 tokens the 32 x 32 tile goes through shared memory (4 KB per warp, granules of four
+                // floats XOR-swizzled by the row) so that a lane then holds one token row of 32 columns and
+                // reads o / writes h with 16-byte vectors
+                float *tile = reinterpret_cast<float *>(Ts) + cw * 1024;
+                const __nv_bfloat16 *__restrict__ op = p.o;
+                __nv_bfloat16 *__restrict__ hp = p.h;
+                uint4 ou[L / 64][4];                      // output gate of this lane's token rows, loaded first
+#pragma unroll
+                for (int u = 0; u < L / 64; ++u) {
+                    const int tau = hf * (L / 2) + u * 32 + lane;
+                    const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8)
+                        ou[u][c8] = (op && tau < len) ? *reinterpret_cast<const uint4 *>(op + off + c8 * 8)
+                                                       : make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+                }
+                if (ct == 0) WALK_TRACE(20);
 #pragma unroll
                 for (int u = 0; u < L / 64; ++u) {
                     const int tb = hf * (L / 2) + u * 32;
+                    if (ct == 0 && u == 1) WALK_TRACE(21);
                     uint32_t r[32];
                     tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + tb), r);
                     tmem_wait_ld();
+                    // lane = value column j (= lane): element (token e, column lane)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int tau = tb + e;
-                        if (tau < len) {
-                            const size_t off = rowbase + (size_t)tau * p.DV;
-                            const float o = p.o ? __bfloat162float(p.o[off]) : 1.f;
-                            p.h[off] = __float2bfloat16_rn(o * __uint_as_float(r[e]) * inv[tau]);
+                    for (int e = 0; e < 32; ++e)
+                        tile[e * 32 + ((((lane >> 2) ^ (e & 7)) << 2) | (lane & 3))] = __uint_as_float(r[e]);
+                    __syncwarp();
+                    // lane = token tb + lane: its 32 columns
+                    const int tau = tb + lane;
+                    float hv[32];
+#pragma unroll
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 v4 = *reinterpret_cast<const float4 *>(tile + lane * 32 + ((gq ^ (lane & 7)) << 2));
+                        hv[4 * gq] = v4.x; hv[4 * gq + 1] = v4.y; hv[4 * gq + 2] = v4.z; hv[4 * gq + 3] = v4.w;
+                    }
+                    __syncwarp();
+                    if (tau < len) {
+                        const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32;
+                        const float iv = inv[tau];
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8) {
+                            float og[8];     // bf16 1.0 = 0x3F80 when there is no output gate
+                            const float2 a0 = unpack_bf16(ou[u][c8].x), a1 = unpack_bf16(ou[u][c8].y),
+                                         a2 = unpack_bf16(ou[u][c8].z), a3 = unpack_bf16(ou[u][c8].w);
+                            og[0] = a0.x; og[1] = a0.y; og[2] = a1.x; og[3] = a1.y;
+                            og[4] = a2.x; og[5] = a2.y; og[6] = a3.x; og[7] = a3.y;
+                            const float *hh = hv + c8 * 8;
+                            *reinterpret_cast<uint4 *>(hp + off + c8 * 8) =
+                                make_uint4(pack_bf16(og[0] * hh[0] * iv, og[1] * hh[1] * iv),
+                                           pack_bf16(og[2] * hh[2] * iv, og[3] * hh[3] * iv),
+                                           pack_bf16(og[4] * hh[4] * iv, og[5] * hh[5] * iv),
+                                           pack_bf16(og[6] * hh[6] * iv, og[7] * hh[7] * iv));
                         }
                     }
                 }
@@ -834,7 +992,8 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     if ((e = mark(2)) != cudaSuccess) return e;
 
     const int nquad = DK * a.DHV / 4;
-    seg_scan_kernel<<<dim3((nquad + 255) / 256, a.BH), 256, 0, a.stream>>>(p, a.C_final, a.n_final, a.m_final);
+    seg_scan_kernel<<<dim3((nquad + 255) / 256, a.BH), 256, 0, a.stream>>>(p, a.C_final, a.n_final, a.m_final,
+                                                                         a.C0, a.n0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = mark(3)) != cudaSuccess) return e;
 
@@ -867,7 +1026,7 @@ int tc_num_segments(int BH, int DHV, int NC)
     const long long ctas_per_seg = (long long)BH * ntile;
     long long best_cost = -1;
     int best = 1;
-    for (int nseg = 1; nseg <= NC; ++nseg) {
+    for (int nseg = 1; nseg <= NC && nseg <= tcfwd::SCAN_MAX_SEG; ++nseg) {
         const int R = (NC + nseg - 1) / nseg;
         const int ns = (NC + R - 1) / R;
         if (ns != nseg) continue;

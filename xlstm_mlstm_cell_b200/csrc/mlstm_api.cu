@@ -89,14 +89,15 @@ extern "C" int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV
 {
     if (mlstm_fwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dt) == 0) return 0;
     if (B == 0 || NH == 0 || S == 0) return 0;
-    // gate preprocessing + (segment sums, segment scan, walk) or (carry walk, outputs)
-    return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 4 : 3;
+    // gate preprocessing (2) + (segment sums, segment scan, walk) or (carry walk, outputs)
+    return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 5 : 4;
 }
 
 namespace {
 
 mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
                       const void *ogate, mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                      const float *C0, const float *n0, const float *m0,
                       void *h_out, float *C_final, float *n_final, float *m_final, void *workspace,
                       size_t workspace_bytes, void *stream, void *const *events)
 {
@@ -115,6 +116,11 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     }
     if ((C_final && !aligned16(C_final)) || (n_final && !aligned16(n_final)) || (m_final && !aligned16(m_final)))
         return MLSTM_ERR_INVALID_ARG;
+    const bool has_state = C0 || n0 || m0;
+    if (has_state && BH > 0) {   // the initial state comes whole or not at all
+        if (!C0 || !n0 || !m0) return MLSTM_ERR_INVALID_ARG;
+        if (!aligned16(C0) || !aligned16(n0) || !aligned16(m0)) return MLSTM_ERR_INVALID_ARG;
+    }
     const bool bf16 = dt == MLSTM_BF16;
     const size_t need = plan_workspace(nullptr, BH, S, DHQK, DHV, chunk, bf16, nullptr);
     if (!workspace || workspace_bytes < need) return MLSTM_ERR_WORKSPACE;
@@ -126,10 +132,20 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     if (BH == 0) return MLSTM_OK;
-    if (S == 0) {   // the zero state
-        if (C_final) e = cudaMemsetAsync(C_final, 0, sizeof(float) * (size_t)BH * DHQK * DHV, st);
-        if (e == cudaSuccess && n_final) e = cudaMemsetAsync(n_final, 0, sizeof(float) * (size_t)BH * DHQK, st);
-        if (e == cudaSuccess && m_final) e = cudaMemsetAsync(m_final, 0, sizeof(float) * (size_t)BH, st);
+    if (S == 0) {   // no tokens: the final state is the initial one (zero state by default)
+        const size_t bC = sizeof(float) * (size_t)BH * DHQK * DHV, bn = sizeof(float) * (size_t)BH * DHQK,
+                     bm = sizeof(float) * (size_t)BH;
+        if (has_state) {
+            if (C_final && C_final != C0) e = cudaMemcpyAsync(C_final, C0, bC, cudaMemcpyDeviceToDevice, st);
+            if (e == cudaSuccess && n_final && n_final != n0)
+                e = cudaMemcpyAsync(n_final, n0, bn, cudaMemcpyDeviceToDevice, st);
+            if (e == cudaSuccess && m_final && m_final != m0)
+                e = cudaMemcpyAsync(m_final, m0, bm, cudaMemcpyDeviceToDevice, st);
+        } else {
+            if (C_final) e = cudaMemsetAsync(C_final, 0, bC, st);
+            if (e == cudaSuccess && n_final) e = cudaMemsetAsync(n_final, 0, bn, st);
+            if (e == cudaSuccess && m_final) e = cudaMemsetAsync(m_final, 0, bm, st);
+        }
         return cuda_status(e);
     }
 
@@ -137,11 +153,11 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     mark.events = events;
     mark.stream = st;
     if (mark(0) != cudaSuccess) return MLSTM_ERR_CUDA;
-    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, w.R, w.NSEG, w.GP, w.SGb, st};
+    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, w.R, w.NSEG, w.GP, w.SGb, m0, st};
     e = launch_gate_prep(gp);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     if (mark(1) != cudaSuccess) return MLSTM_ERR_CUDA;
-    FwdArgs fa{q, k, v, ogate, igate, fgate, h_out, C_final, n_final, m_final, BH, S, DHQK, DHV, chunk,
+    FwdArgs fa{q, k, v, ogate, igate, fgate, h_out, C_final, n_final, m_final, C0, n0, BH, S, DHQK, DHV, chunk,
                dt == MLSTM_BF16, st};
     e = w.tc ? launch_fwd_tc(fa, w, mark) : launch_fwd_simt(fa, w, mark);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
@@ -157,8 +173,17 @@ mlstm_status mlstm_fwd(const void *q, const void *k, const void *v, const float 
                        void *h_out, float *C_final, float *n_final, float *m_final, void *workspace,
                        size_t workspace_bytes, void *stream)
 {
-    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, h_out, C_final, n_final,
-                    m_final, workspace, workspace_bytes, stream, nullptr);
+    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, nullptr, nullptr, nullptr, h_out,
+                    C_final, n_final, m_final, workspace, workspace_bytes, stream, nullptr);
+}
+
+mlstm_status mlstm_fwd_state(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
+                             const void *ogate, mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                             const float *C0, const float *n0, const float *m0, void *h_out, float *C_final,
+                             float *n_final, float *m_final, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, C0, n0, m0, h_out, C_final,
+                    n_final, m_final, workspace, workspace_bytes, stream, nullptr);
 }
 
 mlstm_status mlstm_fwd_profiled(const void *q, const void *k, const void *v, const float *igate,
@@ -170,8 +195,8 @@ mlstm_status mlstm_fwd_profiled(const void *q, const void *k, const void *v, con
     if (!events) return MLSTM_ERR_INVALID_ARG;
     for (int p = 0; p <= MLSTM_FWD_PHASES; ++p)
         if (!events[p]) return MLSTM_ERR_INVALID_ARG;
-    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, h_out, C_final, n_final,
-                    m_final, workspace, workspace_bytes, stream, events);
+    return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, nullptr, nullptr, nullptr, h_out,
+                    C_final, n_final, m_final, workspace, workspace_bytes, stream, events);
 }
 
 mlstm_status mlstm_fwd_status(const void *workspace, void *stream)

@@ -23,6 +23,7 @@ struct GatePrepArgs {
     float *A, *M, *G, *Bc, *MC;
     int R, NSEG;             // segments of R chunks (tensor-core path; NSEG = 0 otherwise)
     float *GP, *SGb;         // [BH][NC] in-segment prefix of chunk decays, [BH][NSEG][2] segment maps
+    const float *m0;         // [BH] initial stabilizer, NULL = 0
     cudaStream_t stream;
 };
 
@@ -31,6 +32,7 @@ struct FwdArgs {
     const float *igate, *fgate;
     void *h;
     float *C_final, *n_final, *m_final;
+    const float *C0, *n0;    // initial state [BH][DHQK][DHV], [BH][DHQK]; NULL = zero
     int BH, S, DHQK, DHV, chunk;
     bool bf16;
     cudaStream_t stream;
@@ -40,7 +42,7 @@ struct FwdArgs {
 struct FwdWorkspace {
     uint32_t *status;      // bounded-wait status word (0 = fine)
     int NC;                // chunks
-    float *A, *M;          // [BH][S] chunk-local cumulative log decay, per-token stabilizer
+    float *A, *M;          // [BH][S] chunk-local cumulative log decay and prefix maximum of i~ - a
     float *G, *Bc;         // [BH][NC] chunk log decay, chunk max-plus offset
     float *MC;             // [BH][NC+1] stabilizer at chunk starts (last = final m)
     float *CS, *NS;        // SIMT path: state at every chunk start
