@@ -26,7 +26,7 @@ def gpu_state(C, n, m):
 
 @pytest.mark.parametrize("B,NH,DHQK,DHV,dt", [
     (2, 3, 16, 16, "f32"), (1, 2, 64, 100, "f32"), (3, 2, 256, 512, "bf16"), (2, 2, 128, 1024, "bf16"),
-    (1, 1, 8, 4, "f32"), (4, 1, 512, 256, "bf16")])
+    (1, 1, 8, 4, "f32"), (4, 1, 512, 256, "bf16"), (10, 8, 64, 64, "f32")])
 def test_step_chain(cuda_lib, B, NH, DHQK, DHV, dt):
     """Ten steps in a row from an oracle-made state; every h and the final state match."""
     C, n, m = oracle_prefill(B, NH, 40, DHQK, DHV, dt, seed=DHQK + DHV, ig=(-1.0, 2.0), fg=(4.0, 1.0))

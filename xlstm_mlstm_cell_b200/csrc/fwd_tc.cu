@@ -83,20 +83,25 @@ struct Params {
 
 // ---------------------------------------------------------------- segsum
 
-template <int DK>
+// NT value tiles of 128 columns per CTA (one TMEM accumulator of DK columns each): with NT = 2
+// a K tile loaded and scaled once serves 256 value columns.
+template <int DK, int NT>
 struct SegSmem {
+    static constexpr int STAGES = NT == 2 ? 3 : SS_STAGES;
     static constexpr uint32_t K_BYTES = DK * TB * 2;
-    static constexpr uint32_t V_BYTES = DVT * TB * 2;
+    static constexpr uint32_t V_BYTES = NT * DVT * TB * 2;
     static constexpr uint32_t STAGE = K_BYTES + V_BYTES;
-    static constexpr uint32_t BAR_OFF = STAGE * SS_STAGES;
+    static constexpr uint32_t BAR_OFF = STAGE * STAGES;
     static constexpr uint32_t TOTAL = BAR_OFF + 128 + TB * 4 + 1024;   // + barriers, weights, alignment slack
+    static constexpr uint32_t TMEM_COLS = NT * DK < 32 ? 32 : NT * DK;
 };
 
-template <int DK>
+template <int DK, int NT>
 __global__ void __launch_bounds__(192, 1)
 segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Params p)
 {
-    using SM = SegSmem<DK>;
+    using SM = SegSmem<DK, NT>;
+    constexpr int SS_STAGES = SM::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
@@ -108,7 +113,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     float *wst = reinterpret_cast<float *>(smem + SM::BAR_OFF + 128);   // [TB] weights of the stage
 
     const int tile = blockIdx.x, seg = blockIdx.y, bh = blockIdx.z;
-    const int j0 = tile * DVT;
+    const int j0 = tile * DVT * NT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t_begin = seg * p.R * p.L;
     const int t_end = min(t_begin + p.R * p.L, p.S);
@@ -128,7 +133,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         tma_prefetch(&tm_v);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, SM::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -149,7 +154,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const int t0 = t_begin + it * TB;
                 mbar_arrive_expect_tx(&full[st], SM::STAGE);
                 for (int b = 0; b < DK / 64; ++b) tma_load_3d(kb + b * TB * 128, &tm_k, b * 64, t0, bh, &full[st]);
-                for (int b = 0; b < DVT / 64; ++b)
+                for (int b = 0; b < NT * DVT / 64; ++b)
                     tma_load_3d(vb + b * TB * 128, &tm_v, j0 + b * 64, t0, bh, &full[st]);
             }
             for (int it = issued > SS_STAGES ? issued - SS_STAGES : 0; it < issued; ++it)   // drain
@@ -167,11 +172,13 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const uint32_t kb = smem_u32(smem + st * SM::STAGE);
                 const uint32_t vb = kb + SM::K_BYTES;
 #pragma unroll
-                for (int k = 0; k < TB / 16; ++k) {
-                    const uint64_t a = smem_desc(vb + k * 2048, TB * 128, 1024);
-                    const uint64_t b = smem_desc(kb + k * 2048, TB * 128, 1024);
-                    mma_ss(tmem, a, b, IDESC, (it > 0 || k > 0) ? 1u : 0u);
-                }
+                for (int t = 0; t < NT; ++t)
+#pragma unroll
+                    for (int k = 0; k < TB / 16; ++k) {
+                        const uint64_t a = smem_desc(vb + t * 2 * TB * 128 + k * 2048, TB * 128, 1024);
+                        const uint64_t b = smem_desc(kb + k * 2048, TB * 128, 1024);
+                        mma_ss(tmem + t * DK, a, b, IDESC, (it > 0 || k > 0) ? 1u : 0u);
+                    }
                 mma_commit(&empty[st]);
             }
             mma_commit(acc_full);
@@ -262,11 +269,12 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         if (ok && mbar_wait(acc_full, 0, wc)) {
             tc_fence_after();
             const int q = warp & 3;
-            const int j = q * 32 + lane;
             float *dst = p.DC + ((size_t)bh * p.NSEG + seg) * (size_t)DK * p.DV;
-            for (int c0 = 0; c0 < DK; c0 += 32) {
+            for (int tc = 0; tc < NT * DK; tc += 32) {
+                const int t = tc / DK, c0 = tc % DK;
+                const int j = t * DVT + q * 32 + lane;
                 uint32_t r[32];
-                tmem_ld32(tmem_addr(tmem, q * 32, c0), r);
+                tmem_ld32(tmem_addr(tmem, q * 32, tc), r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
@@ -281,7 +289,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, SM::TMEM_COLS);
     }
 }
 
@@ -367,19 +375,21 @@ struct WalkSmem {
     static constexpr uint32_t K_OFF = Q_OFF + DK * L * 2;
     static constexpr uint32_t V_OFF = K_OFF + DK * L * 2;
     static constexpr uint32_t P_OFF = V_OFF + DVT * L * 2;
-    // transpose staging of the output epilogue (8 warps x 4 KB): the P tile when it is 32 KB
+    // transpose staging of the output epilogue (16 warps x 2 KB): the P tile when it is 32 KB
     static constexpr uint32_t T_OFF = (L * L * 2 >= 32768) ? P_OFF : P_OFF + L * L * 2;
     static constexpr uint32_t F_OFF = T_OFF == P_OFF ? P_OFF + L * L * 2 : T_OFF + 32768;   // float arrays
-    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [2][L]; dint, inv, qexp, rrow [L]; nX [DK];
-    // red [16]; npart [2048] (n partial sums of the row pass)
-    static constexpr uint32_t NF = L * 11 + DK + 16 + 2048;
+    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [4][L]; dint, inv, qexp, rrow [L]; nX [DK];
+    // red [16]; npart [4096] (n partial sums of the row pass: 16 warps x RPW rows x DK)
+    static constexpr uint32_t NF = L * 13 + DK + 16 + 4096;
     static constexpr uint32_t BAR_OFF = F_OFF + NF * 4;
     static constexpr uint32_t TOTAL = BAR_OFF + 16 * 8 + 16 + 1024;
     static constexpr uint32_t C_COL = 0, CB_COL = DK, HS_COL = DK + DK / 2;
 };
 
+constexpr int WALK_THREADS = 64 + 16 * 32;   // producer warp, MMA warp, 16 epilogue warps
+
 template <int DK, int L>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(WALK_THREADS, 1)
 walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, Params p)
 {
@@ -393,8 +403,8 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint8_t *Ts = smem + SM::T_OFF;
     float *F = reinterpret_cast<float *>(smem + SM::F_OFF);
     float *arow = F, *mrow = F + L, *icol = F + 2 * L, *srow = F + 3 * L, *wcol = F + 4 * L;
-    float *rs = F + 5 * L, *dint = F + 7 * L, *inv = F + 8 * L;
-    float *qexp = F + 9 * L, *rrow = F + 10 * L, *nX = F + 11 * L, *red = nX + DK, *npart = red + 16;
+    float *rs = F + 5 * L, *dint = F + 9 * L, *inv = F + 10 * L;
+    float *qexp = F + 11 * L, *rrow = F + 12 * L, *nX = F + 13 * L, *red = nX + DK, *npart = red + 16;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
     uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *h_full = bars + 4;
     uint64_t *c_upd = bars + 5, *q_empty = bars + 6, *k_empty = bars + 7, *v_empty = bars + 8, *ep1 = bars + 9;
@@ -419,10 +429,10 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(q_empty, 1);
         mbar_init(k_empty, 1);
         mbar_init(v_empty, 1);
-        mbar_init(ep1, 8);
-        mbar_init(hs_free, 8);
+        mbar_init(ep1, 16);
+        mbar_init(hs_free, 16);
         mbar_init(drain, 1);
-        mbar_init(kready, 8);
+        mbar_init(kready, 16);
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch(&tm_q);
@@ -524,11 +534,11 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             mbar_wait_drain(drain, 0);
         }
     } else {
-        // compute warps 2..9: two per TMEM lane quadrant
-        const int ct = threadIdx.x - 64;          // 0..255
-        const int cw = ct >> 5;                   // compute warp 0..7
+        // compute warps 2..17: four per TMEM lane quadrant
+        const int ct = threadIdx.x - 64;          // 0..511
+        const int cw = ct >> 5;                   // compute warp 0..15
         const int q = warp & 3;                   // TMEM lane quadrant
-        const int hf = (warp - 2) >> 2;           // which half of the columns
+        const int hq = (warp - 2) >> 2;           // which quarter of the columns / tokens
         const float scale = rsqrtf((float)DK);
         const float *Ab = p.A + (size_t)bh * p.S;
         const float *Mb = p.Mtok + (size_t)bh * p.S;   // chunk-local prefix maxima p
@@ -539,25 +549,27 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         constexpr int CPR = DK / 8;               // chunks per row
         constexpr int RPW = 32 / CPR;             // rows per warp step
         const int rsub = lane / CPR, jc = lane % CPR;
+        constexpr int CQ = DK / 4;                // state columns of a warp (a quarter of DK)
+        static_assert(CQ % 16 == 0, "state quarter");
 
         // the segment's start state -> TMEM (C^T, lane = value column) and shared (n)
         {
             const float *src = p.DC + ((size_t)bh * p.NSEG + seg) * (size_t)DK * p.DV;
             const int j = q * 32 + lane;
-            for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
-                uint32_t r[32];
+            for (int c0 = hq * CQ; c0 < (hq + 1) * CQ; c0 += 16) {
+                uint32_t r[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     const float4 v4 = *reinterpret_cast<const float4 *>(src + ((size_t)((c0 >> 2) + u) * p.DV + j0 + j) * 4);
                     r[4 * u] = __float_as_uint(v4.x);
                     r[4 * u + 1] = __float_as_uint(v4.y);
                     r[4 * u + 2] = __float_as_uint(v4.z);
                     r[4 * u + 3] = __float_as_uint(v4.w);
                 }
-                tmem_st32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
             }
             tmem_wait_st();
-            for (int i = ct; i < DK; i += 256) nX[i] = p.DN[((size_t)bh * p.NSEG + seg) * DK + i];
+            for (int i = ct; i < DK; i += 512) nX[i] = p.DN[((size_t)bh * p.NSEG + seg) * DK + i];
         }
         float rho = MCb[c_begin];
         bool ok = true;
@@ -571,6 +583,10 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             pm = Mb[t];
             pi = igb[t];
         }
+        // output epilogue mapping: a warp takes 16-token blocks of its quarter of the chunk; a lane
+        // then holds token (lane >> 1) of the block and 16 of the warp's 32 value columns
+        constexpr int TQ = L / 4;                 // tokens of a warp's quarter (32 or 16)
+        constexpr int NBLK = TQ / 16;             // 16-token blocks per warp (2 or 1)
 
         for (int i = 0; i < nck && ok; ++i) {
             const int c = c_begin + i;
@@ -598,13 +614,14 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
             if (p.o) {   // bring this thread's output-gate rows of the epilogue into L2 early
 #pragma unroll
-                for (int u = 0; u < L / 64; ++u) {
-                    const int tau = hf * (L / 2) + u * 32 + lane;
+                for (int u = 0; u < NBLK; ++u) {
+                    const int tau = hq * TQ + u * 16 + (lane >> 1);
                     if (tau < len)
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32));
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + ((size_t)bh * p.S + t0 + tau) * p.DV + j0 +
+                                                                        q * 32 + (lane & 1) * 16));
                 }
             }
-            named_sync(1, 256);   // previous chunk's readers of the per-row arrays are done
+            named_sync(1, 512);   // previous chunk's readers of the per-row arrays are done
             if (ct == 0) WALK_TRACE(10);
             if (ct < L) {
                 if (ct < len) {
@@ -629,7 +646,6 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     wcol[ct] = 0.f;
                 }
             }
-            named_sync(1, 256);
 
             // (b) Cb = fp16(C_c 2^-kc) into TMEM, kc from max |C_c| over the tile; rescale the
             //     fp32 state when the frame moves
@@ -638,20 +654,22 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (ct == 0) WALK_TRACE(12);
             tc_fence_after();
             float cmax = 0.f;
-            for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+#pragma unroll
+            for (int uc = 0; uc < CQ / 16; ++uc) {
+                const int c0 = hq * CQ + uc * 16;
+                uint32_t r[16];
+                tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 32; ++u) cmax = fmaxf(cmax, fabsf(__uint_as_float(r[u])));
+                for (int u = 0; u < 16; ++u) cmax = fmaxf(cmax, fabsf(__uint_as_float(r[u])));
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
-            if (lane == 0) red[ct >> 5] = cmax;
-            named_sync(1, 256);
+            if (lane == 0) red[cw] = cmax;
+            named_sync(1, 512);                   // red[] and the per-row arrays are complete
             cmax = red[0];
 #pragma unroll
-            for (int w8 = 1; w8 < 8; ++w8) cmax = fmaxf(cmax, red[w8]);
+            for (int w16 = 1; w16 < 16; ++w16) cmax = fmaxf(cmax, red[w16]);
             cmax *= alpha;
             int kc = 0;
             if (cmax > 0.f) {
@@ -660,84 +678,83 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 kc = min(max(ex - 8, -120), 14);         // |Cb| < 2^8
             }
             const float cbs = ldexpf(alpha, -kc);
-            for (int c0 = hf * (DK / 2); c0 < (hf + 1) * (DK / 2); c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
-                tmem_wait_ld();
-                uint32_t pk[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u)
+            for (int uc = 0; uc < CQ / 16; ++uc) {
+                const int c0 = hq * CQ + uc * 16;
+                uint32_t r[16];
+                tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                tmem_wait_ld();
+                uint32_t pk[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
                     pk[u] = pack_f16(__uint_as_float(r[2 * u]) * cbs, __uint_as_float(r[2 * u + 1]) * cbs);
-                tmem_st16(tmem_addr(tmem, q * 32, SM::CB_COL + c0 / 2), pk);
+                tmem_st8(tmem_addr(tmem, q * 32, SM::CB_COL + c0 / 2), pk);
                 if (rescale) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
-                    tmem_st32(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                    for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
+                    tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
                 }
             }
             tmem_wait_st();
 
-            // (c) S -> P (bf16, shared, K-major swizzled), row sums
+            // (c) S -> P (bf16, shared, K-major swizzled), partial row sums over a quarter of the columns
             if (ct == 0) WALK_TRACE(13);
             if (!mbar_wait(s_full, ph, wc)) { ok = false; break; }
             if (ct == 0) WALK_TRACE(14);
             tc_fence_after();
             if (L == 128) {
                 const int tau = q * 32 + lane;
+                const int s0 = hq * 32;
                 float sum = 0.f;
+                uint32_t pk[16];
+                if (s0 > q * 32) {                 // whole 32 x 32 block above the diagonal: zeros
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int s0 = hf * 64 + u * 32;
-                    uint32_t pk[16];
-                    if (s0 > q * 32) {                 // whole 32 x 32 block above the diagonal: zeros
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                } else {
+                    uint32_t r[32];
+                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                    tmem_wait_ld();
+                    const float at = arow[tau];
+                    const float ri = 1.f / rrow[tau];
+                    const bool diag = (s0 == q * 32);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                    } else {
-                        uint32_t r[32];
-                        tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
-                        tmem_wait_ld();
-                        const float at = arow[tau];
-                        const float ri = 1.f / rrow[tau];
-                        const bool diag = (s0 == q * 32);
+                    for (int e = 0; e < 16; ++e) {
+                        float v2[2];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            float v2[2];
-#pragma unroll
-                            for (int z = 0; z < 2; ++z) {
-                                const int sg = s0 + 2 * e + z;
-                                float d = exp2f(at + icol[sg]);
-                                if (diag && sg > tau) d = 0.f;
-                                v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
-                                sum += v2[z];
-                            }
-                            pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
+                        for (int z = 0; z < 2; ++z) {
+                            const int sg = s0 + 2 * e + z;
+                            float d = exp2f(at + icol[sg]);
+                            if (diag && sg > tau) d = 0.f;
+                            v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
+                            sum += v2[z];
                         }
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int jc = (s0 >> 3) + e;          // 16-byte chunk index within the row
-                        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jc, L)) =
-                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
                     }
                 }
-                rs[hf * L + tau] = sum;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int jcs = (s0 >> 3) + e;          // 16-byte chunk index within the row
+                    *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jcs, L)) =
+                        make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+                rs[hq * L + tau] = sum;
             } else {   // L == 64: M = 64 accumulator, rows 16q..16q+15 in lanes 0..15 of quadrant q
                 const int tau = q * 16 + (lane & 15);
-                const int s0 = hf * 32;
-                const bool above = s0 > q * 16 + 15;   // the whole 16 x 32 block is masked
-                const bool below = s0 + 31 < q * 16;   // the whole block is causal
-                uint32_t r[32];
+                const int s0 = hq * 16;
+                const bool above = s0 > q * 16 + 15;   // the whole 16 x 16 block is masked
+                const bool below = s0 + 15 < q * 16;   // the whole block is causal
+                uint32_t r[16];
                 if (!above) {
-                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                    tmem_ld16(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
                     tmem_wait_ld();
                 }
                 if (lane < 16) {
                     float sum = 0.f;
                     const float at = arow[tau];
                     const float ri = 1.f / rrow[tau];
-                    uint32_t pk[16];
+                    uint32_t pk[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
+                    for (int e = 0; e < 8; ++e) {
                         float v2[2];
 #pragma unroll
                         for (int z = 0; z < 2; ++z) {
@@ -753,19 +770,19 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
                     }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int jc = (s0 >> 3) + e;
-                        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jc, L)) =
+                    for (int e = 0; e < 2; ++e) {
+                        const int jcs = (s0 >> 3) + e;
+                        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jcs, L)) =
                             make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                     }
-                    rs[hf * L + tau] = sum;
+                    rs[hq * L + tau] = sum;
                 }
             }
 
             if (ct == 0) WALK_TRACE(15);
-            constexpr int RSTEP = 8 * RPW;            // row stride of a warp in the row passes
+            constexpr int RSTEP = 16 * RPW;           // row stride of a warp in the row passes
             constexpr int NB = (L / RSTEP) < 4 ? (L / RSTEP) : 4;   // rows in flight per iteration
-            static_assert(L % (RSTEP * NB) == 0, "row pass unroll");
+            static_assert(NB >= 1 && L % (RSTEP * NB) == 0, "row pass unroll");
             // (d) Q row pass (a warp per row, a 16-byte chunk per lane): den_inter = alpha sc (q . nX)
             //     from the unscaled bf16 q (fp32, warp reduction), then Q' = 2^(e + kc) q in fp16 (exact),
             //     in place as the MMA operand
@@ -806,7 +823,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             fence_proxy_async();
             tc_fence_before();
-            named_sync(1, 256);
+            named_sync(1, 512);
             if (lane == 0) mbar_arrive(ep1);         // P, Q' and Cb are ready: the output MMA can start
             if (ct == 0) WALK_TRACE(16);
 
@@ -841,21 +858,21 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int z = 0; z < 8; ++z) np[z] = nacc[z];
             }
-            named_sync(1, 256);
+            named_sync(1, 512);
             // normalizer for the next chunk; 1 / denominator (times r) of this chunk
             if (!last) {
-                for (int d = ct; d < DK; d += 256) {
+                for (int d = ct; d < DK; d += 512) {
                     float acc = nX[d] * beta;
 #pragma unroll 8
-                    for (int pr = 0; pr < 8 * RPW; ++pr) acc += npart[pr * DK + d];
+                    for (int pr = 0; pr < 16 * RPW; ++pr) acc += npart[pr * DK + d];
                     nX[d] = acc;
                 }
             }
             if (ct < L) {
-                const float den = rs[ct] + rs[L + ct] + dint[ct];
+                const float den = rs[ct] + rs[L + ct] + rs[2 * L + ct] + rs[3 * L + ct] + dint[ct];
                 inv[ct] = rrow[ct] / fmaxf(fabsf(den), expf(-mrow[ct]));
             }
-            named_sync(1, 256);
+            named_sync(1, 512);
             if (ct == 0) WALK_TRACE(17);
 
             // (g) outputs: H^T (lane = value column j, columns = tokens)
@@ -863,50 +880,52 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (ct == 0) WALK_TRACE(18);
             tc_fence_after();
             {
-                // each warp owns value columns [32q, 32q + 32) and tokens [hf L/2, (hf+1) L/2); per block of
-                // 32 tokens the 32 x 32 tile goes through shared memory (4 KB per warp, granules of four
-                // floats XOR-swizzled by the row) so that a lane then holds one token row of 32 columns and
+                // each warp owns value columns [32q, 32q + 32) and the tokens of its quarter; per block of
+                // 16 tokens the 16 x 32 tile goes through shared memory (2 KB per warp, granules of four
+                // floats XOR-swizzled by the row) so that a lane then holds 16 columns of one token and
                 // reads o / writes h with 16-byte vectors
-                float *tile = reinterpret_cast<float *>(Ts) + cw * 1024;
+                float *tile = reinterpret_cast<float *>(Ts) + cw * 512;
                 const __nv_bfloat16 *__restrict__ op = p.o;
                 __nv_bfloat16 *__restrict__ hp = p.h;
-                uint4 ou[L / 64][4];                      // output gate of this lane's token rows, loaded first
+                const int er = lane >> 1, jh = lane & 1;   // token row of the block, column half
+                uint4 ou[NBLK][2];                         // output gate, loaded before the TMEM reads
 #pragma unroll
-                for (int u = 0; u < L / 64; ++u) {
-                    const int tau = hf * (L / 2) + u * 32 + lane;
-                    const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32;
+                for (int u = 0; u < NBLK; ++u) {
+                    const int tau = hq * TQ + u * 16 + er;
+                    const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32 + jh * 16;
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8)
+                    for (int c8 = 0; c8 < 2; ++c8)
                         ou[u][c8] = (op && tau < len) ? *reinterpret_cast<const uint4 *>(op + off + c8 * 8)
                                                        : make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
                 }
                 if (ct == 0) WALK_TRACE(20);
 #pragma unroll
-                for (int u = 0; u < L / 64; ++u) {
-                    const int tb = hf * (L / 2) + u * 32;
+                for (int u = 0; u < NBLK; ++u) {
+                    const int tb = hq * TQ + u * 16;
                     if (ct == 0 && u == 1) WALK_TRACE(21);
-                    uint32_t r[32];
-                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + tb), r);
+                    uint32_t r[16];
+                    tmem_ld16(tmem_addr(tmem, q * 32, SM::HS_COL + tb), r);
                     tmem_wait_ld();
-                    // lane = value column j (= lane): element (token e, column lane)
+                    // lane = value column j: element (token e, column lane), 16 tokens
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
+                    for (int e = 0; e < 16; ++e)
                         tile[e * 32 + ((((lane >> 2) ^ (e & 7)) << 2) | (lane & 3))] = __uint_as_float(r[e]);
                     __syncwarp();
-                    // lane = token tb + lane: its 32 columns
-                    const int tau = tb + lane;
-                    float hv[32];
+                    // lane -> token er of the block, columns [16 jh, 16 jh + 16)
+                    float hv[16];
 #pragma unroll
-                    for (int gq = 0; gq < 8; ++gq) {
-                        const float4 v4 = *reinterpret_cast<const float4 *>(tile + lane * 32 + ((gq ^ (lane & 7)) << 2));
+                    for (int gq = 0; gq < 4; ++gq) {
+                        const float4 v4 =
+                            *reinterpret_cast<const float4 *>(tile + er * 32 + (((jh * 4 + gq) ^ (er & 7)) << 2));
                         hv[4 * gq] = v4.x; hv[4 * gq + 1] = v4.y; hv[4 * gq + 2] = v4.z; hv[4 * gq + 3] = v4.w;
                     }
                     __syncwarp();
+                    const int tau = tb + er;
                     if (tau < len) {
-                        const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32;
+                        const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32 + jh * 16;
                         const float iv = inv[tau];
 #pragma unroll
-                        for (int c8 = 0; c8 < 4; ++c8) {
+                        for (int c8 = 0; c8 < 2; ++c8) {
                             float og[8];     // bf16 1.0 = 0x3F80 when there is no output gate
                             const float2 a0 = unpack_bf16(ou[u][c8].x), a1 = unpack_bf16(ou[u][c8].y),
                                          a2 = unpack_bf16(ou[u][c8].z), a3 = unpack_bf16(ou[u][c8].w);
@@ -986,8 +1005,16 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     const int ntile = a.DHV / DVT;
     cudaError_t e;
 
-    if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK>, SegSmem<DK>::TOTAL)) != cudaSuccess) return e;
-    segsum_kernel<DK><<<dim3(ntile, w.NSEG, a.BH), 192, SegSmem<DK>::TOTAL, a.stream>>>(mk64, mv64, p);
+    // two value tiles per segment-sum CTA when that costs fewer whole waves of 148 SMs
+    const long long ctas1 = (long long)ntile * w.NSEG * a.BH;
+    const bool two = ntile % 2 == 0 && 1.4 * ((ctas1 / 2 + 147) / 148) < (double)((ctas1 + 147) / 148);
+    if (two) {
+        if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK, 2>, SegSmem<DK, 2>::TOTAL)) != cudaSuccess) return e;
+        segsum_kernel<DK, 2><<<dim3(ntile / 2, w.NSEG, a.BH), 192, SegSmem<DK, 2>::TOTAL, a.stream>>>(mk64, mv64, p);
+    } else {
+        if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK, 1>, SegSmem<DK, 1>::TOTAL)) != cudaSuccess) return e;
+        segsum_kernel<DK, 1><<<dim3(ntile, w.NSEG, a.BH), 192, SegSmem<DK, 1>::TOTAL, a.stream>>>(mk64, mv64, p);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;
 
@@ -999,7 +1026,7 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
 
     using WS = WalkSmem<DK, L>;
     if ((e = ensure_dynamic_smem((const void *)walk_kernel<DK, L>, WS::TOTAL)) != cudaSuccess) return e;
-    walk_kernel<DK, L><<<dim3(ntile, w.NSEG, a.BH), 320, WS::TOTAL, a.stream>>>(mq, mk, mv, p);
+    walk_kernel<DK, L><<<dim3(ntile, w.NSEG, a.BH), WALK_THREADS, WS::TOTAL, a.stream>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
