@@ -20,6 +20,7 @@ same workload instead, on rank 0 only.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -264,10 +265,22 @@ def traffic_for(kernel: str):
         return None
 
 
+def workload_for(args) -> Workload:
+    """The named workload, with its sequence length (``--seq``) or batch (``--batch``) replaced
+    when given (other cases of the same shapes for profiler captures; the JSON line's config shows
+    the sizes used)."""
+    w = WORKLOADS[args.workload]
+    if args.seq:
+        w = dataclasses.replace(w, S=args.seq)
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch)
+    return w
+
+
 def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    w = WORKLOADS[args.workload]
+    w = workload_for(args)
     peaks = load_peaks()
     dist = world > 1
     if dist:
@@ -281,6 +294,8 @@ def run_ours(args, rank, world, local_rank):
     one_set = w.B * w.NH * w.S * ((2 * w.DHQK + 2 * w.DHV) * (4 if w.dtype == "f32" else 2) + 8)
     nsets = max(2, math.ceil(3 * L2_BYTES / max(one_set, 1)))
     nsets = min(nsets, 16)
+    if args.sets:
+        nsets = max(2, min(nsets, args.sets))
     sets = device_inputs(w, nsets, device, seed=w.seed + 7919 * rank)
     run = Runner(w, device)
     stream = torch.cuda.current_stream()
@@ -337,26 +352,53 @@ def run_ours(args, rank, world, local_rank):
                 for p, name in enumerate(binding.PHASE_NAMES)}
     phase_ms["decode_step"] = sum(st_ev[s][0].elapsed_time(st_ev[s][1]) for s in range(args.steps)) / args.steps
 
-    # ---- end to end through the public API with host buffers (pinned), eager
+    # ---- end to end through the public API with host buffers (pinned), eager.  Every step copies
+    # its inputs host -> device and its outputs (h of the prefill and of the decode step) back.
+    # Steps are pipelined over three streams: the inputs of step s + 1 go up while step s computes
+    # and the outputs of step s - 1 come down; two input buffers and two output sets alternate.
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in sets[0].items()}
-    dev = sets[0]
+    devs = [sets[0], sets[1 % nsets]]
+    runs = [run, Runner(w, device)]
     h_host = torch.empty(run.h.shape, dtype=run.h.dtype).pin_memory()
     hd_host = torch.empty(run.hd.shape, dtype=run.hd.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = h_host.numel() * h_host.element_size() + hd_host.numel() * hd_host.element_size()
+    s_up, s_comp, s_down = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    up_done, comp_done, down_done = [None] * args.steps, [None] * args.steps, [None] * args.steps
     te0 = time.time()
-    e0.record()
+    e0.record(stream)
+    for st in (s_up, s_comp, s_down):
+        st.wait_event(e0)
     for s in range(args.steps):
-        for key, hv in host.items():
-            if hv is not None:
-                dev[key].copy_(hv, non_blocking=True)
-        run.step(dev)
-        h_host.copy_(run.h, non_blocking=True)
-        hd_host.copy_(run.hd, non_blocking=True)
-    e1.record()
+        b = s & 1
+        if s >= 2:
+            s_up.wait_event(comp_done[s - 2])        # the buffer's previous step has read its inputs
+        with torch.cuda.stream(s_up):
+            for key, hv in host.items():
+                if hv is not None:
+                    devs[b][key].copy_(hv, non_blocking=True)
+        up_done[s] = ev()
+        up_done[s].record(s_up)
+        s_comp.wait_event(up_done[s])
+        if s >= 2:
+            s_comp.wait_event(down_done[s - 2])      # the output set's previous results are on the host
+        with torch.cuda.stream(s_comp):
+            runs[b].step(devs[b])
+        comp_done[s] = ev()
+        comp_done[s].record(s_comp)
+        s_down.wait_event(comp_done[s])
+        with torch.cuda.stream(s_down):
+            h_host.copy_(runs[b].h, non_blocking=True)
+            hd_host.copy_(runs[b].hd, non_blocking=True)
+        down_done[s] = ev()
+        down_done[s].record(s_down)
+    for st in (s_up, s_comp, s_down):
+        stream.wait_stream(st)
+    e1.record(stream)
     torch.cuda.synchronize()
     te1 = time.time()
     clocks.stop()
@@ -414,7 +456,8 @@ def run_ours(args, rank, world, local_rank):
                    "timing": "CUDA graph replay" if use_graph else "eager"},
         "roofline": roof,
         "cpu_baseline": None,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipeline": "upload, compute and download of consecutive steps on three streams"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(tw0, tw1),
         "phases_us": {k: round(v * 1e3, 2) for k, v in phase_ms.items()},
@@ -534,7 +577,7 @@ def cpu_baseline(w: Workload):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = workload_for(args)
     import oracle
     from xlstm_mlstm_cell_b200.workloads import make_fwd_inputs
     oracle.build()
@@ -575,6 +618,9 @@ def main():
     ap.add_argument("--extras", type=int, default=1, help="also time the other workloads (rank 0)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq", type=int, default=0, help="override the workload's sequence length (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling)")
+    ap.add_argument("--sets", type=int, default=0, help="cap the number of rotated input sets (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -378,9 +378,9 @@ struct WalkSmem {
     // transpose staging of the output epilogue (16 warps x 2 KB): the P tile when it is 32 KB
     static constexpr uint32_t T_OFF = (L * L * 2 >= 32768) ? P_OFF : P_OFF + L * L * 2;
     static constexpr uint32_t F_OFF = T_OFF == P_OFF ? P_OFF + L * L * 2 : T_OFF + 32768;   // float arrays
-    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [4][L]; dint, inv, qexp, rrow [L]; nX [DK];
-    // red [16]; npart [4096] (n partial sums of the row pass: 16 warps x RPW rows x DK)
-    static constexpr uint32_t NF = L * 13 + DK + 16 + 4096;
+    // float arrays: arow, mrow, icol, srow, wcol [L]; rs [4][L]; inv, qexp, rrow, ccol [L];
+    // dpart [512] (partial q . n of the Q pass); bcol [16]; nX [DK]; red [16]
+    static constexpr uint32_t NF = L * 13 + 512 + 16 + DK + 16;
     static constexpr uint32_t BAR_OFF = F_OFF + NF * 4;
     static constexpr uint32_t TOTAL = BAR_OFF + 16 * 8 + 16 + 1024;
     static constexpr uint32_t C_COL = 0, CB_COL = DK, HS_COL = DK + DK / 2;
@@ -403,8 +403,8 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint8_t *Ts = smem + SM::T_OFF;
     float *F = reinterpret_cast<float *>(smem + SM::F_OFF);
     float *arow = F, *mrow = F + L, *icol = F + 2 * L, *srow = F + 3 * L, *wcol = F + 4 * L;
-    float *rs = F + 5 * L, *dint = F + 9 * L, *inv = F + 10 * L;
-    float *qexp = F + 11 * L, *rrow = F + 12 * L, *nX = F + 13 * L, *red = nX + DK, *npart = red + 16;
+    float *rs = F + 5 * L, *inv = F + 9 * L, *qexp = F + 10 * L, *rrow = F + 11 * L, *ccol = F + 12 * L;
+    float *dpart = F + 13 * L, *bcol = dpart + 512, *nX = bcol + 16, *red = nX + DK;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR_OFF);
     uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *h_full = bars + 4;
     uint64_t *c_upd = bars + 5, *q_empty = bars + 6, *k_empty = bars + 7, *v_empty = bars + 8, *ep1 = bars + 9;
@@ -545,10 +545,6 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float *igb = p.ig + (size_t)bh * p.S;
         const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
         const float *Gb = p.G + (size_t)bh * p.NC;
-        // row pass mapping: a warp takes RPW rows at a time, one 16-byte chunk (8 columns) per lane
-        constexpr int CPR = DK / 8;               // chunks per row
-        constexpr int RPW = 32 / CPR;             // rows per warp step
-        const int rsub = lane / CPR, jc = lane % CPR;
         constexpr int CQ = DK / 4;                // state columns of a warp (a quarter of DK)
         static_assert(CQ % 16 == 0, "state quarter");
 
@@ -645,6 +641,15 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     rrow[ct] = 1.f;
                     wcol[ct] = 0.f;
                 }
+                // column factors for the blocks of S below the diagonal: 2^(icol - bcol) with bcol
+                // the maximum of icol over the block's L/4 columns (so the factor is at most 1)
+                constexpr int BW = L / 4;
+                const float ic = ct < len ? (ci - ca) * LOG2E : -INFINITY;
+                float bm = ic;
+#pragma unroll
+                for (int o = BW / 2; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+                ccol[ct] = bm == -INFINITY ? 0.f : exp2f(ic - bm);
+                if ((ct & (BW - 1)) == 0) bcol[ct / BW] = bm;
             }
 
             // (b) Cb = fp16(C_c 2^-kc) into TMEM, kc from max |C_c| over the tile; rescale the
@@ -716,19 +721,29 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     tmem_wait_ld();
                     const float at = arow[tau];
                     const float ri = 1.f / rrow[tau];
-                    const bool diag = (s0 == q * 32);
+                    if (s0 == q * 32) {            // diagonal block: the decay per element, causal mask
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float v2[2];
+                        for (int e = 0; e < 16; ++e) {
+                            float v2[2];
 #pragma unroll
-                        for (int z = 0; z < 2; ++z) {
-                            const int sg = s0 + 2 * e + z;
-                            float d = exp2f(at + icol[sg]);
-                            if (diag && sg > tau) d = 0.f;
-                            v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
-                            sum += v2[z];
+                            for (int z = 0; z < 2; ++z) {
+                                const int sg = s0 + 2 * e + z;
+                                float d = exp2f(at + icol[sg]);
+                                if (sg > tau) d = 0.f;
+                                v2[z] = __uint_as_float(r[2 * e + z]) * d * scale;
+                                sum += v2[z];
+                            }
+                            pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
                         }
-                        pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
+                    } else {                       // below the diagonal: row factor x column factor
+                        const float rf = tau < len ? exp2f(at + bcol[hq]) * scale : 0.f;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float v0 = __uint_as_float(r[2 * e]) * (ccol[s0 + 2 * e] * rf);
+                            const float v1 = __uint_as_float(r[2 * e + 1]) * (ccol[s0 + 2 * e + 1] * rf);
+                            sum += v0 + v1;
+                            pk[e] = pack_bf16(v0 * ri, v1 * ri);
+                        }
                     }
                 }
 #pragma unroll
@@ -753,21 +768,32 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const float at = arow[tau];
                     const float ri = 1.f / rrow[tau];
                     uint32_t pk[8];
+                    if (below) {                   // row factor x column factor
+                        const float rf = tau < len ? exp2f(at + bcol[hq]) * scale : 0.f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float v2[2];
-#pragma unroll
-                        for (int z = 0; z < 2; ++z) {
-                            const int sg = s0 + 2 * e + z;
-                            float d = 0.f;
-                            if (!above) {
-                                d = exp2f(at + icol[sg]);
-                                if (!below && sg > tau) d = 0.f;
-                            }
-                            v2[z] = above ? 0.f : __uint_as_float(r[2 * e + z]) * d * scale;
-                            sum += v2[z];
+                        for (int e = 0; e < 8; ++e) {
+                            const float v0 = __uint_as_float(r[2 * e]) * (ccol[s0 + 2 * e] * rf);
+                            const float v1 = __uint_as_float(r[2 * e + 1]) * (ccol[s0 + 2 * e + 1] * rf);
+                            sum += v0 + v1;
+                            pk[e] = pack_bf16(v0 * ri, v1 * ri);
                         }
-                        pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            float v2[2];
+#pragma unroll
+                            for (int z = 0; z < 2; ++z) {
+                                const int sg = s0 + 2 * e + z;
+                                float d = 0.f;
+                                if (!above) {
+                                    d = exp2f(at + icol[sg]);
+                                    if (sg > tau) d = 0.f;
+                                }
+                                v2[z] = above ? 0.f : __uint_as_float(r[2 * e + z]) * d * scale;
+                                sum += v2[z];
+                            }
+                            pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
+                        }
                     }
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
@@ -780,46 +806,33 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
 
             if (ct == 0) WALK_TRACE(15);
-            constexpr int RSTEP = 16 * RPW;           // row stride of a warp in the row passes
-            constexpr int NB = (L / RSTEP) < 4 ? (L / RSTEP) : 4;   // rows in flight per iteration
-            static_assert(NB >= 1 && L % (RSTEP * NB) == 0, "row pass unroll");
-            // (d) Q row pass (a warp per row, a 16-byte chunk per lane): den_inter = alpha sc (q . nX)
-            //     from the unscaled bf16 q (fp32, warp reduction), then Q' = 2^(e + kc) q in fp16 (exact),
-            //     in place as the MMA operand
+            // (d) Q pass, a thread per (row, range of CPT 16-byte chunks): the partial inter-chunk
+            //     denominator q . nX from the unscaled bf16 q (fp32), then Q' = 2^(e + kc) q in fp16
+            //     (exact), in place as the MMA operand
             {
-                float nx[8];
+                constexpr int CPT = DK * L / 4096;       // chunks per thread
+                constexpr int PARTS = 512 / L;           // threads per row
+                static_assert(CPT >= 1 && CPT <= 8 && PARTS * CPT * 8 == DK, "Q pass mapping");
+                const int row = ct % L, part = ct / L;
+                const int jc0 = part * CPT;
+                const int qe = (int)qexp[row] + kc;
+                const float s2 = qe >= -126 ? __int_as_float((qe + 127) << 23) : 0.f;
+                float dot = 0.f;
 #pragma unroll
-                for (int z = 0; z < 8; ++z) nx[z] = nX[jc * 8 + z];
-                for (int row0 = cw * RPW + rsub; row0 < L; row0 += RSTEP * NB) {
-                    uint4 uq[NB];
-#pragma unroll
-                    for (int b = 0; b < NB; ++b)
-                        uq[b] = *reinterpret_cast<const uint4 *>(Qs + sw128_chunk(row0 + b * RSTEP, jc, L));
-                    float dot[NB];
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const float2 f0 = unpack_bf16(uq[b].x), f1 = unpack_bf16(uq[b].y), f2 = unpack_bf16(uq[b].z),
-                                     f3 = unpack_bf16(uq[b].w);
-                        dot[b] = f0.x * nx[0] + f0.y * nx[1] + f1.x * nx[2] + f1.y * nx[3] + f2.x * nx[4] +
-                                 f2.y * nx[5] + f3.x * nx[6] + f3.y * nx[7];
-                    }
-#pragma unroll
-                    for (int o = CPR / 2; o > 0; o >>= 1)
-#pragma unroll
-                        for (int b = 0; b < NB; ++b) dot[b] += __shfl_xor_sync(0xffffffffu, dot[b], o);
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const int row = row0 + b * RSTEP;
-                        if (jc == 0) dint[row] = dot[b] * alpha * srow[row];
-                        const int qe = (int)qexp[row] + kc;
-                        const float s2 = qe >= -126 ? __int_as_float((qe + 127) << 23) : 0.f;
-                        const float2 f0 = unpack_bf16(uq[b].x), f1 = unpack_bf16(uq[b].y), f2 = unpack_bf16(uq[b].z),
-                                     f3 = unpack_bf16(uq[b].w);
-                        *reinterpret_cast<uint4 *>(Qs + sw128_chunk(row, jc, L)) =
-                            make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
-                                       pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
-                    }
+                for (int u = 0; u < CPT; ++u) {
+                    const uint32_t off = sw128_chunk(row, jc0 + u, L);
+                    const uint4 uq = *reinterpret_cast<const uint4 *>(Qs + off);
+                    const float4 na = *reinterpret_cast<const float4 *>(nX + (jc0 + u) * 8);
+                    const float4 nb = *reinterpret_cast<const float4 *>(nX + (jc0 + u) * 8 + 4);
+                    const float2 f0 = unpack_bf16(uq.x), f1 = unpack_bf16(uq.y), f2 = unpack_bf16(uq.z),
+                                 f3 = unpack_bf16(uq.w);
+                    dot += f0.x * na.x + f0.y * na.y + f1.x * na.z + f1.y * na.w + f2.x * nb.x + f2.y * nb.y +
+                           f3.x * nb.z + f3.y * nb.w;
+                    *reinterpret_cast<uint4 *>(Qs + off) =
+                        make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
+                                   pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
                 }
+                dpart[part * L + row] = dot;
             }
             fence_proxy_async();
             tc_fence_before();
@@ -827,49 +840,99 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (lane == 0) mbar_arrive(ep1);         // P, Q' and Cb are ready: the output MMA can start
             if (ct == 0) WALK_TRACE(16);
 
-            // (e) while the output MMA runs: K row pass, n partial sums W k from the unscaled bf16 k
-            //     (fp32) and K' = W k in bf16 in place, the operand of the state update
+            // (e) while the output MMA runs: K pass, n sums W k from the unscaled bf16 k (fp32) and
+            //     K' = W k in bf16 in place, the operand of the state update.  A warp owns CPW 16-byte
+            //     chunks of every row (lane = row), so that its n sums reduce inside the warp and go
+            //     straight into nX
             if (!last) {
-                float nacc[8];
+                constexpr int NCH = DK / 8;                   // chunks per row
+                constexpr int CPW = NCH >= 16 ? NCH / 16 : 1; // chunks per warp
+                constexpr int NV = 8 * CPW;                   // n sums per lane before the reduction
+                static_assert(NV == 8 || NV == 16, "K pass mapping");
+                if (cw < NCH) {                               // DK = 64: warps 8..15 have no chunk
+                    float nacc[NV];
 #pragma unroll
-                for (int z = 0; z < 8; ++z) nacc[z] = 0.f;
-                for (int row0 = cw * RPW + rsub; row0 < L; row0 += RSTEP * NB) {
-                    uint4 uk[NB];
+                    for (int z = 0; z < NV; ++z) nacc[z] = 0.f;
 #pragma unroll
-                    for (int b = 0; b < NB; ++b)
-                        uk[b] = *reinterpret_cast<const uint4 *>(Ks + sw128_chunk(row0 + b * RSTEP, jc, L));
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const int row = row0 + b * RSTEP;
+                    for (int rg = 0; rg < L / 32; ++rg) {
+                        const int row = rg * 32 + lane;
                         const float w = wcol[row];
-                        const float2 f0 = unpack_bf16(uk[b].x), f1 = unpack_bf16(uk[b].y), f2 = unpack_bf16(uk[b].z),
-                                     f3 = unpack_bf16(uk[b].w);
-                        nacc[0] += w * f0.x; nacc[1] += w * f0.y; nacc[2] += w * f1.x; nacc[3] += w * f1.y;
-                        nacc[4] += w * f2.x; nacc[5] += w * f2.y; nacc[6] += w * f3.x; nacc[7] += w * f3.y;
-                        *reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, jc, L)) =
-                            make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
-                                       pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
-                    }
-                }
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(kready);  // K' is ready: the state update can start
-                float *np = npart + (size_t)(cw * RPW + rsub) * DK + jc * 8;
+                        uint4 uk[CPW];
 #pragma unroll
-                for (int z = 0; z < 8; ++z) np[z] = nacc[z];
-            }
-            named_sync(1, 512);
-            // normalizer for the next chunk; 1 / denominator (times r) of this chunk
-            if (!last) {
-                for (int d = ct; d < DK; d += 512) {
-                    float acc = nX[d] * beta;
-#pragma unroll 8
-                    for (int pr = 0; pr < 16 * RPW; ++pr) acc += npart[pr * DK + d];
-                    nX[d] = acc;
+                        for (int cc = 0; cc < CPW; ++cc)
+                            uk[cc] = *reinterpret_cast<const uint4 *>(Ks + sw128_chunk(row, cw * CPW + cc, L));
+#pragma unroll
+                        for (int cc = 0; cc < CPW; ++cc) {
+                            const float2 f0 = unpack_bf16(uk[cc].x), f1 = unpack_bf16(uk[cc].y),
+                                         f2 = unpack_bf16(uk[cc].z), f3 = unpack_bf16(uk[cc].w);
+                            float *na = nacc + cc * 8;
+                            na[0] += w * f0.x; na[1] += w * f0.y; na[2] += w * f1.x; na[3] += w * f1.y;
+                            na[4] += w * f2.x; na[5] += w * f2.y; na[6] += w * f3.x; na[7] += w * f3.y;
+                            *reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, cw * CPW + cc, L)) =
+                                make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
+                                           pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
+                        }
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(kready);      // K' is ready: the state update can start
+                    // transposed reduction over the 32 lanes: each exchange halves the values a lane
+                    // holds, so that lane l ends with the sum of value l / (32 / NV)
+                    int nv = NV;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) {
+                        if (nv > 1) {
+                            const bool up = (lane & o) != 0;
+                            const int h = nv / 2;
+#pragma unroll
+                            for (int z = 0; z < NV / 2; ++z) {
+                                if (z < h) {
+                                    const float send = up ? nacc[z] : nacc[z + h];
+                                    const float keep = up ? nacc[z + h] : nacc[z];
+                                    nacc[z] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                                }
+                            }
+                            nv = h;
+                        } else {
+                            nacc[0] += __shfl_xor_sync(0xffffffffu, nacc[0], o);
+                        }
+                    }
+                    if ((lane & (32 / NV - 1)) == 0) {
+                        const int d = cw * NV + lane / (32 / NV);
+                        nX[d] = nX[d] * beta + nacc[0];
+                    }
+                } else {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(kready);
                 }
             }
+            // output gate of this thread's epilogue rows, loaded after the K pass so that the loads overlap the
+            // normalizer update and the wait for the output MMA
+            // (rows past the end of the sequence read the last row; their outputs are not stored)
+            uint4 ou[NBLK][2];
+            if (p.o) {
+                const int er = lane >> 1, jh = lane & 1;
+#pragma unroll
+                for (int u = 0; u < NBLK; ++u) {
+                    const int tau = min(hq * TQ + u * 16 + er, len - 1);
+                    const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32 + jh * 16;
+#pragma unroll
+                    for (int c8 = 0; c8 < 2; ++c8) ou[u][c8] = *reinterpret_cast<const uint4 *>(p.o + off + c8 * 8);
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < NBLK; ++u)
+#pragma unroll
+                    for (int c8 = 0; c8 < 2; ++c8)   // bf16 1.0 = 0x3F80 when there is no output gate
+                        ou[u][c8] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+            }
+
+            // 1 / denominator (times r) of this chunk (rs, dpart and the row arrays are complete since ep1)
             if (ct < L) {
-                const float den = rs[ct] + rs[L + ct] + rs[2 * L + ct] + rs[3 * L + ct] + dint[ct];
+                float qn = 0.f;
+#pragma unroll
+                for (int pp = 0; pp < 512 / L; ++pp) qn += dpart[pp * L + ct];
+                const float den = rs[ct] + rs[L + ct] + rs[2 * L + ct] + rs[3 * L + ct] + qn * alpha * srow[ct];
                 inv[ct] = rrow[ct] / fmaxf(fabsf(den), expf(-mrow[ct]));
             }
             named_sync(1, 512);
@@ -885,24 +948,12 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 // floats XOR-swizzled by the row) so that a lane then holds 16 columns of one token and
                 // reads o / writes h with 16-byte vectors
                 float *tile = reinterpret_cast<float *>(Ts) + cw * 512;
-                const __nv_bfloat16 *__restrict__ op = p.o;
                 __nv_bfloat16 *__restrict__ hp = p.h;
                 const int er = lane >> 1, jh = lane & 1;   // token row of the block, column half
-                uint4 ou[NBLK][2];                         // output gate, loaded before the TMEM reads
-#pragma unroll
-                for (int u = 0; u < NBLK; ++u) {
-                    const int tau = hq * TQ + u * 16 + er;
-                    const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32 + jh * 16;
-#pragma unroll
-                    for (int c8 = 0; c8 < 2; ++c8)
-                        ou[u][c8] = (op && tau < len) ? *reinterpret_cast<const uint4 *>(op + off + c8 * 8)
-                                                       : make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-                }
-                if (ct == 0) WALK_TRACE(20);
 #pragma unroll
                 for (int u = 0; u < NBLK; ++u) {
                     const int tb = hq * TQ + u * 16;
-                    if (ct == 0 && u == 1) WALK_TRACE(21);
+                    if (ct == 0 && u == 1) WALK_TRACE(20);
                     uint32_t r[16];
                     tmem_ld16(tmem_addr(tmem, q * 32, SM::HS_COL + tb), r);
                     tmem_wait_ld();

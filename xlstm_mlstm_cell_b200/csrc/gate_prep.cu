@@ -74,7 +74,7 @@ gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fga
     }
 }
 
-constexpr int GS_THREADS = 1024;
+constexpr int GS_THREADS = 1024;   // most threads of gate_scan_kernel; a launch uses a multiple of 32 up to this
 
 __global__ void __launch_bounds__(GS_THREADS)
 gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ Bc, float *__restrict__ MC,
@@ -83,12 +83,13 @@ gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ 
     __shared__ float sa[GS_THREADS], sb[GS_THREADS];
     const int bh = blockIdx.x;
     const int tid = threadIdx.x;
+    const int nthr = blockDim.x;
     const float *g_in = G + (size_t)bh * NC;
     const float *b_in = Bc + (size_t)bh * NC;
     float *mc_out = MC + (size_t)bh * (NC + 1);
 
     // each thread composes the maps of a contiguous range of chunks
-    const int per = (NC + GS_THREADS - 1) / GS_THREADS;
+    const int per = (NC + nthr - 1) / nthr;
     const int c0 = min(tid * per, NC), c1 = min(c0 + per, NC);
     float ga = 0.f, gb = -INFINITY;
     for (int c = c0; c < c1; ++c) {
@@ -100,7 +101,7 @@ gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ 
     sa[tid] = ga;
     sb[tid] = gb;
     __syncthreads();
-    for (int o = 1; o < GS_THREADS; o <<= 1) {
+    for (int o = 1; o < nthr; o <<= 1) {
         float pa = 0.f, pb = -INFINITY;
         const bool has = tid >= o;
         if (has) {
@@ -129,7 +130,7 @@ gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ 
     if (NC == 0 && tid == 0) mc_out[0] = m_init;
 
     // segments of R chunks: in-segment prefix of the chunk decays and the composed segment map
-    for (int sg = tid; sg < NSEG; sg += GS_THREADS) {
+    for (int sg = tid; sg < NSEG; sg += nthr) {
         float sga = 0.f, sgb = -INFINITY;
         const int e1 = min((sg + 1) * R, NC);
         for (int c = sg * R; c < e1; ++c) {
@@ -150,7 +151,8 @@ cudaError_t launch_gate_prep(const GatePrepArgs &a)
     gate_local_kernel<<<g1, GL_WARPS * 32, 0, a.stream>>>(a.igate, a.fgate, a.S, a.L, a.NC, a.A, a.M, a.G, a.Bc);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    gate_scan_kernel<<<a.BH, GS_THREADS, 0, a.stream>>>(a.NC, a.G, a.Bc, a.MC, a.R, a.NSEG, a.GP, a.SGb, a.m0);
+    const int scan_threads = a.NC >= GS_THREADS ? GS_THREADS : (a.NC + 31) / 32 * 32;
+    gate_scan_kernel<<<a.BH, scan_threads, 0, a.stream>>>(a.NC, a.G, a.Bc, a.MC, a.R, a.NSEG, a.GP, a.SGb, a.m0);
     return cudaGetLastError();
 }
 
