@@ -482,8 +482,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 def path_is_tensor(w: Workload) -> bool:
-    """True when the library takes its tensor-core path for this workload (5 launches)."""
-    return binding.fwd_kernel_launches(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 5
+    """True when the library takes its tensor-core path for this workload."""
+    return binding.fwd_tensor_path(w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 1
 
 
 def extras(device, peaks):

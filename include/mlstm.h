@@ -134,6 +134,14 @@ mlstm_status mlstm_fwd_profiled(const void *q, const void *k, const void *v,
 int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
 
 /*
+ * 1 when mlstm_fwd takes its tensor-core path for these head sizes, chunk and
+ * element type (bf16 inputs, DHQK in {64, 128, 256}, DHV a multiple of 128,
+ * chunk in {64, 128}), 0 when it takes the fp32 CUDA-core path, -1 when the
+ * combination is not supported at all.  No GPU work; a host-side query.
+ */
+int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt);
+
+/*
  * Reports whether the last mlstm_fwd that used `workspace` ran to completion:
  * synchronizes `stream`, reads the status word kept in the workspace and
  * returns MLSTM_OK or MLSTM_ERR_TIMEOUT (a bounded device-side wait gave up;

@@ -122,3 +122,26 @@ def test_fwd_state_needs_the_whole_state(lib):
 
 def test_fwd_status_rejects_null(lib):
     assert lib.mlstm_fwd_status(None, None) == 1
+
+
+def test_tensor_path_query(lib):
+    bf, f32 = binding.MLSTM_BF16, binding.MLSTM_F32
+    assert lib.mlstm_fwd_tensor_path(256, 512, 64, bf) == 1
+    assert lib.mlstm_fwd_tensor_path(64, 128, 128, bf) == 1
+    assert lib.mlstm_fwd_tensor_path(256, 512, 64, f32) == 0     # fp32 inputs: CUDA-core path
+    assert lib.mlstm_fwd_tensor_path(256, 200, 64, bf) == 0      # DHV not a multiple of 128
+    assert lib.mlstm_fwd_tensor_path(256, 512, 32, bf) == 0      # chunk 32
+    assert lib.mlstm_fwd_tensor_path(256, 512, 48, bf) == -1     # unsupported chunk
+    assert lib.mlstm_fwd_tensor_path(256, 512, 64, 7) == -1      # unsupported dtype
+
+
+def test_kernel_launch_counts(lib):
+    bf, f32 = binding.MLSTM_BF16, binding.MLSTM_F32
+    # gate preprocessing is one kernel up to 4096 tokens per head, two beyond
+    assert lib.mlstm_fwd_kernel_launches(4, 4, 2048, 256, 256, 64, bf) == 1 + 3
+    assert lib.mlstm_fwd_kernel_launches(4, 4, 4096, 256, 256, 64, bf) == 1 + 3
+    assert lib.mlstm_fwd_kernel_launches(1, 8, 4097, 256, 512, 64, bf) == 2 + 3
+    assert lib.mlstm_fwd_kernel_launches(1, 8, 131072, 256, 512, 128, bf) == 2 + 3
+    assert lib.mlstm_fwd_kernel_launches(1, 2, 64, 16, 16, 16, f32) == 1 + 2
+    assert lib.mlstm_fwd_kernel_launches(1, 2, 64 * 200, 16, 16, 64, f32) == 2 + 2
+    assert lib.mlstm_fwd_kernel_launches(0, 2, 64, 16, 16, 16, f32) == 0

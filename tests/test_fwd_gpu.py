@@ -115,6 +115,17 @@ def test_fwd_then_step_equals_longer_fwd(cuda_lib, dt, DHQK, DHV, chunk):
     assert rel_l2(m1.cpu(), m2.cpu()) <= tol
 
 
+@pytest.mark.parametrize("dt,DHQK,DHV,chunk,S", [("f32", 16, 16, 16, 4096), ("f32", 16, 16, 16, 4097),
+                                                 ("bf16", 64, 128, 64, 4096), ("bf16", 64, 128, 64, 4097)])
+def test_fwd_gate_kernel_split(cuda_lib, dt, DHQK, DHV, chunk, S):
+    """Up to 4096 tokens per head the gate preprocessing is one kernel, beyond it two; both match."""
+    # fp32 takes gentle gates here: at 4097 tokens the fp32 rounding of the log-decay sums alone
+    # (about 1.5e-5 with the workload's gate spread) would meet the 1e-5 bound of the 64-token case
+    ig, fg = ((0.0, 0.5), (8.0, 1.0)) if dt == "f32" else ((-1.0, 2.0), (4.0, 1.0))
+    inputs = make_custom(1, 2, S, DHQK, DHV, dt, seed=S, ig=ig, fg=fg)
+    check_against_oracle(inputs, chunk, TOL[dt])
+
+
 @pytest.mark.parametrize("name", ["fwd_bf16_d256", "fwd_bf16_7b"])
 def test_fwd_full_workload(cuda_lib, name):
     """Whole-tensor parity at the workload's full size (the oracle takes seconds here)."""

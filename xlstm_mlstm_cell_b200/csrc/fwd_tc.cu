@@ -63,14 +63,15 @@ constexpr float LOG2E = 1.4426950408889634f;
 #ifdef MLSTM_WALK_TRACE
 constexpr int TR_SLOTS = 24, TR_CHUNKS = 256, TR_SEGS = 64;
 __device__ long long g_walk_trace[TR_SEGS * TR_CHUNKS * TR_SLOTS];
-#define WALK_TRACE(slot)                                                                                   \
+#define WALK_TRACE_AT(slot, ci)                                                                            \
     do {                                                                                                   \
-        if (tile == 0 && bh == 0 && seg < TR_SEGS && i < TR_CHUNKS)                                        \
-            g_walk_trace[((size_t)seg * TR_CHUNKS + i) * TR_SLOTS + (slot)] = clock64();                   \
+        if (tile == 0 && bh == 0 && seg < TR_SEGS && (ci) < TR_CHUNKS)                                     \
+            g_walk_trace[((size_t)seg * TR_CHUNKS + (ci)) * TR_SLOTS + (slot)] = clock64();                \
     } while (0)
 #else
-#define WALK_TRACE(slot) do { } while (0)
+#define WALK_TRACE_AT(slot, ci) do { } while (0)
 #endif
+#define WALK_TRACE(slot) WALK_TRACE_AT(slot, i)
 
 struct Params {
     int S, L, NC, R, NSEG, DK, DV, BH;
@@ -371,19 +372,33 @@ seg_scan_kernel(Params p, float *C_final, float *n_final, float *__restrict__ m_
 
 template <int DK, int L>
 struct WalkSmem {
+    static constexpr bool TF = (L == 64);           // see Q32_OFF
+    static constexpr int KB = TF ? 2 : 1;           // K tiles in flight (chunk 64: the next chunk's K
+                                                    // loads while this chunk's K' feeds the state update)
+    static constexpr uint32_t KBYTES = DK * L * 2;
     static constexpr uint32_t Q_OFF = 0;
     static constexpr uint32_t K_OFF = Q_OFF + DK * L * 2;
-    static constexpr uint32_t V_OFF = K_OFF + DK * L * 2;
+    static constexpr uint32_t V_OFF = K_OFF + KB * KBYTES;
     static constexpr uint32_t P_OFF = V_OFF + DVT * L * 2;
     // transpose staging of the output epilogue (16 warps x 2 KB): the P tile when it is 32 KB
     static constexpr uint32_t T_OFF = (L * L * 2 >= 32768) ? P_OFF : P_OFF + L * L * 2;
-    static constexpr uint32_t F_OFF = T_OFF == P_OFF ? P_OFF + L * L * 2 : T_OFF + 32768;   // float arrays
+    static constexpr uint32_t T_END = T_OFF == P_OFF ? P_OFF + L * L * 2 : T_OFF + 32768;
+    // chunk 64: the inter-chunk product runs in tf32 straight from the fp32 state in TMEM, with
+    // Q' in fp32 (a 128-byte-swizzled K-major tile of DK / 32 blocks); chunk 128 keeps the fp16
+    // state copy in TMEM and Q' in fp16 in place of Q (an fp32 Q' would not fit in shared memory)
+    static constexpr uint32_t Q32_OFF = T_END;
+    static constexpr uint32_t F_OFF = Q32_OFF + (TF ? DK * L * 4 : 0);   // float arrays
     // float arrays: arow, mrow, icol, srow, wcol [L]; rs [4][L]; inv, qexp, rrow, ccol [L];
     // dpart [512] (partial q . n of the Q pass); bcol [16]; nX [DK]; red [16]
     static constexpr uint32_t NF = L * 13 + 512 + 16 + DK + 16;
     static constexpr uint32_t BAR_OFF = F_OFF + NF * 4;
     static constexpr uint32_t TOTAL = BAR_OFF + 16 * 8 + 16 + 1024;
-    static constexpr uint32_t C_COL = 0, CB_COL = DK, HS_COL = DK + DK / 2;
+    static constexpr uint32_t C_COL = 0, CB_COL = DK, HS_COL = TF ? DK : DK + DK / 2;
+    // chunk 128: S and H^T share one accumulator; chunk 64: separate ones, so that the next chunk's
+    // S = Q K^T runs while this chunk's outputs are read
+    static constexpr uint32_t S_COL = HS_COL, H_COL = TF ? HS_COL + L : HS_COL;
+    static constexpr uint32_t TMEM_USED = H_COL + L;
+    static constexpr uint32_t TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
 };
 
 constexpr int WALK_THREADS = 64 + 16 * 32;   // producer warp, MMA warp, 16 epilogue warps
@@ -409,6 +424,9 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint64_t *q_full = bars + 0, *k_full = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *h_full = bars + 4;
     uint64_t *c_upd = bars + 5, *q_empty = bars + 6, *k_empty = bars + 7, *v_empty = bars + 8, *ep1 = bars + 9;
     uint64_t *hs_free = bars + 10, *drain = bars + 11, *kready = bars + 12;
+    // per K buffer b: full and empty barriers (b = 0: k_full, k_empty; b = 1: bars 13, 14)
+    auto kf = [&](int b) { return b ? bars + 13 : k_full; };
+    auto ke = [&](int b) { return b ? bars + 14 : k_empty; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
     uint32_t *abort_flag = tmem_slot + 1;
 
@@ -426,8 +444,10 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(s_full, 1);
         mbar_init(h_full, 1);
         mbar_init(c_upd, 1);
-        mbar_init(q_empty, 1);
+        mbar_init(q_empty, SM::TF ? 16 : 1);   // chunk 64: released by the compute warps at ep1
         mbar_init(k_empty, 1);
+        mbar_init(bars + 13, 1);
+        mbar_init(bars + 14, 1);
         mbar_init(v_empty, 1);
         mbar_init(ep1, 16);
         mbar_init(hs_free, 16);
@@ -440,7 +460,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_prefetch(&tm_v);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, SM::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -450,7 +470,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (warp == 0) {
         if (lane == 0) {   // TMA producer: Q, K (all DK) and the V tile of every chunk
-            int nq = 0, nk = 0, nv = 0;
+            int nq = 0, nv = 0, nk0 = 0, nk1 = 0;   // loads issued per buffer
             for (int i = 0; i < nck; ++i) {
                 const int t0 = (c_begin + i) * L;
                 const uint32_t pp = (uint32_t)(i - 1) & 1u;
@@ -459,11 +479,13 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 mbar_arrive_expect_tx(q_full, DK * L * 2);
                 for (int b = 0; b < DK / 64; ++b) tma_load_3d(Qs + b * L * 128, &tm_q, b * 64, t0, bh, q_full);
                 ++nq;
-                if (i > 0 && !mbar_wait(k_empty, pp, wc)) break;
+                const int kb = i % SM::KB;
+                if (i >= SM::KB && !mbar_wait(ke(kb), (uint32_t)(i / SM::KB - 1) & 1u, wc)) break;
                 WALK_TRACE(1);
-                mbar_arrive_expect_tx(k_full, DK * L * 2);
-                for (int b = 0; b < DK / 64; ++b) tma_load_3d(Ks + b * L * 128, &tm_k, b * 64, t0, bh, k_full);
-                ++nk;
+                mbar_arrive_expect_tx(kf(kb), DK * L * 2);
+                for (int b = 0; b < DK / 64; ++b)
+                    tma_load_3d(Ks + kb * SM::KBYTES + b * L * 128, &tm_k, b * 64, t0, bh, kf(kb));
+                (kb ? nk1 : nk0) += 1;
                 if (i > 0 && !mbar_wait(v_empty, pp, wc)) break;
                 WALK_TRACE(2);
                 mbar_arrive_expect_tx(v_full, DVT * L * 2);
@@ -473,17 +495,81 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             // drain: the last load issued into each buffer has landed
             if (nq > 0) mbar_wait_drain(q_full, (uint32_t)(nq - 1) & 1u);
-            if (nk > 0) mbar_wait_drain(k_full, (uint32_t)(nk - 1) & 1u);
+            if (nk0 > 0) mbar_wait_drain(kf(0), (uint32_t)(nk0 - 1) & 1u);
+            if (nk1 > 0) mbar_wait_drain(kf(1), (uint32_t)(nk1 - 1) & 1u);
             if (nv > 0) mbar_wait_drain(v_full, (uint32_t)(nv - 1) & 1u);
         }
     } else if (warp == 1) {
         if (lane == 0) {   // MMA issuer
             constexpr uint32_t ID_S = idesc_bf16(L, L, 0, 0);       // S  = Q K^T
-            constexpr uint32_t ID_HC = idesc_f16(DVT, L, 0, 0);     // H^T = Cb^T Q'^T   (fp16, A in TMEM)
+            constexpr uint32_t ID_HC = SM::TF ? idesc_tf32(DVT, L)  // H^T = C^T Q'^T    (tf32, A in TMEM)
+                                              : idesc_f16(DVT, L, 0, 0);  // H^T = Cb^T Q'^T (fp16, A in TMEM)
             constexpr uint32_t ID_HP = idesc_bf16(DVT, L, 1, 0);    // H^T += V^T P^T
             constexpr uint32_t ID_C = idesc_bf16(DVT, DK, 1, 1);    // C^T += V^T K'
             const uint32_t qa = smem_u32(Qs), ka = smem_u32(Ks), va = smem_u32(Vs), pa = smem_u32(Ps);
             const uint32_t hs = tmem + SM::HS_COL;
+            if constexpr (SM::TF) {
+                // chunk 64: S(i + 1) is issued right after the state update of chunk i (separate S and
+                // H^T accumulators, K double-buffered), so it runs while chunk i's outputs are read
+                const uint32_t sa = tmem + SM::S_COL, ha = tmem + SM::H_COL;
+                const uint32_t q32 = smem_u32(smem + SM::Q32_OFF);
+                auto issue_s = [&](int ci) -> bool {
+                    if (!mbar_wait(q_full, (uint32_t)ci & 1u, wc)) return false;
+                    WALK_TRACE_AT(3, ci);
+                    if (!mbar_wait(kf(ci % SM::KB), (uint32_t)(ci / SM::KB) & 1u, wc)) return false;
+                    WALK_TRACE_AT(4, ci);
+                    tc_fence_after();
+                    const uint32_t kab = ka + (ci % SM::KB) * SM::KBYTES;
+#pragma unroll
+                    for (int k = 0; k < DK / 16; ++k) {
+                        const uint32_t off = (k >> 2) * L * 128 + (k & 3) * 32;
+                        mma_ss(sa, smem_desc(qa + off, 16, 1024), smem_desc(kab + off, 16, 1024), ID_S,
+                               k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(s_full);
+                    WALK_TRACE_AT(5, ci);
+                    return true;
+                };
+                bool run = nck > 0 && issue_s(0);
+                for (int i = 0; i < nck && run; ++i) {
+                    const uint32_t ph = (uint32_t)i & 1u;
+                    // the compute warps arrive on ep1 after their last reads of the previous H^T
+                    if (!mbar_wait(ep1, ph, wc)) break;
+                    WALK_TRACE(6);
+                    if (!mbar_wait(v_full, ph, wc)) break;
+                    WALK_TRACE(7);
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < DK / 8; ++k) {     // 8 tf32 = 32 bytes of a 128-byte row per step
+                        const uint32_t off = (k >> 2) * L * 128 + (k & 3) * 32;
+                        mma_ts_tf32(ha, tmem + SM::C_COL + k * 8, smem_desc(q32 + off, 16, 1024), ID_HC,
+                                    k > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int k = 0; k < L / 16; ++k) {
+                        const uint32_t poff = (k >> 2) * L * 128 + (k & 3) * 32;
+                        mma_ss(ha, smem_desc(va + k * 2048, L * 128, 1024), smem_desc(pa + poff, 16, 1024), ID_HP,
+                               1u);
+                    }
+                    mma_commit(h_full);
+                    WALK_TRACE(8);
+                    const int kb = i % SM::KB;
+                    if (i < nck - 1) {
+                        if (!mbar_wait(kready, ph, wc)) break;
+                        WALK_TRACE(9);
+                        tc_fence_after();
+                        const uint32_t kab = ka + kb * SM::KBYTES;
+#pragma unroll
+                        for (int k = 0; k < L / 16; ++k)
+                            mma_ss(tmem + SM::C_COL, smem_desc(va + k * 2048, L * 128, 1024),
+                                   smem_desc(kab + k * 2048, L * 128, 1024), ID_C, 1u);
+                        mma_commit(c_upd);
+                    }
+                    mma_commit(ke(kb));
+                    mma_commit(v_empty);
+                    if (i < nck - 1 && !issue_s(i + 1)) break;
+                }
+            } else
             for (int i = 0; i < nck; ++i) {
                 const uint32_t ph = (uint32_t)i & 1u;
                 if (!mbar_wait(q_full, ph, wc)) break;
@@ -607,6 +693,8 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float rho_new = rescale ? (mn - g) : rho;
             const float alpha = expf(rho - mc);
             const float beta = expf(rho - rho_new);
+            // scale of the TMEM state (after this chunk's rescale) as the tf32 inter product reads it
+            const float ahc = SM::TF ? expf(rho_new - mc) : 1.f;
 
             if (p.o) {   // bring this thread's output-gate rows of the epilogue into L2 early
 #pragma unroll
@@ -627,10 +715,11 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     icol[ct] = (ci - ca) * LOG2E;
                     const float sc = expf(ca + mc - mt) * scale;
                     srow[ct] = sc;
+                    const float sct = sc * ahc;                 // row scale of the inter product
                     int ex = 0;
-                    const float fr = frexpf(sc, &ex);            // sc = fr 2^ex, fr in [0.5, 1)
-                    qexp[ct] = sc > 0.f ? (float)(ex - 1) : -1000.f;
-                    rrow[ct] = sc > 0.f ? 2.f * fr : 1.f;
+                    const float fr = frexpf(sct, &ex);           // sct = fr 2^ex, fr in [0.5, 1)
+                    qexp[ct] = sct > 0.f ? (float)(ex - 1) : -1000.f;
+                    rrow[ct] = sct > 0.f ? 2.f * fr : 1.f;
                     wcol[ct] = last ? 0.f : expf(ci - ca - rho_new);
                 } else {
                     arow[ct] = 0.f;
@@ -658,6 +747,23 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (i > 0 && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
             if (ct == 0) WALK_TRACE(12);
             tc_fence_after();
+            int kc = 0;
+            if constexpr (SM::TF) {   // tf32 inter product: only the frame move touches the state here
+                if (rescale) {
+#pragma unroll
+                    for (int uc = 0; uc < CQ / 16; ++uc) {
+                        const int c0 = hq * CQ + uc * 16;
+                        uint32_t r[16];
+                        tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
+                        tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                    }
+                    tmem_wait_st();
+                }
+                named_sync(1, 512);                   // the per-row arrays are complete
+            } else {
             float cmax = 0.f;
 #pragma unroll
             for (int uc = 0; uc < CQ / 16; ++uc) {
@@ -676,7 +782,6 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int w16 = 1; w16 < 16; ++w16) cmax = fmaxf(cmax, red[w16]);
             cmax *= alpha;
-            int kc = 0;
             if (cmax > 0.f) {
                 int ex = 0;
                 frexpf(cmax, &ex);                       // cmax < 2^ex
@@ -701,6 +806,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
             tmem_wait_st();
+            }
 
             // (c) S -> P (bf16, shared, K-major swizzled), partial row sums over a quarter of the columns
             if (ct == 0) WALK_TRACE(13);
@@ -717,7 +823,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 } else {
                     uint32_t r[32];
-                    tmem_ld32(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                    tmem_ld32(tmem_addr(tmem, q * 32, SM::S_COL + s0), r);
                     tmem_wait_ld();
                     const float at = arow[tau];
                     const float ri = 1.f / rrow[tau];
@@ -760,7 +866,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const bool below = s0 + 15 < q * 16;   // the whole block is causal
                 uint32_t r[16];
                 if (!above) {
-                    tmem_ld16(tmem_addr(tmem, q * 32, SM::HS_COL + s0), r);
+                    tmem_ld16(tmem_addr(tmem, q * 32, SM::S_COL + s0), r);
                     tmem_wait_ld();
                 }
                 if (lane < 16) {
@@ -828,16 +934,28 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                  f3 = unpack_bf16(uq.w);
                     dot += f0.x * na.x + f0.y * na.y + f1.x * na.z + f1.y * na.w + f2.x * nb.x + f2.y * nb.y +
                            f3.x * nb.z + f3.y * nb.w;
-                    *reinterpret_cast<uint4 *>(Qs + off) =
-                        make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
-                                   pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
+                    if constexpr (SM::TF) {   // fp32 Q': the chunk's 8 values are two 16-byte chunks of the tile
+                        const int j32 = ((jc0 + u) >> 2) * 8 + ((jc0 + u) & 3) * 2;
+                        uint8_t *q32 = smem + SM::Q32_OFF;
+                        *reinterpret_cast<float4 *>(q32 + sw128_chunk(row, j32, L)) =
+                            make_float4(f0.x * s2, f0.y * s2, f1.x * s2, f1.y * s2);
+                        *reinterpret_cast<float4 *>(q32 + sw128_chunk(row, j32 + 1, L)) =
+                            make_float4(f2.x * s2, f2.y * s2, f3.x * s2, f3.y * s2);
+                    } else {
+                        *reinterpret_cast<uint4 *>(Qs + off) =
+                            make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
+                                       pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
+                    }
                 }
                 dpart[part * L + row] = dot;
             }
             fence_proxy_async();
             tc_fence_before();
             named_sync(1, 512);
-            if (lane == 0) mbar_arrive(ep1);         // P, Q' and Cb are ready: the output MMA can start
+            if (lane == 0) {
+                mbar_arrive(ep1);                    // P, Q' and Cb are ready: the output MMA can start
+                if constexpr (SM::TF) mbar_arrive(q_empty);   // the bf16 Q tile has been read
+            }
             if (ct == 0) WALK_TRACE(16);
 
             // (e) while the output MMA runs: K pass, n sums W k from the unscaled bf16 k (fp32) and
@@ -849,6 +967,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 constexpr int CPW = NCH >= 16 ? NCH / 16 : 1; // chunks per warp
                 constexpr int NV = 8 * CPW;                   // n sums per lane before the reduction
                 static_assert(NV == 8 || NV == 16, "K pass mapping");
+                uint8_t *Kc = Ks + (i % SM::KB) * SM::KBYTES;  // this chunk's K tile
                 if (cw < NCH) {                               // DK = 64: warps 8..15 have no chunk
                     float nacc[NV];
 #pragma unroll
@@ -860,7 +979,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         uint4 uk[CPW];
 #pragma unroll
                         for (int cc = 0; cc < CPW; ++cc)
-                            uk[cc] = *reinterpret_cast<const uint4 *>(Ks + sw128_chunk(row, cw * CPW + cc, L));
+                            uk[cc] = *reinterpret_cast<const uint4 *>(Kc + sw128_chunk(row, cw * CPW + cc, L));
 #pragma unroll
                         for (int cc = 0; cc < CPW; ++cc) {
                             const float2 f0 = unpack_bf16(uk[cc].x), f1 = unpack_bf16(uk[cc].y),
@@ -868,7 +987,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                             float *na = nacc + cc * 8;
                             na[0] += w * f0.x; na[1] += w * f0.y; na[2] += w * f1.x; na[3] += w * f1.y;
                             na[4] += w * f2.x; na[5] += w * f2.y; na[6] += w * f3.x; na[7] += w * f3.y;
-                            *reinterpret_cast<uint4 *>(Ks + sw128_chunk(row, cw * CPW + cc, L)) =
+                            *reinterpret_cast<uint4 *>(Kc + sw128_chunk(row, cw * CPW + cc, L)) =
                                 make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
                                            pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
                         }
@@ -955,7 +1074,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const int tb = hq * TQ + u * 16;
                     if (ct == 0 && u == 1) WALK_TRACE(20);
                     uint32_t r[16];
-                    tmem_ld16(tmem_addr(tmem, q * 32, SM::HS_COL + tb), r);
+                    tmem_ld16(tmem_addr(tmem, q * 32, SM::H_COL + tb), r);
                     tmem_wait_ld();
                     // lane = value column j: element (token e, column lane), 16 tokens
 #pragma unroll
@@ -994,7 +1113,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(hs_free);
+            if (!SM::TF && lane == 0) mbar_arrive(hs_free);
             if (ct == 0) WALK_TRACE(19);
             rho = rho_new + g;
         }
@@ -1003,7 +1122,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, SM::TMEM_COLS);
     }
 }
 

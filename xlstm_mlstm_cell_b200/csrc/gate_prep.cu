@@ -14,10 +14,10 @@
 // scan across chunks is a parallel max-plus scan, the "low-overhead
 // associative scan" of the guide's "Exploit Chunkwise Hardware Kernels".
 //
-// Two kernels.  gate_local_kernel is parallel over all chunks of all heads (a
-// warp per chunk, 32 tokens per pass, warp shuffles for the sums and maxima)
-// and writes a and p per token, g and b per chunk.  gate_scan_kernel runs one
-// CTA per head: it scans the chunk maps (m_c for every chunk start from the initial m_0),
+// Two kernels (one, gate_fused_kernel, for heads of at most 4096 tokens).
+// gate_local_kernel is parallel over all chunks of all heads (a warp per chunk,
+// 32 tokens per pass, warp shuffles for the sums and maxima) and writes a and p
+// per token, g and b per chunk.  gate_scan_kernel runs one CTA per head: it scans the chunk maps (m_c for every chunk start from the initial m_0),
 // and, for the tensor-core path, composes the maps of each segment of R chunks
 // and the in-segment prefix of the chunk decays.  The per-token stabilizer m_tau
 // is not stored: the consumers form it from a_tau, p_tau and m_c.
@@ -28,14 +28,11 @@ namespace mlstm {
 
 constexpr int GL_WARPS = 8;   // chunks per CTA of gate_local_kernel
 
-__global__ void __launch_bounds__(GL_WARPS * 32)
-gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fgate, int S, int L, int NC,
-                  float *__restrict__ A, float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc)
+// One warp: chunk c of head bh.
+__device__ __forceinline__ void local_chunk(const float *__restrict__ igate, const float *__restrict__ fgate, int S,
+                                            int L, int NC, int bh, int c, int lane, float *__restrict__ A,
+                                            float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc)
 {
-    const int bh = blockIdx.y;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int c = blockIdx.x * GL_WARPS + warp;
-    if (c >= NC) return;
     const float *ig = igate + (size_t)bh * S;
     const float *fg = fgate + (size_t)bh * S;
     float *a_out = A + (size_t)bh * S;
@@ -74,14 +71,25 @@ gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fga
     }
 }
 
-constexpr int GS_THREADS = 1024;   // most threads of gate_scan_kernel; a launch uses a multiple of 32 up to this
+__global__ void __launch_bounds__(GL_WARPS * 32)
+gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fgate, int S, int L, int NC,
+                  float *__restrict__ A, float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc)
+{
+    const int c = blockIdx.x * GL_WARPS + (threadIdx.x >> 5);
+    if (c < NC) local_chunk(igate, fgate, S, L, NC, blockIdx.y, c, threadIdx.x & 31, A, P, G, Bc);
+}
 
-__global__ void __launch_bounds__(GS_THREADS)
-gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ Bc, float *__restrict__ MC,
-                 int R, int NSEG, float *__restrict__ GP, float *__restrict__ SGb, const float *__restrict__ m0)
+constexpr int GS_THREADS = 1024;   // most threads of gate_scan_kernel; a launch uses a multiple of 32 up to this
+// One kernel does both steps when a head has at most FUSED_MAX_S tokens: its warps then walk at
+// most FUSED_MAX_S / 1024 serial passes of 32 tokens, fewer than the second launch costs.
+constexpr int FUSED_MAX_S = 4096;
+
+// One CTA: the chunk maps of head bh (G, Bc written before by this CTA or an earlier kernel).
+__device__ __forceinline__ void scan_head(int NC, const float *__restrict__ G, const float *__restrict__ Bc,
+                                          float *__restrict__ MC, int R, int NSEG, float *__restrict__ GP,
+                                          float *__restrict__ SGb, const float *__restrict__ m0, int bh)
 {
     __shared__ float sa[GS_THREADS], sb[GS_THREADS];
-    const int bh = blockIdx.x;
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
     const float *g_in = G + (size_t)bh * NC;
@@ -144,9 +152,41 @@ gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ 
     }
 }
 
+__global__ void __launch_bounds__(GS_THREADS)
+gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ Bc, float *__restrict__ MC,
+                 int R, int NSEG, float *__restrict__ GP, float *__restrict__ SGb, const float *__restrict__ m0)
+{
+    scan_head(NC, G, Bc, MC, R, NSEG, GP, SGb, m0, blockIdx.x);
+}
+
+// Both steps in one CTA per head for short sequences (at most FUSED_MAX_S tokens): the CTA's
+// warps take the chunks in turn, then the CTA scans the maps it has just written.
+__global__ void __launch_bounds__(GS_THREADS)
+gate_fused_kernel(const float *__restrict__ igate, const float *__restrict__ fgate, int S, int L, int NC,
+                  float *__restrict__ A, float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc,
+                  float *__restrict__ MC, int R, int NSEG, float *__restrict__ GP, float *__restrict__ SGb,
+                  const float *__restrict__ m0)
+{
+    const int bh = blockIdx.x;
+    for (int c = threadIdx.x >> 5; c < NC; c += GS_THREADS / 32)
+        local_chunk(igate, fgate, S, L, NC, bh, c, threadIdx.x & 31, A, P, G, Bc);
+    __syncthreads();   // G and Bc of this head are written (global memory, visible within the CTA)
+    scan_head(NC, G, Bc, MC, R, NSEG, GP, SGb, m0, bh);
+}
+
+int gate_prep_launches(int S, int NC)
+{
+    return NC == 0 ? 0 : (S <= FUSED_MAX_S ? 1 : 2);
+}
+
 cudaError_t launch_gate_prep(const GatePrepArgs &a)
 {
     if (a.NC == 0) return cudaSuccess;
+    if (a.S <= FUSED_MAX_S) {
+        gate_fused_kernel<<<a.BH, GS_THREADS, 0, a.stream>>>(a.igate, a.fgate, a.S, a.L, a.NC, a.A, a.M, a.G, a.Bc,
+                                                             a.MC, a.R, a.NSEG, a.GP, a.SGb, a.m0);
+        return cudaGetLastError();
+    }
     dim3 g1((a.NC + GL_WARPS - 1) / GL_WARPS, a.BH);
     gate_local_kernel<<<g1, GL_WARPS * 32, 0, a.stream>>>(a.igate, a.fgate, a.S, a.L, a.NC, a.A, a.M, a.G, a.Bc);
     cudaError_t e = cudaGetLastError();

@@ -89,8 +89,16 @@ extern "C" int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV
 {
     if (mlstm_fwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dt) == 0) return 0;
     if (B == 0 || NH == 0 || S == 0) return 0;
-    // gate preprocessing (2) + (segment sums, segment scan, walk) or (carry walk, outputs)
-    return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 5 : 4;
+    // gate preprocessing (1 or 2) + (segment sums, segment scan, walk) or (carry walk, outputs)
+    const int NC = (S + chunk - 1) / chunk;
+    return gate_prep_launches(S, NC) + (tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 3 : 2);
+}
+
+extern "C" int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if (dt != MLSTM_F32 && dt != MLSTM_BF16) return -1;
+    if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return -1;
+    return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 1 : 0;
 }
 
 namespace {

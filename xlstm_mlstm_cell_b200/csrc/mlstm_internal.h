@@ -67,6 +67,7 @@ struct PhaseMark {
 
 cudaError_t launch_step(const StepArgs &a);
 cudaError_t launch_gate_prep(const GatePrepArgs &a);
+int gate_prep_launches(int S, int NC);   // kernels launch_gate_prep launches for S tokens, NC chunks per head
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark);
 size_t simt_state_bytes(int BH, int NC, int DHQK, int DHV);
 bool tc_path_supported(bool bf16, int DHQK, int DHV, int chunk);

@@ -49,6 +49,17 @@ step_kernel(float *__restrict__ C, float *__restrict__ n, float *__restrict__ m,
     const int tx = tid % (DHV / 4);   // column group
     const int g = tid / (DHV / 4);    // row group
 
+    // the thread's first UNROLL rows of C are requested before the gate arithmetic, so that their
+    // latency overlaps it (the rest follow UNROLL at a time)
+    const int j = tx * 4;
+    float *Cb = C + ((size_t)bh * DHQK + r0) * DHV + j;
+    float4 c[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+        const int i = g + u * RG;
+        if (i < rows) c[u] = __ldcs(reinterpret_cast<const float4 *>(Cb + (size_t)i * DHV));
+    }
+
     const float lf = log_sigmoid(fgate[bh]);
     const float it = igate[bh];
     const float m_old = m[bh];
@@ -79,44 +90,35 @@ step_kernel(float *__restrict__ C, float *__restrict__ n, float *__restrict__ m,
         if (tid == 0) red[0] = x;
     }
 
-    const int j = tx * 4;
     const float4 v4 = load4(v + (size_t)bh * DHV + j);
     const float4 iv = make_float4(ip * v4.x, ip * v4.y, ip * v4.z, ip * v4.w);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float *Cb = C + ((size_t)bh * DHQK + r0) * DHV + j;
 
-    int i = g;
-    for (; i + (UNROLL - 1) * RG < rows; i += UNROLL * RG) {
-        float4 c[UNROLL];
+    // UNROLL rows in flight per thread: all loads of a group are issued before any is used
+    for (int i0 = g; i0 < rows; i0 += UNROLL * RG) {
+        if (i0 != g) {
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u)
-            c[u] = __ldcs(reinterpret_cast<const float4 *>(Cb + (size_t)(i + u * RG) * DHV));
+            for (int u = 0; u < UNROLL; ++u) {
+                const int i = i0 + u * RG;
+                if (i < rows) c[u] = __ldcs(reinterpret_cast<const float4 *>(Cb + (size_t)i * DHV));
+            }
+        }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const float kk = ks[i + u * RG], qq = qs[i + u * RG];
-            c[u].x = fmaf(fp, c[u].x, kk * iv.x);
-            c[u].y = fmaf(fp, c[u].y, kk * iv.y);
-            c[u].z = fmaf(fp, c[u].z, kk * iv.z);
-            c[u].w = fmaf(fp, c[u].w, kk * iv.w);
-            __stcs(reinterpret_cast<float4 *>(Cb + (size_t)(i + u * RG) * DHV), c[u]);
-            acc.x = fmaf(qq, c[u].x, acc.x);
-            acc.y = fmaf(qq, c[u].y, acc.y);
-            acc.z = fmaf(qq, c[u].z, acc.z);
-            acc.w = fmaf(qq, c[u].w, acc.w);
+            const int i = i0 + u * RG;
+            if (i < rows) {
+                const float kk = ks[i], qq = qs[i];
+                c[u].x = fmaf(fp, c[u].x, kk * iv.x);
+                c[u].y = fmaf(fp, c[u].y, kk * iv.y);
+                c[u].z = fmaf(fp, c[u].z, kk * iv.z);
+                c[u].w = fmaf(fp, c[u].w, kk * iv.w);
+                __stcs(reinterpret_cast<float4 *>(Cb + (size_t)i * DHV), c[u]);
+                acc.x = fmaf(qq, c[u].x, acc.x);
+                acc.y = fmaf(qq, c[u].y, acc.y);
+                acc.z = fmaf(qq, c[u].z, acc.z);
+                acc.w = fmaf(qq, c[u].w, acc.w);
+            }
         }
-    }
-    for (; i < rows; i += RG) {
-        float4 c = __ldcs(reinterpret_cast<const float4 *>(Cb + (size_t)i * DHV));
-        const float kk = ks[i], qq = qs[i];
-        c.x = fmaf(fp, c.x, kk * iv.x);
-        c.y = fmaf(fp, c.y, kk * iv.y);
-        c.z = fmaf(fp, c.z, kk * iv.z);
-        c.w = fmaf(fp, c.w, kk * iv.w);
-        __stcs(reinterpret_cast<float4 *>(Cb + (size_t)i * DHV), c);
-        acc.x = fmaf(qq, c.x, acc.x);
-        acc.y = fmaf(qq, c.y, acc.y);
-        acc.z = fmaf(qq, c.z, acc.z);
-        acc.w = fmaf(qq, c.w, acc.w);
     }
     *reinterpret_cast<float4 *>(part + (size_t)g * DHV + j) = acc;
     __syncthreads();

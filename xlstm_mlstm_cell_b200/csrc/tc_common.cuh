@@ -182,6 +182,18 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem] with tf32 operands (fp32 storage; the MMA uses the upper 19 bits).
+__device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrives on `bar` once every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
@@ -275,6 +287,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// kind::tf32 instruction descriptor: tf32 A and B (format 2), fp32 accumulator, both K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N)
+{
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Same with fp16 A and B (both operands of one MMA always share their type).
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn)
 {
@@ -306,6 +324,50 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi)
 {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): two floats in one 64-bit register, one instruction
+// for both lanes of a multiply, add or fused multiply-add (each rounded to nearest like the scalar op).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t r)
+{
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// bf16x2 (low half = first element) -> packed fp32 pair, exact.
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t u)
+{
+    return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+// packed fp32 pair -> bf16x2 (round to nearest even), first element in the low half.
+__device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t r)
+{
+    const float2 v = f2_unpack(r);
+    return pack_bf16(v.x, v.y);
 }
 
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u)
