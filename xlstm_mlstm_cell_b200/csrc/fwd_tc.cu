@@ -843,13 +843,18 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         }
                     } else {                       // below the diagonal: row factor x column factor
                         const float rf = tau < len ? exp2f(at + bcol[hq]) * scale : 0.f;
+                        const uint64_t rf2 = f2_pack(rf, rf), ri2 = f2_pack(ri, ri);
+                        const uint64_t *cc2 = reinterpret_cast<const uint64_t *>(ccol + s0);
+                        uint64_t sum2 = 0ull;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float v0 = __uint_as_float(r[2 * e]) * (ccol[s0 + 2 * e] * rf);
-                            const float v1 = __uint_as_float(r[2 * e + 1]) * (ccol[s0 + 2 * e + 1] * rf);
-                            sum += v0 + v1;
-                            pk[e] = pack_bf16(v0 * ri, v1 * ri);
+                            const uint64_t v = f2_mul(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])),
+                                                      f2_mul(cc2[e], rf2));
+                            sum2 = f2_add(sum2, v);
+                            pk[e] = f2_to_bf16x2(f2_mul(v, ri2));
                         }
+                        const float2 sd = f2_unpack(sum2);
+                        sum = sd.x + sd.y;
                     }
                 }
 #pragma unroll
@@ -923,31 +928,36 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int jc0 = part * CPT;
                 const int qe = (int)qexp[row] + kc;
                 const float s2 = qe >= -126 ? __int_as_float((qe + 127) << 23) : 0.f;
-                float dot = 0.f;
+                const uint64_t ss = f2_pack(s2, s2);
+                uint64_t dot2 = 0ull;                    // packed pair of partial dot products
 #pragma unroll
                 for (int u = 0; u < CPT; ++u) {
                     const uint32_t off = sw128_chunk(row, jc0 + u, L);
                     const uint4 uq = *reinterpret_cast<const uint4 *>(Qs + off);
-                    const float4 na = *reinterpret_cast<const float4 *>(nX + (jc0 + u) * 8);
-                    const float4 nb = *reinterpret_cast<const float4 *>(nX + (jc0 + u) * 8 + 4);
-                    const float2 f0 = unpack_bf16(uq.x), f1 = unpack_bf16(uq.y), f2 = unpack_bf16(uq.z),
-                                 f3 = unpack_bf16(uq.w);
-                    dot += f0.x * na.x + f0.y * na.y + f1.x * na.z + f1.y * na.w + f2.x * nb.x + f2.y * nb.y +
-                           f3.x * nb.z + f3.y * nb.w;
+                    const ulonglong2 na = *reinterpret_cast<const ulonglong2 *>(nX + (jc0 + u) * 8);
+                    const ulonglong2 nb = *reinterpret_cast<const ulonglong2 *>(nX + (jc0 + u) * 8 + 4);
+                    const uint64_t q0 = f2_from_bf16x2(uq.x), q1 = f2_from_bf16x2(uq.y), q2 = f2_from_bf16x2(uq.z),
+                                   q3 = f2_from_bf16x2(uq.w);
+                    dot2 = f2_fma(q0, na.x, dot2);
+                    dot2 = f2_fma(q1, na.y, dot2);
+                    dot2 = f2_fma(q2, nb.x, dot2);
+                    dot2 = f2_fma(q3, nb.y, dot2);
                     if constexpr (SM::TF) {   // fp32 Q': the chunk's 8 values are two 16-byte chunks of the tile
                         const int j32 = ((jc0 + u) >> 2) * 8 + ((jc0 + u) & 3) * 2;
                         uint8_t *q32 = smem + SM::Q32_OFF;
-                        *reinterpret_cast<float4 *>(q32 + sw128_chunk(row, j32, L)) =
-                            make_float4(f0.x * s2, f0.y * s2, f1.x * s2, f1.y * s2);
-                        *reinterpret_cast<float4 *>(q32 + sw128_chunk(row, j32 + 1, L)) =
-                            make_float4(f2.x * s2, f2.y * s2, f3.x * s2, f3.y * s2);
+                        *reinterpret_cast<ulonglong2 *>(q32 + sw128_chunk(row, j32, L)) =
+                            make_ulonglong2(f2_mul(q0, ss), f2_mul(q1, ss));
+                        *reinterpret_cast<ulonglong2 *>(q32 + sw128_chunk(row, j32 + 1, L)) =
+                            make_ulonglong2(f2_mul(q2, ss), f2_mul(q3, ss));
                     } else {
-                        *reinterpret_cast<uint4 *>(Qs + off) =
-                            make_uint4(pack_f16(f0.x * s2, f0.y * s2), pack_f16(f1.x * s2, f1.y * s2),
-                                       pack_f16(f2.x * s2, f2.y * s2), pack_f16(f3.x * s2, f3.y * s2));
+                        const float2 a0 = f2_unpack(f2_mul(q0, ss)), a1 = f2_unpack(f2_mul(q1, ss)),
+                                     a2 = f2_unpack(f2_mul(q2, ss)), a3 = f2_unpack(f2_mul(q3, ss));
+                        *reinterpret_cast<uint4 *>(Qs + off) = make_uint4(pack_f16(a0.x, a0.y), pack_f16(a1.x, a1.y),
+                                                                          pack_f16(a2.x, a2.y), pack_f16(a3.x, a3.y));
                     }
                 }
-                dpart[part * L + row] = dot;
+                const float2 dd = f2_unpack(dot2);
+                dpart[part * L + row] = dd.x + dd.y;
             }
             fence_proxy_async();
             tc_fence_before();
@@ -969,28 +979,38 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 static_assert(NV == 8 || NV == 16, "K pass mapping");
                 uint8_t *Kc = Ks + (i % SM::KB) * SM::KBYTES;  // this chunk's K tile
                 if (cw < NCH) {                               // DK = 64: warps 8..15 have no chunk
-                    float nacc[NV];
+                    uint64_t nacc2[NV / 2];                   // packed pairs of n sums
 #pragma unroll
-                    for (int z = 0; z < NV; ++z) nacc[z] = 0.f;
+                    for (int z = 0; z < NV / 2; ++z) nacc2[z] = 0ull;
 #pragma unroll
                     for (int rg = 0; rg < L / 32; ++rg) {
                         const int row = rg * 32 + lane;
                         const float w = wcol[row];
+                        const uint64_t ww = f2_pack(w, w);
                         uint4 uk[CPW];
 #pragma unroll
                         for (int cc = 0; cc < CPW; ++cc)
                             uk[cc] = *reinterpret_cast<const uint4 *>(Kc + sw128_chunk(row, cw * CPW + cc, L));
 #pragma unroll
                         for (int cc = 0; cc < CPW; ++cc) {
-                            const float2 f0 = unpack_bf16(uk[cc].x), f1 = unpack_bf16(uk[cc].y),
-                                         f2 = unpack_bf16(uk[cc].z), f3 = unpack_bf16(uk[cc].w);
-                            float *na = nacc + cc * 8;
-                            na[0] += w * f0.x; na[1] += w * f0.y; na[2] += w * f1.x; na[3] += w * f1.y;
-                            na[4] += w * f2.x; na[5] += w * f2.y; na[6] += w * f3.x; na[7] += w * f3.y;
+                            const uint64_t k0 = f2_from_bf16x2(uk[cc].x), k1 = f2_from_bf16x2(uk[cc].y),
+                                           k2 = f2_from_bf16x2(uk[cc].z), k3 = f2_from_bf16x2(uk[cc].w);
+                            uint64_t *na = nacc2 + cc * 4;
+                            na[0] = f2_fma(ww, k0, na[0]);
+                            na[1] = f2_fma(ww, k1, na[1]);
+                            na[2] = f2_fma(ww, k2, na[2]);
+                            na[3] = f2_fma(ww, k3, na[3]);
                             *reinterpret_cast<uint4 *>(Kc + sw128_chunk(row, cw * CPW + cc, L)) =
-                                make_uint4(pack_bf16(f0.x * w, f0.y * w), pack_bf16(f1.x * w, f1.y * w),
-                                           pack_bf16(f2.x * w, f2.y * w), pack_bf16(f3.x * w, f3.y * w));
+                                make_uint4(f2_to_bf16x2(f2_mul(k0, ww)), f2_to_bf16x2(f2_mul(k1, ww)),
+                                           f2_to_bf16x2(f2_mul(k2, ww)), f2_to_bf16x2(f2_mul(k3, ww)));
                         }
+                    }
+                    float nacc[NV];
+#pragma unroll
+                    for (int z = 0; z < NV / 2; ++z) {
+                        const float2 v = f2_unpack(nacc2[z]);
+                        nacc[2 * z] = v.x;
+                        nacc[2 * z + 1] = v.y;
                     }
                     fence_proxy_async();
                     __syncwarp();
@@ -1095,18 +1115,17 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32 + jh * 16;
                         const float iv = inv[tau];
 #pragma unroll
+                        const uint64_t iv2 = f2_pack(iv, iv);
                         for (int c8 = 0; c8 < 2; ++c8) {
-                            float og[8];     // bf16 1.0 = 0x3F80 when there is no output gate
-                            const float2 a0 = unpack_bf16(ou[u][c8].x), a1 = unpack_bf16(ou[u][c8].y),
-                                         a2 = unpack_bf16(ou[u][c8].z), a3 = unpack_bf16(ou[u][c8].w);
-                            og[0] = a0.x; og[1] = a0.y; og[2] = a1.x; og[3] = a1.y;
-                            og[4] = a2.x; og[5] = a2.y; og[6] = a3.x; og[7] = a3.y;
+                            // o h / den in packed pairs (bf16 1.0 = 0x3F80 when there is no output gate)
                             const float *hh = hv + c8 * 8;
-                            *reinterpret_cast<uint4 *>(hp + off + c8 * 8) =
-                                make_uint4(pack_bf16(og[0] * hh[0] * iv, og[1] * hh[1] * iv),
-                                           pack_bf16(og[2] * hh[2] * iv, og[3] * hh[3] * iv),
-                                           pack_bf16(og[4] * hh[4] * iv, og[5] * hh[5] * iv),
-                                           pack_bf16(og[6] * hh[6] * iv, og[7] * hh[7] * iv));
+                            uint32_t w4[4];
+                            const uint32_t og4[4] = {ou[u][c8].x, ou[u][c8].y, ou[u][c8].z, ou[u][c8].w};
+#pragma unroll
+                            for (int z = 0; z < 4; ++z)
+                                w4[z] = f2_to_bf16x2(f2_mul(f2_from_bf16x2(og4[z]),
+                                                            f2_mul(f2_pack(hh[2 * z], hh[2 * z + 1]), iv2)));
+                            *reinterpret_cast<uint4 *>(hp + off + c8 * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                         }
                     }
                 }
