@@ -97,8 +97,11 @@ struct SegSmem {
     static constexpr uint32_t TMEM_COLS = NT * DK < 32 ? 32 : NT * DK;
 };
 
+constexpr int SS_SCALERS = 8;                     // scaler warps of segsum_kernel
+constexpr int SS_THREADS = 64 + SS_SCALERS * 32;  // producer warp, MMA warp, scalers
+
 template <int DK, int NT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(SS_THREADS, 1)
 segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Params p)
 {
     using SM = SegSmem<DK, NT>;
@@ -124,7 +127,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SS_STAGES; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&scaled[i], 4);
+            mbar_init(&scaled[i], SS_SCALERS);
             mbar_init(&empty[i], 1);
         }
         mbar_init(acc_full, 1);
@@ -186,14 +189,15 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             mbar_wait_drain(acc_full, 0);
         }
     } else {
-        // scalers (warps 2..5): K rows *= w in place; tile 0 also sums dn = sum_t w_t k_t in fp32 from
+        // scalers (warps 2..): K rows *= w in place; tile 0 also sums dn = sum_t w_t k_t in fp32 from
         // the unrounded bf16 k.  A warp takes RPW rows at a time, one 16-byte chunk per lane.
-        const int ct = threadIdx.x - 64;                 // 0..127
-        const int sw = ct >> 5;                          // scaler warp 0..3
+        constexpr int NST = SS_SCALERS * 32;             // scaler threads
+        const int ct = threadIdx.x - 64;                 // 0..NST-1
+        const int sw = ct >> 5;                          // scaler warp
         constexpr int CPR = DK / 8;                      // 16-byte chunks per row
         constexpr int RPW = 32 / CPR;                    // rows per warp step
-        constexpr int RSTEP = 4 * RPW;
-        constexpr int NB = 4;                            // rows in flight per iteration
+        constexpr int RSTEP = SS_SCALERS * RPW;
+        constexpr int NB = (TB / RSTEP) < 4 ? (TB / RSTEP) : 4;   // rows in flight per iteration
         static_assert(TB % (RSTEP * NB) == 0, "segsum row pass unroll");
         const int rsub = lane / CPR, jc = lane % CPR;
         const float Gs = p.SGb[((size_t)bh * p.NSEG + seg) * 2 + 0];
@@ -222,9 +226,9 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 pi = igb[t + TB];
                 pgp = GPb[(t + TB) / p.L];
             }
-            named_sync(1, 128);                          // the previous stage's readers of wst are done
+            named_sync(1, NST);                          // the previous stage's readers of wst are done
             if (ct < TB) wst[ct] = (t < t_end) ? expf(Gs - cgp - ca + ci - bs) : 0.f;
-            named_sync(1, 128);
+            named_sync(1, NST);
             if (!mbar_wait(&full[st], ph, wc)) { ok = false; break; }
             uint8_t *kb = smem + st * SM::STAGE;
             for (int row0 = sw * RPW + rsub; row0 < TB; row0 += RSTEP * NB) {
@@ -257,11 +261,11 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
                 for (int z = 0; z < 8; ++z) npart[(sw * RPW + rsub) * DK + jc * 8 + z] = nacc[z];
             }
-            named_sync(1, 128);
+            named_sync(1, NST);
             if (ok) {
-                for (int d = ct; d < DK; d += 128) {
+                for (int d = ct; d < DK; d += NST) {
                     float acc = 0.f;
-                    for (int pr = 0; pr < 4 * RPW; ++pr) acc += npart[pr * DK + d];
+                    for (int pr = 0; pr < SS_SCALERS * RPW; ++pr) acc += npart[pr * DK + d];
                     p.DN[((size_t)bh * p.NSEG + seg) * DK + d] = acc;
                 }
             }
@@ -269,9 +273,10 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         // epilogue: TMEM (lane = value column, columns = DK) -> workspace, quad layout [DK/4][DV][4]
         if (ok && mbar_wait(acc_full, 0, wc)) {
             tc_fence_after();
-            const int q = warp & 3;
+            const int q = warp & 3;                      // TMEM lane quadrant of the warp
+            const int half = (warp - 2) >> 2;            // two scaler warps per quadrant share its columns
             float *dst = p.DC + ((size_t)bh * p.NSEG + seg) * (size_t)DK * p.DV;
-            for (int tc = 0; tc < NT * DK; tc += 32) {
+            for (int tc = half * 32; tc < NT * DK; tc += 64) {
                 const int t = tc / DK, c0 = tc % DK;
                 const int j = t * DVT + q * 32 + lane;
                 uint32_t r[32];
@@ -1199,10 +1204,10 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     const bool two = ntile % 2 == 0 && 1.4 * ((ctas1 / 2 + 147) / 148) < (double)((ctas1 + 147) / 148);
     if (two) {
         if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK, 2>, SegSmem<DK, 2>::TOTAL)) != cudaSuccess) return e;
-        segsum_kernel<DK, 2><<<dim3(ntile / 2, w.NSEG, a.BH), 192, SegSmem<DK, 2>::TOTAL, a.stream>>>(mk64, mv64, p);
+        segsum_kernel<DK, 2><<<dim3(ntile / 2, w.NSEG, a.BH), SS_THREADS, SegSmem<DK, 2>::TOTAL, a.stream>>>(mk64, mv64, p);
     } else {
         if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK, 1>, SegSmem<DK, 1>::TOTAL)) != cudaSuccess) return e;
-        segsum_kernel<DK, 1><<<dim3(ntile, w.NSEG, a.BH), 192, SegSmem<DK, 1>::TOTAL, a.stream>>>(mk64, mv64, p);
+        segsum_kernel<DK, 1><<<dim3(ntile, w.NSEG, a.BH), SS_THREADS, SegSmem<DK, 1>::TOTAL, a.stream>>>(mk64, mv64, p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;

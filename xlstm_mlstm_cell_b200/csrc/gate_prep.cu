@@ -80,6 +80,7 @@ gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fga
 }
 
 constexpr int GS_THREADS = 1024;   // most threads of gate_scan_kernel; a launch uses a multiple of 32 up to this
+constexpr int GS_STAGE = 4096;     // chunk maps per head staged in shared memory by the scan
 // One kernel does both steps when a head has at most FUSED_MAX_S tokens: its warps then walk at
 // most FUSED_MAX_S / 1024 serial passes of 32 tokens, fewer than the second launch costs.
 constexpr int FUSED_MAX_S = 4096;
@@ -89,12 +90,24 @@ __device__ __forceinline__ void scan_head(int NC, const float *__restrict__ G, c
                                           float *__restrict__ MC, int R, int NSEG, float *__restrict__ GP,
                                           float *__restrict__ SGb, const float *__restrict__ m0, int bh)
 {
-    __shared__ float sa[GS_THREADS], sb[GS_THREADS];
+    __shared__ float wa[32], wb[32];                 // per-warp totals, then their exclusive prefixes
+    __shared__ float g_st[GS_STAGE], b_st[GS_STAGE];
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
     const float *g_in = G + (size_t)bh * NC;
     const float *b_in = Bc + (size_t)bh * NC;
     float *mc_out = MC + (size_t)bh * (NC + 1);
+    // the chunk maps go to shared memory first (parallel, coalesced loads) when they fit, so that
+    // the serial loops below read shared memory instead of waiting on one global load after another
+    if (NC <= GS_STAGE) {
+        for (int c = tid; c < NC; c += nthr) {
+            g_st[c] = g_in[c];
+            b_st[c] = b_in[c];
+        }
+        __syncthreads();
+        g_in = g_st;
+        b_in = b_st;
+    }
 
     // each thread composes the maps of a contiguous range of chunks
     const int per = (NC + nthr - 1) / nthr;
@@ -105,29 +118,50 @@ __device__ __forceinline__ void scan_head(int NC, const float *__restrict__ G, c
         ga += g;
         gb = fmaxf(gb + g, b_in[c]);
     }
-    // inclusive Hillis-Steele scan of the maps across threads, (earlier) then (later)
-    sa[tid] = ga;
-    sb[tid] = gb;
+    // exclusive scan of the maps across threads, composing (earlier) then (later):
+    // (a1, b1) then (a2, b2) = (a1 + a2, max(b1 + a2, b2)).  Shuffle scan inside each warp, then
+    // the first warp scans the warp totals.
+    const int lane = tid & 31, warp = tid >> 5, nwarp = (nthr + 31) >> 5;
+    float ia = ga, ib = gb;            // inclusive within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float pa = __shfl_up_sync(0xffffffffu, ia, o), pb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ib = fmaxf(pb + ia, ib);
+            ia = pa + ia;
+        }
+    }
+    float xa = __shfl_up_sync(0xffffffffu, ia, 1), xb = __shfl_up_sync(0xffffffffu, ib, 1);
+    if (lane == 0) {                   // exclusive within the warp
+        xa = 0.f;
+        xb = -INFINITY;
+    }
+    if (lane == 31) {
+        wa[warp] = ia;
+        wb[warp] = ib;
+    }
     __syncthreads();
-    for (int o = 1; o < nthr; o <<= 1) {
-        float pa = 0.f, pb = -INFINITY;
-        const bool has = tid >= o;
-        if (has) {
-            pa = sa[tid - o];
-            pb = sb[tid - o];
+    if (warp == 0) {
+        float ta = lane < nwarp ? wa[lane] : 0.f, tb = lane < nwarp ? wb[lane] : -INFINITY;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float pa = __shfl_up_sync(0xffffffffu, ta, o), pb = __shfl_up_sync(0xffffffffu, tb, o);
+            if (lane >= o) {
+                tb = fmaxf(pb + ta, tb);
+                ta = pa + ta;
+            }
         }
-        __syncthreads();
-        if (has) {
-            sb[tid] = fmaxf(pb + sa[tid], sb[tid]);
-            sa[tid] = pa + sa[tid];
+        float ua = __shfl_up_sync(0xffffffffu, ta, 1), ub = __shfl_up_sync(0xffffffffu, tb, 1);
+        if (lane == 0) {
+            ua = 0.f;
+            ub = -INFINITY;
         }
-        __syncthreads();
+        wa[lane] = ua;                 // exclusive prefix of the warp totals
+        wb[lane] = ub;
     }
-    float ea = 0.f, eb = -INFINITY;   // exclusive prefix map
-    if (tid > 0) {
-        ea = sa[tid - 1];
-        eb = sb[tid - 1];
-    }
+    __syncthreads();
+    // the thread's exclusive prefix: the warp's prefix, then the lanes before it
+    const float ea = wa[warp] + xa, eb = fmaxf(wb[warp] + xa, xb);
     const float m_init = m0 ? m0[bh] : 0.f;
     float mm = fmaxf(m_init + ea, eb);   // m at this thread's first chunk
     for (int c = c0; c < c1; ++c) {
