@@ -51,6 +51,42 @@ MLSTM_DEVINL float warp_sum(float x)
     return x;
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched with programmatic
+// stream serialization, so that its launch and its prologue (barrier set-up, TMEM allocation,
+// descriptor prefetch: nothing that touches global memory) overlap the tail of the kernel before
+// it.  griddep_wait() returns once the preceding grid has completed and its memory is visible;
+// it must come before the kernel's first global load or store.  griddep_launch_dependents()
+// lets the next kernel in the stream start launching (it still waits for this one to finish).
+// Both are no-ops for a kernel launched without the attribute.
+MLSTM_DEVINL void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MLSTM_DEVINL void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 int cluster_x, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (cluster_x > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)cluster_x;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)na;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device), so that
 // launches stay free of attribute calls after the first one.
 inline cudaError_t ensure_dynamic_smem(const void *kernel, int bytes)

@@ -39,6 +39,8 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
                   float *__restrict__ CS, float *__restrict__ NS,
                   float *C_final, float *n_final, float *__restrict__ m_final, const float *C0, const float *n0)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ float sm[];
     float *ks = sm;                    // [L][ST]
     float *vs = ks + L * ST;           // [L][ST]
@@ -120,6 +122,8 @@ output_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
                    const float *__restrict__ CS, const float *__restrict__ NS,
                    int S, int L, int NC, int DHQK, int DHV, T *__restrict__ h)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ float sm[];
     const int LP = L + 1;
     float *P = sm;                       // [L][L+1]
@@ -254,10 +258,9 @@ static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, co
     const int L = a.chunk;
     dim3 g1(a.BH, (a.DHQK + ST - 1) / ST, (a.DHV + ST - 1) / ST);
     const size_t sm1 = sizeof(float) * (2 * (size_t)L * ST + L);
-    carry_simt_kernel<T><<<g1, 256, sm1, a.stream>>>((const T *)a.k, (const T *)a.v, a.igate, w.A, w.G, w.MC,
-                                                     a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS, a.C_final,
-                                                     a.n_final, a.m_final, a.C0, a.n0);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(carry_simt_kernel<T>, g1, dim3(256), sm1, a.stream, 1, (const T *)a.k,
+                                  (const T *)a.v, a.igate, w.A, w.G, w.MC, a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS,
+                                  a.C_final, a.n_final, a.m_final, a.C0, a.n0);
     if (e != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;   // the chunk scan is fused into the carry walk
     if ((e = mark(3)) != cudaSuccess) return e;
@@ -265,10 +268,9 @@ static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, co
     const size_t sm2 = sizeof(float) * ((size_t)L * (L + 1) + 2 * (size_t)L * 33 + 32 * 33 + 5 * (size_t)L);
     if (sm2 > 48 * 1024 && (e = ensure_dynamic_smem((const void *)output_simt_kernel<T>, (int)sm2)) != cudaSuccess)
         return e;
-    output_simt_kernel<T><<<g2, 256, sm2, a.stream>>>((const T *)a.q, (const T *)a.k, (const T *)a.v, a.igate,
-                                                      (const T *)a.ogate, w.A, w.M, w.MC, w.CS, w.NS, a.S, L,
-                                                      w.NC, a.DHQK, a.DHV, (T *)a.h);
-    return cudaGetLastError();
+    return launch_kernel(output_simt_kernel<T>, g2, dim3(256), sm2, a.stream, 1, (const T *)a.q, (const T *)a.k,
+                         (const T *)a.v, a.igate, (const T *)a.ogate, w.A, w.M, w.MC, w.CS, w.NS, a.S, L, w.NC,
+                         a.DHQK, a.DHV, (T *)a.h);
 }
 
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark)

@@ -144,6 +144,8 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_wait();                  // the preceding kernel's outputs are visible from here on
+    griddep_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {   // TMA producer
@@ -307,6 +309,8 @@ __global__ void __launch_bounds__(256)
 seg_scan_kernel(Params p, float *C_final, float *n_final, float *__restrict__ m_final, const float *C0,
                 const float *n0)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     __shared__ float gam[SCAN_MAX_SEG], bet[SCAN_MAX_SEG];
     const int bh = blockIdx.y;
     const int nquad = p.DK * p.DV / 4;
@@ -472,6 +476,8 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_wait();                  // the preceding kernel's outputs are visible from here on
+    griddep_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {   // TMA producer: Q, K (all DK) and the V tile of every chunk
@@ -1204,24 +1210,26 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     const bool two = ntile % 2 == 0 && 1.4 * ((ctas1 / 2 + 147) / 148) < (double)((ctas1 + 147) / 148);
     if (two) {
         if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK, 2>, SegSmem<DK, 2>::TOTAL)) != cudaSuccess) return e;
-        segsum_kernel<DK, 2><<<dim3(ntile / 2, w.NSEG, a.BH), SS_THREADS, SegSmem<DK, 2>::TOTAL, a.stream>>>(mk64, mv64, p);
+        e = launch_kernel(segsum_kernel<DK, 2>, dim3(ntile / 2, w.NSEG, a.BH), dim3(SS_THREADS), SegSmem<DK, 2>::TOTAL,
+                          a.stream, 1, mk64, mv64, p);
     } else {
         if ((e = ensure_dynamic_smem((const void *)segsum_kernel<DK, 1>, SegSmem<DK, 1>::TOTAL)) != cudaSuccess) return e;
-        segsum_kernel<DK, 1><<<dim3(ntile, w.NSEG, a.BH), SS_THREADS, SegSmem<DK, 1>::TOTAL, a.stream>>>(mk64, mv64, p);
+        e = launch_kernel(segsum_kernel<DK, 1>, dim3(ntile, w.NSEG, a.BH), dim3(SS_THREADS), SegSmem<DK, 1>::TOTAL,
+                          a.stream, 1, mk64, mv64, p);
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;
 
     const int nquad = DK * a.DHV / 4;
-    seg_scan_kernel<<<dim3((nquad + 255) / 256, a.BH), 256, 0, a.stream>>>(p, a.C_final, a.n_final, a.m_final,
-                                                                         a.C0, a.n0);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_kernel(seg_scan_kernel, dim3((nquad + 255) / 256, a.BH), dim3(256), 0, a.stream, 1, p, a.C_final,
+                      a.n_final, a.m_final, a.C0, a.n0);
+    if (e != cudaSuccess) return e;
     if ((e = mark(3)) != cudaSuccess) return e;
 
     using WS = WalkSmem<DK, L>;
     if ((e = ensure_dynamic_smem((const void *)walk_kernel<DK, L>, WS::TOTAL)) != cudaSuccess) return e;
-    walk_kernel<DK, L><<<dim3(ntile, w.NSEG, a.BH), WALK_THREADS, WS::TOTAL, a.stream>>>(mq, mk, mv, p);
-    return cudaGetLastError();
+    return launch_kernel(walk_kernel<DK, L>, dim3(ntile, w.NSEG, a.BH), dim3(WALK_THREADS), WS::TOTAL, a.stream, 1,
+                         mq, mk, mv, p);
 }
 
 }  // namespace tcfwd

@@ -73,8 +73,12 @@ __device__ __forceinline__ void local_chunk(const float *__restrict__ igate, con
 
 __global__ void __launch_bounds__(GL_WARPS * 32)
 gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fgate, int S, int L, int NC,
-                  float *__restrict__ A, float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc)
+                  float *__restrict__ A, float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc,
+                  uint32_t *__restrict__ status)
 {
+    griddep_wait();
+    griddep_launch_dependents();
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0u;   // this call's status word
     const int c = blockIdx.x * GL_WARPS + (threadIdx.x >> 5);
     if (c < NC) local_chunk(igate, fgate, S, L, NC, blockIdx.y, c, threadIdx.x & 31, A, P, G, Bc);
 }
@@ -190,6 +194,8 @@ __global__ void __launch_bounds__(GS_THREADS)
 gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ Bc, float *__restrict__ MC,
                  int R, int NSEG, float *__restrict__ GP, float *__restrict__ SGb, const float *__restrict__ m0)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     scan_head(NC, G, Bc, MC, R, NSEG, GP, SGb, m0, blockIdx.x);
 }
 
@@ -199,9 +205,12 @@ __global__ void __launch_bounds__(GS_THREADS)
 gate_fused_kernel(const float *__restrict__ igate, const float *__restrict__ fgate, int S, int L, int NC,
                   float *__restrict__ A, float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc,
                   float *__restrict__ MC, int R, int NSEG, float *__restrict__ GP, float *__restrict__ SGb,
-                  const float *__restrict__ m0)
+                  const float *__restrict__ m0, uint32_t *__restrict__ status)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     const int bh = blockIdx.x;
+    if (bh == 0 && threadIdx.x == 0) *status = 0u;   // this call's status word
     for (int c = threadIdx.x >> 5; c < NC; c += GS_THREADS / 32)
         local_chunk(igate, fgate, S, L, NC, bh, c, threadIdx.x & 31, A, P, G, Bc);
     __syncthreads();   // G and Bc of this head are written (global memory, visible within the CTA)
@@ -217,17 +226,16 @@ cudaError_t launch_gate_prep(const GatePrepArgs &a)
 {
     if (a.NC == 0) return cudaSuccess;
     if (a.S <= FUSED_MAX_S) {
-        gate_fused_kernel<<<a.BH, GS_THREADS, 0, a.stream>>>(a.igate, a.fgate, a.S, a.L, a.NC, a.A, a.M, a.G, a.Bc,
-                                                             a.MC, a.R, a.NSEG, a.GP, a.SGb, a.m0);
-        return cudaGetLastError();
+        return launch_kernel(gate_fused_kernel, dim3(a.BH), dim3(GS_THREADS), 0, a.stream, 1, a.igate, a.fgate, a.S,
+                             a.L, a.NC, a.A, a.M, a.G, a.Bc, a.MC, a.R, a.NSEG, a.GP, a.SGb, a.m0, a.status);
     }
     dim3 g1((a.NC + GL_WARPS - 1) / GL_WARPS, a.BH);
-    gate_local_kernel<<<g1, GL_WARPS * 32, 0, a.stream>>>(a.igate, a.fgate, a.S, a.L, a.NC, a.A, a.M, a.G, a.Bc);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(gate_local_kernel, g1, dim3(GL_WARPS * 32), 0, a.stream, 1, a.igate, a.fgate, a.S,
+                                  a.L, a.NC, a.A, a.M, a.G, a.Bc, a.status);
     if (e != cudaSuccess) return e;
     const int scan_threads = a.NC >= GS_THREADS ? GS_THREADS : (a.NC + 31) / 32 * 32;
-    gate_scan_kernel<<<a.BH, scan_threads, 0, a.stream>>>(a.NC, a.G, a.Bc, a.MC, a.R, a.NSEG, a.GP, a.SGb, a.m0);
-    return cudaGetLastError();
+    return launch_kernel(gate_scan_kernel, dim3(a.BH), dim3(scan_threads), 0, a.stream, 1, a.NC, a.G, a.Bc, a.MC,
+                         a.R, a.NSEG, a.GP, a.SGb, a.m0);
 }
 
 }  // namespace mlstm

@@ -137,8 +137,11 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     FwdWorkspace w;
     plan_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, bf16, &w);
-    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
-    if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+    cudaError_t e = cudaSuccess;
+    if (BH == 0 || S == 0) {   // no kernel runs: reset the status word here (else the first gate kernel does)
+        e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+        if (e != cudaSuccess) return MLSTM_ERR_CUDA;
+    }
     if (BH == 0) return MLSTM_OK;
     if (S == 0) {   // no tokens: the final state is the initial one (zero state by default)
         const size_t bC = sizeof(float) * (size_t)BH * DHQK * DHV, bn = sizeof(float) * (size_t)BH * DHQK,
@@ -161,7 +164,8 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     mark.events = events;
     mark.stream = st;
     if (mark(0) != cudaSuccess) return MLSTM_ERR_CUDA;
-    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, w.R, w.NSEG, w.GP, w.SGb, m0, st};
+    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, w.R, w.NSEG, w.GP, w.SGb, m0, w.status,
+                    st};
     e = launch_gate_prep(gp);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     if (mark(1) != cudaSuccess) return MLSTM_ERR_CUDA;

@@ -24,6 +24,7 @@ struct GatePrepArgs {
     int R, NSEG;             // segments of R chunks (tensor-core path; NSEG = 0 otherwise)
     float *GP, *SGb;         // [BH][NC] in-segment prefix of chunk decays, [BH][NSEG][2] segment maps
     const float *m0;         // [BH] initial stabilizer, NULL = 0
+    uint32_t *status;        // bounded-wait status word, reset to 0 by the first gate kernel
     cudaStream_t stream;
 };
 

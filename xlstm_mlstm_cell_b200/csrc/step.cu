@@ -47,6 +47,8 @@ step_kernel(float *__restrict__ C, float *__restrict__ n, float *__restrict__ m,
     const int g = tid / (CW / 4);     // row group
     const int jl = tx * 4;            // first column of the thread in the CTA's slice
     const int j = rank * CW + jl;     // ... and in the head
+    griddep_wait();
+    griddep_launch_dependents();
 
     // the thread's first UNROLL rows of C and the small per-head inputs are requested together,
     // so that their latencies overlap (the remaining rows follow UNROLL at a time)
@@ -150,26 +152,9 @@ step_kernel(float *__restrict__ C, float *__restrict__ n, float *__restrict__ m,
 template <typename T, int G>
 static cudaError_t launch_step_g(const StepArgs &a, int RG, int threads, size_t smem)
 {
-    auto kern = step_kernel<T, 8, G>;
-    if (G == 1) {
-        kern<<<a.BH, threads, smem, a.stream>>>(a.C, a.n, a.m, (const T *)a.q, (const T *)a.k, (const T *)a.v,
-                                                a.igate, a.fgate, (const T *)a.ogate, a.DHQK, a.DHV, RG, (T *)a.h);
-        return cudaGetLastError();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.BH * G);
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = a.stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a.C, a.n, a.m, (const T *)a.q, (const T *)a.k, (const T *)a.v, a.igate,
-                              a.fgate, (const T *)a.ogate, a.DHQK, a.DHV, RG, (T *)a.h);
+    return launch_kernel(step_kernel<T, 8, G>, dim3(a.BH * G), dim3(threads), smem, a.stream, G, a.C, a.n, a.m,
+                         (const T *)a.q, (const T *)a.k, (const T *)a.v, a.igate, a.fgate, (const T *)a.ogate, a.DHQK,
+                         a.DHV, RG, (T *)a.h);
 }
 
 // Value columns of one head are split over G CTAs when there are too few heads for two waves of CTAs
