@@ -716,7 +716,10 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                                                         q * 32 + (lane & 1) * 16));
                 }
             }
-            named_sync(1, 512);   // previous chunk's readers of the per-row arrays are done
+            // No barrier here: the previous chunk's last reads of the per-row arrays written below (in
+            // (c), (d), the K pass and the denominators) all precede the barrier before its output
+            // epilogue, which reads only inv[] and the staging tile; inv[] and the P tile (the staging
+            // tile at chunk 128) are next written after the barrier of (b).
             if (ct == 0) WALK_TRACE(10);
             if (ct < L) {
                 if (ct < len) {
