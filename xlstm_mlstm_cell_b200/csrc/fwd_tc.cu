@@ -68,8 +68,16 @@ __device__ long long g_walk_trace[TR_SEGS * TR_CHUNKS * TR_SLOTS];
         if (tile == 0 && bh == 0 && seg < TR_SEGS && (ci) < TR_CHUNKS)                                     \
             g_walk_trace[((size_t)seg * TR_CHUNKS + (ci)) * TR_SLOTS + (slot)] = clock64();                \
     } while (0)
+// segment sums of CTA (0, 1, 0): clock64 per stage (rows 0..63) and per kernel phase (row 64)
+__device__ long long g_seg_trace[65 * 8];
+#define SEG_TRACE(row, slot)                                                                               \
+    do {                                                                                                   \
+        if (blockIdx.x == 0 && blockIdx.y == 1 && blockIdx.z == 0 && (row) < 65)                           \
+            g_seg_trace[(row) * 8 + (slot)] = clock64();                                                   \
+    } while (0)
 #else
 #define WALK_TRACE_AT(slot, ci) do { } while (0)
+#define SEG_TRACE(row, slot) do { } while (0)
 #endif
 #define WALK_TRACE(slot) WALK_TRACE_AT(slot, i)
 
@@ -146,6 +154,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
     griddep_wait();                  // the preceding kernel's outputs are visible from here on
     griddep_launch_dependents();
+    if (threadIdx.x == 0) SEG_TRACE(64, 0);
 
     if (warp == 0) {
         if (lane == 0) {   // TMA producer
@@ -154,6 +163,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const int st = it % SS_STAGES;
                 const uint32_t ph = (uint32_t)(it / SS_STAGES) & 1u;
                 if (it >= SS_STAGES && !mbar_wait(&empty[st], ph ^ 1u, wc)) break;
+                SEG_TRACE(it, 0);
                 ++issued;
                 uint8_t *kb = smem + st * SM::STAGE;
                 uint8_t *vb = kb + SM::K_BYTES;
@@ -174,6 +184,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 const int st = it % SS_STAGES;
                 const uint32_t ph = (uint32_t)(it / SS_STAGES) & 1u;
                 if (!mbar_wait(&scaled[st], ph, wc)) break;
+                SEG_TRACE(it, 3);
                 tc_fence_after();
                 const uint32_t kb = smem_u32(smem + st * SM::STAGE);
                 const uint32_t vb = kb + SM::K_BYTES;
@@ -186,6 +197,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                         mma_ss(tmem + t * DK, a, b, IDESC, (it > 0 || k > 0) ? 1u : 0u);
                     }
                 mma_commit(&empty[st]);
+                SEG_TRACE(it, 4);
             }
             mma_commit(acc_full);
             mbar_wait_drain(acc_full, 0);
@@ -232,6 +244,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (ct < TB) wst[ct] = (t < t_end) ? expf(Gs - cgp - ca + ci - bs) : 0.f;
             named_sync(1, NST);
             if (!mbar_wait(&full[st], ph, wc)) { ok = false; break; }
+            if (ct == 0) SEG_TRACE(it, 1);
             uint8_t *kb = smem + st * SM::STAGE;
             for (int row0 = sw * RPW + rsub; row0 < TB; row0 += RSTEP * NB) {
                 uint4 uk[NB];
@@ -256,6 +269,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&scaled[st]);
+            if (ct == 0) SEG_TRACE(it, 2);
         }
         if (tile == 0) {    // reduce the n partial sums of the scaler warps (and lanes sharing a chunk)
             float *npart = reinterpret_cast<float *>(smem);      // stage buffers are idle once acc_full fires
@@ -274,6 +288,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
         // epilogue: TMEM (lane = value column, columns = DK) -> workspace, quad layout [DK/4][DV][4]
         if (ok && mbar_wait(acc_full, 0, wc)) {
+            if (ct == 0) SEG_TRACE(64, 1);
             tc_fence_after();
             const int q = warp & 3;                      // TMEM lane quadrant of the warp
             const int half = (warp - 2) >> 2;            // two scaler warps per quadrant share its columns
@@ -293,6 +308,7 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             }
         }
     }
+    if (threadIdx.x == 64) SEG_TRACE(64, 2);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -1241,6 +1257,10 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
 extern "C" int mlstm_walk_trace_copy(void *dst, size_t bytes)
 {
     return (int)cudaMemcpyFromSymbol(dst, tcfwd::g_walk_trace, bytes);
+}
+extern "C" int mlstm_seg_trace_copy(void *dst, size_t bytes)
+{
+    return (int)cudaMemcpyFromSymbol(dst, tcfwd::g_seg_trace, bytes);
 }
 #endif
 
