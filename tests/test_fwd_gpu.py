@@ -57,6 +57,10 @@ SMALL = [
     (1, 2, 384, 256, 512, 128, "bf16"),
     (1, 2, 200, 64, 128, 32, "bf16"),
     (1, 1, 130, 256, 512, 64, "bf16"),
+    # the tensor-core walk at DK 64 and 128 with both chunk sizes
+    (1, 2, 333, 64, 128, 64, "bf16"),
+    (1, 2, 333, 64, 128, 128, "bf16"),
+    (2, 1, 400, 128, 256, 128, "bf16"),
 ]
 
 

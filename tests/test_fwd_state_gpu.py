@@ -26,7 +26,8 @@ def oracle_state(B, NH, DK, DV, dt, seed):
 
 @pytest.mark.parametrize("B,NH,S,DK,DV,chunk,dt", [
     (1, 2, 100, 16, 16, 16, "f32"), (2, 2, 333, 64, 48, 32, "f32"),
-    (1, 2, 512, 256, 256, 64, "bf16"), (1, 2, 700, 256, 512, 128, "bf16"), (2, 1, 260, 128, 128, 64, "bf16")])
+    (1, 2, 512, 256, 256, 64, "bf16"), (1, 2, 700, 256, 512, 128, "bf16"), (2, 1, 260, 128, 128, 64, "bf16"),
+    (1, 2, 300, 64, 128, 64, "bf16")])
 def test_fwd_from_state_matches_oracle(cuda_lib, B, NH, S, DK, DV, chunk, dt):
     C0, n0, m0 = oracle_state(B, NH, DK, DV, dt, seed=DK + S)
     inp = make_custom(B, NH, S, DK, DV, dt, seed=S + 5, ig=(-1.0, 2.0), fg=(4.0, 1.0))
