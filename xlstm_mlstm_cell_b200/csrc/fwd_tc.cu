@@ -333,6 +333,15 @@ seg_scan_kernel(Params p, float *C_final, float *n_final, float *__restrict__ m_
     const int e = blockIdx.x * blockDim.x + threadIdx.x;    // quad index: (i4, j) = (e / DV, e % DV)
     const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
     const float *SG = p.SGb + (size_t)bh * p.NSEG * 2;
+    constexpr int BATCH = 8;                           // contributions loaded ahead of the stores
+    float4 *__restrict__ slot0 = reinterpret_cast<float4 *>(p.DC + (size_t)bh * p.NSEG * p.DK * p.DV) + e;
+    const size_t stride = (size_t)p.DK * p.DV / 4;
+    // the first batch of contributions is requested before the per-segment factors are formed,
+    // so that the two memory latencies overlap
+    float4 d[BATCH];
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u)
+        if (e < nquad && u < p.NSEG) d[u] = __ldcs(slot0 + u * stride);
     // decay of the running state and weight of the segment's contribution, per segment
     for (int s = threadIdx.x; s < p.NSEG; s += blockDim.x) {
         const float Ms = MCb[s * p.R], Mn = MCb[min((s + 1) * p.R, p.NC)];
@@ -341,8 +350,6 @@ seg_scan_kernel(Params p, float *C_final, float *n_final, float *__restrict__ m_
     }
     __syncthreads();
     if (e < nquad) {
-        float4 *__restrict__ slot0 = reinterpret_cast<float4 *>(p.DC + (size_t)bh * p.NSEG * p.DK * p.DV) + e;
-        const size_t stride = (size_t)p.DK * p.DV / 4;
         float4 C = make_float4(0.f, 0.f, 0.f, 0.f);
         if (C0) {   // initial state (user layout); C_final may alias C0: each element is read before written
             const int i4 = e / p.DV, j = e % p.DV;
@@ -350,12 +357,12 @@ seg_scan_kernel(Params p, float *C_final, float *n_final, float *__restrict__ m_
             C = make_float4(c0[(size_t)(4 * i4 + 0) * p.DV + j], c0[(size_t)(4 * i4 + 1) * p.DV + j],
                             c0[(size_t)(4 * i4 + 2) * p.DV + j], c0[(size_t)(4 * i4 + 3) * p.DV + j]);
         }
-        constexpr int BATCH = 8;                       // contributions loaded ahead of the stores
         for (int s0 = 0; s0 < p.NSEG; s0 += BATCH) {
-            float4 d[BATCH];
+            if (s0 > 0) {
 #pragma unroll
-            for (int u = 0; u < BATCH; ++u)
-                if (s0 + u < p.NSEG) d[u] = __ldcs(slot0 + (s0 + u) * stride);
+                for (int u = 0; u < BATCH; ++u)
+                    if (s0 + u < p.NSEG) d[u] = __ldcs(slot0 + (s0 + u) * stride);
+            }
 #pragma unroll
             for (int u = 0; u < BATCH; ++u) {
                 const int s = s0 + u;

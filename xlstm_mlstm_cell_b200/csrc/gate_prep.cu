@@ -31,7 +31,8 @@ constexpr int GL_WARPS = 8;   // chunks per CTA of gate_local_kernel
 // One warp: chunk c of head bh.
 __device__ __forceinline__ void local_chunk(const float *__restrict__ igate, const float *__restrict__ fgate, int S,
                                             int L, int NC, int bh, int c, int lane, float *__restrict__ A,
-                                            float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc)
+                                            float *__restrict__ P, float *__restrict__ G, float *__restrict__ Bc,
+                                            float *g_sm = nullptr, float *b_sm = nullptr)
 {
     const float *ig = igate + (size_t)bh * S;
     const float *fg = fgate + (size_t)bh * S;
@@ -39,18 +40,30 @@ __device__ __forceinline__ void local_chunk(const float *__restrict__ igate, con
     float *p_out = P + (size_t)bh * S;
     const int t0 = c * L;
     const int t1 = min(t0 + L, S);
+    // the chunk's gate values (at most four passes of 32 tokens: L <= 128) are requested before
+    // the serial passes, so that one memory latency covers them all
+    float fv[4], iv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * 32 + lane;
+        fv[u] = t < t1 ? fg[t] : 0.f;
+        iv[u] = t < t1 ? ig[t] : 0.f;
+    }
     float carry_a = 0.f, carry_p = -INFINITY;
-    for (int base = t0; base < t1; base += 32) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int base = t0 + u * 32;
+        if (base >= t1) break;
         const int t = base + lane;
         const bool ok = t < t1;
-        float x = ok ? log_sigmoid(fg[t]) : 0.f;
+        float x = ok ? log_sigmoid(fv[u]) : 0.f;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
         const float a = carry_a + x;
-        float p = ok ? ig[t] - a : -INFINITY;
+        float p = ok ? iv[u] - a : -INFINITY;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, p, o);
@@ -68,6 +81,10 @@ __device__ __forceinline__ void local_chunk(const float *__restrict__ igate, con
     if (lane == 0) {
         G[(size_t)bh * NC + c] = carry_a;
         Bc[(size_t)bh * NC + c] = carry_a + carry_p;
+        if (g_sm) {              // the fused kernel's scan reads them from shared memory
+            g_sm[c] = carry_a;
+            b_sm[c] = carry_a + carry_p;
+        }
     }
 }
 
@@ -90,28 +107,16 @@ constexpr int GS_STAGE = 4096;     // chunk maps per head staged in shared memor
 constexpr int FUSED_MAX_S = 4096;
 
 // One CTA: the chunk maps of head bh (G, Bc written before by this CTA or an earlier kernel).
-__device__ __forceinline__ void scan_head(int NC, const float *__restrict__ G, const float *__restrict__ Bc,
-                                          float *__restrict__ MC, int R, int NSEG, float *__restrict__ GP,
-                                          float *__restrict__ SGb, const float *__restrict__ m0, int bh)
+// g_in, b_in: the head's chunk maps, in shared memory when they fit (the serial loops below then
+// read shared memory instead of waiting on one global load after another), else in global memory.
+__device__ __forceinline__ void scan_head(int NC, const float *g_in, const float *b_in, float *__restrict__ MC,
+                                          int R, int NSEG, float *__restrict__ GP, float *__restrict__ SGb,
+                                          const float *__restrict__ m0, int bh)
 {
     __shared__ float wa[32], wb[32];                 // per-warp totals, then their exclusive prefixes
-    __shared__ float g_st[GS_STAGE], b_st[GS_STAGE];
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
-    const float *g_in = G + (size_t)bh * NC;
-    const float *b_in = Bc + (size_t)bh * NC;
     float *mc_out = MC + (size_t)bh * (NC + 1);
-    // the chunk maps go to shared memory first (parallel, coalesced loads) when they fit, so that
-    // the serial loops below read shared memory instead of waiting on one global load after another
-    if (NC <= GS_STAGE) {
-        for (int c = tid; c < NC; c += nthr) {
-            g_st[c] = g_in[c];
-            b_st[c] = b_in[c];
-        }
-        __syncthreads();
-        g_in = g_st;
-        b_in = b_st;
-    }
 
     // each thread composes the maps of a contiguous range of chunks
     const int per = (NC + nthr - 1) / nthr;
@@ -196,7 +201,19 @@ gate_scan_kernel(int NC, const float *__restrict__ G, const float *__restrict__ 
 {
     griddep_wait();
     griddep_launch_dependents();
-    scan_head(NC, G, Bc, MC, R, NSEG, GP, SGb, m0, blockIdx.x);
+    __shared__ float g_st[GS_STAGE], b_st[GS_STAGE];
+    const int bh = blockIdx.x;
+    const float *g_in = G + (size_t)bh * NC, *b_in = Bc + (size_t)bh * NC;
+    if (NC <= GS_STAGE) {   // parallel, coalesced loads into shared memory
+        for (int c = threadIdx.x; c < NC; c += blockDim.x) {
+            g_st[c] = g_in[c];
+            b_st[c] = b_in[c];
+        }
+        __syncthreads();
+        g_in = g_st;
+        b_in = b_st;
+    }
+    scan_head(NC, g_in, b_in, MC, R, NSEG, GP, SGb, m0, bh);
 }
 
 // Both steps in one CTA per head for short sequences (at most FUSED_MAX_S tokens): the CTA's
@@ -211,10 +228,11 @@ gate_fused_kernel(const float *__restrict__ igate, const float *__restrict__ fga
     griddep_launch_dependents();
     const int bh = blockIdx.x;
     if (bh == 0 && threadIdx.x == 0) *status = 0u;   // this call's status word
+    __shared__ float g_st[FUSED_MAX_S / 16], b_st[FUSED_MAX_S / 16];   // chunk 16 at most 256 chunks
     for (int c = threadIdx.x >> 5; c < NC; c += GS_THREADS / 32)
-        local_chunk(igate, fgate, S, L, NC, bh, c, threadIdx.x & 31, A, P, G, Bc);
-    __syncthreads();   // G and Bc of this head are written (global memory, visible within the CTA)
-    scan_head(NC, G, Bc, MC, R, NSEG, GP, SGb, m0, bh);
+        local_chunk(igate, fgate, S, L, NC, bh, c, threadIdx.x & 31, A, P, G, Bc, g_st, b_st);
+    __syncthreads();   // the head's chunk maps are in shared memory
+    scan_head(NC, g_st, b_st, MC, R, NSEG, GP, SGb, m0, bh);
 }
 
 int gate_prep_launches(int S, int NC)
