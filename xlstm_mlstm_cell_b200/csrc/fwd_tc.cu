@@ -152,7 +152,12 @@ segsum_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    griddep_wait();                  // the preceding kernel's outputs are visible from here on
+    // The TMA producer (warp 0) loads only the inputs q, k, v, which no kernel of this call writes
+    // (this kernel launches only once every earlier grid of the stream has passed its own
+    // griddepcontrol.wait, so their producers have finished), and the MMA warp (warp 1) reads
+    // shared memory and TMEM only: their first loads and MMAs go out while the preceding kernel
+    // is still running.  The warps that read its outputs wait for them.
+    if (warp >= 2) griddep_wait();
     griddep_launch_dependents();
     if (threadIdx.x == 0) SEG_TRACE(64, 0);
 
@@ -499,7 +504,12 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    griddep_wait();                  // the preceding kernel's outputs are visible from here on
+    // The TMA producer (warp 0) loads only the inputs q, k, v, which no kernel of this call writes
+    // (this kernel launches only once every earlier grid of the stream has passed its own
+    // griddepcontrol.wait, so their producers have finished), and the MMA warp (warp 1) reads
+    // shared memory and TMEM only: their first loads and MMAs go out while the preceding kernel
+    // is still running.  The warps that read its outputs wait for them.
+    if (warp >= 2) griddep_wait();
     griddep_launch_dependents();
 
     if (warp == 0) {
