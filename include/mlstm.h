@@ -111,6 +111,61 @@ mlstm_status mlstm_fwd_state(const void *q, const void *k, const void *v,
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Sequence-parallel forward pass, the pieces.  A sequence split into R
+ * consecutive slices (rank r holds slice r) is run in three steps:
+ *   1. every rank: the final state of its slice from the zero state
+ *      (mlstm_fwd_final_state) and the slice's total log forget decay
+ *      (mlstm_log_decay_sum);
+ *   2. the caller all-gathers these summaries over the ranks (NCCL);
+ *   3. every rank: its start state from the summaries of the slices before it
+ *      (mlstm_state_prefix), then mlstm_fwd_state over its slice from it.
+ * The state after a slice is the state before it decayed by the product of the
+ * slice's forget gates plus the slice's own contribution, the recurrence of
+ * "Recurrent Formulation (Inference Mode)" (xLSTM guide) over the slice; this
+ * is the exchange of chunk summaries the guide's "Exploit Chunkwise Hardware
+ * Kernels" scan across chunks implies at the granularity of a GPU.  The
+ * composed state's stabilizer m can be above the one of a single pass (the
+ * slices start from m_0 = 0); C and n are scaled to match, so h and the
+ * unstabilized state exp(m) C, exp(m) n are the same.
+ */
+
+/*
+ * mlstm_fwd without the output stage: the final state (C, n, m) of the slice
+ * from the zero state, for step 1.  Same arguments and workspace as mlstm_fwd
+ * without q, ogate and h (k, v, igate, fgate as there; the final-state
+ * pointers as there, each may be NULL).  No extra entry point in the pages:
+ * it is mlstm_fwd with its last phase left out.
+ */
+mlstm_status mlstm_fwd_final_state(const void *k, const void *v,
+                                   const float *igate, const float *fgate,
+                                   mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                                   float *C_final, float *n_final, float *m_final,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * g_out[b][h] = sum over the S tokens of logsigmoid(fgate[b][h][t]) (float32,
+ * device; fgate [B][NH][S]).  0 for S == 0.  Errors: MLSTM_ERR_INVALID_ARG for
+ * negative sizes or NULL pointers, MLSTM_ERR_CUDA for a launch failure.
+ */
+mlstm_status mlstm_log_decay_sum(const float *fgate, int B, int NH, int S, float *g_out, void *stream);
+
+/*
+ * Start state of slice `rank` (0 <= rank < R) from the gathered summaries of
+ * the R slices: C_parts [R][B][NH][DHQK][DHV], n_parts [R][B][NH][DHQK],
+ * m_parts [R][B][NH] (the zero-start final states of step 1) and g_parts
+ * [R][B][NH] (the log decay sums), float32 device arrays, C_parts and C0
+ * 16-byte aligned.  Only slices 0 .. rank-1 are read.  Writes C0, n0, m0 in
+ * the layouts of mlstm_fwd_state's initial state (rank 0 gets the zero state,
+ * m = 0).  DHQK, DHV as for mlstm_fwd.  Errors: MLSTM_ERR_INVALID_ARG for a
+ * bad rank, NULL or misaligned pointers; MLSTM_ERR_UNSUPPORTED for head sizes
+ * mlstm_fwd rejects or more than 65535 heads; MLSTM_ERR_CUDA for a launch
+ * failure.
+ */
+mlstm_status mlstm_state_prefix(const float *C_parts, const float *n_parts, const float *m_parts,
+                                const float *g_parts, int R, int rank, int B, int NH, int DHQK, int DHV,
+                                float *C0, float *n0, float *m0, void *stream);
+
+/*
  * mlstm_fwd with per-phase timing: identical work and results, and in addition
  * records CUDA events (cudaEvent_t passed as void*, created by the caller) on
  * `stream`: events[p] just before phase p and events[MLSTM_FWD_PHASES] after

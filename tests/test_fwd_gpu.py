@@ -155,3 +155,27 @@ def test_fwd_long_context_sampled(cuda_lib):
         assert_close("m[head %d]" % hd, m[:, hd:hd + 1], mr, tol)
         pos = np.sort(rng.choice(w.S, size=1024 // len(heads), replace=False))
         assert_close("h[head %d, 512 positions]" % hd, h[0, hd][pos][:, cols], hr[0, 0][pos], tol)
+
+
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_chained_calls_read_previous_outputs(cuda_lib, chunk):
+    """Calls issued back to back on one stream, each reading the previous call's output h as its q,
+    k and v (no synchronization in between): every call sees its inputs complete, as with plain
+    stream order, although the library's kernels start before their predecessors finish."""
+    B, NH, S, D = 1, 2, 5 * chunk + 9, 256
+    q, k, v, i, f, o = make_custom(B, NH, S, D, D, "bf16", seed=chunk, ig=(-1.0, 2.0), fg=(4.0, 1.0))
+    gen = torch.Generator().manual_seed(chunk + 1)
+    gates = [(torch.randn(B, NH, S, generator=gen) * 2 - 1, torch.randn(B, NH, S, generator=gen) + 4)
+             for _ in range(2)]
+    h1, _, _, _ = binding.fwd(q.cuda(), k.cuda(), v.cuda(), i.cuda(), f.cuda(), o.cuda(), chunk=chunk)
+    (i2, f2), (i3, f3) = gates
+    h2, _, _, _ = binding.fwd(h1, h1, h1, i2.cuda(), f2.cuda(), None, chunk=chunk)
+    h3, C3, n3, m3 = binding.fwd(h2, h1, h2, i3.cuda(), f3.cuda(), None, chunk=chunk)
+    torch.cuda.synchronize()
+    h1c, h2c = h1.cpu(), h2.cpu()
+    hr2, _, _, _ = oracle.mlstm_fwd(h1c, h1c, h1c, i2, f2, None)
+    assert_close("h of the second call", h2.cpu(), hr2, TOL["bf16"])
+    hr3, Cr3, nr3, mr3 = oracle.mlstm_fwd(h2c, h1c, h2c, i3, f3, None)
+    assert_close("h of the third call", h3.cpu(), hr3, TOL["bf16"])
+    assert_close("C of the third call", C3.cpu(), Cr3, TOL["bf16"])
+    assert_close("n of the third call", n3.cpu(), nr3, TOL["bf16"])

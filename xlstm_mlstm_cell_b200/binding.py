@@ -38,6 +38,9 @@ SIGNATURES = {
     "mlstm_fwd_tensor_path": (_i, [_i, _i, _i, _i]),
     "mlstm_step": (_i, [_fp, _fp, _fp, _vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "mlstm_status_string": (ctypes.c_char_p, [_i]),
+    "mlstm_fwd_final_state": (_i, [_vp, _vp, _fp, _fp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _sz, _vp]),
+    "mlstm_log_decay_sum": (_i, [_fp, _i, _i, _i, _fp, _vp]),
+    "mlstm_state_prefix": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp]),
 }
 
 _lib = None
@@ -158,6 +161,46 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
         arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[e.cuda_event for e in events])
         _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
     return h_out, C_final, n_final, m_final
+
+
+def fwd_final_state(k, v, igate, fgate, chunk: int = 64, workspace=None, stream=None):
+    """mlstm_fwd_final_state: ``(C, n, m)`` of the sequence from the zero state, no outputs."""
+    lib = load()
+    B, NH, S, DHQK = k.shape
+    DHV = v.shape[-1]
+    C = torch.empty((B, NH, DHQK, DHV), dtype=torch.float32, device=k.device)
+    n = torch.empty((B, NH, DHQK), dtype=torch.float32, device=k.device)
+    m = torch.empty((B, NH), dtype=torch.float32, device=k.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, NH, S, DHQK, DHV, chunk, k.dtype, k.device)
+    _check("mlstm_fwd_final_state",
+           lib.mlstm_fwd_final_state(_ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _dt(k), B, NH, S, DHQK, DHV, chunk,
+                                     _ptr(C), _ptr(n), _ptr(m), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return C, n, m
+
+
+def log_decay_sum(fgate, stream=None):
+    """mlstm_log_decay_sum: per (b, h) the sum over tokens of logsigmoid(f~), ``[B, NH]``."""
+    lib = load()
+    B, NH, S = fgate.shape
+    g = torch.empty((B, NH), dtype=torch.float32, device=fgate.device)
+    _check("mlstm_log_decay_sum", lib.mlstm_log_decay_sum(_ptr(fgate), B, NH, S, _ptr(g), _stream(stream)))
+    return g
+
+
+def state_prefix(C_parts, n_parts, m_parts, g_parts, rank: int, stream=None):
+    """mlstm_state_prefix: the start state ``(C0, n0, m0)`` of slice ``rank`` from the gathered
+    summaries ``C_parts [R, B, NH, DHQK, DHV]``, ``n_parts [R, B, NH, DHQK]``, ``m_parts`` and
+    ``g_parts [R, B, NH]``."""
+    lib = load()
+    R, B, NH, DHQK, DHV = C_parts.shape
+    C0 = torch.empty((B, NH, DHQK, DHV), dtype=torch.float32, device=C_parts.device)
+    n0 = torch.empty((B, NH, DHQK), dtype=torch.float32, device=C_parts.device)
+    m0 = torch.empty((B, NH), dtype=torch.float32, device=C_parts.device)
+    _check("mlstm_state_prefix",
+           lib.mlstm_state_prefix(_ptr(C_parts), _ptr(n_parts), _ptr(m_parts), _ptr(g_parts), R, rank, B, NH, DHQK,
+                                  DHV, _ptr(C0), _ptr(n0), _ptr(m0), _stream(stream)))
+    return C0, n0, m0
 
 
 NOALLOC_MAX_BYTES = 32 * 1024 * 1024

@@ -264,6 +264,7 @@ static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, co
     if (e != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;   // the chunk scan is fused into the carry walk
     if ((e = mark(3)) != cudaSuccess) return e;
+    if (!a.outputs) return cudaSuccess;   // the final state is complete after the carry walk
     dim3 g2(a.BH, w.NC, (a.DHV + ST - 1) / ST);
     const size_t sm2 = sizeof(float) * ((size_t)L * (L + 1) + 2 * (size_t)L * 33 + 32 * 33 + 5 * (size_t)L);
     if (sm2 > 48 * 1024 && (e = ensure_dynamic_smem((const void *)output_simt_kernel<T>, (int)sm2)) != cudaSuccess)

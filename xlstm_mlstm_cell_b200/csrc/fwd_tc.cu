@@ -791,7 +791,10 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             // (b) Cb = fp16(C_c 2^-kc) into TMEM, kc from max |C_c| over the tile; rescale the
             //     fp32 state when the frame moves
             if (ct == 0) WALK_TRACE(11);
-            if (i > 0 && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
+            // the previous chunk's state update must be complete before the state is read or
+            // rescaled here; at chunk 64 without a rescale nothing here touches it (the inter-chunk
+            // MMA is ordered after the update in the MMA pipe, and Q', P are free since h_full)
+            if (i > 0 && (!SM::TF || rescale) && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
             if (ct == 0) WALK_TRACE(12);
             tc_fence_after();
             int kc = 0;
@@ -1234,7 +1237,7 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     p.status = w.status;
 
     CUtensorMap mq, mk, mv, mk64, mv64;
-    if (!make_map(&mq, a.q, DK, a.S, a.BH, L) || !make_map(&mk, a.k, DK, a.S, a.BH, L) ||
+    if (!make_map(&mq, a.outputs ? a.q : a.k, DK, a.S, a.BH, L) || !make_map(&mk, a.k, DK, a.S, a.BH, L) ||
         !make_map(&mv, a.v, a.DHV, a.S, a.BH, L) || !make_map(&mk64, a.k, DK, a.S, a.BH, TB) ||
         !make_map(&mv64, a.v, a.DHV, a.S, a.BH, TB))
         return cudaErrorInvalidValue;
@@ -1262,6 +1265,7 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     if (e != cudaSuccess) return e;
     if ((e = mark(3)) != cudaSuccess) return e;
 
+    if (!a.outputs) return cudaSuccess;   // the final state is complete after the segment scan
     using WS = WalkSmem<DK, L>;
     if ((e = ensure_dynamic_smem((const void *)walk_kernel<DK, L>, WS::TOTAL)) != cudaSuccess) return e;
     return launch_kernel(walk_kernel<DK, L>, dim3(ntile, w.NSEG, a.BH), dim3(WALK_THREADS), WS::TOTAL, a.stream, 1,

@@ -107,7 +107,7 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
                       const void *ogate, mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
                       const float *C0, const float *n0, const float *m0,
                       void *h_out, float *C_final, float *n_final, float *m_final, void *workspace,
-                      size_t workspace_bytes, void *stream, void *const *events)
+                      size_t workspace_bytes, void *stream, void *const *events, bool outputs = true)
 {
     if (B < 0 || NH < 0 || S < 0) return MLSTM_ERR_INVALID_ARG;
     if (dt != MLSTM_F32 && dt != MLSTM_BF16) return MLSTM_ERR_UNSUPPORTED;
@@ -115,12 +115,18 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     if ((long long)B * NH > (1LL << 30) || (long long)S * DHV > (1LL << 40)) return MLSTM_ERR_UNSUPPORTED;
     const int BH = B * NH;
     const bool has_tokens = BH > 0 && S > 0;
-    if (has_tokens) {
+    if (has_tokens && outputs) {
         if (!q || !k || !v || !igate || !fgate || !h_out) return MLSTM_ERR_INVALID_ARG;
         const void *ptrs[] = {q, k, v, igate, fgate, h_out};
         for (const void *p : ptrs)
             if (!aligned16(p)) return MLSTM_ERR_INVALID_ARG;
         if (ogate && !aligned16(ogate)) return MLSTM_ERR_INVALID_ARG;
+    }
+    if (has_tokens && !outputs) {   // the final state only: q, ogate and h are not used
+        if (!k || !v || !igate || !fgate) return MLSTM_ERR_INVALID_ARG;
+        const void *ptrs[] = {k, v, igate, fgate};
+        for (const void *p : ptrs)
+            if (!aligned16(p)) return MLSTM_ERR_INVALID_ARG;
     }
     if ((C_final && !aligned16(C_final)) || (n_final && !aligned16(n_final)) || (m_final && !aligned16(m_final)))
         return MLSTM_ERR_INVALID_ARG;
@@ -170,7 +176,7 @@ mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     if (mark(1) != cudaSuccess) return MLSTM_ERR_CUDA;
     FwdArgs fa{q, k, v, ogate, igate, fgate, h_out, C_final, n_final, m_final, C0, n0, BH, S, DHQK, DHV, chunk,
-               dt == MLSTM_BF16, st};
+               dt == MLSTM_BF16, st, outputs};
     e = w.tc ? launch_fwd_tc(fa, w, mark) : launch_fwd_simt(fa, w, mark);
     if (e != cudaSuccess) return MLSTM_ERR_CUDA;
     return cuda_status(mark(MLSTM_FWD_PHASES));
@@ -187,6 +193,15 @@ mlstm_status mlstm_fwd(const void *q, const void *k, const void *v, const float 
 {
     return fwd_impl(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, nullptr, nullptr, nullptr, h_out,
                     C_final, n_final, m_final, workspace, workspace_bytes, stream, nullptr);
+}
+
+mlstm_status mlstm_fwd_final_state(const void *k, const void *v, const float *igate, const float *fgate,
+                                   mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                                   float *C_final, float *n_final, float *m_final, void *workspace,
+                                   size_t workspace_bytes, void *stream)
+{
+    return fwd_impl(nullptr, k, v, igate, fgate, nullptr, dt, B, NH, S, DHQK, DHV, chunk, nullptr, nullptr, nullptr,
+                    nullptr, C_final, n_final, m_final, workspace, workspace_bytes, stream, nullptr, false);
 }
 
 mlstm_status mlstm_fwd_state(const void *q, const void *k, const void *v, const float *igate, const float *fgate,

@@ -37,6 +37,7 @@ struct FwdArgs {
     int BH, S, DHQK, DHV, chunk;
     bool bf16;
     cudaStream_t stream;
+    bool outputs;            // false: the final state only (no output stage; q, ogate, h unused)
 };
 
 // Device workspace of one mlstm_fwd call, carved from the caller's buffer.
