@@ -205,6 +205,18 @@ int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt);
 mlstm_status mlstm_fwd_status(const void *workspace, void *stream);
 
 /*
+ * Self-test of the failure detection above (no counterpart in the pages): one
+ * CTA waits, through the kernels' own bounded wait, on a barrier that nothing
+ * completes; after the wait limit (2 s) it records a timeout in the status word
+ * of `workspace` (a workspace of mlstm_fwd, 256-byte aligned, device) and exits.
+ * A following mlstm_fwd_status on that workspace returns MLSTM_ERR_TIMEOUT, and
+ * the GPU context stays usable (the next mlstm_fwd with the workspace resets
+ * the word).  Asynchronous on `stream`.  Errors: MLSTM_ERR_INVALID_ARG for a
+ * NULL or misaligned workspace, MLSTM_ERR_CUDA for a launch failure.
+ */
+mlstm_status mlstm_selftest_wait_timeout(void *workspace, void *stream);
+
+/*
  * One recurrent decode step for every (b, h): reads the state (C, n, m),
  * applies one token and writes the new state back IN PLACE, plus h_out
  * [B][NH][DHV].  Token inputs: q, k [B][NH][DHQK] and v, ogate [B][NH][DHV]

@@ -41,6 +41,7 @@ SIGNATURES = {
     "mlstm_fwd_final_state": (_i, [_vp, _vp, _fp, _fp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _sz, _vp]),
     "mlstm_log_decay_sum": (_i, [_fp, _i, _i, _i, _fp, _vp]),
     "mlstm_state_prefix": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp]),
+    "mlstm_selftest_wait_timeout": (_i, [_vp, _vp]),
 }
 
 _lib = None
