@@ -94,8 +94,9 @@ gate_local_kernel(const float *__restrict__ igate, const float *__restrict__ fga
                   uint32_t *__restrict__ status)
 {
     griddep_wait();
+    // this call's status word, reset before any kernel that may report into it starts
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0u;
     griddep_launch_dependents();
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0u;   // this call's status word
     const int c = blockIdx.x * GL_WARPS + (threadIdx.x >> 5);
     if (c < NC) local_chunk(igate, fgate, S, L, NC, blockIdx.y, c, threadIdx.x & 31, A, P, G, Bc);
 }
@@ -225,9 +226,10 @@ gate_fused_kernel(const float *__restrict__ igate, const float *__restrict__ fga
                   const float *__restrict__ m0, uint32_t *__restrict__ status)
 {
     griddep_wait();
-    griddep_launch_dependents();
     const int bh = blockIdx.x;
-    if (bh == 0 && threadIdx.x == 0) *status = 0u;   // this call's status word
+    // this call's status word, reset before any kernel that may report into it starts
+    if (bh == 0 && threadIdx.x == 0) *status = 0u;
+    griddep_launch_dependents();
     __shared__ float g_st[FUSED_MAX_S / 16], b_st[FUSED_MAX_S / 16];   // chunk 16 at most 256 chunks
     for (int c = threadIdx.x >> 5; c < NC; c += GS_THREADS / 32)
         local_chunk(igate, fgate, S, L, NC, bh, c, threadIdx.x & 31, A, P, G, Bc, g_st, b_st);
