@@ -543,7 +543,44 @@ def extras(device, peaks):
     sw = step_work(w.B, w.NH, w.DHQK, w.DHV)
     res["step_bf16"] = {"us_per_step": ts * 1e6, "gbs": sw["bytes"] / ts / 1e9, "frac_hbm": sw["bytes"] / ts / 1e9 / bw,
                         "steps": nsteps}
+    res["slstm_f32"] = slstm_extra(device, peaks)
     return res
+
+
+def slstm_work(B, S, NH, DH, esize):
+    """Algorithmic work of one slstm_fwd call: the recurrent products (2 x 4 DH^2 flops per cell
+    group and step) and the bytes of wx read and h written once."""
+    return {"flops": 2.0 * 4 * DH * DH * NH * B * S, "bytes": (4 + 1) * NH * DH * B * S * esize}
+
+
+def slstm_extra(device, peaks):
+    """The sLSTM recurrence on its workload: one slstm_fwd call over the whole sequence."""
+    from xlstm_mlstm_cell_b200.workloads import SLSTM_WORKLOADS, make_slstm_inputs
+    w = SLSTM_WORKLOADS["slstm_f32"]
+    wx, R = make_slstm_inputs(w.B, w.S, w.NH, w.DH, w.dtype, w.seed, w.f_loc)
+    wx, R = wx.to(device), R.to(device)
+    h_out = torch.empty((w.B, w.S, w.NH, w.DH), dtype=wx.dtype, device=device)
+    state = tuple(torch.zeros((w.B, w.NH, w.DH), device=device) for _ in range(4))
+    for _ in range(2):
+        for x in state:
+            x.zero_()
+        binding.slstm_fwd(wx, R, forget=w.forget, state=state, h_out=h_out)
+    torch.cuda.synchronize()
+    reps = 5
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        binding.slstm_fwd(wx, R, forget=w.forget, state=state, h_out=h_out)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / reps / 1e3
+    sw = slstm_work(w.B, w.S, w.NH, w.DH, wx.element_size())
+    fp32_peak = N_SM * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    return {"workload": "B%d S%d NH%d DH%d %s, %s forget gate" % (w.B, w.S, w.NH, w.DH, w.dtype, w.forget),
+            "ms": t * 1e3, "tokens_per_s": w.B * w.S / t, "us_per_step": t / w.S * 1e6,
+            "tflops": sw["flops"] / t / 1e12, "bound": "alu", "frac_fp32_peak": sw["flops"] / t / 1e12 / fp32_peak,
+            "fp32_peak_tflops": fp32_peak, "hbm_gbs": sw["bytes"] / t / 1e9,
+            "batch_per_cluster": binding.slstm_batch_per_cluster(w.B, w.NH, w.DH, wx.dtype)}
 
 
 # ---------------------------------------------------------------- the oracle as CPU baseline / reference arm

@@ -36,7 +36,7 @@ state c, n, m, h [B, NH, DH]; outputs h_seq [B, S, NH, DH].  Inputs are widened
 to float64 exactly (fp32 or bf16 data); the arithmetic is float64 throughout.
 
 Parity pins (tests/test_oracle_pins_slstm.py): hand-derived values for two tiny
-cases (tests/golden/hand_slstm_*.json), the closed form of equal gates (a
+cases (tests/golden/slstm_hand_*.json), the closed form of equal gates (a
 running mean of tanh(z~)), the stabilizer's cancellation in c / n, the feedback
 decomposition of R, and the independence of heads.
 """

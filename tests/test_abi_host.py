@@ -25,13 +25,13 @@ def declared_functions():
         if fname.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fname)).read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-            names += re.findall(r"\b(mlstm_\w+)\s*\(", text)
+            names += re.findall(r"\b((?:mlstm|slstm)_\w+)\s*\(", text)
     return sorted(set(names))
 
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert "mlstm_fwd" in names and "mlstm_step" in names
+    assert "mlstm_fwd" in names and "mlstm_step" in names and "slstm_fwd" in names
     for name in names:
         assert hasattr(lib, name), name
         assert name in binding.SIGNATURES, "binding lacks " + name
@@ -145,3 +145,37 @@ def test_kernel_launch_counts(lib):
     assert lib.mlstm_fwd_kernel_launches(1, 2, 64, 16, 16, 16, f32) == 1 + 2
     assert lib.mlstm_fwd_kernel_launches(1, 2, 64 * 200, 16, 16, 64, f32) == 2 + 2
     assert lib.mlstm_fwd_kernel_launches(0, 2, 64, 16, 16, 16, f32) == 0
+
+
+def slstm_args(**over):
+    a = dict(wx=FAKE, R=FAKE, dt=0, B=2, S=5, NH=2, DH=64, fs=0, c=FAKE, n=FAKE, m=FAKE, h=FAKE, ho=FAKE)
+    a.update(over)
+    return a
+
+
+def call_slstm(lib, a):
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return lib.slstm_fwd(v(a["wx"]), v(a["R"]), a["dt"], a["B"], a["S"], a["NH"], a["DH"], a["fs"], v(a["c"]),
+                         v(a["n"]), v(a["m"]), v(a["h"]), v(a["ho"]), None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(wx=None), 1), (dict(R=None), 1), (dict(c=None), 1), (dict(n=None), 1), (dict(m=None), 1),
+    (dict(h=None), 1), (dict(R=FAKE + 8), 1), (dict(wx=FAKE + 2), 1), (dict(dt=1, wx=FAKE + 1), 1),
+    (dict(c=FAKE + 2), 1), (dict(B=-1), 1), (dict(S=-3), 1), (dict(NH=0), 1), (dict(dt=7), 2),
+    (dict(DH=48), 2), (dict(DH=512), 2), (dict(DH=16), 2),
+])
+def test_slstm_rejects_bad_arguments(lib, over, expect):
+    assert call_slstm(lib, slstm_args(**over)) == expect
+
+
+def test_slstm_empty_work_is_a_no_op(lib):
+    # nothing to run: no launch, and the pointers are not looked at
+    assert call_slstm(lib, slstm_args(B=0, wx=None, R=None, c=None, n=None, m=None, h=None, ho=None)) == 0
+    assert call_slstm(lib, slstm_args(S=0, wx=None, R=None, ho=None)) == 0
+
+
+def test_slstm_batch_per_cluster_rejects_unsupported(lib):
+    assert lib.slstm_batch_per_cluster(4, 2, 48, 0) == 0
+    assert lib.slstm_batch_per_cluster(4, 0, 64, 0) == 0
+    assert lib.slstm_batch_per_cluster(4, 2, 64, 5) == 0

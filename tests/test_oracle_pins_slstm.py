@@ -1,6 +1,6 @@
 """Pins of the sLSTM oracle (oracle/slstm.py) to facts that do not come from the oracle itself.
 
-* hand-derived values for two tiny cases (tests/golden/hand_slstm_*.json): memory mixing through
+* hand-derived values for two tiny cases (tests/golden/slstm_hand_*.json): memory mixing through
   an asymmetric R (a transposed R fails), the stabilizer shifting between steps, an exponential
   forget gate above 1, and the sigmoid forget gate;
 * closed form: with i~ = f~ = 0 (exponential forget) and R = 0 every weight is 1, so
@@ -31,7 +31,7 @@ def _rand(shape, rng, loc=0.0, scale=1.0):
     return (rng.standard_normal(shape) * scale + loc).astype(np.float32)
 
 
-@pytest.mark.parametrize("name", ["hand_slstm_mixing_three_steps.json", "hand_slstm_sigmoid_forget.json"])
+@pytest.mark.parametrize("name", ["slstm_hand_mixing_three_steps.json", "slstm_hand_sigmoid_forget.json"])
 def test_hand_derived(name):
     g = json.load(open(os.path.join(GOLDEN, name)))
     wx = np.asarray(g["wx"], dtype=np.float32)[None]          # [1, S, 4, NH, DH]

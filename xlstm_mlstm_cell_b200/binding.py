@@ -21,7 +21,7 @@ MLSTM_F32, MLSTM_BF16 = 0, 1
 STATUS = {0: "MLSTM_OK", 1: "MLSTM_ERR_INVALID_ARG", 2: "MLSTM_ERR_UNSUPPORTED", 3: "MLSTM_ERR_WORKSPACE",
           4: "MLSTM_ERR_CUDA", 5: "MLSTM_ERR_TIMEOUT"}
 
-# Every symbol include/mlstm.h declares, with its ctypes signature.
+# Every symbol include/mlstm.h and include/slstm.h declare, with its ctypes signature.
 _vp, _fp, _i, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
     "mlstm_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
@@ -42,6 +42,8 @@ SIGNATURES = {
     "mlstm_log_decay_sum": (_i, [_fp, _i, _i, _i, _fp, _vp]),
     "mlstm_state_prefix": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp]),
     "mlstm_selftest_wait_timeout": (_i, [_vp, _vp]),
+    "slstm_fwd": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
+    "slstm_batch_per_cluster": (_i, [_i, _i, _i, _i]),
 }
 
 _lib = None
@@ -247,3 +249,30 @@ def step(C, n, m, q, k, v, igate, fgate, ogate=None, h_out=None, stream=None):
                         _ptr(ogate), _dt(q), B, NH, DHQK, DHV, _ptr(h_out), _stream(stream))
     _check("mlstm_step", st)
     return h_out
+
+
+def slstm_fwd(wx, R, forget: str = "exp", state=None, h_out=None, want_h: bool = True, stream=None):
+    """slstm_fwd on device tensors: S steps of the sLSTM recurrence.
+
+    wx [B, S, 4, NH, DH] gate pre-activations (i, f, z, o), R [NH, 4, DH, DH], both float32 or
+    bfloat16; forget "exp" or "sigmoid"; state (c, n, m, h) fp32 [B, NH, DH] updated in place
+    (zeros when None).  Returns (h_seq [B, S, NH, DH] or None, (c, n, m, h)).
+    """
+    if forget not in ("exp", "sigmoid"):
+        raise ValueError("forget must be 'exp' or 'sigmoid'")
+    lib = load()
+    B, S, _, NH, DH = wx.shape
+    if state is None:
+        state = tuple(torch.zeros((B, NH, DH), dtype=torch.float32, device=wx.device) for _ in range(4))
+    c, n, m, h = state
+    if want_h and h_out is None:
+        h_out = torch.empty((B, S, NH, DH), dtype=wx.dtype, device=wx.device)
+    st = lib.slstm_fwd(_ptr(wx), _ptr(R), _dt(wx), B, S, NH, DH, 1 if forget == "sigmoid" else 0, _ptr(c), _ptr(n),
+                       _ptr(m), _ptr(h), _ptr(h_out if want_h else None), _stream(stream))
+    _check("slstm_fwd", st)
+    return (h_out if want_h else None), (c, n, m, h)
+
+
+def slstm_batch_per_cluster(B, NH, DH, dtype) -> int:
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().slstm_batch_per_cluster(B, NH, DH, dt))

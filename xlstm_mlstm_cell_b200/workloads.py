@@ -96,3 +96,42 @@ def make_custom(B, NH, S, DHQK, DHV, dtype, seed, qkv_scale=1.0, ig=(0.0, 1.0), 
     gen = torch.Generator().manual_seed(seed)
     dt = torch.float32 if dtype == "f32" else torch.bfloat16
     return draw((B, NH, S, DHQK), (B, NH, S, DHV), (B, NH, S), dt, qkv_scale, ig, fg, ogate, gen)
+
+
+# ---------------------------------------------------------------- sLSTM recurrence
+
+@dataclasses.dataclass(frozen=True)
+class SlstmWorkload:
+    """Inputs of the sLSTM recurrence: gate pre-activations wx [B, S, 4, NH, DH] (gate order
+    i, f, z, o; i, z, o ~ N(0, 1), f ~ N(f_loc, 1)) and recurrent weights R [NH, 4, DH, DH]
+    ~ N(0, 1 / DH), so that R h is of order one."""
+    name: str
+    dtype: str
+    B: int
+    S: int
+    NH: int
+    DH: int
+    forget: str         # "exp" or "sigmoid"
+    f_loc: float
+    seed: int
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+# a 4-head sLSTM layer of a 1024-wide model over 1024 tokens, 16 sequences; sigmoid forget gate
+# with pre-activations ~ N(3, 1) (forget gates near 0.95, a slowly decaying memory)
+SLSTM_WORKLOADS = {
+    "slstm_f32": SlstmWorkload("slstm_f32", "f32", 16, 1024, 4, 256, "sigmoid", 3.0, 1006),
+}
+
+
+def make_slstm_inputs(B, S, NH, DH, dtype, seed, f_loc=3.0):
+    """(wx, R) on the CPU, drawn in that order from a generator seeded with ``seed``."""
+    gen = torch.Generator().manual_seed(seed)
+    wx = torch.randn(B, S, 4, NH, DH, generator=gen)
+    wx[:, :, 1] += f_loc
+    R = torch.randn(NH, 4, DH, DH, generator=gen) / DH ** 0.5
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    return wx.to(dt), R.to(dt)
