@@ -553,10 +553,13 @@ def slstm_work(B, S, NH, DH, esize):
     return {"flops": 2.0 * 4 * DH * DH * NH * B * S, "bytes": (4 + 1) * NH * DH * B * S * esize}
 
 
-def slstm_extra(device, peaks):
-    """The sLSTM recurrence on its workload: one slstm_fwd call over the whole sequence."""
+def slstm_extra(device, peaks, B=None, S=None):
+    """The sLSTM recurrence on its workload: one slstm_fwd call over the whole sequence (batch
+    and sequence length overridable for profiling)."""
+    import dataclasses
     from xlstm_mlstm_cell_b200.workloads import SLSTM_WORKLOADS, make_slstm_inputs
     w = SLSTM_WORKLOADS["slstm_f32"]
+    w = dataclasses.replace(w, B=B or w.B, S=S or w.S)
     wx, R = make_slstm_inputs(w.B, w.S, w.NH, w.DH, w.dtype, w.seed, w.f_loc)
     wx, R = wx.to(device), R.to(device)
     h_out = torch.empty((w.B, w.S, w.NH, w.DH), dtype=wx.dtype, device=device)
@@ -658,6 +661,8 @@ def main():
     ap.add_argument("--seq", type=int, default=0, help="override the workload's sequence length (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling)")
     ap.add_argument("--sets", type=int, default=0, help="cap the number of rotated input sets (profiling)")
+    ap.add_argument("--slstm", action="store_true",
+                    help="time only the sLSTM recurrence workload (sizes from --batch / --seq) and print its numbers")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -670,6 +675,11 @@ def main():
         run_reference(args, rank, world)
         return
     binding.load()
+    if args.slstm:
+        torch.cuda.set_device(local_rank)
+        print(json.dumps(slstm_extra(torch.device("cuda", local_rank), load_peaks(), B=args.batch or None,
+                                     S=args.seq or None)))
+        return
     run_ours(args, rank, world, local_rank)
 
 

@@ -16,9 +16,11 @@
 //      (shared memory, fp32) for the BG batch items; lanes 0..3 add wx of gate i, f, z, o;
 //   2. a butterfly over the cell's 8 lanes leaves the four sums in every lane, and all of
 //      them update the cell's (c, n, m) in registers;
-//   3. lane r of the cell stores h_t into the shared memory of cluster rank r (distributed
-//      shared memory), and lane b writes h_out of batch item b;
-//   4. a cluster barrier (release / acquire) publishes h_t to every CTA of the head.
+//   3. the lanes of a cell store h_t into the shared memory of every cluster rank
+//      (distributed shared memory);
+//   4. a cluster barrier (release / acquire) publishes h_t to every CTA of the head; h_out
+//      and the next step's wx loads are issued between its arrive and its wait, so that the
+//      release does not wait for them.
 // h_{t-1} and h_t live in two shared buffers that alternate between steps: a CTA writes
 // step t's buffer only after the barrier of step t - 1, by which every CTA has finished
 // reading it.
@@ -57,6 +59,26 @@ MLSTM_DEVINL void st_cluster(const float *local, uint32_t rank, float v)
 
 MLSTM_DEVINL float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
 
+// Packed pairs of fp32 (low half = first element): one instruction for two fused multiply-adds.
+MLSTM_DEVINL uint64_t pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+MLSTM_DEVINL float sum2(uint64_t r)
+{
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+    return lo + hi;
+}
+MLSTM_DEVINL uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 template <typename T, int DH, int BG>
 __global__ void __launch_bounds__(THREADS, 1)
 slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, int NH, int forget_sigmoid,
@@ -80,17 +102,16 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
 
     // the four gate rows of cell j over this lane's k: k = 32 q + 4 l8 + e (the 8 lanes of a
     // cell read 8 consecutive 16-byte pieces of h, so one load instruction covers 128 bytes)
-    float wr[4][NQ * 4];
+    // (as packed pairs (k, k + 1), the operands of the paired multiply-adds)
+    uint64_t wr[4][NQ * 2];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         const T *row = R + (((size_t)head * 4 + g) * DH + j) * DH + 4 * l8;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
             const float4 v = load4(row + 32 * q);
-            wr[g][4 * q] = v.x;
-            wr[g][4 * q + 1] = v.y;
-            wr[g][4 * q + 2] = v.z;
-            wr[g][4 * q + 3] = v.w;
+            wr[g][2 * q] = pack2(v.x, v.y);
+            wr[g][2 * q + 1] = pack2(v.z, v.w);
         }
     }
     // lane l8 of a cell keeps the state of batch item it = l8 mod BG (the 8 / BG lanes with the
@@ -124,37 +145,36 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
 
     const bool exp_forget = forget_sigmoid == 0;
     float hv = 0.f;
+    float xsel[4];                      // 1 for the gate whose wx this lane adds, else 0 (no branch)
+#pragma unroll
+    for (int g = 0; g < 4; ++g) xsel[g] = (g == l8) ? 1.f : 0.f;
     for (int t = 0; t < S; ++t) {
         const int cur = t & 1;
-        float nx[BG];
-#pragma unroll
-        for (int b = 0; b < BG; ++b) {
-            const bool ld = has_x && b0 + b < B && t + 1 < S;
-            const size_t off = ((size_t)(b0 + b) * S + t + 1) * 4 * HD;
-            nx[b] = ld ? to_f32(wxr[off]) : 0.f;
-            if (ld && t + 16 < S)                              // warm L2 further ahead
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(wxr + off + 15 * 4 * HD));
-        }
-        // 1. partial gate pre-activations over this lane's k (wx added by lanes 0..3)
+        // 1. partial gate pre-activations over this lane's k (wx added by lanes 0..3 afterwards,
+        //    so that its load, issued during the previous step's barrier, has the products' time)
         float acc[BG][4];
+        {
+            uint64_t acc2[BG][4];            // even and odd k summed apart, added at the end
 #pragma unroll
-        for (int b = 0; b < BG; ++b)
+            for (int b = 0; b < BG; ++b)
 #pragma unroll
-            for (int g = 0; g < 4; ++g) acc[b][g] = (g == l8) ? xw[b] : 0.f;
+                for (int g = 0; g < 4; ++g) acc2[b][g] = 0ull;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
+            for (int q = 0; q < NQ; ++q) {
 #pragma unroll
-            for (int b = 0; b < BG; ++b) {
-                const float4 h4 = *reinterpret_cast<const float4 *>(&hs[cur][b][32 * q + 4 * l8]);
+                for (int b = 0; b < BG; ++b) {
+                    const ulonglong2 h4 = *reinterpret_cast<const ulonglong2 *>(&hs[cur][b][32 * q + 4 * l8]);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float &a = acc[b][g];
-                    a = fmaf(wr[g][4 * q], h4.x, a);
-                    a = fmaf(wr[g][4 * q + 1], h4.y, a);
-                    a = fmaf(wr[g][4 * q + 2], h4.z, a);
-                    a = fmaf(wr[g][4 * q + 3], h4.w, a);
+                    for (int g = 0; g < 4; ++g) {
+                        acc2[b][g] = fma2(wr[g][2 * q], h4.x, acc2[b][g]);
+                        acc2[b][g] = fma2(wr[g][2 * q + 1], h4.y, acc2[b][g]);
+                    }
                 }
             }
+#pragma unroll
+            for (int b = 0; b < BG; ++b)
+#pragma unroll
+                for (int g = 0; g < 4; ++g) acc[b][g] = fmaf(xsel[g], xw[b], sum2(acc2[b][g]));
         }
         // 2. sum over the cell's 8 lanes: a butterfly over the lane bits above the batch items'
         //    and a halving exchange over the others, after which slot 0 of lane l8 holds the four
@@ -192,8 +212,8 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
             m = mn;
             hv = sigmoidf_(go) * (c / n);
         }
-        // 3. publish h_t: the copies of item it share the cluster ranks (copy ci writes ranks ci,
-        //    ci + 8 / BG, ...); copy 0 writes h_out
+        // 3. publish h_t to the CTAs of the cluster: the copies of item it share the ranks (copy ci
+        //    writes ranks ci, ci + 8 / BG, ...)
         const int nxt = cur ^ 1;
         if (item_ok) {
 #pragma unroll
@@ -205,14 +225,24 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
                         hs[nxt][it][j] = hv;
                 }
             }
-            if (h_out != nullptr && ci == 0)
-                h_out[(((size_t)(b0 + it) * S + t) * NH + head) * DH + j] = from_f32<T>(hv);
         }
-#pragma unroll
-        for (int b = 0; b < BG; ++b) xw[b] = nx[b];
-        // 4. every CTA of the head has h_t before any reads it
+        // 4. every CTA of the head has h_t before any reads it.  The release orders only what
+        //    precedes the arrive, so h_out and the next step's wx go out between arrive and
+        //    wait: the barrier does not wait for their round trips to memory.
         if (G > 1)
-            cluster_sync_release_acquire();
+            asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        if (item_ok && h_out != nullptr && ci == 0)
+            h_out[(((size_t)(b0 + it) * S + t) * NH + head) * DH + j] = from_f32<T>(hv);
+#pragma unroll
+        for (int b = 0; b < BG; ++b) {
+            const bool ld = has_x && b0 + b < B && t + 1 < S;
+            const size_t off = ((size_t)(b0 + b) * S + t + 1) * 4 * HD;
+            xw[b] = ld ? to_f32(wxr[off]) : 0.f;
+            if (ld && t + 16 < S)                              // warm L2 further ahead
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(wxr + off + 15 * 4 * HD));
+        }
+        if (G > 1)
+            asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
         else
             __syncthreads();
     }
