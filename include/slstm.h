@@ -44,6 +44,9 @@ extern "C" {
  *   h_out   [B][S][NH][DH] device, dtype dt: h of every step, or NULL (state only).
  *   DH      32, 64, 128, 192 or 256 (the cells of one head are spread over a thread-
  *           block cluster of DH / 32 CTAs).
+ *   status  device uint32 or NULL, 4-byte aligned: set to MLSTM_ERR_TIMEOUT if one of the
+ *           kernel's bounded waits (2 s each, for the other CTAs' h of a step) gave up; the
+ *           outputs are then not valid.  The call never clears it.
  *   stream  cudaStream_t, or NULL for the default stream.  Asynchronous.
  *
  * Arithmetic is fp32 (bf16 inputs are widened exactly; h_out is rounded to dt).
@@ -54,7 +57,8 @@ extern "C" {
  * pointers); the state is left as it is.
  */
 mlstm_status slstm_fwd(const void *wx, const void *R, mlstm_dtype dt, int B, int S, int NH, int DH,
-                       int forget_sigmoid, float *c, float *n, float *m, float *h, void *h_out, void *stream);
+                       int forget_sigmoid, float *c, float *n, float *m, float *h, void *h_out,
+                       unsigned int *status, void *stream);
 
 /* The batch items one cluster carries through the recurrence for this shape on
  * the current device (1, 2, 4 or 8), or 0 for an unsupported shape: the launch

@@ -148,7 +148,7 @@ def test_kernel_launch_counts(lib):
 
 
 def slstm_args(**over):
-    a = dict(wx=FAKE, R=FAKE, dt=0, B=2, S=5, NH=2, DH=64, fs=0, c=FAKE, n=FAKE, m=FAKE, h=FAKE, ho=FAKE)
+    a = dict(wx=FAKE, R=FAKE, dt=0, B=2, S=5, NH=2, DH=64, fs=0, c=FAKE, n=FAKE, m=FAKE, h=FAKE, ho=FAKE, st=None)
     a.update(over)
     return a
 
@@ -156,14 +156,14 @@ def slstm_args(**over):
 def call_slstm(lib, a):
     v = lambda p: None if p is None else ctypes.c_void_p(p)
     return lib.slstm_fwd(v(a["wx"]), v(a["R"]), a["dt"], a["B"], a["S"], a["NH"], a["DH"], a["fs"], v(a["c"]),
-                         v(a["n"]), v(a["m"]), v(a["h"]), v(a["ho"]), None)
+                         v(a["n"]), v(a["m"]), v(a["h"]), v(a["ho"]), v(a["st"]), None)
 
 
 @pytest.mark.parametrize("over,expect", [
     (dict(wx=None), 1), (dict(R=None), 1), (dict(c=None), 1), (dict(n=None), 1), (dict(m=None), 1),
     (dict(h=None), 1), (dict(R=FAKE + 8), 1), (dict(wx=FAKE + 2), 1), (dict(dt=1, wx=FAKE + 1), 1),
     (dict(c=FAKE + 2), 1), (dict(B=-1), 1), (dict(S=-3), 1), (dict(NH=0), 1), (dict(dt=7), 2),
-    (dict(DH=48), 2), (dict(DH=512), 2), (dict(DH=16), 2),
+    (dict(DH=48), 2), (dict(DH=512), 2), (dict(DH=16), 2), (dict(st=FAKE + 2), 1),
 ])
 def test_slstm_rejects_bad_arguments(lib, over, expect):
     assert call_slstm(lib, slstm_args(**over)) == expect

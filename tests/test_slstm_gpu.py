@@ -42,8 +42,11 @@ def make_state(B, NH, DH, seed):
 
 def run_gpu(wx, R, forget, state=None, want_h=True):
     st = None if state is None else tuple(x.clone().cuda() for x in state)
-    h, (c, n, m, hl) = binding.slstm_fwd(wx.cuda(), R.cuda(), forget=forget, state=st, want_h=want_h)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    h, (c, n, m, hl) = binding.slstm_fwd(wx.cuda(), R.cuda(), forget=forget, state=st, want_h=want_h,
+                                         status=status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, "a bounded wait of the sLSTM kernel gave up"
     return (None if h is None else h.cpu()), (c.cpu(), n.cpu(), m.cpu(), hl.cpu())
 
 

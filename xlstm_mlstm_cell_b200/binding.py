@@ -42,7 +42,7 @@ SIGNATURES = {
     "mlstm_log_decay_sum": (_i, [_fp, _i, _i, _i, _fp, _vp]),
     "mlstm_state_prefix": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp]),
     "mlstm_selftest_wait_timeout": (_i, [_vp, _vp]),
-    "slstm_fwd": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp]),
+    "slstm_fwd": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _fp, _vp, _vp, _vp]),
     "slstm_batch_per_cluster": (_i, [_i, _i, _i, _i]),
 }
 
@@ -251,12 +251,13 @@ def step(C, n, m, q, k, v, igate, fgate, ogate=None, h_out=None, stream=None):
     return h_out
 
 
-def slstm_fwd(wx, R, forget: str = "exp", state=None, h_out=None, want_h: bool = True, stream=None):
+def slstm_fwd(wx, R, forget: str = "exp", state=None, h_out=None, want_h: bool = True, status=None, stream=None):
     """slstm_fwd on device tensors: S steps of the sLSTM recurrence.
 
     wx [B, S, 4, NH, DH] gate pre-activations (i, f, z, o), R [NH, 4, DH, DH], both float32 or
     bfloat16; forget "exp" or "sigmoid"; state (c, n, m, h) fp32 [B, NH, DH] updated in place
-    (zeros when None).  Returns (h_seq [B, S, NH, DH] or None, (c, n, m, h)).
+    (zeros when None); status: an optional int32 device tensor that a timed-out wait sets to
+    MLSTM_ERR_TIMEOUT.  Returns (h_seq [B, S, NH, DH] or None, (c, n, m, h)).
     """
     if forget not in ("exp", "sigmoid"):
         raise ValueError("forget must be 'exp' or 'sigmoid'")
@@ -268,7 +269,7 @@ def slstm_fwd(wx, R, forget: str = "exp", state=None, h_out=None, want_h: bool =
     if want_h and h_out is None:
         h_out = torch.empty((B, S, NH, DH), dtype=wx.dtype, device=wx.device)
     st = lib.slstm_fwd(_ptr(wx), _ptr(R), _dt(wx), B, S, NH, DH, 1 if forget == "sigmoid" else 0, _ptr(c), _ptr(n),
-                       _ptr(m), _ptr(h), _ptr(h_out if want_h else None), _stream(stream))
+                       _ptr(m), _ptr(h), _ptr(h_out if want_h else None), _ptr(status), _stream(stream))
     _check("slstm_fwd", st)
     return (h_out if want_h else None), (c, n, m, h)
 

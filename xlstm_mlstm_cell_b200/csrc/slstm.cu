@@ -16,17 +16,17 @@
 //      (shared memory, fp32) for the BG batch items; lanes 0..3 add wx of gate i, f, z, o;
 //   2. a butterfly over the cell's 8 lanes leaves the four sums in every lane, and all of
 //      them update the cell's (c, n, m) in registers;
-//   3. the lanes of a cell store h_t into the shared memory of every cluster rank
-//      (distributed shared memory);
-//   4. a cluster barrier (release / acquire) publishes h_t to every CTA of the head; h_out
-//      and the next step's wx loads are issued between its arrive and its wait, so that the
-//      release does not wait for them.
-// h_{t-1} and h_t live in two shared buffers that alternate between steps: a CTA writes
-// step t's buffer only after the barrier of step t - 1, by which every CTA has finished
-// reading it.
+//   3. the lanes of a cell send h_t into the shared memory of every cluster rank with st.async
+//      stores that count their bytes on that rank's mbarrier for the buffer;
+//   4. the next step waits on its own mbarrier until the whole head's h_t has arrived (no
+//      cluster-wide barrier and no release fence per step).
+// h_{t-1} and h_t live in two shared buffers that alternate between steps.  A CTA sends into a
+// peer's buffer for step t + 1 only after it has received h_t from every CTA, that is after every
+// CTA has finished its step-t reads of that buffer.
 #include "common.cuh"
 #include "mlstm.h"
 #include "slstm.h"
+#include "tc_common.cuh"
 
 namespace mlstm {
 namespace slstm {
@@ -48,13 +48,47 @@ MLSTM_DEVINL void cluster_sync_release_acquire()
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Stores v at the same shared-memory offset as `local` in the CTA of cluster rank `rank`.
-MLSTM_DEVINL void st_cluster(const float *local, uint32_t rank, float v)
+MLSTM_DEVINL uint32_t map_rank(const void *local, uint32_t rank)
 {
-    const uint32_t la = (uint32_t)__cvta_generic_to_shared(local);
     uint32_t ra;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"((uint32_t)__cvta_generic_to_shared(local)),
+                 "r"(rank));
+    return ra;
+}
+
+// Stores v at the offset of `local` in the CTA of cluster rank `rank` and counts its 4 bytes on
+// that CTA's mbarrier at the offset of `bar` (asynchronous; no fence on this side).
+MLSTM_DEVINL void st_async_cluster(const float *local, const uint64_t *bar, uint32_t rank, float v)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                     map_rank(local, rank)),
+                 "r"(__float_as_uint(v)), "r"(map_rank(bar, rank))
+                 : "memory");
+}
+
+// Bounded wait for the phase of parity `parity` of a local mbarrier whose bytes come from other
+// CTAs of the cluster (acquire at cluster scope).  False once the limit has passed.
+MLSTM_DEVINL bool wait_cluster_fill(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(bar);
+    unsigned long long t0 = 0ull;
+    for (uint32_t it = 0;; ++it) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done)
+                     : "r"(a), "r"(parity)
+                     : "memory");
+        if (done) return true;
+        if ((it & 15u) == 0u) {
+            const unsigned long long now = tc::global_timer();
+            if (t0 == 0ull)
+                t0 = now;
+            else if (now - t0 > tc::WAIT_LIMIT_NS)
+                return false;
+        }
+    }
 }
 
 MLSTM_DEVINL float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
@@ -83,11 +117,14 @@ template <typename T, int DH, int BG>
 __global__ void __launch_bounds__(THREADS, 1)
 slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, int NH, int forget_sigmoid,
              float *__restrict__ c_st, float *__restrict__ n_st, float *__restrict__ m_st, float *__restrict__ h_st,
-             T *__restrict__ h_out)
+             T *__restrict__ h_out, uint32_t *__restrict__ status)
 {
     constexpr int G = DH / CELLS;        // CTAs per head (cluster size)
     constexpr int NQ = DH / 32;          // 4-value groups of k per lane
     __shared__ __align__(16) float hs[2][BG][DH];
+    __shared__ __align__(8) uint64_t fill[2];      // hs[p] holds the whole head's h of a step
+    __shared__ uint32_t stuck;                     // a wait gave up: later waits are skipped
+    constexpr uint32_t FILL_BYTES = (uint32_t)(BG * DH * 4);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cl = lane >> 3, l8 = lane & 7;                 // cell of the warp, eighth of k
@@ -98,6 +135,16 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
     const int j = (int)rank * CELLS + warp * 4 + cl;        // this lane's cell in the head
     const size_t HD = (size_t)NH * DH;                      // stride of one gate in wx
 
+    if (tid == 0) {
+        stuck = 0u;
+        if constexpr (G > 1) {
+            tc::mbar_init(&fill[0], 1);
+            tc::mbar_init(&fill[1], 1);
+            tc::fence_barrier_init();
+            tc::mbar_arrive_expect_tx(&fill[0], FILL_BYTES);   // the first fill of each buffer
+            tc::mbar_arrive_expect_tx(&fill[1], FILL_BYTES);
+        }
+    }
     griddep_wait();
 
     // the four gate rows of cell j over this lane's k: k = 32 q + 4 l8 + e (the 8 lanes of a
@@ -150,6 +197,17 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
     for (int g = 0; g < 4; ++g) xsel[g] = (g == l8) ? 1.f : 0.f;
     for (int t = 0; t < S; ++t) {
         const int cur = t & 1;
+        if constexpr (G > 1) {
+            // h_{t-1} of the whole head: fill (t - 1) / 2 of buffer cur, written by every CTA of
+            // the cluster during step t - 1
+            if (t > 0) {
+                if (!*(volatile uint32_t *)&stuck && !wait_cluster_fill(&fill[cur], (uint32_t)((t - 1) >> 1) & 1u)) {
+                    stuck = 1u;
+                    if (status != nullptr) atomicExch(status, (uint32_t)MLSTM_ERR_TIMEOUT);
+                }
+                if (tid == 0) tc::mbar_arrive_expect_tx(&fill[cur], FILL_BYTES);   // its next fill
+            }
+        }
         // 1. partial gate pre-activations over this lane's k (wx added by lanes 0..3 afterwards,
         //    so that its load, issued during the previous step's barrier, has the products' time)
         float acc[BG][4];
@@ -212,25 +270,21 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
             m = mn;
             hv = sigmoidf_(go) * (c / n);
         }
-        // 3. publish h_t to the CTAs of the cluster: the copies of item it share the ranks (copy ci
-        //    writes ranks ci, ci + 8 / BG, ...)
+        // 3. publish h_t to every CTA of the cluster (not after the last step: nobody reads it).
+        //    The copies of item it share the ranks (copy ci writes ranks ci, ci + 8 / BG, ...);
+        //    every (item, cell) slot is written, so that each fill is exactly FILL_BYTES.  A CTA
+        //    writes buffer nxt of a peer only after it has h_t of every CTA, that is after every
+        //    CTA has finished step t's reads of that buffer's previous contents.
         const int nxt = cur ^ 1;
-        if (item_ok) {
+        if constexpr (G > 1) {
+            if (t + 1 < S) {
 #pragma unroll
-            for (int r = 0; r < G; r += DUP) {
-                if (r + ci < G) {
-                    if (G > 1)
-                        st_cluster(&hs[nxt][it][j], (uint32_t)(r + ci), hv);
-                    else
-                        hs[nxt][it][j] = hv;
-                }
+                for (int r = 0; r < G; r += DUP)
+                    if (r + ci < G) st_async_cluster(&hs[nxt][it][j], &fill[nxt], (uint32_t)(r + ci), hv);
             }
+        } else {
+            hs[nxt][it][j] = hv;
         }
-        // 4. every CTA of the head has h_t before any reads it.  The release orders only what
-        //    precedes the arrive, so h_out and the next step's wx go out between arrive and
-        //    wait: the barrier does not wait for their round trips to memory.
-        if (G > 1)
-            asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         if (item_ok && h_out != nullptr && ci == 0)
             h_out[(((size_t)(b0 + it) * S + t) * NH + head) * DH + j] = from_f32<T>(hv);
 #pragma unroll
@@ -241,11 +295,10 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
             if (ld && t + 16 < S)                              // warm L2 further ahead
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(wxr + off + 15 * 4 * HD));
         }
-        if (G > 1)
-            asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-        else
-            __syncthreads();
+        if constexpr (G == 1) __syncthreads();
     }
+    // no CTA leaves while a peer may still address its shared memory
+    if (G > 1) cluster_sync_release_acquire();
     griddep_launch_dependents();
     // the state after step S (copy 0 of each item)
     if (item_ok && ci == 0) {
@@ -259,13 +312,13 @@ slstm_kernel(const T *__restrict__ wx, const T *__restrict__ R, int B, int S, in
 
 template <typename T, int DH, int BG>
 static cudaError_t launch_bg(const void *wx, const void *R, int B, int S, int NH, int fs, float *c, float *n, float *m,
-                             float *h, void *h_out, cudaStream_t st)
+                             float *h, void *h_out, uint32_t *status, cudaStream_t st)
 {
     constexpr int G = DH / CELLS;
     const int ngrp = (B + BG - 1) / BG;
     const dim3 grid((unsigned)(NH * ngrp * G));
     return launch_kernel(slstm_kernel<T, DH, BG>, grid, dim3(THREADS), 0, st, G, static_cast<const T *>(wx),
-                         static_cast<const T *>(R), B, S, NH, fs, c, n, m, h, static_cast<T *>(h_out));
+                         static_cast<const T *>(R), B, S, NH, fs, c, n, m, h, static_cast<T *>(h_out), status);
 }
 
 // Clusters of this kernel that fit on the device at once (cached per kernel and device).
@@ -325,26 +378,26 @@ static int choose_bg(int B, int NH)
 
 template <typename T, int DH>
 static cudaError_t launch_dh(const void *wx, const void *R, int B, int S, int NH, int fs, float *c, float *n, float *m,
-                             float *h, void *h_out, cudaStream_t st)
+                             float *h, void *h_out, uint32_t *status, cudaStream_t st)
 {
     switch (choose_bg<T, DH>(B, NH)) {
-    case 1: return launch_bg<T, DH, 1>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    case 2: return launch_bg<T, DH, 2>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    case 4: return launch_bg<T, DH, 4>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    default: return launch_bg<T, DH, 8>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
+    case 1: return launch_bg<T, DH, 1>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    case 2: return launch_bg<T, DH, 2>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    case 4: return launch_bg<T, DH, 4>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    default: return launch_bg<T, DH, 8>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
     }
 }
 
 template <typename T>
 static cudaError_t launch_t(const void *wx, const void *R, int B, int S, int NH, int DH, int fs, float *c, float *n,
-                            float *m, float *h, void *h_out, cudaStream_t st)
+                            float *m, float *h, void *h_out, uint32_t *status, cudaStream_t st)
 {
     switch (DH) {
-    case 32: return launch_dh<T, 32>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    case 64: return launch_dh<T, 64>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    case 128: return launch_dh<T, 128>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    case 192: return launch_dh<T, 192>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
-    default: return launch_dh<T, 256>(wx, R, B, S, NH, fs, c, n, m, h, h_out, st);
+    case 32: return launch_dh<T, 32>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    case 64: return launch_dh<T, 64>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    case 128: return launch_dh<T, 128>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    case 192: return launch_dh<T, 192>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
+    default: return launch_dh<T, 256>(wx, R, B, S, NH, fs, c, n, m, h, h_out, status, st);
     }
 }
 
@@ -368,7 +421,8 @@ static bool aligned(const void *p, unsigned a) { return (reinterpret_cast<uintpt
 }  // namespace mlstm
 
 extern "C" mlstm_status slstm_fwd(const void *wx, const void *R, mlstm_dtype dt, int B, int S, int NH, int DH,
-                                  int forget_sigmoid, float *c, float *n, float *m, float *h, void *h_out, void *stream)
+                                  int forget_sigmoid, float *c, float *n, float *m, float *h, void *h_out,
+                                  unsigned int *status, void *stream)
 {
     using namespace mlstm::slstm;
     if (B < 0 || S < 0 || NH < 1 || DH < 1) return MLSTM_ERR_INVALID_ARG;
@@ -379,11 +433,13 @@ extern "C" mlstm_status slstm_fwd(const void *wx, const void *R, mlstm_dtype dt,
     const unsigned es = dt == MLSTM_F32 ? 4u : 2u;
     if (!aligned(wx, es) || !aligned(R, 16u) || (h_out && !aligned(h_out, es))) return MLSTM_ERR_INVALID_ARG;
     if (!aligned(c, 4u) || !aligned(n, 4u) || !aligned(m, 4u) || !aligned(h, 4u)) return MLSTM_ERR_INVALID_ARG;
+    if (status && !aligned(status, 4u)) return MLSTM_ERR_INVALID_ARG;
     if ((long long)B * NH * (DH / CELLS) > (1ll << 31) - 1) return MLSTM_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = dt == MLSTM_F32 ? launch_t<float>(wx, R, B, S, NH, DH, forget_sigmoid, c, n, m, h, h_out, st)
-                                          : launch_t<__nv_bfloat16>(wx, R, B, S, NH, DH, forget_sigmoid, c, n, m, h,
-                                                                    h_out, st);
+    uint32_t *sw = reinterpret_cast<uint32_t *>(status);
+    const cudaError_t e = dt == MLSTM_F32
+                              ? launch_t<float>(wx, R, B, S, NH, DH, forget_sigmoid, c, n, m, h, h_out, sw, st)
+                              : launch_t<__nv_bfloat16>(wx, R, B, S, NH, DH, forget_sigmoid, c, n, m, h, h_out, sw, st);
     return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
 }
 
