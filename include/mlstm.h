@@ -173,6 +173,11 @@ mlstm_status mlstm_state_prefix(const float *C_parts, const float *n_parts, cons
  * state contributions, 2 scan of the states across chunks or segments,
  * 3 outputs (and, on the tensor-core path, the in-segment state walk).  A
  * phase that launches nothing on a given path has two events back to back.
+ * Entries of `events` may be NULL (that boundary is not recorded); the array
+ * itself may not.  events[MLSTM_FWD_PHASES - 1], recorded before the outputs
+ * phase, completes once C_final, n_final and m_final are written: a consumer of
+ * the final state (a decode step on another stream) can wait for it while the
+ * outputs are still being computed.
  */
 #define MLSTM_FWD_PHASES 4
 mlstm_status mlstm_fwd_profiled(const void *q, const void *k, const void *v,

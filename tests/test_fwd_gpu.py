@@ -179,3 +179,21 @@ def test_chained_calls_read_previous_outputs(cuda_lib, chunk):
     assert_close("h of the third call", h3.cpu(), hr3, TOL["bf16"])
     assert_close("C of the third call", C3.cpu(), Cr3, TOL["bf16"])
     assert_close("n of the third call", n3.cpu(), nr3, TOL["bf16"])
+
+
+def test_state_ready_event_with_other_phase_events_null(cuda_lib):
+    """mlstm_fwd_profiled with only the event before the outputs phase: same results as mlstm_fwd, and
+    a second stream that waits on that event reads the complete final state."""
+    q, k, v, i, f, o = (x.cuda() for x in make_custom(1, 2, 333, 256, 256, "bf16", seed=21, ig=(-1.0, 2.0),
+                                                       fg=(4.0, 1.0)))
+    h1, C1, n1, m1 = binding.fwd(q, k, v, i, f, o, chunk=64)
+    ready = torch.cuda.Event()
+    events = [None] * (binding.FWD_PHASES - 1) + [ready, None]
+    h2, C2, n2, m2 = binding.fwd(q, k, v, i, f, o, chunk=64, events=events)
+    side = torch.cuda.Stream()
+    side.wait_event(ready)
+    with torch.cuda.stream(side):
+        C_copy = C2.clone()
+    torch.cuda.synchronize()
+    assert torch.equal(h1, h2) and torch.equal(C1, C2) and torch.equal(n1, n2) and torch.equal(m1, m2)
+    assert torch.equal(C_copy, C1)

@@ -128,8 +128,9 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
     """mlstm_fwd on device tensors; returns ``(h, C, n, m)`` (states None unless requested).
 
     ``state=(C0, n0, m0)`` starts from that state (mlstm_fwd_state) instead of the zero state.
-    With ``events`` (FWD_PHASES + 1 ``torch.cuda.Event(enable_timing=True)``) the call goes
-    through mlstm_fwd_profiled, which records them around its phases on the stream.
+    With ``events`` (FWD_PHASES + 1 ``torch.cuda.Event`` or None) the call goes through
+    mlstm_fwd_profiled, which records them around its phases on the stream; ``events[FWD_PHASES
+    - 1]`` completes once the final state is written.
     """
     lib = load()
     B, NH, S, DHQK = q.shape
@@ -159,9 +160,9 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
     else:
         assert len(events) == FWD_PHASES + 1
         for e in events:            # torch creates the CUDA event lazily, on its first record
-            if not e.cuda_event:
+            if e is not None and not e.cuda_event:
                 e.record()
-        arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[e.cuda_event for e in events])
+        arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[None if e is None else e.cuda_event for e in events])
         _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
     return h_out, C_final, n_final, m_final
 

@@ -63,7 +63,8 @@ struct PhaseMark {
     cudaStream_t stream = nullptr;
     cudaError_t operator()(int phase) const
     {
-        return events ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[phase]), stream) : cudaSuccess;
+        return events && events[phase] ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[phase]), stream)
+                                       : cudaSuccess;
     }
 };
 
