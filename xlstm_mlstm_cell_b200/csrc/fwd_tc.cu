@@ -914,56 +914,48 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
                 rs[hq * L + tau] = sum;
-            } else {   // L == 64: M = 64 accumulator, rows 16q..16q+15 in lanes 0..15 of quadrant q
+            } else {   // L == 64: M = 64 accumulator, rows 16q..16q+15 in lanes 0..15 of quadrant q.
+                // The four warps of a quadrant share all of its blocks by columns: warp hq takes
+                // columns 4 hq .. 4 hq + 3 of every 16-column block, so that the diagonal block's
+                // per-element decay is spread over the four warps instead of falling on one
                 const int tau = q * 16 + (lane & 15);
-                const int s0 = hq * 16;
-                const bool above = s0 > q * 16 + 15;   // the whole 16 x 16 block is masked
-                const bool below = s0 + 15 < q * 16;   // the whole block is causal
-                uint32_t r[16];
-                if (!above) {
-                    tmem_ld16(tmem_addr(tmem, q * 32, SM::S_COL + s0), r);
-                    tmem_wait_ld();
-                }
-                if (lane < 16) {
-                    float sum = 0.f;
-                    const float at = arow[tau];
-                    const float ri = 1.f / rrow[tau];
-                    uint32_t pk[8];
-                    if (below) {                   // row factor x column factor
-                        const float rf = tau < len ? exp2f(at + bcol[hq]) * scale : 0.f;
+                const float at = arow[tau];
+                const float ri = 1.f / rrow[tau];
+                float sum = 0.f;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float v0 = __uint_as_float(r[2 * e]) * (ccol[s0 + 2 * e] * rf);
-                            const float v1 = __uint_as_float(r[2 * e + 1]) * (ccol[s0 + 2 * e + 1] * rf);
-                            sum += v0 + v1;
-                            pk[e] = pack_bf16(v0 * ri, v1 * ri);
-                        }
-                    } else {
+                for (int blk = 0; blk < 4; ++blk) {
+                    const int s0 = blk * 16 + hq * 4;          // this warp's first column of the block
+                    const bool above = blk > q;                // the whole block is masked
+                    uint32_t r[4];
+                    if (!above) {
+                        tmem_ld4(tmem_addr(tmem, q * 32, SM::S_COL + s0), r);
+                        tmem_wait_ld();
+                    }
+                    if (lane < 16) {
+                        float v[4];
+                        if (above) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            float v2[2];
+                            for (int z = 0; z < 4; ++z) v[z] = 0.f;
+                        } else if (blk < q) {                  // row factor x column factor
+                            const float rf = tau < len ? exp2f(at + bcol[blk]) * scale : 0.f;
 #pragma unroll
-                            for (int z = 0; z < 2; ++z) {
-                                const int sg = s0 + 2 * e + z;
-                                float d = 0.f;
-                                if (!above) {
-                                    d = exp2f(at + icol[sg]);
-                                    if (sg > tau) d = 0.f;
-                                }
-                                v2[z] = above ? 0.f : __uint_as_float(r[2 * e + z]) * d * scale;
-                                sum += v2[z];
+                            for (int z = 0; z < 4; ++z) v[z] = __uint_as_float(r[z]) * (ccol[s0 + z] * rf);
+                        } else {                               // diagonal block: per element, causal mask
+#pragma unroll
+                            for (int z = 0; z < 4; ++z) {
+                                const int sg = s0 + z;
+                                float d = exp2f(at + icol[sg]);
+                                if (sg > tau) d = 0.f;
+                                v[z] = __uint_as_float(r[z]) * d * scale;
                             }
-                            pk[e] = pack_bf16(v2[0] * ri, v2[1] * ri);
                         }
+                        sum += (v[0] + v[1]) + (v[2] + v[3]);
+                        // 4 bf16 = the first or second half of the row's 16-byte chunk s0 / 8
+                        *reinterpret_cast<uint2 *>(Ps + sw128_chunk(tau, s0 >> 3, L) + ((s0 >> 2) & 1) * 8) =
+                            make_uint2(pack_bf16(v[0] * ri, v[1] * ri), pack_bf16(v[2] * ri, v[3] * ri));
                     }
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int jcs = (s0 >> 3) + e;
-                        *reinterpret_cast<uint4 *>(Ps + sw128_chunk(tau, jcs, L)) =
-                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                    }
-                    rs[hq * L + tau] = sum;
                 }
+                if (lane < 16) rs[hq * L + tau] = sum;
             }
 
             if (ct == 0) WALK_TRACE(15);
