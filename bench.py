@@ -300,10 +300,14 @@ def run_ours(args, rank, world, local_rank):
     run = Runner(w, device)
     stream = torch.cuda.current_stream()
 
-    # warm-up (eager), also sets kernel attributes before any capture
+    # warm-up (eager), also sets kernel attributes before any capture.  NVTX ranges name the
+    # bench's parts for a timeline profiler
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push("bench/warmup")
     for s in range(args.warmup):
         run.step(sets[s % nsets])
     torch.cuda.synchronize()
+    nvtx.range_pop()
 
     # capture one graph per input set
     graphs = []
@@ -325,6 +329,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nvtx.range_push("bench/timed")
     tw0 = time.time()
     ev0.record()
     for s in range(args.steps):
@@ -335,6 +340,7 @@ def run_ours(args, rank, world, local_rank):
     ev1.record()
     torch.cuda.synchronize()
     tw1 = time.time()
+    nvtx.range_pop()
     barrier()
     ms_max = max_over_ranks(ev0.elapsed_time(ev1), device)
 
@@ -343,11 +349,13 @@ def run_ours(args, rank, world, local_rank):
     ph_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
     st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     torch.cuda.synchronize()
+    nvtx.range_push("bench/phases")
     tp0 = time.time()
     for s in range(args.steps):
         run.step(sets[s % nsets], events=ph_ev[s], step_events=st_ev[s])
     torch.cuda.synchronize()
     tp1 = time.time()
+    nvtx.range_pop()
     phase_ms = {name: sum(ph_ev[s][p].elapsed_time(ph_ev[s][p + 1]) for s in range(args.steps)) / args.steps
                 for p, name in enumerate(binding.PHASE_NAMES)}
     phase_ms["decode_step"] = sum(st_ev[s][0].elapsed_time(st_ev[s][1]) for s in range(args.steps)) / args.steps
@@ -369,6 +377,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     up_done, comp_done, down_done = [None] * args.steps, [None] * args.steps, [None] * args.steps
+    nvtx.range_push("bench/e2e")
     te0 = time.time()
     e0.record(stream)
     for st in (s_up, s_comp, s_down):
@@ -401,6 +410,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     te1 = time.time()
+    nvtx.range_pop()
     clocks.stop()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
 
@@ -470,7 +480,9 @@ def run_ours(args, rank, world, local_rank):
         "peaks": {"hbm_gbs": bw, "bf16_tflops": tc, "source": peaks["source"]},
     }
     if args.extras and rank == 0:
+        nvtx.range_push("bench/extras")
         out["workloads"] = extras(device, peaks)
+        nvtx.range_pop()
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
     graphs.clear()

@@ -179,3 +179,30 @@ def test_slstm_batch_per_cluster_rejects_unsupported(lib):
     assert lib.slstm_batch_per_cluster(4, 2, 48, 0) == 0
     assert lib.slstm_batch_per_cluster(4, 0, 64, 0) == 0
     assert lib.slstm_batch_per_cluster(4, 2, 64, 5) == 0
+
+
+# ---------------------------------------------------------------- launch failures (no GPU)
+# On a machine without a CUDA device every launch fails.  Calls with valid arguments must then
+# return MLSTM_ERR_CUDA (4) through the launch-error path instead of crashing; the fake device
+# pointers are never dereferenced on the host.  Skipped where a device is present, since there
+# the fake pointers would reach real kernels.
+def _no_device():
+    import torch
+    return not torch.cuda.is_available()
+
+
+@pytest.mark.skipif(not _no_device(), reason="needs a machine without a CUDA device")
+@pytest.mark.parametrize("over", [
+    dict(),                                        # tensor-core path (bf16, d 64, chunk 64)
+    dict(dt=binding.MLSTM_F32, chunk=16),          # fp32 CUDA-core path
+    dict(S=5000, DHQK=128, DHV=128, chunk=128),    # gate preprocessing in two kernels
+])
+def test_fwd_reports_launch_failure(lib, over):
+    assert call_fwd(lib, fwd_args(**over)) == 4
+
+
+@pytest.mark.skipif(not _no_device(), reason="needs a machine without a CUDA device")
+def test_step_and_slstm_report_launch_failure(lib):
+    assert call_step(lib, step_args()) == 4
+    assert call_slstm(lib, slstm_args()) == 4
+    assert lib.slstm_batch_per_cluster(4, 2, 64, 0) == 0      # no device to size the clusters for
