@@ -40,7 +40,7 @@ def _worker(rank, world, port, results):
 
 def test_max_over_ranks_and_whole_job_value():
     world = 2
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         results = man.dict()
         mp.spawn(_worker, args=(world, _free_port(), results), nprocs=world, join=True)
         res = dict(results)

@@ -105,7 +105,7 @@ def _worker(rank, world, port, S, results):
 @pytest.mark.parametrize("world", [2, 3])
 def test_sequence_parallel_protocol_on_cpu_ranks(world):
     S = 12 * world
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         results = man.dict()
         mp.spawn(_worker, args=(world, _free_port(), S, results), nprocs=world, join=True)
         res = dict(results)
