@@ -5,6 +5,10 @@ this package.  The CUDA library and its binding never do.  The arithmetic lives
 in ``mlstm_oracle.c`` (plain C, double precision, one head at a time, token by
 token); this module compiles it with gcc and marshals numpy arrays.
 
+Two more modules live beside it, for the library's other entry points: ``oracle.slstm`` (the
+sLSTM cell's recurrence, numpy float64) and ``oracle.mlstm_bwd`` (gradients of the forward pass,
+float64 torch autograd of the plain recurrence).
+
 Layouts follow the library: q, k ``[B, NH, T, DHQK]``; v, o ``[B, NH, T, DHV]``;
 gates ``[B, NH, T]``; state C ``[B, NH, DHQK, DHV]``, n ``[B, NH, DHQK]``,
 m ``[B, NH]``.  Inputs are converted to float32 (exact for fp32 and bf16
