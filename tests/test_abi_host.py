@@ -206,3 +206,51 @@ def test_step_and_slstm_report_launch_failure(lib):
     assert call_step(lib, step_args()) == 4
     assert call_slstm(lib, slstm_args()) == 4
     assert lib.slstm_batch_per_cluster(4, 2, 64, 0) == 0      # no device to size the clusters for
+
+
+# ---------------------------------------------------------------- sequence-parallel pieces, profiled fwd
+def test_log_decay_sum_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+    assert lib.mlstm_log_decay_sum(v(FAKE), -1, 2, 8, v(FAKE), None) == 1
+    assert lib.mlstm_log_decay_sum(v(FAKE), 1, 2, -8, v(FAKE), None) == 1
+    assert lib.mlstm_log_decay_sum(v(FAKE), 1, 2, 8, None, None) == 1          # no output
+    assert lib.mlstm_log_decay_sum(None, 1, 2, 8, v(FAKE), None) == 1          # tokens but no gates
+    assert lib.mlstm_log_decay_sum(None, 0, 2, 8, None, None) == 0             # no heads: no launch
+
+
+def _prefix(lib, **over):
+    a = dict(Cp=FAKE, np_=FAKE, mp=FAKE, gp=FAKE, R=2, rank=1, B=1, NH=2, DK=64, DV=64, C0=FAKE, n0=FAKE, m0=FAKE)
+    a.update(over)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return lib.mlstm_state_prefix(v(a["Cp"]), v(a["np_"]), v(a["mp"]), v(a["gp"]), a["R"], a["rank"], a["B"],
+                                  a["NH"], a["DK"], a["DV"], v(a["C0"]), v(a["n0"]), v(a["m0"]), None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(R=0), 1), (dict(rank=2), 1), (dict(rank=-1), 1), (dict(B=-1), 1),
+    (dict(DK=12), 2), (dict(DV=1024), 2), (dict(C0=None), 1), (dict(m0=None), 1),
+    (dict(Cp=None), 1), (dict(gp=None), 1), (dict(C0=FAKE + 4), 1), (dict(Cp=FAKE + 8), 1),
+])
+def test_state_prefix_rejects_bad_arguments(lib, over, expect):
+    assert _prefix(lib, **over) == expect
+
+
+def test_state_prefix_empty_batch_is_a_no_op(lib):
+    assert _prefix(lib, B=0, C0=None, n0=None, m0=None) == 0
+
+
+def test_final_state_checks_only_the_inputs_it_reads(lib):
+    v = ctypes.c_void_p
+    args = lambda k, vv, i, f, ws, wsb: lib.mlstm_fwd_final_state(k, vv, i, f, binding.MLSTM_BF16, 1, 2, 128, 64, 64,
+                                                                     64, None, None, None, ws, wsb, None)
+    assert args(None, v(FAKE), v(FAKE), v(FAKE), v(FAKE), 1 << 40) == 1        # k missing
+    assert args(v(FAKE + 4), v(FAKE), v(FAKE), v(FAKE), v(FAKE), 1 << 40) == 1 # k misaligned
+    assert args(v(FAKE), v(FAKE), v(FAKE), v(FAKE), None, 1 << 40) == 3        # no workspace
+
+
+def test_profiled_needs_the_event_array(lib):
+    a = fwd_args()
+    st = lib.mlstm_fwd_profiled(a["q"], a["k"], a["v"], a["ig"], a["fg"], a["og"], a["dt"], a["B"], a["NH"], a["S"],
+                                a["DHQK"], a["DHV"], a["chunk"], a["h"], a["C"], a["n"], a["m"], a["ws"], a["wsb"],
+                                a["stream"], None)
+    assert st == 1
