@@ -36,6 +36,10 @@
 //    cancellation in the denominator, and the fp16 inter-chunk product keeps
 //    inputs with one dominant token (huge input gates) within the error budget.
 //
+//    At chunk 64 the inter-chunk product instead reads the fp32 state in TMEM
+//    directly as a tf32 operand (kind::tf32, Q' in fp32 shared memory), so no
+//    fp16 copy Cb is made per chunk.
+//
 //    The state in TMEM is kept in a lazily rescaled frame: TMEM holds
 //    X = Cbar exp(-rho) (Cbar the unstabilized state), the chunk decay is folded
 //    into rho instead of rescaling TMEM, and new tokens enter with weight
