@@ -141,3 +141,68 @@ def test_sigmoid_helpers_are_stable():
     assert np.all(np.isfinite(ls))
     assert ls[2] == -math.log(2.0)
     assert ls[0] == -800.0 and ls[4] == 0.0
+
+
+# ---------------------------------------------------------------- planted mistakes
+# Mutated copies of the oracle (one plausible slip each) must fail at least one pin.
+
+MUTATIONS = {
+    "transposed_R": ('rec = np.einsum("egjk,bek->bgej", R, h)', 'rec = np.einsum("egkj,bek->bgej", R, h)'),
+    "heads_mix": ('rec = np.einsum("egjk,bek->bgej", R, h)', 'rec = np.einsum("egjk,bfk->bgej", R, h)'),
+    "forget_ignores_stabilizer": ("fw = np.exp(lf + m - m_new)", "fw = np.exp(lf)"),
+    "normalizer_drops_input": ("n = fw * n + iw", "n = fw * n + 1.0"),
+    "no_tanh_on_z": ("c = fw * c + iw * np.tanh(zg)", "c = fw * c + iw * zg"),
+    "raw_output_gate": ("h = sigmoid(og) * c / n", "h = og * c / n"),
+    "sigmoid_forget_as_exp": ('lf = fg if forget == "exp" else log_sigmoid(fg)', "lf = fg"),
+}
+
+
+def pin_errors(run):
+    """Largest deviation of each pin for an implementation `run` with slstm_run's signature."""
+    errs = {}
+    for name in ("slstm_hand_mixing_three_steps.json", "slstm_hand_sigmoid_forget.json"):
+        g = json.load(open(os.path.join(GOLDEN, name)))
+        wx = np.asarray(g["wx"], dtype=np.float32)[None]
+        h_seq, (c, n, m, h) = run(wx, np.asarray(g["R"], dtype=np.float32), forget=g["forget"])
+        errs[name] = max(np.abs(h_seq[0, :, 0] - np.asarray(g["h_expected"])).max(),
+                         np.abs(c[0, 0] - g["c_expected"]).max(), np.abs(n[0, 0] - g["n_expected"]).max())
+    rng = np.random.default_rng(2)
+    B, S, NH, DH = 1, 12, 2, 4
+    wx = _rand((B, S, 4, NH, DH), rng, scale=0.8)
+    R = _rand((NH, 4, DH, DH), rng, scale=0.3)
+    for forget in ("exp", "sigmoid"):
+        h_seq, _ = run(wx, R, forget=forget)
+        w64, R64 = wx.astype(np.float64), R.astype(np.float64)
+        c = np.zeros((B, NH, DH))
+        n = np.zeros((B, NH, DH))
+        h = np.zeros((B, NH, DH))
+        worst = 0.0
+        for t in range(S):
+            pre = w64[:, t].copy()
+            for e in range(NH):
+                for g in range(4):
+                    pre[:, g, e] += h[:, e] @ R64[e, g].T
+            F = np.exp(pre[:, 1]) if forget == "exp" else 1.0 / (1.0 + np.exp(-pre[:, 1]))
+            c = F * c + np.exp(pre[:, 0]) * np.tanh(pre[:, 2])
+            n = F * n + np.exp(pre[:, 0])
+            h = c / n / (1.0 + np.exp(-pre[:, 3]))
+            worst = max(worst, np.abs(h_seq[:, t] - h).max())
+        errs["unstabilized_" + forget] = worst
+    return errs
+
+
+def test_pins_hold_for_the_oracle():
+    errs = pin_errors(slstm_run)
+    assert max(errs.values()) <= 1e-6, errs
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(mutation):
+    import oracle.slstm as mod
+    src = open(mod.__file__).read()
+    old, new = MUTATIONS[mutation]
+    assert src.count(old) == 1, "mutation anchor not found: %s" % old
+    ns = {"__name__": "slstm_mutant"}
+    exec(compile(src.replace(old, new), "slstm_mutant.py", "exec"), ns)
+    errs = pin_errors(ns["slstm_run"])
+    assert max(errs.values()) > 1e-4, (mutation, errs)
