@@ -12,9 +12,10 @@ n_t = f' n_{t-1} + i' k_t, h_t = o_t * (C_t^T qh_t) / max(|n_t . qh_t|, exp(-m_t
 qh = q / sqrt(DHQK), from the zero state.  It is written here token by token with plain torch
 float64 operations, and the gradients of a loss L = sum(dh * h) with respect to q, k, v, i~, f~
 and o are torch.autograd's derivatives of exactly that computation (the library primitive that
-differentiates it; no step is reordered or fused).  h does not depend on the stabilizer except
-through the floor, which in unstabilized terms is max(|nbar . qh|, 1): the gradient through m
-cancels wherever the max picks |n . qh| and is the floor's own derivative elsewhere.
+differentiates it; no step is reordered or fused).  h does not depend on the stabilizer: in
+unstabilized terms h = o * (Cbar^T qh) / max(|nbar . qh|, 1), so the gradient paths through m
+cancel (holding m fixed gives the same gradient).  The derivative of the max in the denominator
+is taken on the branch the forward pass picked.
 
 Pins (tests/test_oracle_bwd_pins.py): central finite differences of the C oracle's forward pass;
 dL/do = dh * h / o (h is linear in o); dL/dv from the causal decay matrix of the guide's dual

@@ -108,3 +108,60 @@ def test_value_gradient_from_the_dual_form(scale):
             W[t] /= max(abs(W[t].sum()), 1.0)
         dv_ref[0, hd] = W.T @ (dhn[0, hd] * on[0, hd])
     assert np.abs(grads[2] - dv_ref).max() <= 1e-11 * np.abs(dv_ref).max()
+
+
+# ---------------------------------------------------------------- planted mistakes
+# Mutated copies of the gradient oracle must fail at least one of the checks below: a slip in the
+# forward shows against the C oracle, a cut gradient path against finite differences.  (Cutting
+# the gradient through the stabilizer m is not a slip: h does not depend on m, so the gradient
+# with m held fixed is the same.)
+
+MUTATIONS = {
+    "denominator_detached": ("den = torch.maximum(torch.abs((n * qh[..., t, :]).sum(-1)), torch.exp(-m_new))",
+                             "den = torch.maximum(torch.abs((n * qh[..., t, :]).sum(-1)), torch.exp(-m_new)).detach()"),
+    "no_q_scale": ("qh = q / math.sqrt(dk)", "qh = q"),
+    "raw_forget_gate": ("lf = torch.nn.functional.logsigmoid(fgate)", "lf = fgate"),
+    "normalizer_detached": ("n = fw[..., None] * n + iw[..., None] * k[..., t, :]",
+                            "n = (fw[..., None] * n + iw[..., None] * k[..., t, :]).detach()"),
+}
+
+
+def _worst_check(mod):
+    """Largest relative deviation of the forward check and of finite differences (both branches)."""
+    (q, k, v, i, f, o), _ = _inputs(1, 2, 9, 3, 2, seed=11)
+    hc, _, _, _ = oracle.run(q, k, v, i, f, o, nthreads=1)
+    worst = np.abs(mod.mlstm_fwd64(q, k, v, i, f, o) - hc).max() / np.abs(hc).max()
+    for scale in (1.5, 0.02):
+        (q, k, v, i, f, o), dh = _inputs(1, 1, 5, 3, 2, seed=7, scale=scale)
+        xs = [q, k, v, i, f, o]
+        grads = mod.mlstm_bwd(q, k, v, i, f, o, dh)
+
+        def loss(ys):
+            with torch.no_grad():
+                return float((mod.forward(*ys) * dh).sum())
+        eps = 1e-6
+        for idx, x in enumerate(xs):
+            for j in range(x.numel()):
+                xp = [y.clone() for y in xs]
+                xm = [y.clone() for y in xs]
+                xp[idx].reshape(-1)[j] += eps
+                xm[idx].reshape(-1)[j] -= eps
+                fd = (loss(xp) - loss(xm)) / (2 * eps)
+                g = grads[idx].reshape(-1)[j]
+                worst = max(worst, abs(g - fd) / max(1.0, abs(fd)))
+    return worst
+
+
+def test_checks_pass_for_the_oracle():
+    assert _worst_check(mlstm_bwd) <= 1e-6
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(mutation):
+    src = open(mlstm_bwd.__file__).read()
+    old, new = MUTATIONS[mutation]
+    assert src.count(old) == 1, "mutation anchor not found: %s" % old
+    import types
+    mod = types.ModuleType("mlstm_bwd_mutant")
+    exec(compile(src.replace(old, new), "mlstm_bwd_mutant.py", "exec"), mod.__dict__)
+    assert _worst_check(mod) > 1e-4, mutation
