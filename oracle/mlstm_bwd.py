@@ -17,9 +17,10 @@ unstabilized terms h = o * (Cbar^T qh) / max(|nbar . qh|, 1), so the gradient pa
 cancel (holding m fixed gives the same gradient).  The derivative of the max in the denominator
 is taken on the branch the forward pass picked.
 
-Pins (tests/test_oracle_bwd_pins.py): central finite differences of the C oracle's forward pass;
-dL/do = dh * h / o (h is linear in o); dL/dv from the causal decay matrix of the guide's dual
-form (h is linear in v for fixed gates, q and k); the forward part against the C oracle.
+Pins (tests/test_oracle_bwd_pins.py): the forward part against the C oracle; central finite
+differences of that forward pass for every input; dL/do = dh * h / o (h is linear in o); dL/dv
+from the causal decay matrix of the guide's dual form (h is linear in v for fixed gates, q and
+k); planted mistakes that must fail them.
 """
 from __future__ import annotations
 
