@@ -59,20 +59,9 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 
-def tc_num_segments(BH: int, DHV: int, NC: int) -> int:
-    """Segments per head of the tensor-core path (mirrors the library's planner)."""
-    ctas_per_seg = BH * (DHV // 128)
-    best, best_cost = 1, None
-    for nseg in range(1, min(NC, 256) + 1):
-        R = -(-NC // nseg)
-        ns = -(-NC // R)
-        if ns != nseg:
-            continue
-        rounds = -(-(ctas_per_seg * ns) // 148)
-        cost = rounds * (R + 1) * 100 + ns
-        if best_cost is None or cost < best_cost:
-            best, best_cost = ns, cost
-    return best
+def segments(w: Workload) -> int:
+    """Segments per head of the library's tensor-core path for the workload (its own planner)."""
+    return binding.fwd_segments(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.torch_dtype)
 
 
 def fwd_work(w: Workload, tensor_path: bool):
@@ -90,7 +79,7 @@ def fwd_work(w: Workload, tensor_path: bool):
     dk, dv, L = w.DHQK, w.DHV, w.chunk
     heads = w.B * w.NH
     NC = math.ceil(w.S / L)
-    nstate = tc_num_segments(heads, dv, NC) if tensor_path else NC
+    nstate = segments(w) if tensor_path else NC
     state = heads * nstate * 4 * (dk * dv + dk)
     in_bytes = tok * (e * (2 * dk + dv) + (e * dv if w.ogate else 0) + 8)
     out_bytes = tok * e * dv + heads * 4 * (dk * dv + dk + 1)

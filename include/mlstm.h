@@ -202,6 +202,14 @@ int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV, int chunk
 int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt);
 
 /*
+ * Segments per head that mlstm_fwd's tensor-core path cuts the sequence into for
+ * this shape (each segment's contribution is one long GEMM; the walk runs one
+ * CTA per segment and 128 value columns), or 0 when the shape does not take the
+ * tensor-core path or has no tokens.  No GPU work; a host-side query.
+ */
+int mlstm_fwd_segments(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
+
+/*
  * Reports whether the last mlstm_fwd that used `workspace` ran to completion:
  * synchronizes `stream`, reads the status word kept in the workspace and
  * returns MLSTM_OK or MLSTM_ERR_TIMEOUT (a bounded device-side wait gave up;

@@ -12,8 +12,7 @@ from xlstm_mlstm_cell_b200.workloads import WORKLOADS
 def _walk_bytes_per_token_head(w):
     fw = bench.fwd_work(w, True)
     heads = w.B * w.NH
-    NC = -(-w.S // w.chunk)
-    nseg = bench.tc_num_segments(heads, w.DHV, NC)
+    nseg = bench.segments(w)
     state = heads * nseg * 4 * (w.DHQK * w.DHV + w.DHQK)
     return (fw["phases"]["outputs"]["bytes"] - state) / (heads * w.S)
 
@@ -46,13 +45,22 @@ def test_slstm_work():
 
 
 def test_segment_planner_fills_whole_waves():
-    # the bench workload: 16 heads x 2 value tiles, 32 chunks: four segments of eight chunks fill
-    # 128 of the 148 SMs in one wave
-    assert bench.tc_num_segments(16, 256, 32) == 4
-    for BH, DHV, NC in [(8, 512, 128), (8, 512, 1024), (1, 128, 8), (64, 512, 64)]:
-        ns = bench.tc_num_segments(BH, DHV, NC)
+    # the library's planner (a host query): the bench workload's 16 heads x 2 value tiles and 32
+    # chunks take four segments of eight chunks, 128 CTAs on the 148 SMs in one wave
+    assert bench.segments(WORKLOADS["fwd_bf16_d256"]) == 4
+    from xlstm_mlstm_cell_b200 import binding
+    import torch
+    for B, NH, S, DK, DV, L in [(1, 8, 8192, 256, 512, 64), (1, 8, 131072, 256, 512, 128), (1, 1, 512, 64, 128, 64),
+                                (8, 8, 4096, 128, 512, 64), (2, 3, 333, 256, 256, 64)]:
+        ns = binding.fwd_segments(B, NH, S, DK, DV, L, torch.bfloat16)
+        NC = -(-S // L)
         R = -(-NC // ns)
         assert 1 <= ns <= min(NC, 256) and -(-NC // R) == ns
+    # off the tensor-core path, or nothing to compute
+    assert binding.fwd_segments(1, 8, 8192, 256, 512, 64, torch.float32) == 0
+    assert binding.fwd_segments(1, 8, 8192, 96, 512, 64, torch.bfloat16) == 0
+    assert binding.fwd_segments(0, 8, 8192, 256, 512, 64, torch.bfloat16) == 0
+    assert binding.fwd_segments(1, 8, 0, 256, 512, 64, torch.bfloat16) == 0
 
 
 def test_workload_overrides_for_captures():

@@ -36,6 +36,7 @@ SIGNATURES = {
                                _vp]),
     "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_fwd_tensor_path": (_i, [_i, _i, _i, _i]),
+    "mlstm_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_step": (_i, [_fp, _fp, _fp, _vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "mlstm_status_string": (ctypes.c_char_p, [_i]),
     "mlstm_fwd_final_state": (_i, [_vp, _vp, _fp, _fp, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _fp, _vp, _sz, _vp]),
@@ -110,6 +111,12 @@ def fwd_tensor_path(DHQK, DHV, chunk, dtype) -> int:
     """1: tensor-core path, 0: fp32 CUDA-core path, -1: unsupported (mlstm_fwd_tensor_path)."""
     dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
     return int(load().mlstm_fwd_tensor_path(DHQK, DHV, chunk, dt))
+
+
+def fwd_segments(B, NH, S, DHQK, DHV, chunk, dtype) -> int:
+    """Segments per head of the tensor-core path for this shape (0 off that path)."""
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().mlstm_fwd_segments(B, NH, S, DHQK, DHV, chunk, dt))
 
 
 def alloc_workspace(B, NH, S, DHQK, DHV, chunk, dtype, device="cuda") -> torch.Tensor:

@@ -101,6 +101,15 @@ extern "C" int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype d
     return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 1 : 0;
 }
 
+extern "C" int mlstm_fwd_segments(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if (B < 0 || NH < 0 || S < 0 || mlstm_fwd_tensor_path(DHQK, DHV, chunk, dt) != 1) return 0;
+    if ((long long)B * NH > (1LL << 30) || B * NH == 0 || S == 0) return 0;
+    FwdWorkspace w;
+    plan_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, true, &w);
+    return w.NSEG;
+}
+
 namespace {
 
 mlstm_status fwd_impl(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
