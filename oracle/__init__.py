@@ -74,11 +74,13 @@ def _ptr(a, t):
 
 
 def run(q, k, v, igate, fgate, ogate=None, C=None, n=None, m=None,
-        want_h: bool = True, nthreads: int = 0, lib=None):
+        want_h: bool = True, nthreads: int = 0, lib=None, inplace: bool = False):
     """Runs the recurrence over the T tokens of the inputs from state (C, n, m).
 
     A missing state is the zero state (C = 0, n = 0, m = 0).  Returns
-    ``(h, C, n, m)`` in float64 (h is None when ``want_h`` is False).
+    ``(h, C, n, m)`` in float64 (h is None when ``want_h`` is False).  With
+    ``inplace`` the given state arrays (float64, C-contiguous numpy) are updated
+    in place and returned instead of copied first (large decode states).
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     ig, fg, og = _f32(igate), _f32(fgate), _f32(ogate)
@@ -87,9 +89,14 @@ def run(q, k, v, igate, fgate, ogate=None, C=None, n=None, m=None,
     assert k.shape == (B, NH, T, dk) and v.shape == (B, NH, T, dv)
     assert ig.shape == (B, NH, T) and fg.shape == (B, NH, T)
     assert og is None or og.shape == (B, NH, T, dv)
-    Cs = np.zeros((B, NH, dk, dv)) if C is None else np.array(C, dtype=np.float64, order="C")
-    ns = np.zeros((B, NH, dk)) if n is None else np.array(n, dtype=np.float64, order="C")
-    ms = np.zeros((B, NH)) if m is None else np.array(m, dtype=np.float64, order="C")
+    def state(x, shape):
+        if x is None:
+            return np.zeros(shape)
+        if inplace:
+            assert isinstance(x, np.ndarray) and x.dtype == np.float64 and x.flags["C_CONTIGUOUS"]
+            return x
+        return np.array(x, dtype=np.float64, order="C")
+    Cs, ns, ms = state(C, (B, NH, dk, dv)), state(n, (B, NH, dk)), state(m, (B, NH))
     assert Cs.shape == (B, NH, dk, dv) and ns.shape == (B, NH, dk) and ms.shape == (B, NH)
     h = np.empty((B, NH, T, dv)) if want_h else None
     rc = (lib or _load()).oracle_mlstm_run(B * NH, T, dk, dv, _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p),
@@ -106,14 +113,15 @@ def mlstm_fwd(q, k, v, igate, fgate, ogate=None, nthreads: int = 0):
     return run(q, k, v, igate, fgate, ogate, nthreads=nthreads)
 
 
-def mlstm_step(C, n, m, q, k, v, igate, fgate, ogate=None, nthreads: int = 0):
+def mlstm_step(C, n, m, q, k, v, igate, fgate, ogate=None, nthreads: int = 0, inplace: bool = False):
     """One decode step on a state; token inputs are ``[B, NH, D]`` and ``[B, NH]``.
 
-    Returns ``(h [B, NH, DHV], C', n', m')``.
+    Returns ``(h [B, NH, DHV], C', n', m')`` (with ``inplace``, the given float64 state arrays,
+    updated).
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     og = _f32(ogate)
     h, C2, n2, m2 = run(q[:, :, None], k[:, :, None], v[:, :, None],
                         _f32(igate)[:, :, None], _f32(fgate)[:, :, None],
-                        None if og is None else og[:, :, None], C, n, m, nthreads=nthreads)
+                        None if og is None else og[:, :, None], C, n, m, nthreads=nthreads, inplace=inplace)
     return h[:, :, 0], C2, n2, m2

@@ -34,3 +34,22 @@ def assert_close(name: str, x, ref, tol: float):
     assert np.all(np.isfinite(to64(x))), "%s has non-finite values" % name
     assert err <= tol, "%s: rel-L2 %.3e > %.1e" % (name, err, tol)
     return err
+
+
+class L2Acc:
+    """Relative L2 error of a tensor compared piece by piece (sum of squared differences and of
+    squared reference values over the pieces), for outputs too large to hold twice in fp64."""
+
+    def __init__(self):
+        self.diff = 0.0
+        self.ref = 0.0
+
+    def add(self, x, ref):
+        x, ref = to64(x), to64(ref)
+        assert x.shape == ref.shape, (x.shape, ref.shape)
+        assert np.all(np.isfinite(x)), "non-finite values"
+        self.diff += float(np.sum(np.square(x - ref)))
+        self.ref += float(np.sum(np.square(ref)))
+
+    def rel(self) -> float:
+        return float(np.sqrt(self.diff) / np.sqrt(self.ref)) if self.ref > 0 else float(np.sqrt(self.diff))

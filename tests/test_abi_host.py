@@ -53,6 +53,9 @@ def test_workspace_size(lib):
     assert lib.mlstm_fwd_workspace_size(-1, 8, 8192, 256, 512, 64, binding.MLSTM_BF16) == 0
     assert lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 512, 64, 7) == 0                    # dtype
     assert lib.mlstm_fwd_workspace_size(1, 8, 0, 256, 512, 64, binding.MLSTM_BF16) > 0
+    # beyond the sizes mlstm_fwd accepts (B * NH > 2^30, which would also overflow an int): 0
+    assert lib.mlstm_fwd_workspace_size(1 << 16, 1 << 15, 64, 64, 64, 64, binding.MLSTM_BF16) == 0
+    assert lib.mlstm_fwd_workspace_size(1 << 15, 1 << 15, 64, 64, 64, 64, binding.MLSTM_BF16) > 0
 
 
 FAKE = 1 << 20   # a 16-byte-aligned non-NULL address that is never dereferenced
@@ -254,3 +257,42 @@ def test_profiled_needs_the_event_array(lib):
                                 a["DHQK"], a["DHV"], a["chunk"], a["h"], a["C"], a["n"], a["m"], a["ws"], a["wsb"],
                                 a["stream"], None)
     assert st == 1
+
+
+# ---------------------------------------------------------------- concurrent host callers (no GPU)
+@pytest.mark.skipif(not _no_device(), reason="needs a machine without a CUDA device")
+def test_concurrent_host_callers(lib):
+    """Eight host threads call the library at once (ctypes releases the GIL): the host-side caches
+    (per-kernel shared-memory limits, the tensor-map encoder, the sLSTM cluster capacity, the
+    no-alloc array's address) are filled under a lock, and every call returns its status."""
+    import threading
+    results, errors = [], []
+
+    def worker(tid):
+        try:
+            for it in range(20):
+                ws = lib.mlstm_fwd_workspace_size(1, 8, 4096 + tid, 256, 512, 64, binding.MLSTM_BF16)
+                assert ws > 0 and ws % 256 == 0
+                r = [call_fwd(lib, fwd_args()),
+                     call_fwd(lib, fwd_args(dt=binding.MLSTM_F32, chunk=16)),
+                     call_fwd(lib, fwd_args(DHQK=256, DHV=512, chunk=128)),
+                     call_step(lib, step_args()),
+                     call_slstm(lib, slstm_args(DH=32 << (it % 4))),
+                     lib.mlstm_fwd_noalloc_status(None)]
+                results.append(tuple(r))
+        except Exception as e:   # noqa: BLE001 - reported below
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(t,)) for t in range(8)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    assert len(results) == 8 * 20
+    assert set(results) == {(4, 4, 4, 4, 4, 4)}
+
+
+@pytest.mark.skipif(not _no_device(), reason="needs a machine without a CUDA device")
+def test_noalloc_status_without_device(lib):
+    assert lib.mlstm_fwd_noalloc_status(None) == 4

@@ -9,18 +9,32 @@ import bench
 from xlstm_mlstm_cell_b200.workloads import WORKLOADS
 
 
-def _walk_bytes_per_token_head(w):
-    fw = bench.fwd_work(w, True)
-    heads = w.B * w.NH
-    nseg = bench.segments(w)
-    state = heads * nseg * 4 * (w.DHQK * w.DHV + w.DHQK)
-    return (fw["phases"]["outputs"]["bytes"] - state) / (heads * w.S)
-
-
 def test_walk_bytes_per_token_and_head():
-    # q, k, v (and o) read, h written, 12 bytes of gate values: 2 (2 dk + dv) + 2 dv [o] + 2 dv + 12
-    assert _walk_bytes_per_token_head(WORKLOADS["fwd_bf16_d256"]) == 2 * (512 + 256) + 2 * 256 + 12
-    assert _walk_bytes_per_token_head(WORKLOADS["fwd_bf16_7b"]) == 4108
+    # the per-token figure of the algorithmic bytes: q, k, v (and o) read, h written, two gate
+    # pre-activations read: 2 (2 dk + dv) + 2 dv [o] + 2 dv + 8
+    assert bench.bytes_per_token_head(WORKLOADS["fwd_bf16_d256"]) == 2 * (512 + 256) + 2 * 256 + 8
+    assert bench.bytes_per_token_head(WORKLOADS["fwd_bf16_7b"]) == 4104
+    w = WORKLOADS["fwd_bf16_long"]
+    assert bench.bytes_per_token_head(w) == 4104
+    fw = bench.fwd_work(w, True)
+    tok = w.B * w.NH * w.S
+    # the walk's algorithmic bytes are that figure times the token-heads of one launch: 4.30 GB at
+    # 131072 tokens x 8 heads; the segment states it reads are reported apart, not counted
+    assert fw["phases"]["outputs"]["bytes"] == 4104 * tok
+    assert abs(fw["phases"]["outputs"]["bytes"] / 1e9 - 4.303) < 1e-3
+    nseg = bench.segments(w)
+    assert fw["phases"]["outputs"]["state_traffic"] == w.B * w.NH * nseg * 4 * (256 * 512 + 256)
+    # the whole pass adds the final state written once
+    assert fw["bytes"] == 4104 * tok + w.B * w.NH * 4 * (256 * 512 + 256 + 1)
+
+
+def test_roofline_object():
+    peaks = {"hbm_gbs": 6452.8, "bf16_tflops": 1662.0, "source": "measured"}
+    r = bench.roofline({"bytes": 4.303e9, "flops": 6.5e11}, 1.0e-3, peaks, True)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - 4303.0) < 1e-6 and abs(r["frac"] - 4303.0 / 6452.8) < 1e-12
+    r = bench.roofline({"bytes": 1e6, "flops": 1.662e12}, 2.0e-3, peaks, True)
+    assert r["bound"] == "tensor" and abs(r["frac"] - 0.5) < 1e-12
 
 
 def test_forward_flops_per_token_and_head():
@@ -70,6 +84,8 @@ def test_workload_overrides_for_captures():
     assert dataclasses.replace(w, S=WORKLOADS["fwd_bf16_7b"].S, B=1) == WORKLOADS["fwd_bf16_7b"]
     args = argparse.Namespace(workload="fwd_bf16_d256", seq=0, batch=0)
     assert bench.workload_for(args) == WORKLOADS["fwd_bf16_d256"]
+    # the headline workload is the largest forward configuration
+    assert bench.DEFAULT_WORKLOAD == "fwd_bf16_long"
 
 
 def test_whole_job_throughput():

@@ -77,27 +77,24 @@ def prefill_state_full(w):
     return Cs, ns, ms
 
 
-def test_step_full_workload_sampled(cuda_lib):
+def test_step_full_workload(cuda_lib):
     """B256 NH8 d256/512 state from the oracle's 512-token prefill; 1000 steps on all 2048 heads.
 
-    h is compared at every step and the state after step 1000, on 16 seeded sampled heads.
+    h of every head is compared at every step, and the whole state after step 1000.
     """
     w = WORKLOADS["step_bf16"]
     Cs, ns, ms = prefill_state_full(w)
     Cg, ng, mg = (torch.from_numpy(x).cuda() for x in (Cs, ns, ms))
-    rng = np.random.default_rng(99)
-    flat = np.sort(rng.choice(w.B * w.NH, size=16, replace=False))
-    bi, hi = flat // w.NH, flat % w.NH
-    Cr, nr, mr = (x[bi, hi][:, None].astype(np.float64) for x in (Cs, ns, ms))   # [16, 1, ...]
+    Cr, nr, mr = (np.ascontiguousarray(x, dtype=np.float64) for x in (Cs, ns, ms))
+    del Cs
     tol = TOL[w.dtype]
     worst = 0.0
     for s in range(w.steps):
         q, k, v, i, f, o = make_step_inputs(w, s)
         h = binding.step(Cg, ng, mg, q.cuda(), k.cuda(), v.cuda(), i.cuda(), f.cuda(), o.cuda())
-        sel = lambda x: x[bi, hi][:, None]
-        hr, Cr, nr, mr = oracle.mlstm_step(Cr, nr, mr, sel(q), sel(k), sel(v), sel(i), sel(f), sel(o))
-        worst = max(worst, assert_close("h step %d" % s, h.cpu()[bi, hi][:, None], hr, tol))
+        hr, _, _, _ = oracle.mlstm_step(Cr, nr, mr, q, k, v, i, f, o, inplace=True)
+        worst = max(worst, assert_close("h step %d" % s, h.cpu(), hr, tol))
     torch.cuda.synchronize()
-    assert_close("C after %d steps" % w.steps, Cg.cpu()[bi, hi][:, None], Cr, tol)
-    assert_close("n after %d steps" % w.steps, ng.cpu()[bi, hi][:, None], nr, tol)
-    assert_close("m after %d steps" % w.steps, mg.cpu()[bi, hi][:, None], mr, tol)
+    assert_close("C after %d steps" % w.steps, Cg.cpu(), Cr, tol)
+    assert_close("n after %d steps" % w.steps, ng.cpu(), nr, tol)
+    assert_close("m after %d steps" % w.steps, mg.cpu(), mr, tol)

@@ -45,3 +45,15 @@ def test_noalloc_matches_fwd_on_two_calls_in_a_row(cuda_lib, B, NH, S, DK, DV, c
         for name, x, r in zip("hCnm", out, ref):
             err = rel_l2(x.cpu(), r.cpu())
             assert err <= TOL[dt], "call %d, %s: rel-L2 %.3e" % (call, name, err)
+
+
+@pytest.mark.gpu
+def test_noalloc_status_after_a_completed_call(cuda_lib):
+    """mlstm_fwd_noalloc_status reads the status word that the last no-alloc call left in the
+    built-in array: MLSTM_OK after a call that ran to completion."""
+    inputs = [None if x is None else x.cuda() for x in
+              make_custom(1, 2, 300, 128, 128, "bf16", seed=33, ig=(-1.0, 2.0), fg=(4.0, 1.0))]
+    binding.fwd_noalloc(*inputs, chunk=64)
+    assert binding.fwd_noalloc_status() == 0
+    binding.fwd_noalloc(*inputs, chunk=128)
+    assert binding.fwd_noalloc_status() == 0

@@ -34,6 +34,7 @@ SIGNATURES = {
     "mlstm_fwd_status": (_i, [_vp, _vp]),
     "mlstm_fwd_noalloc": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp,
                                _vp]),
+    "mlstm_fwd_noalloc_status": (_i, [_vp]),
     "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_fwd_tensor_path": (_i, [_i, _i, _i, _i]),
     "mlstm_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _i]),
@@ -240,6 +241,12 @@ def fwd_noalloc(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, 
                                _stream(stream))
     _check("mlstm_fwd_noalloc", st)
     return h_out, C_final, n_final, m_final
+
+
+def fwd_noalloc_status(stream=None) -> int:
+    """mlstm_fwd_noalloc_status: 0 when the last mlstm_fwd_noalloc on this device completed, else the
+    status code (MLSTM_ERR_TIMEOUT after a bounded wait gave up); synchronizes the stream."""
+    return int(load().mlstm_fwd_noalloc_status(_stream(stream)))
 
 
 def fwd_status(workspace, stream=None) -> int:

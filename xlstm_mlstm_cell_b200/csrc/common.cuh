@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #define MLSTM_DEVINL __device__ __forceinline__
 
 namespace mlstm {
@@ -87,8 +89,17 @@ inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// One lock for the library's host-side caches (the per-kernel shared-memory limits set so far,
+// the sLSTM kernel's cluster capacity, the tensor-map encoder), so that host threads may call the
+// library at the same time.  An inline function's static is one object across translation units.
+inline std::mutex &host_cache_mutex()
+{
+    static std::mutex m;
+    return m;
+}
+
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device), so that
-// launches stay free of attribute calls after the first one.
+// launches stay free of attribute calls after the first one.  Thread-safe.
 inline cudaError_t ensure_dynamic_smem(const void *kernel, int bytes)
 {
     struct Entry { const void *fn; int dev; int bytes; };
@@ -96,6 +107,7 @@ inline cudaError_t ensure_dynamic_smem(const void *kernel, int bytes)
     static int used = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    std::lock_guard<std::mutex> guard(host_cache_mutex());
     for (int i = 0; i < used; ++i)
         if (reg[i].fn == kernel && reg[i].dev == dev && reg[i].bytes >= bytes) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

@@ -17,6 +17,8 @@
 #include "mlstm.h"
 #include "mlstm_internal.h"
 
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 namespace {
@@ -25,11 +27,45 @@ constexpr size_t kScratchBytes = (size_t)MLSTM_FWD_NOALLOC_MAX_BYTES;
 
 __device__ __align__(256) unsigned char g_fwd_scratch[kScratchBytes];
 
+// The array's device address per device, with the identity of the context it was looked up in:
+// after the primary context is destroyed and created again (cudaDeviceReset), the module is
+// loaded anew and the address is looked up again.
+struct Slot {
+    void *ptr = nullptr;
+    unsigned long long ctx = 0;
+    bool ctx_known = false;
+};
 constexpr int kMaxDevices = 64;
-void *g_scratch_ptr[kMaxDevices] = {};
+Slot g_slots[kMaxDevices];
 std::mutex g_scratch_lock;
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Unique id of the context current on this thread (false when none is current or the driver
+// does not offer the query).
+bool current_context_id(unsigned long long *id)
+{
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {   // under g_scratch_lock
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+        looked_up = true;
+    }
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array on the current device: looked up with
+// cudaGetSymbolAddress the first time on a device (and again if that device's context has been
+// replaced since), then taken from the cache.
 cudaError_t scratch_address(void **out)
 {
     int dev = 0;
@@ -37,13 +73,22 @@ cudaError_t scratch_address(void **out)
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> guard(g_scratch_lock);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_fwd_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+    Slot &s = g_slots[dev];
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    if (s.ptr && s.ctx_known && have_id && s.ctx == id) {
+        *out = s.ptr;
+        return cudaSuccess;
     }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fwd_scratch);   // creates the device's primary context if needed
+    if (e != cudaSuccess) {
+        s = Slot();
+        return e;
+    }
+    s.ptr = p;
+    s.ctx_known = current_context_id(&s.ctx);
+    *out = p;
     return cudaSuccess;
 }
 
@@ -62,4 +107,11 @@ extern "C" mlstm_status mlstm_fwd_noalloc(const void *q, const void *k, const vo
     if (scratch_address(&scratch) != cudaSuccess) return MLSTM_ERR_CUDA;
     return mlstm_fwd(q, k, v, igate, fgate, ogate, dt, B, NH, S, DHQK, DHV, chunk, h_out, C_final, n_final,
                      m_final, scratch, kScratchBytes, stream);
+}
+
+extern "C" mlstm_status mlstm_fwd_noalloc_status(void *stream)
+{
+    void *scratch = nullptr;
+    if (scratch_address(&scratch) != cudaSuccess) return MLSTM_ERR_CUDA;
+    return mlstm_fwd_status(scratch, stream);
 }

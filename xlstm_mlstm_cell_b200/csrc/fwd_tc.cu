@@ -1193,9 +1193,11 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 // ---------------------------------------------------------------- host side
 
+// The driver's tensor-map encoder, looked up once (a failed lookup is retried on the next call).
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::lock_guard<std::mutex> guard(host_cache_mutex());
     if (!fn) {
         cudaDriverEntryPointQueryResult q;
         void *ptr = nullptr;

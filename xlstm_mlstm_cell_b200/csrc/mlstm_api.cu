@@ -82,6 +82,8 @@ extern "C" size_t mlstm_fwd_workspace_size(int B, int NH, int S, int DHQK, int D
 {
     if (B < 0 || NH < 0 || S < 0 || (dt != MLSTM_F32 && dt != MLSTM_BF16)) return 0;
     if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return 0;
+    // the limits mlstm_fwd applies: larger shapes are unsupported (and B * NH would overflow)
+    if ((long long)B * NH > (1LL << 30) || (long long)S * DHV > (1LL << 40)) return 0;
     return plan_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, dt == MLSTM_BF16, nullptr);
 }
 

@@ -321,7 +321,8 @@ static cudaError_t launch_bg(const void *wx, const void *R, int B, int S, int NH
                          static_cast<const T *>(R), B, S, NH, fs, c, n, m, h, static_cast<T *>(h_out), status);
 }
 
-// Clusters of this kernel that fit on the device at once (cached per kernel and device).
+// Clusters of this kernel that fit on the device at once (cached per kernel and device, under the
+// library's host-cache lock).
 template <typename T, int DH, int BG>
 static int max_clusters()
 {
@@ -330,6 +331,7 @@ static int max_clusters()
     static int used = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> guard(host_cache_mutex());
     for (int i = 0; i < used; ++i)
         if (cache[i].dev == dev) return cache[i].v;
     constexpr int G = DH / CELLS;
