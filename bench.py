@@ -637,6 +637,52 @@ def step_extra(device, peaks, nsteps: int = 200):
             "steps": nsteps, "roofline": roof}
 
 
+def bwd_work(w: Workload):
+    """Algorithmic work of one mlstm_bwd: per token and head the products of the chunkwise gradient
+    (the forward read-out recomputed, 2 dk dv; the chunk-start states recomputed, 2 dk dv; the
+    read-out's state gradient and the dq, dk, dv inter-chunk terms, 4 x 2 dk dv; the causal half of
+    the intra-chunk products, 3 (L + 1)(dk + dv)), i.e. 14 dk dv + 3 (L + 1)(dk + dv) flops; bytes:
+    q, k, v, o, dh and both gates read once, dq, dk, dv, do and both gate gradients written once."""
+    e = 4 if w.dtype == "f32" else 2
+    tok = w.B * w.NH * w.S
+    dk, dv, L = w.DHQK, w.DHV, w.chunk
+    flops = tok * (14 * dk * dv + 3 * (L + 1) * (dk + dv))
+    io = e * (2 * dk + dv) + (e * dv if w.ogate else 0) + e * dv + 8
+    out = e * (2 * dk + dv) + (e * dv if w.ogate else 0) + 8
+    return {"flops": flops, "bytes": tok * (io + out)}
+
+
+def bwd_extra(w: Workload, device, peaks, reps: int = 5):
+    """The backward pass on a forward workload's shape (dh ~ N(0, 1)), timed alone with events."""
+    s = device_inputs(w, 1, device, seed=w.seed)[0]
+    g = torch.Generator(device=device).manual_seed(w.seed + 1)
+    dh = torch.randn((w.B, w.NH, w.S, w.DHV), generator=g, device=device).to(w.torch_dtype)
+    ws = torch.empty(binding.bwd_workspace_size(w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk, w.torch_dtype),
+                     dtype=torch.uint8, device=device)
+    out = (torch.empty_like(s["q"]), torch.empty_like(s["k"]), torch.empty_like(s["v"]), torch.empty_like(s["i"]),
+           torch.empty_like(s["f"]), None if s["o"] is None else torch.empty_like(s["o"]))
+    call = lambda: binding.bwd(s["q"], s["k"], s["v"], s["i"], s["f"], s["o"], dh, chunk=w.chunk, workspace=ws, out=out)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / reps / 1e3
+    bw = bwd_work(w)
+    roof = roofline(bw, t, peaks, False)
+    roof["kernel"] = "mlstm_bwd (all kernels of the call)"
+    del s, dh, ws, out
+    torch.cuda.empty_cache()
+    return {"workload": "%s shape (B%d NH%d S%d d%d/%d chunk %d, %s)" % (w.name, w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk,
+                                                                        w.dtype),
+            "ms": t * 1e3, "tokens_per_s": w.B * w.S / t, "tflops": bw["flops"] / t / 1e12,
+            "kernel_launches": "gate preprocessing, chunk-start states, 4 backward kernels", "roofline": roof}
+
+
 def extras(device, peaks, skip=None):
     """Per-workload numbers for the other shapes (eager, events)."""
     res = {}
@@ -644,6 +690,7 @@ def extras(device, peaks, skip=None):
         if name != skip:
             res[name] = fwd_extra(WORKLOADS[name], device, peaks)
     res["step_bf16"] = step_extra(device, peaks)
+    res["bwd_bf16_7b"] = bwd_extra(WORKLOADS["fwd_bf16_7b"], device, peaks)
     res["slstm_f32"] = slstm_extra(device, peaks)
     return res
 
@@ -760,6 +807,8 @@ def main():
     ap.add_argument("--slstm", action="store_true",
                     help="time only the sLSTM recurrence workload (sizes from --batch / --seq) and print its numbers")
     ap.add_argument("--decode", action="store_true", help="time only the decode step workload and print its numbers")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time only the backward pass on the workload's shape (sizes from --batch / --seq)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -772,6 +821,10 @@ def main():
         run_reference(args, rank, world)
         return
     binding.load()
+    if args.bwd:
+        torch.cuda.set_device(local_rank)
+        print(json.dumps(bwd_extra(workload_for(args), torch.device("cuda", local_rank), load_peaks())))
+        return
     if args.slstm or args.decode:
         torch.cuda.set_device(local_rank)
         dev = torch.device("cuda", local_rank)

@@ -258,6 +258,37 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
                         void *h_out, void *stream);
 
 /*
+ * Backward pass of mlstm_fwd (from the zero state): the gradients of a loss
+ * L = sum over b, h, t, j of dh[b][h][t][j] * h[b][h][t][j] with respect to
+ * every input, the training form of the guide's "The Dual Formulation: How
+ * mLSTM Enables Parallel GPU Training" and "Exploit Chunkwise Hardware Kernels
+ * for Production Training".  The stabilizer m carries no gradient (h does not
+ * depend on it); at the denominator's max the derivative follows the branch
+ * the forward pass took.
+ *
+ * Inputs as for mlstm_fwd plus dh [B][NH][S][DHV] (type `dt`).  Outputs (device,
+ * 16-byte aligned, caller-owned): dq, dk [B][NH][S][DHQK] and dv [B][NH][S][DHV]
+ * in `dt`; digate, dfgate [B][NH][S] float32 (gradients of the pre-activations
+ * i~, f~); dogate [B][NH][S][DHV] in `dt` when ogate is non-NULL (required
+ * then; ignored when ogate is NULL).  No gradient flows into or out of the
+ * states: the sequence starts from the zero state and the final state is not
+ * part of L.  The forward pass is recomputed inside (gate preprocessing and
+ * the fp32 chunk-start states); every product is fp32 on the CUDA cores.
+ * Shapes and chunk sizes as for mlstm_fwd.
+ *
+ * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
+ * (it holds the chunk-start states and their gradients, 8 DHQK DHV bytes per
+ * chunk and head, plus 4 DHV + 2 chunk + 8 ceil(DHQK / 32) + 12 bytes per
+ * token and head).  Errors as for mlstm_fwd.
+ */
+size_t mlstm_bwd_workspace_size(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
+mlstm_status mlstm_bwd(const void *q, const void *k, const void *v,
+                       const float *igate, const float *fgate, const void *ogate, const void *dh,
+                       mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,
+                       void *dq, void *dk, void *dv, float *digate, float *dfgate, void *dogate,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * mlstm_fwd for callers that cannot allocate device memory.  The pages have no
  * counterpart to this entry point; it exists for callers that may not call
  * cudaMalloc or any allocating routine: code running inside a host framework

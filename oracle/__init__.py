@@ -5,9 +5,11 @@ this package.  The CUDA library and its binding never do.  The arithmetic lives
 in ``mlstm_oracle.c`` (plain C, double precision, one head at a time, token by
 token); this module compiles it with gcc and marshals numpy arrays.
 
-Two more modules live beside it, for the library's other entry points: ``oracle.slstm`` (the
-sLSTM cell's recurrence, numpy float64) and ``oracle.mlstm_bwd`` (gradients of the forward pass,
-float64 torch autograd of the plain recurrence).
+Beside it, for the library's other entry points: ``oracle.slstm`` (the sLSTM cell's recurrence,
+numpy float64), ``oracle.mlstm_bwd`` (gradients of the forward pass, float64 torch autograd of the
+plain recurrence) and ``mlstm_adjoint.c`` / ``mlstm_adjoint()`` (the same gradients by the
+token-by-token adjoint of the recurrence written out in C, fast enough for full-size shapes; pinned
+against the autograd gradients).
 
 Layouts follow the library: q, k ``[B, NH, T, DHQK]``; v, o ``[B, NH, T, DHV]``;
 gates ``[B, NH, T]``; state C ``[B, NH, DHQK, DHV]``, n ``[B, NH, DHQK]``,
@@ -25,20 +27,28 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mlstm_oracle.c")
 _LIB = os.path.join(_HERE, "libmlstm_oracle.so")
+_ADJ_SRC = os.path.join(_HERE, "mlstm_adjoint.c")
+_ADJ_LIB = os.path.join(_HERE, "libmlstm_adjoint.so")
 _lib = None
+_adj_lib = None
 
 _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
 
 
-def build(force: bool = False) -> str:
-    """Compiles the oracle with gcc (IEEE double, no fast-math) if stale."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
+def _gcc(src: str, lib: str, force: bool) -> str:
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+        tmp = lib + ".tmp%d" % os.getpid()
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared",
-                               "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
-        os.replace(tmp, _LIB)
-    return _LIB
+                               "-ffp-contract=off", "-o", tmp, src, "-lm", "-lpthread"])
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False) -> str:
+    """Compiles the oracle (and the gradient adjoint) with gcc (IEEE double, no fast-math) if stale."""
+    _gcc(_ADJ_SRC, _ADJ_LIB, force)
+    return _gcc(_SRC, _LIB, force)
 
 
 def load_library(path: str):
@@ -125,3 +135,40 @@ def mlstm_step(C, n, m, q, k, v, igate, fgate, ogate=None, nthreads: int = 0, in
                         _f32(igate)[:, :, None], _f32(fgate)[:, :, None],
                         None if og is None else og[:, :, None], C, n, m, nthreads=nthreads, inplace=inplace)
     return h[:, :, 0], C2, n2, m2
+
+
+def load_adjoint_library(path: str):
+    """Loads a gradient library built from ``mlstm_adjoint.c`` (or a variant of it)."""
+    lib = ctypes.CDLL(path)
+    lib.oracle_mlstm_adjoint.restype = ctypes.c_int
+    lib.oracle_mlstm_adjoint.argtypes = [ctypes.c_int] * 4 + [_f32p] * 7 + [_f64p] * 6 + [ctypes.c_int]
+    return lib
+
+
+def mlstm_adjoint(q, k, v, igate, fgate, ogate, dh, nthreads: int = 0, lib=None):
+    """Gradients of sum(dh * h) of the forward pass from the zero state, by the token-by-token
+    adjoint of the recurrence in ``mlstm_adjoint.c``: ``(dq, dk, dv, digate, dfgate, dogate)`` in
+    float64 (dogate None without an output gate)."""
+    global _adj_lib
+    if lib is None:
+        if _adj_lib is None:
+            build()
+            _adj_lib = load_adjoint_library(_ADJ_LIB)
+        lib = _adj_lib
+    q, k, v, dh = _f32(q), _f32(k), _f32(v), _f32(dh)
+    ig, fg, og = _f32(igate), _f32(fgate), _f32(ogate)
+    B, NH, T, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and v.shape == (B, NH, T, dv) and dh.shape == v.shape
+    assert ig.shape == (B, NH, T) and fg.shape == (B, NH, T) and (og is None or og.shape == v.shape)
+    dq, dkk = np.empty(q.shape), np.empty(q.shape)
+    dvv = np.empty(v.shape)
+    dig, dfg = np.empty(ig.shape), np.empty(ig.shape)
+    dog = np.empty(v.shape) if og is not None else None
+    rc = lib.oracle_mlstm_adjoint(B * NH, T, dk, dv, _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p),
+                                  _ptr(ig, _f32p), _ptr(fg, _f32p), _ptr(og, _f32p), _ptr(dh, _f32p),
+                                  _ptr(dq, _f64p), _ptr(dkk, _f64p), _ptr(dvv, _f64p), _ptr(dig, _f64p),
+                                  _ptr(dfg, _f64p), _ptr(dog, _f64p), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_mlstm_adjoint rejected its arguments")
+    return dq, dkk, dvv, dig, dfg, dog

@@ -1,0 +1,137 @@
+"""GPU parity of mlstm_bwd (gradients of sum(dh * h)) against the fp64 gradient oracles, through the
+C ABI.
+
+Every gradient (q, k, v, the input- and forget-gate pre-activations, the output gate) is compared
+with the oracle element by element as a whole-tensor relative L2 error: against the C adjoint of
+the recurrence (oracle/mlstm_adjoint.c, pinned against torch.autograd) on small, ragged and
+adversarial shapes and on the full 8192-token 7B-shaped workload, and against torch.autograd
+(oracle/mlstm_bwd.py) directly on a small case.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import mlstm_bwd
+from tests.parity import TOL, L2Acc, rel_l2
+from xlstm_mlstm_cell_b200 import binding
+from xlstm_mlstm_cell_b200.workloads import WORKLOADS, make_custom, make_dh, make_fwd_inputs
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq", "dk", "dv", "digate", "dfgate", "dogate")
+# Tolerance of a gradient (rel-L2 over the whole tensor against the fp64 oracle).  The pages state
+# none for gradients; it is derived from the forward pass's: every gradient term is a product of two
+# factors that each carry the forward read-out's error (g = o dh / N with the recomputed normalizer,
+# and the recomputed scores or states), so an fp32 gradient is held to twice the forward pass's 1e-5.
+# With bf16 inputs the forward's 1e-2 stands (the bf16 rounding of the inputs and outputs, about
+# 2^-9, dominates both).
+BWD_TOL = {"f32": 2e-5, "bf16": 1e-2}
+
+
+def run_gpu(inputs, dh, chunk):
+    q, k, v, i, f, o = (None if x is None else x.cuda() for x in inputs)
+    out = binding.bwd(q, k, v, i, f, o, dh.cuda(), chunk=chunk)
+    torch.cuda.synchronize()
+    return tuple(None if x is None else x.cpu() for x in out)
+
+
+def check(inputs, dh, chunk, tol):
+    got = run_gpu(inputs, dh, chunk)
+    ref = oracle.mlstm_adjoint(*inputs, dh)
+    errs = {}
+    for name, x, r in zip(NAMES, got, ref):
+        if r is None:
+            assert x is None
+            continue
+        xx = x.double().numpy()
+        assert np.all(np.isfinite(xx)), name
+        errs[name] = rel_l2(xx, r)
+    bad = {n: e for n, e in errs.items() if not e <= tol}
+    assert not bad, "rel-L2 above %.0e: %s (all: %s)" % (tol, bad, errs)
+    return errs
+
+
+SMALL = [
+    # B, NH, S, DHQK, DHV, chunk, dtype
+    (1, 2, 64, 16, 16, 16, "f32"),
+    (2, 1, 100, 32, 48, 32, "f32"),
+    (1, 2, 77, 40, 24, 16, "f32"),
+    (1, 1, 1, 8, 8, 16, "f32"),
+    (1, 2, 257, 64, 64, 64, "bf16"),
+    (1, 2, 300, 128, 128, 64, "bf16"),
+    (2, 1, 260, 256, 256, 128, "bf16"),
+    (1, 1, 200, 64, 128, 32, "bf16"),
+    (1, 2, 130, 256, 512, 64, "bf16"),
+]
+
+
+@pytest.mark.parametrize("B,NH,S,DHQK,DHV,chunk,dt", SMALL)
+def test_bwd_small_shapes(cuda_lib, B, NH, S, DHQK, DHV, chunk, dt):
+    inputs = make_custom(B, NH, S, DHQK, DHV, dt, seed=S * 5 + DHV, ig=(-1.0, 2.0), fg=(3.0, 1.5))
+    check(inputs, make_dh(B, NH, S, DHV, dt, seed=S), chunk, BWD_TOL[dt])
+
+
+@pytest.mark.parametrize("ig,fg", [((0.0, 8.0), (3.0, 1.0)), ((0.0, 1.0), (-4.0, 1.0)),
+                                   ((0.0, 1.0), (10.0, 1.0)), ((-10.0, 1.0), (2.0, 1.0))])
+@pytest.mark.parametrize("dt,DHQK,DHV,chunk", [("f32", 32, 32, 32), ("bf16", 128, 256, 64)])
+def test_bwd_adversarial_gates(cuda_lib, ig, fg, dt, DHQK, DHV, chunk):
+    inputs = make_custom(1, 2, 3 * chunk + 5, DHQK, DHV, dt, seed=13, ig=ig, fg=fg)
+    check(inputs, make_dh(1, 2, 3 * chunk + 5, DHV, dt, seed=14), chunk, BWD_TOL[dt])
+
+
+def test_bwd_floor_binds(cuda_lib):
+    """Small q and k: the denominator's floor exp(-m) binds for many tokens (its branch carries no
+    gradient)."""
+    inputs = make_custom(1, 2, 150, 64, 64, "f32", seed=15, qkv_scale=0.05, ig=(-1.0, 1.0), fg=(3.0, 1.0))
+    check(inputs, make_dh(1, 2, 150, 64, "f32", seed=16), 32, BWD_TOL["f32"])
+
+
+def test_bwd_no_output_gate(cuda_lib):
+    inputs = make_custom(1, 2, 192, 128, 128, "bf16", seed=5, ogate=False)
+    check(inputs, make_dh(1, 2, 192, 128, "bf16", seed=6), 64, BWD_TOL["bf16"])
+
+
+def test_bwd_against_autograd(cuda_lib):
+    """The same gradients straight from torch.autograd of the plain recurrence."""
+    inputs = make_custom(1, 2, 70, 24, 16, "f32", seed=17, ig=(-1.0, 2.0), fg=(3.0, 1.5))
+    dh = make_dh(1, 2, 70, 16, "f32", seed=18)
+    got = run_gpu(inputs, dh, 16)
+    ref = mlstm_bwd.mlstm_bwd(*[x.double() for x in inputs], dh.double())
+    for name, x, r in zip(NAMES, got, ref):
+        assert rel_l2(x, r) <= BWD_TOL["f32"], name
+
+
+def test_bwd_empty_sequence(cuda_lib):
+    inputs = make_custom(2, 2, 0, 64, 64, "bf16", seed=1)
+    out = run_gpu(inputs, make_dh(2, 2, 0, 64, "bf16", seed=2), 64)
+    assert out[0].shape == (2, 2, 0, 64) and out[3].shape == (2, 2, 0)
+
+
+@pytest.mark.parametrize("dt,DHQK,DHV", [("f32", 32, 32), ("bf16", 128, 128)])
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
+def test_bwd_every_chunk_size(cuda_lib, dt, DHQK, DHV, chunk):
+    """One input, every chunk length: each matches the oracle (the chunking is exact in real arithmetic)."""
+    inputs = make_custom(1, 2, 300, DHQK, DHV, dt, seed=3, ig=(-1.0, 2.0), fg=(4.0, 1.0))
+    check(inputs, make_dh(1, 2, 300, DHV, dt, seed=4), chunk, BWD_TOL[dt])
+
+
+def test_bwd_full_workload_7b(cuda_lib):
+    """The 7B-shaped prefill (B1 NH8 S8192 d256/512, chunk 64) at full size: every gradient of every
+    head, whole-tensor rel-L2 (the oracle takes the heads in groups, a thread per head)."""
+    w = WORKLOADS["fwd_bf16_7b"]
+    inputs = make_fwd_inputs(w)
+    dh = make_dh(w.B, w.NH, w.S, w.DHV, w.dtype, seed=w.seed + 1)
+    got = run_gpu(inputs, dh, w.chunk)
+    acc = {n: L2Acc() for n in NAMES}
+    group = max(1, min(w.NH, oracle.default_threads()))
+    for h0 in range(0, w.NH, group):
+        sl = lambda x: None if x is None else x[:, h0:h0 + group]
+        ref = oracle.mlstm_adjoint(*(sl(x) for x in inputs), sl(dh))
+        for name, x, r in zip(NAMES, got, ref):
+            acc[name].add(sl(x), r)
+    errs = {n: a.rel() for n, a in acc.items()}
+    bad = {n: e for n, e in errs.items() if not e <= BWD_TOL["bf16"]}
+    assert not bad, "rel-L2 above 1e-2: %s (all: %s)" % (bad, errs)

@@ -35,6 +35,9 @@ SIGNATURES = {
     "mlstm_fwd_noalloc": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _fp, _fp,
                                _vp]),
     "mlstm_fwd_noalloc_status": (_i, [_vp]),
+    "mlstm_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "mlstm_bwd": (_i, [_vp, _vp, _vp, _fp, _fp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _fp, _fp, _vp,
+                       _vp, _sz, _vp]),
     "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_fwd_tensor_path": (_i, [_i, _i, _i, _i]),
     "mlstm_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _i]),
@@ -173,6 +176,34 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
         arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[None if e is None else e.cuda_event for e in events])
         _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
     return h_out, C_final, n_final, m_final
+
+
+def bwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dtype) -> int:
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().mlstm_bwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dt))
+
+
+def bwd(q, k, v, igate, fgate, ogate, dh, chunk: int = 64, workspace=None, stream=None, out=None):
+    """mlstm_bwd on device tensors: gradients of sum(dh * h) for the forward pass from the zero
+    state.  Returns ``(dq, dk, dv, digate, dfgate, dogate)`` (dogate None without an output gate);
+    ``out`` may give those six tensors to write into."""
+    lib = load()
+    B, NH, S, DHQK = q.shape
+    DHV = v.shape[-1]
+    dt = _dt(q)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(igate),
+               torch.empty_like(fgate), None if ogate is None else torch.empty_like(ogate))
+    dq, dk, dv, dig, dfg, dog = out
+    if workspace is None:
+        n = bwd_workspace_size(B, NH, S, DHQK, DHV, chunk, q.dtype)
+        if n == 0:
+            raise MlstmError("mlstm_bwd_workspace_size", 2)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    _check("mlstm_bwd", lib.mlstm_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(igate), _ptr(fgate), _ptr(ogate), _ptr(dh), dt,
+                                      B, NH, S, DHQK, DHV, chunk, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dig), _ptr(dfg),
+                                      _ptr(dog), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv, dig, dfg, dog
 
 
 def fwd_final_state(k, v, igate, fgate, chunk: int = 64, workspace=None, stream=None):

@@ -63,6 +63,40 @@ size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, b
 
 mlstm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA; }
 
+// Lays out the backward pass's workspace (base may be NULL to size it).  Returns the bytes used.
+size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, BwdWorkspace *w)
+{
+    BwdWorkspace tmp;
+    if (!w) w = &tmp;
+    const int NC = (S + chunk - 1) / chunk;
+    const int NTK = (DHQK + 31) / 32;
+    w->NC = NC;
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char * {
+        char *p = base ? base + off : nullptr;
+        off = align_up(off + bytes, 256);
+        return p;
+    };
+    const size_t f = sizeof(float);
+    w->status = reinterpret_cast<uint32_t *>(take(sizeof(uint32_t)));
+    w->A = reinterpret_cast<float *>(take(f * BH * S));
+    w->M = reinterpret_cast<float *>(take(f * BH * S));
+    w->G = reinterpret_cast<float *>(take(f * BH * NC));
+    w->Bc = reinterpret_cast<float *>(take(f * BH * NC));
+    w->MC = reinterpret_cast<float *>(take(f * BH * (NC + 1)));
+    w->CS = reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
+    w->NS = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
+    w->GS = reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
+    w->GN = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
+    w->Gt = reinterpret_cast<float *>(take(f * BH * S * DHV));
+    w->DD = reinterpret_cast<float *>(take(f * BH * S));
+    w->P2 = reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
+    w->AI = reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
+    w->QD = reinterpret_cast<float *>(take(f * BH * S * NTK));
+    w->KD = reinterpret_cast<float *>(take(f * BH * S * NTK));
+    return off;
+}
+
 }  // namespace
 
 extern "C" const char *mlstm_status_string(mlstm_status s)
@@ -266,3 +300,52 @@ mlstm_status mlstm_step(float *C, float *n, float *m, const void *q, const void 
 }
 
 }  // extern "C"
+
+extern "C" size_t mlstm_bwd_workspace_size(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if (B < 0 || NH < 0 || S < 0 || (dt != MLSTM_F32 && dt != MLSTM_BF16)) return 0;
+    if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return 0;
+    if ((long long)B * NH > (1LL << 30) || (long long)S * DHV > (1LL << 40)) return 0;
+    return plan_bwd_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, nullptr);
+}
+
+extern "C" mlstm_status mlstm_bwd(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
+                                  const void *ogate, const void *dh, mlstm_dtype dt, int B, int NH, int S, int DHQK,
+                                  int DHV, int chunk, void *dq, void *dk, void *dv, float *digate, float *dfgate,
+                                  void *dogate, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || NH < 0 || S < 0) return MLSTM_ERR_INVALID_ARG;
+    if (dt != MLSTM_F32 && dt != MLSTM_BF16) return MLSTM_ERR_UNSUPPORTED;
+    if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return MLSTM_ERR_UNSUPPORTED;
+    if ((long long)B * NH > (1LL << 30) || (long long)S * DHV > (1LL << 40)) return MLSTM_ERR_UNSUPPORTED;
+    const int BH = B * NH;
+    if (BH == 0 || S == 0) return MLSTM_OK;   // no tokens: every gradient is empty
+    const void *ins[] = {q, k, v, igate, fgate, dh, dq, dk, dv, digate, dfgate};
+    for (const void *p : ins)
+        if (!p || !aligned16(p)) return MLSTM_ERR_INVALID_ARG;
+    if (ogate && (!dogate || !aligned16(ogate) || !aligned16(dogate))) return MLSTM_ERR_INVALID_ARG;
+    const size_t need = plan_bwd_workspace(nullptr, BH, S, DHQK, DHV, chunk, nullptr);
+    if (!workspace || workspace_bytes < need) return MLSTM_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLSTM_ERR_INVALID_ARG;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    BwdWorkspace w;
+    plan_bwd_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, &w);
+    const bool bf16 = dt == MLSTM_BF16;
+    // gate preprocessing and the chunk-start states of the forward pass (its fp32 carry)
+    GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, 0, 0, nullptr, nullptr, nullptr,
+                    w.status, st};
+    if (launch_gate_prep(gp) != cudaSuccess) return MLSTM_ERR_CUDA;
+    FwdWorkspace fw{};
+    fw.status = w.status;
+    fw.NC = w.NC;
+    fw.A = w.A; fw.M = w.M; fw.G = w.G; fw.Bc = w.Bc; fw.MC = w.MC;
+    fw.CS = w.CS; fw.NS = w.NS;
+    fw.tc = false;
+    FwdArgs fa{q, k, v, nullptr, igate, fgate, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, BH, S, DHQK, DHV,
+               chunk, bf16, st, false};
+    if (launch_fwd_simt(fa, fw, PhaseMark{}) != cudaSuccess) return MLSTM_ERR_CUDA;
+    BwdArgs ba{q, k, v, ogate, dh, igate, fgate, dq, dk, dv, dogate, digate, dfgate, BH, S, DHQK, DHV, chunk, bf16,
+               st};
+    return cuda_status(launch_bwd(ba, w));
+}

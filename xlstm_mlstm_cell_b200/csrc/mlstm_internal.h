@@ -57,6 +57,29 @@ struct FwdWorkspace {
     float *DN;             // [BH][NSEG][DHQK] same for the normalizer
 };
 
+struct BwdArgs {
+    const void *q, *k, *v, *ogate, *dh;
+    const float *igate, *fgate;
+    void *dq, *dk, *dv, *dogate;
+    float *digate, *dfgate;
+    int BH, S, DHQK, DHV, chunk;
+    bool bf16;
+    cudaStream_t stream;
+};
+
+// Device workspace of one mlstm_bwd call.
+struct BwdWorkspace {
+    uint32_t *status;
+    int NC;
+    float *A, *M, *G, *Bc, *MC;   // gate preprocessing, as for the forward pass
+    float *CS, *NS;               // forward chunk-start states [BH][NC][DHQK][DHV], [BH][NC][DHQK]
+    float *GS, *GN;               // state gradients per chunk, same layouts
+    float *Gt;                    // [BH][S][DHV] gradient of the read-out numerator
+    float *DD;                    // [BH][S] gradient of the denominator
+    float *P2, *AI;               // [BH][NC][chunk][chunk] score gradients and scores
+    float *QD, *KD;               // [BH][S][ceil(DHQK / 32)] partial q . dq, k . dk
+};
+
 // Records the caller's phase events (mlstm_fwd_profiled); a no-op without events.
 struct PhaseMark {
     void *const *events = nullptr;
@@ -76,5 +99,6 @@ size_t simt_state_bytes(int BH, int NC, int DHQK, int DHV);
 bool tc_path_supported(bool bf16, int DHQK, int DHV, int chunk);
 int tc_num_segments(int BH, int DHV, int NC);
 cudaError_t launch_fwd_tc(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark);
+cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w);
 
 }  // namespace mlstm

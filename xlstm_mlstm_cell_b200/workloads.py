@@ -90,6 +90,14 @@ def make_step_inputs(w: Workload, step: int, B: int | None = None, NH: int | Non
                 1.0, w.ig, w.fg, w.ogate, gen)
 
 
+def make_dh(B, NH, S, DHV, dtype, seed):
+    """The gradient of a loss with respect to h, dh ~ N(0, 1) [B, NH, S, DHV], for the backward pass
+    (drawn from its own generator, seeded with ``seed``)."""
+    gen = torch.Generator().manual_seed(seed)
+    dt = torch.float32 if dtype in ("f32", torch.float32) else torch.bfloat16
+    return torch.randn((B, NH, S, DHV), generator=gen).to(dt)
+
+
 def make_custom(B, NH, S, DHQK, DHV, dtype, seed, qkv_scale=1.0, ig=(0.0, 1.0), fg=(3.0, 1.0),
                 ogate=True):
     """Free-form inputs for sweeps and edge cases."""
