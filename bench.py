@@ -368,7 +368,8 @@ def fwd_report(w: Workload, phase_ms: dict, fwd_ms: float, peaks: dict):
     wk = fw["phases"][dom]
     uses_tc = tensor and dom in ("state_contributions", "outputs")
     roof = roofline(wk, phase_ms[dom] / 1e3, peaks, uses_tc)
-    roof["kernel"] = {"outputs": "walk_kernel" if tensor else "output_simt_kernel",
+    paired = tensor and binding.fwd_paired_walk(w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 1
+    roof["kernel"] = {"outputs": ("walk_pair_kernel" if paired else "walk_kernel") if tensor else "output_simt_kernel",
                       "state_contributions": "segsum_kernel" if tensor else "carry_simt_kernel",
                       "state_scan": "seg_scan_kernel", "gate_prep": "gate kernels"}[dom]
     roof["phase"] = dom

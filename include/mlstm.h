@@ -214,6 +214,15 @@ int mlstm_fwd_kernel_launches(int B, int NH, int S, int DHQK, int DHV, int chunk
 int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt);
 
 /*
+ * 1 when mlstm_fwd's tensor-core path runs its in-segment walk as CTA pairs
+ * (tcgen05 .cta_group::2: two CTAs share each chunk's S = Q K^T, P and the passes
+ * over q and k, 256 value columns per pair; DHQK 256, DHV a multiple of 256,
+ * chunk 128), 0 when the walk runs one CTA per 128 value columns, -1 when the
+ * combination does not take the tensor-core path.  No GPU work; a host-side query.
+ */
+int mlstm_fwd_paired_walk(int DHQK, int DHV, int chunk, mlstm_dtype dt);
+
+/*
  * Segments per head that mlstm_fwd's tensor-core path cuts the sequence into for
  * this shape (each segment's contribution is one long GEMM; the walk runs one
  * CTA per segment and 128 value columns), or 0 when the shape does not take the

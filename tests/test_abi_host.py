@@ -138,6 +138,17 @@ def test_tensor_path_query(lib):
     assert lib.mlstm_fwd_tensor_path(256, 512, 64, 7) == -1      # unsupported dtype
 
 
+def test_paired_walk_query(lib):
+    bf, f32 = 1, 0
+    assert lib.mlstm_fwd_paired_walk(256, 512, 128, bf) == 1     # the long-context shape
+    assert lib.mlstm_fwd_paired_walk(256, 256, 128, bf) == 1
+    assert lib.mlstm_fwd_paired_walk(256, 384, 128, bf) == 0     # DHV not a multiple of 256
+    assert lib.mlstm_fwd_paired_walk(256, 512, 64, bf) == 0      # chunk 64: one CTA per value tile
+    assert lib.mlstm_fwd_paired_walk(128, 512, 128, bf) == 0     # DHQK 128
+    assert lib.mlstm_fwd_paired_walk(256, 512, 128, f32) == -1   # fp32: CUDA-core path
+    assert lib.mlstm_fwd_paired_walk(256, 512, 48, bf) == -1     # unsupported chunk
+
+
 def test_kernel_launch_counts(lib):
     bf, f32 = binding.MLSTM_BF16, binding.MLSTM_F32
     # gate preprocessing is one kernel up to 4096 tokens per head, two beyond

@@ -40,6 +40,7 @@ SIGNATURES = {
                        _vp, _sz, _vp]),
     "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_fwd_tensor_path": (_i, [_i, _i, _i, _i]),
+    "mlstm_fwd_paired_walk": (_i, [_i, _i, _i, _i]),
     "mlstm_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_step": (_i, [_fp, _fp, _fp, _vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "mlstm_status_string": (ctypes.c_char_p, [_i]),
@@ -115,6 +116,13 @@ def fwd_tensor_path(DHQK, DHV, chunk, dtype) -> int:
     """1: tensor-core path, 0: fp32 CUDA-core path, -1: unsupported (mlstm_fwd_tensor_path)."""
     dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
     return int(load().mlstm_fwd_tensor_path(DHQK, DHV, chunk, dt))
+
+
+def fwd_paired_walk(DHQK, DHV, chunk, dtype) -> int:
+    """1: the walk runs as CTA pairs, 0: one CTA per value tile, -1: off the tensor-core path
+    (mlstm_fwd_paired_walk)."""
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().mlstm_fwd_paired_walk(DHQK, DHV, chunk, dt))
 
 
 def fwd_segments(B, NH, S, DHQK, DHV, chunk, dtype) -> int:

@@ -48,6 +48,7 @@
 #include "common.cuh"
 #include "mlstm_internal.h"
 #include "tc_common.cuh"
+#include "tc_fwd.h"
 
 #include <cudaTypedefs.h>
 
@@ -85,14 +86,6 @@ __device__ long long g_seg_trace[65 * 8];
 #endif
 #define WALK_TRACE(slot) WALK_TRACE_AT(slot, i)
 
-struct Params {
-    int S, L, NC, R, NSEG, DK, DV, BH;
-    const float *A, *Mtok, *ig, *MC, *G, *GP, *SGb;
-    float *DC, *DN;
-    const __nv_bfloat16 *o;
-    __nv_bfloat16 *h;
-    uint32_t *status;
-};
 
 // ---------------------------------------------------------------- segsum
 
@@ -1264,6 +1257,7 @@ cudaError_t launch_dk_l(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark
     if ((e = mark(3)) != cudaSuccess) return e;
 
     if (!a.outputs) return cudaSuccess;   // the final state is complete after the segment scan
+    if (walk_pair_supported(DK, a.DHV, L)) return launch_walk_pair(p, a.q, a.k, a.v, a.stream);
     using WS = WalkSmem<DK, L>;
     if ((e = ensure_dynamic_smem((const void *)walk_kernel<DK, L>, WS::TOTAL)) != cudaSuccess) return e;
     return launch_kernel(walk_kernel<DK, L>, dim3(ntile, w.NSEG, a.BH), dim3(WALK_THREADS), WS::TOTAL, a.stream, 1,

@@ -5,6 +5,7 @@
 // the caller's stream; nothing here synchronizes except mlstm_fwd_status.
 #include "mlstm.h"
 #include "mlstm_internal.h"
+#include "tc_fwd.h"
 
 #include <stdint.h>
 
@@ -135,6 +136,12 @@ extern "C" int mlstm_fwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype d
     if (dt != MLSTM_F32 && dt != MLSTM_BF16) return -1;
     if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return -1;
     return tc_path_supported(dt == MLSTM_BF16, DHQK, DHV, chunk) ? 1 : 0;
+}
+
+extern "C" int mlstm_fwd_paired_walk(int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if (mlstm_fwd_tensor_path(DHQK, DHV, chunk, dt) != 1) return -1;
+    return tcfwd::walk_pair_supported(DHQK, DHV, chunk) ? 1 : 0;
 }
 
 extern "C" int mlstm_fwd_segments(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt)
