@@ -4,9 +4,10 @@
  * section "The Twin Cells: sLSTM and mLSTM Mathematical Formulations", part 1,
  * the step-by-step recurrent equations) keeps one scalar memory c, normalizer n
  * and stabilizer m per cell and mixes the cells of a head through recurrent
- * matrices R.  Heads do not mix ("xLSTM: Extended Long Short-Term Memory",
- * section 2: memory mixing among the cells of a head, not across heads), so R is
- * block-diagonal: one DH x DH block per head and gate.
+ * matrices R.  Heads do not mix (the hu-po summary "Introduction to xLSTM
+ * architecture", section "xLSTM Architecture Design": the gates pass through a
+ * block-diagonal layer whose diagonal blocks, the heads, keep connectivity inside
+ * a head), so R is block-diagonal: one DH x DH block per head and gate.
  *
  * Per batch item b, head e and cell j, at every step t:
  *   x~[g][j] = wx[b][t][g][e][j] + sum_k R[e][g][j][k] h[k]     (g = i, f, z, o; h = h_{t-1} of head e)

@@ -6,11 +6,13 @@ this module; the CUDA library and its binding never do.
 What it follows: "xLSTM Guide: Extended LSTM Architecture & Matrix Memory",
 section "The Twin Cells: sLSTM and mLSTM Mathematical Formulations", part 1
 "sLSTM: Scalar Memory with Recurrent Cross-Head Mixing" (the step-by-step
-recurrent equations), read together with "xLSTM: Extended Long Short-Term
-Memory", section 2 "Extended Long Short-Term Memory", which states that sLSTM
-heads mix memory among the cells of one head but not across heads.  The guide's
-title speaks of mixing across heads; the paper's statement is taken (R is
-block-diagonal over heads); with one head the two agree.
+recurrent equations), read together with the hu-po summary "Introduction to
+xLSTM architecture", section "xLSTM Architecture Design" (the residual block
+with post-up projection), which says that the sLSTM's cell input and gates pass
+through a block-diagonal linear layer of four diagonal blocks, its "heads", so
+that connectivity stays inside each head.  The guide's title speaks of mixing
+across heads; the hu-po statement is taken (R is block-diagonal over heads);
+with one head the two agree.
 
 Per batch item, head and cell j, at step t (1-based), from the state
 (c, n, m, h) of step t-1:

@@ -208,3 +208,49 @@ def test_state_ready_event_with_other_phase_events_null(cuda_lib):
     torch.cuda.synchronize()
     assert torch.equal(h1, h2) and torch.equal(C1, C2) and torch.equal(n1, n2) and torch.equal(m1, m2)
     assert torch.equal(C_copy, C1)
+
+
+def test_two_host_threads_on_separate_streams(cuda_lib):
+    """Two host threads call mlstm_fwd at once, each on its own stream with its own inputs and
+    workspace, many times over: every result equals the same call made alone (the kernels are
+    deterministic) and the oracle.  Exercises the library's host caches (shared-memory attributes,
+    the tensor-map encoder) under concurrent first use and the per-call workspaces."""
+    import threading
+    shapes = [(1, 2, 520, 256, 512, 128, "bf16"), (2, 2, 300, 128, 256, 64, "bf16")]
+    inputs = [make_custom(*s[:5], s[6], seed=7100 + t) for t, s in enumerate(shapes)]
+    dev = [tuple(None if x is None else x.cuda() for x in inp) for inp in inputs]
+    alone = []
+    for t, s in enumerate(shapes):
+        h, C, n, m = binding.fwd(*dev[t], chunk=s[5])
+        torch.cuda.synchronize()
+        alone.append((h.cpu(), C.cpu(), n.cpu(), m.cpu()))
+    results = [[] for _ in shapes]
+    errors = []
+    start = threading.Barrier(len(shapes))
+
+    def worker(t):
+        try:
+            stream = torch.cuda.Stream()
+            start.wait()
+            with torch.cuda.stream(stream):
+                for _ in range(20):
+                    out = binding.fwd(*dev[t], chunk=shapes[t][5], stream=stream)
+                    stream.synchronize()
+                    results[t].append(tuple(x.cpu() for x in out))
+        except Exception as e:   # reported on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(t,)) for t in range(len(shapes))]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
+    for t, s in enumerate(shapes):
+        assert len(results[t]) == 20
+        for out in results[t]:
+            for a, b in zip(out, alone[t]):
+                assert torch.equal(a, b)
+        hr, Cr, nr, mr = oracle.mlstm_fwd(*inputs[t])
+        assert_close("h", alone[t][0], hr, TOL[s[6]])
+        assert_close("C", alone[t][1], Cr, TOL[s[6]])
