@@ -60,6 +60,11 @@ SMALL = [
     (1, 2, 333, 64, 128, 64, "bf16"),
     (1, 2, 333, 64, 128, 128, "bf16"),
     (2, 1, 400, 128, 256, 128, "bf16"),
+    # the paired walk (chunk 128, DHQK 256, DHV a multiple of 256): several heads and batches with
+    # ragged tails, and one head cut into one-chunk segments (33 segments, the last partial)
+    (2, 3, 333, 256, 512, 128, "bf16"),
+    (3, 1, 200, 256, 512, 128, "bf16"),
+    (1, 1, 4096 + 77, 256, 256, 128, "bf16"),
 ]
 
 
@@ -78,9 +83,10 @@ def test_fwd_adversarial_gates(cuda_lib, ig, fg, dt, DHQK, DHV, chunk):
     check_against_oracle(inputs, chunk, TOL[dt])
 
 
-def test_fwd_no_output_gate(cuda_lib):
-    inputs = make_custom(1, 2, 192, 128, 128, "bf16", seed=5, ogate=False)
-    check_against_oracle(inputs, 64, TOL["bf16"])
+@pytest.mark.parametrize("DHQK,DHV,chunk", [(128, 128, 64), (256, 256, 128), (256, 512, 128)])
+def test_fwd_no_output_gate(cuda_lib, DHQK, DHV, chunk):
+    inputs = make_custom(1, 2, 300, DHQK, DHV, "bf16", seed=5, ogate=False)
+    check_against_oracle(inputs, chunk, TOL["bf16"])
 
 
 def test_fwd_empty_sequence(cuda_lib):
