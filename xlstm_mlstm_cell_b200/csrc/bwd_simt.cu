@@ -57,7 +57,7 @@ struct Params {
 
 // Shared-memory floats of bwd_chunk_kernel and bwd_grad_kernel for chunk length L.
 __host__ __device__ constexpr int chunk_smem_floats(int L) { return 2 * L * (L + 1) + 3 * L * 33 + 32 * 33 + 8 * L; }
-__host__ __device__ constexpr int grad_smem_floats(int L) { return L * (L + 1) + 2 * L * 33 + 2 * 32 * 33 + 4 * L; }
+__host__ __device__ constexpr int grad_smem_floats(int L) { return L * (L + 1) + 2 * L * 36 + 2 * 32 * 36 + 4 * L; }
 
 // Per-token gate terms of chunk c, in forms where the chunk-local cumulative log decay a_t
 // cancels before rounding (m_t = a_t + max(m_c, p_t), so a_t - a_s + i~_s - m_t = x_s - mx_t):
@@ -83,7 +83,7 @@ __device__ __forceinline__ void chunk_rows(const Params &p, int bh, int c, int t
 // grid (BH, NC), NT threads.  Recomputes A, den, N and num of the chunk, writes do, g, dden, dS,
 // A and the read-out's state gradients (dC_c, dn_c).
 template <typename T>
-__global__ void __launch_bounds__(NT) bwd_chunk_kernel(Params p)
+__global__ void __launch_bounds__(NT, 3) bwd_chunk_kernel(Params p)
 {
     griddep_wait();
     griddep_launch_dependents();
@@ -331,7 +331,12 @@ __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
 
 // ---------------------------------------------------------------- per chunk and column tile: dq, dk, dv
 // grid (BH, NC, NTK + NTV), NT threads.  Tiles z < NTK: 32 columns of DK (dq and dk); the rest:
-// 32 columns of DV (dv).
+// 32 columns of DV (dv).  A thread owns column x of the tile for the rows ty + 8 r; the products
+// run with the reduction index outermost, so that a shared value read by the whole warp (a row of
+// the left factor) and one per lane (the lane's column of the right factor) feed the warp's rows,
+// four reduction steps per 16-byte load where the layout allows.
+constexpr int TS = 36;    // row stride of the 32-column tiles (16-byte aligned rows, no bank conflicts)
+
 template <typename T>
 __global__ void __launch_bounds__(NT) bwd_grad_kernel(Params p)
 {
@@ -340,11 +345,11 @@ __global__ void __launch_bounds__(NT) bwd_grad_kernel(Params p)
     extern __shared__ float sm[];
     const int L = p.L, LP = L + 1, DK = p.DK, DV = p.DV;
     float *Ms = sm;               // [L][LP]: dS (key tiles) or A (value tiles)
-    float *as_ = Ms + L * LP;     // [L][33]
-    float *bs = as_ + L * 33;     // [L][33]
-    float *cs = bs + L * 33;      // [32][33]
-    float *cs2 = cs + 32 * 33;    // [32][33]
-    float *xs_ = cs2 + 32 * 33, *mx = xs_ + L, *fl = mx + L, *sc = fl + L;
+    float *as_ = Ms + L * LP;     // [L][TS]
+    float *bs = as_ + L * TS;     // [L][TS]
+    float *cs = bs + L * TS;      // [32][TS]
+    float *cs2 = cs + 32 * TS;    // [32][TS]
+    float *xs_ = cs2 + 32 * TS, *mx = xs_ + L, *fl = mx + L, *sc = fl + L;
 
     const int bh = blockIdx.x, c = blockIdx.y, z = blockIdx.z;
     const int t0 = c * L, len = min(L, p.S - t0);
@@ -376,51 +381,57 @@ __global__ void __launch_bounds__(NT) bwd_grad_kernel(Params p)
         for (int e = tid; e < L * 32; e += NT) {
             const int t = e >> 5, xx = e & 31;
             const bool ok = t < len && i0 + xx < DK;
-            as_[t * 33 + xx] = ok ? to_f32(kb[(size_t)t * DK + i0 + xx]) : 0.f;
-            bs[t * 33 + xx] = ok ? to_f32(qb[(size_t)t * DK + i0 + xx]) * scale : 0.f;
+            as_[t * TS + xx] = ok ? to_f32(kb[(size_t)t * DK + i0 + xx]) : 0.f;
+            bs[t * TS + xx] = ok ? to_f32(qb[(size_t)t * DK + i0 + xx]) * scale : 0.f;
         }
         __syncthreads();
         float aq[16], ak[16], iq[16], ik[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            aq[r] = ak[r] = iq[r] = ik[r] = 0.f;
-            const int t = ty + 8 * r;
-            if (r < RPT) {
-                for (int s = 0; s <= t; ++s) aq[r] = fmaf(Ms[t * LP + s], as_[s * 33 + x], aq[r]);   // dS K
-                for (int u = t; u < L; ++u) ak[r] = fmaf(Ms[u * LP + t], bs[u * 33 + x], ak[r]);     // dS^T qh
+        for (int r = 0; r < 16; ++r) aq[r] = ak[r] = iq[r] = ik[r] = 0.f;
+        // dS K (row t: sum_s dS_ts k_s) and dS^T qh (row t: sum_u dS_ut qh_u); dS is zero above the
+        // diagonal and past the end of the sequence
+        for (int s = 0; s < L; ++s) {
+            const float ks = as_[s * TS + x], qs = bs[s * TS + x];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                if (r < RPT) {
+                    const int t = ty + 8 * r;
+                    aq[r] = fmaf(Ms[t * LP + s], ks, aq[r]);
+                    ak[r] = fmaf(Ms[s * LP + t], qs, ak[r]);
+                }
             }
         }
-        __syncthreads();
         // inter-chunk parts over slices of 32 of DV: g C_c^T (rows t) and V G_end^T (rows s)
         for (int j0 = 0; j0 < DV; j0 += 32) {
+            __syncthreads();
             for (int e = tid; e < L * 32; e += NT) {
                 const int t = e >> 5, xx = e & 31;
                 const bool ok = t < len && j0 + xx < DV;
-                as_[t * 33 + xx] = ok ? gtb[(size_t)t * DV + j0 + xx] : 0.f;
-                bs[t * 33 + xx] = ok ? to_f32(vb[(size_t)t * DV + j0 + xx]) : 0.f;
+                as_[t * TS + xx] = ok ? gtb[(size_t)t * DV + j0 + xx] : 0.f;
+                bs[t * TS + xx] = ok ? to_f32(vb[(size_t)t * DV + j0 + xx]) : 0.f;
             }
             for (int e = tid; e < 32 * 32; e += NT) {
                 const int ii = e >> 5, xx = e & 31;
                 const bool ok = i0 + ii < DK && j0 + xx < DV;
-                cs[ii * 33 + xx] = ok ? Cc[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
-                cs2[ii * 33 + xx] = ok ? Ge[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
+                cs[ii * TS + xx] = ok ? Cc[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
+                cs2[ii * TS + xx] = ok ? Ge[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
             }
             __syncthreads();
+#pragma unroll 2
+            for (int jj = 0; jj < 32; jj += 4) {
+                const float4 c4 = *reinterpret_cast<const float4 *>(cs + x * TS + jj);
+                const float4 e4 = *reinterpret_cast<const float4 *>(cs2 + x * TS + jj);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int t = ty + 8 * r;
-                if (r < RPT) {
-                    float a1 = iq[r], a2 = ik[r];
-#pragma unroll 8
-                    for (int jj = 0; jj < 32; ++jj) {
-                        a1 = fmaf(as_[t * 33 + jj], cs[x * 33 + jj], a1);
-                        a2 = fmaf(bs[t * 33 + jj], cs2[x * 33 + jj], a2);
+                for (int r = 0; r < 16; ++r) {
+                    if (r < RPT) {
+                        const int t = ty + 8 * r;
+                        const float4 g4 = *reinterpret_cast<const float4 *>(as_ + t * TS + jj);
+                        const float4 v4 = *reinterpret_cast<const float4 *>(bs + t * TS + jj);
+                        iq[r] = fmaf(g4.x, c4.x, fmaf(g4.y, c4.y, fmaf(g4.z, c4.z, fmaf(g4.w, c4.w, iq[r]))));
+                        ik[r] = fmaf(v4.x, e4.x, fmaf(v4.y, e4.y, fmaf(v4.z, e4.z, fmaf(v4.w, e4.w, ik[r]))));
                     }
-                    iq[r] = a1;
-                    ik[r] = a2;
                 }
             }
-            __syncthreads();
         }
         const float ncx = i < DK ? nc[i] : 0.f, gex = i < DK ? ge[i] : 0.f;
         T *dqb = static_cast<T *>(p.dq) + ((size_t)bh * p.S + t0) * DK;
@@ -453,37 +464,42 @@ __global__ void __launch_bounds__(NT) bwd_grad_kernel(Params p)
         const int j = j0 + x;
         for (int e = tid; e < L * 32; e += NT) {
             const int t = e >> 5, xx = e & 31;
-            as_[t * 33 + xx] = (t < len && j0 + xx < DV) ? gtb[(size_t)t * DV + j0 + xx] : 0.f;
+            as_[t * TS + xx] = (t < len && j0 + xx < DV) ? gtb[(size_t)t * DV + j0 + xx] : 0.f;
         }
         __syncthreads();
         float av[16], iv[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            av[r] = iv[r] = 0.f;
-            const int s = ty + 8 * r;
-            if (r < RPT)
-                for (int u = s; u < L; ++u) av[r] = fmaf(Ms[u * LP + s], as_[u * 33 + x], av[r]);   // A^T g
+        for (int r = 0; r < 16; ++r) av[r] = iv[r] = 0.f;
+        // A^T g (row s: sum_u A_us g_u); A is zero above the diagonal and past the end
+        for (int u = 0; u < L; ++u) {
+            const float gu = as_[u * TS + x];
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+                if (r < RPT) av[r] = fmaf(Ms[u * LP + ty + 8 * r], gu, av[r]);
         }
-        // K G_end over slices of 32 of DK
+        // K G_end over slices of 32 of DK; the slice of G_end transposed ([value column][DK]) so that
+        // a lane reads its column's four DK entries at once
+        float *gT = cs2;
         for (int i0 = 0; i0 < DK; i0 += 32) {
             __syncthreads();
             for (int e = tid; e < L * 32; e += NT) {
                 const int t = e >> 5, xx = e & 31;
-                bs[t * 33 + xx] = (t < len && i0 + xx < DK) ? to_f32(kb[(size_t)t * DK + i0 + xx]) : 0.f;
+                bs[t * TS + xx] = (t < len && i0 + xx < DK) ? to_f32(kb[(size_t)t * DK + i0 + xx]) : 0.f;
             }
             for (int e = tid; e < 32 * 32; e += NT) {
                 const int ii = e >> 5, xx = e & 31;
-                cs2[ii * 33 + xx] = (i0 + ii < DK && j0 + xx < DV) ? Ge[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
+                gT[xx * TS + ii] = (i0 + ii < DK && j0 + xx < DV) ? Ge[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
             }
             __syncthreads();
+#pragma unroll 2
+            for (int ii = 0; ii < 32; ii += 4) {
+                const float4 e4 = *reinterpret_cast<const float4 *>(gT + x * TS + ii);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int s = ty + 8 * r;
-                if (r < RPT) {
-                    float a2 = iv[r];
-#pragma unroll 8
-                    for (int ii = 0; ii < 32; ++ii) a2 = fmaf(bs[s * 33 + ii], cs2[ii * 33 + x], a2);
-                    iv[r] = a2;
+                for (int r = 0; r < 16; ++r) {
+                    if (r < RPT) {
+                        const float4 k4 = *reinterpret_cast<const float4 *>(bs + (ty + 8 * r) * TS + ii);
+                        iv[r] = fmaf(k4.x, e4.x, fmaf(k4.y, e4.y, fmaf(k4.z, e4.z, fmaf(k4.w, e4.w, iv[r]))));
+                    }
                 }
             }
         }
