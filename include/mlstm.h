@@ -286,9 +286,10 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * Shapes and chunk sizes as for mlstm_fwd.
  *
  * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
- * (it holds the chunk-start states and their gradients, 8 DHQK DHV bytes per
- * chunk and head, plus 4 DHV + 2 chunk + 8 ceil(DHQK / 32) + 12 bytes per
- * token and head).  Errors as for mlstm_fwd.
+ * (it holds the chunk-start states and their gradients and the chunk's scores:
+ * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
+ * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head, each
+ * array 256-byte aligned).  Errors as for mlstm_fwd.
  */
 size_t mlstm_bwd_workspace_size(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
 mlstm_status mlstm_bwd(const void *q, const void *k, const void *v,

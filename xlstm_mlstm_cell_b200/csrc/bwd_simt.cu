@@ -31,6 +31,13 @@
 //   dL/di~_t = k_t . dk_t,  dL/dA_t = q_t . dq_t - k_t . dk_t,
 //   dL/dlog f_j = sum_{t >= j} dL/dA_t,  dL/df~_j = dL/dlog f_j * sigmoid(-f~_j),
 // a reverse cumulative sum over the sequence (accumulated in fp64).
+//
+// Kernels, in launch order (after the gate preprocessing and the forward's fp32 carry that stores
+// the chunk-start states): bwd_scores_kernel (A, den, N per chunk), bwd_num_kernel (the read-out
+// numerator, g and do per chunk and 64 value columns), bwd_ds_kernel (dden, dS, dn of the read-out),
+// bwd_dc_kernel (dC of the read-out per 64 x 64 state tile), bwd_state_scan_kernel (the reverse scan
+// of the state gradients), bwd_grad_kernel (dq, dk, dv per chunk and 64 columns) and
+// bwd_gate_kernel.  The per-chunk products run as 64 x 64 output tiles on the CUDA cores in fp32.
 #include "common.cuh"
 #include "mlstm_internal.h"
 
@@ -38,7 +45,6 @@ namespace mlstm {
 namespace bwd {
 
 constexpr int NT = 256;   // threads of the chunk kernels
-constexpr int TW = 32;    // column tile
 
 struct Params {
     int S, L, NC, DK, DV, NTK;
@@ -49,6 +55,9 @@ struct Params {
     float *GS, *GN;                  // read-out state gradients, then chunk-end gradients (same layout)
     float *Gt;                       // g = o dh / N [BH][S][DV]
     float *DD;                       // dden [BH][S]
+    float *DEN, *NRM;                // den and N = max(|den|, exp(-m)) [BH][S]
+    float *DOTP;                     // partial row sums of g . hh per 64 value columns [BH][S][NJT]
+    int NJT;                         // ceil(DV / 64)
     float *P2, *AI;                  // dS and A per chunk [BH][NC][L][L]
     float *QD, *KD;                  // per dk tile partial q . dq and k . dk [BH][S][NTK]
     void *dq, *dk, *dv, *dog;
@@ -56,8 +65,6 @@ struct Params {
 };
 
 // Shared-memory floats of bwd_chunk_kernel and bwd_grad_kernel for chunk length L.
-__host__ __device__ constexpr int chunk_smem_floats(int L) { return 2 * L * (L + 1) + 3 * L * 33 + 32 * 33 + 8 * L; }
-__host__ __device__ constexpr int grad_smem_floats(int L) { return L * (L + 1) + 2 * L * 36 + 2 * 32 * 36 + 4 * L; }
 
 // Per-token gate terms of chunk c, in forms where the chunk-local cumulative log decay a_t
 // cancels before rounding (m_t = a_t + max(m_c, p_t), so a_t - a_s + i~_s - m_t = x_s - mx_t):
@@ -82,205 +89,339 @@ __device__ __forceinline__ void chunk_rows(const Params &p, int bh, int c, int t
 // ---------------------------------------------------------------- per chunk: read-out recompute
 // grid (BH, NC), NT threads.  Recomputes A, den, N and num of the chunk, writes do, g, dden, dS,
 // A and the read-out's state gradients (dC_c, dn_c).
+// ---------------------------------------------------------------- 64 x 64 tiles of the chunk products
+// The per-chunk products (S = qh K^T, the read-out numerator, g V^T, the read-out's state gradient)
+// run as tiles of 64 x 64 outputs per CTA of 256 threads, a 4 x 4 block per thread, the reduction
+// in steps of 32 staged in shared memory k-major (As[k][m], Bs[k][n], rows padded to 68 floats so
+// that a thread reads its four rows or columns with one 16-byte load).
+constexpr int GM = 64, GK = 32, GSTR = 68;
+static_assert(NT == 256, "the 64 x 64 tiles take 16 x 16 threads");
+
+__device__ __forceinline__ void tile_mma(const float *As, const float *Bs, float (&acc)[4][4])
+{
+    const int tm = threadIdx.x >> 4, tn = threadIdx.x & 15;
+#pragma unroll 8
+    for (int k = 0; k < GK; ++k) {
+        const float4 a = *reinterpret_cast<const float4 *>(As + k * GSTR + 4 * tm);
+        const float4 b = *reinterpret_cast<const float4 *>(Bs + k * GSTR + 4 * tn);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+}
+
+// Runs `nsteps` reduction steps of 32 into acc.  A thread stages 8 elements of each tile per step:
+// get(st, e, a, b) reads element e (0..2047) of step st's A and B tiles from global memory and
+// put(st, e, a, b) stores them into As and Bs.  The next step's reads are issued before this step's
+// products, so their latency overlaps the products.
+template <typename Get, typename Put>
+__device__ __forceinline__ void tile_gemm(int nsteps, Get get, Put put, const float *As, const float *Bs,
+                                          float (&acc)[4][4])
+{
+    float ra[8], rb[8];
+    if (nsteps > 0) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) get(0, threadIdx.x + u * NT, ra[u], rb[u]);
+    }
+    for (int st = 0; st < nsteps; ++st) {
+        __syncthreads();   // the previous step's readers are done
+#pragma unroll
+        for (int u = 0; u < 8; ++u) put(st, threadIdx.x + u * NT, ra[u], rb[u]);
+        __syncthreads();
+        if (st + 1 < nsteps) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) get(st + 1, threadIdx.x + u * NT, ra[u], rb[u]);
+        }
+        tile_mma(As, Bs, acc);
+    }
+}
+
+// Sum over the 16 threads that share a tile row block (tn = lane & 15).
+__device__ __forceinline__ float sum16(float v)
+{
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ---------------------------------------------------------------- per chunk: scores and denominators
+// grid (BH, NC): A = D * S with S = qh K^T on the causal triangle (-> AI), den_t = rowsum(A)_t +
+// sc_t n_c . qh_t and N_t = max(|den_t|, exp(-m_t)) (-> DEN, NRM).
 template <typename T>
-__global__ void __launch_bounds__(NT, 3) bwd_chunk_kernel(Params p)
+__global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
 {
     griddep_wait();
     griddep_launch_dependents();
-    extern __shared__ float sm[];
-    const int L = p.L, LP = L + 1, DK = p.DK, DV = p.DV;
-    float *Sm = sm;               // [L][LP]: S, then A = D * S
-    float *dAg = Sm + L * LP;     // [L][LP]: g v^T over the value tiles
-    float *qs = dAg + L * LP;     // [L][33]
-    float *xs = qs + L * 33;      // [L][33]: k slice, then v tile
-    float *gs = xs + L * 33;      // [L][33]: g tile
-    float *cs = gs + L * 33;      // [32][33]: slice of C_c
-    float *xs_ = cs + 32 * 33, *mx = xs_ + L, *fl = mx + L, *sc = fl + L;
-    float *den = sc + L, *nrm = den + L, *dot = nrm + L, *dd = dot + L;
-
+    __shared__ __align__(16) float As[GK * GSTR], Bs[GK * GSTR];
+    __shared__ float xs_[128], mx[128], fl[128], sc[128], rsum[128];
+    const int L = p.L, DK = p.DK;
     const int bh = blockIdx.x, c = blockIdx.y;
     const int t0 = c * L, len = min(L, p.S - t0);
-    const int tid = threadIdx.x, x = tid & 31, ty = tid >> 5;
+    const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15, lane = tid & 31, warp = tid >> 5;
     const float scale = rsqrtf((float)DK);
     const T *qb = static_cast<const T *>(p.q) + ((size_t)bh * p.S + t0) * DK;
     const T *kb = static_cast<const T *>(p.k) + ((size_t)bh * p.S + t0) * DK;
+    const float *nc = p.NS + ((size_t)bh * p.NC + c) * DK;
+    float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
+
+    chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
+    for (int t = tid; t < L; t += NT) rsum[t] = 0.f;
+    const int nmt = (L + GM - 1) / GM;
+    for (int mt = 0; mt < nmt; ++mt)
+        for (int nt = 0; nt <= mt; ++nt) {   // tiles on or below the diagonal
+            float acc[4][4] = {};
+            for (int d0 = 0; d0 < DK; d0 += GK) {   // (a small product: staged without prefetch)
+                __syncthreads();
+                for (int e = tid; e < GK * GM; e += NT) {
+                    const int m = e >> 5, k = e & 31;   // consecutive threads: consecutive d
+                    const int ta = mt * GM + m, tb = nt * GM + m;
+                    As[k * GSTR + m] = (ta < len && d0 + k < DK) ? to_f32(qb[(size_t)ta * DK + d0 + k]) * scale : 0.f;
+                    Bs[k * GSTR + m] = (tb < len && d0 + k < DK) ? to_f32(kb[(size_t)tb * DK + d0 + k]) : 0.f;
+                }
+                __syncthreads();
+                tile_mma(As, Bs, acc);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int t = mt * GM + 4 * tm + a;
+                float part = 0.f;
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2) {
+                    const int s2 = nt * GM + 4 * tn + b2;
+                    float av = 0.f;
+                    if (s2 <= t && t < len) av = acc[a][b2] * expf(xs_[s2] - mx[t]);
+                    if (t < L && s2 < L) AIg[(size_t)t * L + s2] = av;
+                    part += av;
+                }
+                part = sum16(part);
+                if (tn == 0 && t < L) atomicAdd(&rsum[t], part);
+            }
+            // tiles above the diagonal (s > t everywhere) hold zeros
+            if (nt < mt) {
+                for (int e = tid; e < GM * GM; e += NT) {
+                    const int t = nt * GM + e / GM, s2 = mt * GM + e % GM;
+                    if (t < L && s2 < L) AIg[(size_t)t * L + s2] = 0.f;
+                }
+            }
+        }
+    __syncthreads();
+    // den and N: a warp per row, lanes over DK
+    for (int t = warp; t < L; t += NT / 32) {
+        float qn = 0.f;
+        if (t < len)
+            for (int d = lane; d < DK; d += 32) qn = fmaf(nc[d], to_f32(qb[(size_t)t * DK + d]), qn);
+        qn = warp_sum(qn);
+        if (lane == 0 && t < len) {
+            const float den = rsum[t] + qn * scale * sc[t];
+            p.DEN[(size_t)bh * p.S + t0 + t] = den;
+            p.NRM[(size_t)bh * p.S + t0 + t] = fmaxf(fabsf(den), fl[t]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- per chunk and 64 value columns: the read-out
+// grid (BH, NC, NJT): num = sc qh C_c + A V (one product over [sc qh | A] and [C_c ; V], K = DK + L),
+// hh = num / N, do = dh hh, g = o dh / N (-> Gt) and the partial row sums of g . hh (-> DOTP).
+template <typename T>
+__global__ void __launch_bounds__(NT) bwd_num_kernel(Params p)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ __align__(16) float As[GK * GSTR], Bs[GK * GSTR];
+    __shared__ float sc[128], xs_[128], mx[128], fl[128];
+    const int L = p.L, DK = p.DK, DV = p.DV;
+    const int bh = blockIdx.x, c = blockIdx.y, jt = blockIdx.z, j0 = jt * GM;
+    const int t0 = c * L, len = min(L, p.S - t0);
+    const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15;
+    const float scale = rsqrtf((float)DK);
+    const T *qb = static_cast<const T *>(p.q) + ((size_t)bh * p.S + t0) * DK;
     const T *vb = static_cast<const T *>(p.v) + ((size_t)bh * p.S + t0) * DV;
     const T *ob = p.o ? static_cast<const T *>(p.o) + ((size_t)bh * p.S + t0) * DV : nullptr;
     const T *dhb = static_cast<const T *>(p.dh) + ((size_t)bh * p.S + t0) * DV;
     T *dob = p.dog ? static_cast<T *>(p.dog) + ((size_t)bh * p.S + t0) * DV : nullptr;
     float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
     const float *Cc = p.CS + ((size_t)bh * p.NC + c) * DK * DV;
-    const float *nc = p.NS + ((size_t)bh * p.NC + c) * DK;
+    const float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
+    const float *nrm = p.NRM + (size_t)bh * p.S + t0;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
-    for (int t = tid; t < L; t += NT) dot[t] = 0.f;
-    for (int e = tid; e < L * LP; e += NT) {
-        Sm[e] = 0.f;
-        dAg[e] = 0.f;
-    }
-    __syncthreads();
-
-    // S = qh K^T over slices of 32 of DK (lower triangle)
-    for (int d0 = 0; d0 < DK; d0 += 32) {
-        for (int e = tid; e < L * 32; e += NT) {
-            const int t = e >> 5, xx = e & 31;
-            const bool ok = t < len && d0 + xx < DK;
-            qs[t * 33 + xx] = ok ? to_f32(qb[(size_t)t * DK + d0 + xx]) * scale : 0.f;
-            xs[t * 33 + xx] = ok ? to_f32(kb[(size_t)t * DK + d0 + xx]) : 0.f;
-        }
-        __syncthreads();
-        for (int e = tid; e < L * L; e += NT) {
-            const int t = e / L, s = e % L;
-            if (s <= t) {
-                float acc = Sm[t * LP + s];
-#pragma unroll 8
-                for (int xx = 0; xx < 32; ++xx) acc = fmaf(qs[t * 33 + xx], xs[s * 33 + xx], acc);
-                Sm[t * LP + s] = acc;
-            }
-        }
-        __syncthreads();
-    }
-    // A = D * S on the causal triangle (zero elsewhere and past the end of the sequence)
-    for (int e = tid; e < L * L; e += NT) {
-        const int t = e / L, s = e % L;
-        Sm[t * LP + s] = (s <= t && t < len) ? Sm[t * LP + s] * expf(xs_[s] - mx[t]) : 0.f;
-    }
-    __syncthreads();
-    // den and the normalizer N
-    for (int t = tid; t < L; t += NT) {
-        float r = 0.f;
-        for (int s = 0; s <= t; ++s) r += Sm[t * LP + s];
-        float qn = 0.f;
-        if (t < len) {
-            for (int d = 0; d < DK; ++d) qn = fmaf(nc[d], to_f32(qb[(size_t)t * DK + d]), qn);
-            qn *= scale * sc[t];
-        }
-        den[t] = r + qn;
-        nrm[t] = t < len ? fmaxf(fabsf(r + qn), fl[t]) : 1.f;
-    }
-    __syncthreads();
-
-    // value tiles of 32 columns: num, hh = num / N, do, g; sum of g . hh per row; g v^T
-    const int RPT = L / 8;   // rows per thread: t = ty + 8 r
-    for (int j0 = 0; j0 < DV; j0 += 32) {
-        float acc[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
-        for (int d0 = 0; d0 < DK; d0 += 32) {
-            for (int e = tid; e < L * 32; e += NT) {
-                const int t = e >> 5, xx = e & 31;
-                qs[t * 33 + xx] = (t < len && d0 + xx < DK) ? to_f32(qb[(size_t)t * DK + d0 + xx]) * scale : 0.f;
-            }
-            for (int e = tid; e < 32 * 32; e += NT) {
-                const int d = e >> 5, xx = e & 31;
-                cs[d * 33 + xx] = (d0 + d < DK && j0 + xx < DV) ? Cc[(size_t)(d0 + d) * DV + j0 + xx] : 0.f;
+    __syncthreads();   // sc is read by the tile loads
+    const int nmt = (L + GM - 1) / GM;
+    for (int mt = 0; mt < nmt; ++mt) {
+        float acc[4][4] = {};
+        for (int d0 = 0; d0 < DK; d0 += GK) {   // sc qh C_c
+            __syncthreads();
+            for (int e = tid; e < GK * GM; e += NT) {
+                const int m = e >> 5, k = e & 31;
+                const int t = mt * GM + m;
+                As[k * GSTR + m] = (t < len && d0 + k < DK) ? to_f32(qb[(size_t)t * DK + d0 + k]) * scale * sc[t] : 0.f;
+                const int kk = e >> 6, n = e & 63;   // consecutive threads: consecutive value columns
+                Bs[kk * GSTR + n] = (d0 + kk < DK && j0 + n < DV) ? Cc[(size_t)(d0 + kk) * DV + j0 + n] : 0.f;
             }
             __syncthreads();
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int t = ty + 8 * r;
-                if (r < RPT) {
-                    float a2 = 0.f;
-#pragma unroll 8
-                    for (int d = 0; d < 32; ++d) a2 = fmaf(qs[t * 33 + d], cs[d * 33 + x], a2);
-                    acc[r] = fmaf(sc[t], a2, acc[r]);
-                }
+            tile_mma(As, Bs, acc);
+        }
+        for (int s0 = 0; s0 < L; s0 += GK) {    // A V (A is zero past the end and above the diagonal)
+            __syncthreads();
+            for (int e = tid; e < GK * GM; e += NT) {
+                const int m = e >> 5, k = e & 31;
+                const int t = mt * GM + m;
+                As[k * GSTR + m] = (t < L && s0 + k < L) ? AIg[(size_t)t * L + s0 + k] : 0.f;
+                const int kk = e >> 6, n = e & 63;
+                Bs[kk * GSTR + n] = (s0 + kk < len && j0 + n < DV) ? to_f32(vb[(size_t)(s0 + kk) * DV + j0 + n]) : 0.f;
             }
             __syncthreads();
-        }
-        for (int e = tid; e < L * 32; e += NT) {
-            const int s = e >> 5, xx = e & 31;
-            xs[s * 33 + xx] = (s < len && j0 + xx < DV) ? to_f32(vb[(size_t)s * DV + j0 + xx]) : 0.f;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int t = ty + 8 * r;
-            if (r < RPT) {
-                float a2 = 0.f;
-                for (int s = 0; s <= t; ++s) a2 = fmaf(Sm[t * LP + s], xs[s * 33 + x], a2);
-                acc[r] += a2;
-            }
+            tile_mma(As, Bs, acc);
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int t = ty + 8 * r;
-            if (r < RPT) {
-                const int j = j0 + x;
-                float g = 0.f, hh = 0.f;
-                if (t < len && j < DV) {
-                    const size_t off = (size_t)t * DV + j;
-                    hh = acc[r] / nrm[t];
-                    const float dhv = to_f32(dhb[off]);
-                    const float ov = ob ? to_f32(ob[off]) : 1.f;
-                    if (dob) dob[off] = from_f32<T>(dhv * hh);
-                    g = ov * dhv / nrm[t];
-                    gtb[off] = g;
+        for (int a = 0; a < 4; ++a) {
+            const int t = mt * GM + 4 * tm + a;
+            float part = 0.f;
+            if (t < len) {
+                const float N = nrm[t];
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2) {
+                    const int j = j0 + 4 * tn + b2;
+                    if (j < DV) {
+                        const size_t off = (size_t)t * DV + j;
+                        const float hh = acc[a][b2] / N;
+                        const float dhv = to_f32(dhb[off]);
+                        const float ov = ob ? to_f32(ob[off]) : 1.f;
+                        if (dob) dob[off] = from_f32<T>(dhv * hh);
+                        const float g = ov * dhv / N;
+                        gtb[off] = g;
+                        part = fmaf(g, hh, part);
+                    }
                 }
-                gs[t * 33 + x] = g;
-                const float pr = warp_sum(g * hh);   // the warp holds one row t
-                if (x == 0) dot[t] += pr;
             }
+            part = sum16(part);
+            if (tn == 0 && t < len) p.DOTP[((size_t)bh * p.S + t0 + t) * p.NJT + jt] = part;
         }
-        __syncthreads();
-        for (int e = tid; e < L * L; e += NT) {
-            const int t = e / L, s = e % L;
-            if (s <= t && t < len) {
-                float a2 = dAg[t * LP + s];
-#pragma unroll 8
-                for (int xx = 0; xx < 32; ++xx) a2 = fmaf(gs[t * 33 + xx], xs[s * 33 + xx], a2);
-                dAg[t * LP + s] = a2;
-            }
-        }
-        __syncthreads();
     }
+}
 
-    // dden (the branch of the max that the forward pass took), then dS = (g v^T + dden) * D and A
-    for (int t = tid; t < L; t += NT) {
-        const bool live = t < len && fabsf(den[t]) > fl[t];
-        dd[t] = live ? -dot[t] * copysignf(1.f, den[t]) : 0.f;
-        if (t < len) p.DD[(size_t)bh * p.S + t0 + t] = dd[t];
-    }
-    __syncthreads();
+// ---------------------------------------------------------------- per chunk: dden and dS
+// grid (BH, NC): dden_t = -(g_t . hh_t) sign(den_t) where the floor does not bind (-> DD),
+// dS = (g V^T + dden) * D on the causal triangle (-> P2), and the read-out's normalizer gradient
+// dn_c = sum_t sc_t dden_t qh_t (-> GN).
+template <typename T>
+__global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ __align__(16) float As[GK * GSTR], Bs[GK * GSTR];
+    __shared__ float xs_[128], mx[128], fl[128], sc[128], dd[128];
+    const int L = p.L, DK = p.DK, DV = p.DV;
+    const int bh = blockIdx.x, c = blockIdx.y;
+    const int t0 = c * L, len = min(L, p.S - t0);
+    const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15;
+    const float scale = rsqrtf((float)DK);
+    const T *qb = static_cast<const T *>(p.q) + ((size_t)bh * p.S + t0) * DK;
+    const T *vb = static_cast<const T *>(p.v) + ((size_t)bh * p.S + t0) * DV;
+    const float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
     float *P2g = p.P2 + ((size_t)bh * p.NC + c) * L * L;
-    float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
-    for (int e = tid; e < L * L; e += NT) {
-        const int t = e / L, s = e % L;
-        float pv = 0.f;
-        if (s <= t && t < len) pv = (dAg[t * LP + s] + dd[t]) * expf(xs_[s] - mx[t]);
-        P2g[e] = pv;
-        AIg[e] = Sm[t * LP + s];
-    }
 
-    // the read-out's state gradients: dC[i][j] = sum_t sc_t qh_t[i] g_t[j], dn[i] = sum_t sc_t dd_t qh_t[i]
-    float *GSc = p.GS + ((size_t)bh * p.NC + c) * DK * DV;
-    float *GNc = p.GN + ((size_t)bh * p.NC + c) * DK;
-    for (int i0 = 0; i0 < DK; i0 += 32) {
-        __syncthreads();
-        for (int e = tid; e < L * 32; e += NT) {
-            const int t = e >> 5, xx = e & 31;
-            qs[t * 33 + xx] = (t < len && i0 + xx < DK) ? sc[t] * to_f32(qb[(size_t)t * DK + i0 + xx]) * scale : 0.f;
+    chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
+    for (int t = tid; t < L; t += NT) {
+        float v = 0.f;
+        if (t < len) {
+            const size_t r = (size_t)bh * p.S + t0 + t;
+            float dot = 0.f;
+            for (int u = 0; u < p.NJT; ++u) dot += p.DOTP[r * p.NJT + u];
+            const float den = p.DEN[r];
+            if (fabsf(den) > fl[t]) v = -dot * copysignf(1.f, den);
+            p.DD[r] = v;
         }
-        __syncthreads();
-        if (tid < 32 && i0 + tid < DK) {
-            float a2 = 0.f;
-            for (int t = 0; t < len; ++t) a2 = fmaf(qs[t * 33 + tid], dd[t], a2);
-            GNc[i0 + tid] = a2;
-        }
-        for (int j0 = 0; j0 < DV; j0 += 32) {
-            for (int e = tid; e < L * 32; e += NT) {
-                const int t = e >> 5, xx = e & 31;
-                gs[t * 33 + xx] = (t < len && j0 + xx < DV) ? __ldcg(gtb + (size_t)t * DV + j0 + xx) : 0.f;
+        dd[t] = v;
+    }
+    const int nmt = (L + GM - 1) / GM;
+    for (int mt = 0; mt < nmt; ++mt)
+        for (int nt = 0; nt < nmt; ++nt) {
+            if (nt > mt) {   // above the diagonal: zeros
+                for (int e = tid; e < GM * GM; e += NT) {
+                    const int t = mt * GM + e / GM, s2 = nt * GM + e % GM;
+                    if (t < L && s2 < L) P2g[(size_t)t * L + s2] = 0.f;
+                }
+                continue;
             }
-            __syncthreads();
+            float acc[4][4] = {};
+            tile_gemm((DV + GK - 1) / GK,   // g V^T
+                      [&](int st, int e, float &av, float &bv) {
+                          const int m = e >> 5, k = e & 31, j = st * GK + k;
+                          const int ta = mt * GM + m, tb = nt * GM + m;
+                          av = (ta < len && j < DV) ? gtb[(size_t)ta * DV + j] : 0.f;
+                          bv = (tb < len && j < DV) ? to_f32(vb[(size_t)tb * DV + j]) : 0.f;
+                      },
+                      [&](int, int e, float av, float bv) {
+                          As[(e & 31) * GSTR + (e >> 5)] = av;
+                          Bs[(e & 31) * GSTR + (e >> 5)] = bv;
+                      },
+                      As, Bs, acc);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int i = ty + 8 * r;
-                float a2 = 0.f;
-                for (int t = 0; t < len; ++t) a2 = fmaf(qs[t * 33 + i], gs[t * 33 + x], a2);
-                if (i0 + i < DK && j0 + x < DV) GSc[(size_t)(i0 + i) * DV + j0 + x] = a2;
+            for (int a = 0; a < 4; ++a) {
+                const int t = mt * GM + 4 * tm + a;
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2) {
+                    const int s2 = nt * GM + 4 * tn + b2;
+                    float pv = 0.f;
+                    if (s2 <= t && t < len) pv = (acc[a][b2] + dd[t]) * expf(xs_[s2] - mx[t]);
+                    if (t < L && s2 < L) P2g[(size_t)t * L + s2] = pv;
+                }
             }
-            __syncthreads();
+        }
+    __syncthreads();
+    float *GNc = p.GN + ((size_t)bh * p.NC + c) * DK;
+    for (int i = tid; i < DK; i += NT) {
+        float a2 = 0.f;
+        for (int t = 0; t < len; ++t) a2 = fmaf(sc[t] * dd[t], to_f32(qb[(size_t)t * DK + i]) * scale, a2);
+        GNc[i] = a2;
+    }
+}
+
+// ---------------------------------------------------------------- per chunk and 64 x 64 state tile: dC of the read-out
+// grid (BH NC, ceil(DK / 64), NJT): GS[i][j] = sum_t sc_t qh_t[i] g_t[j].
+template <typename T>
+__global__ void __launch_bounds__(NT) bwd_dc_kernel(Params p)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ __align__(16) float As[GK * GSTR], Bs[GK * GSTR];
+    __shared__ float xs_[128], mx[128], fl[128], sc[128];
+    const int L = p.L, DK = p.DK, DV = p.DV;
+    const int bh = blockIdx.x / p.NC, c = blockIdx.x % p.NC;
+    const int i0 = blockIdx.y * GM, j0 = blockIdx.z * GM;
+    const int t0 = c * L, len = min(L, p.S - t0);
+    const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15;
+    const float scale = rsqrtf((float)DK);
+    const T *qb = static_cast<const T *>(p.q) + ((size_t)bh * p.S + t0) * DK;
+    const float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
+    float *GSc = p.GS + ((size_t)bh * p.NC + c) * DK * DV;
+
+    chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
+    __syncthreads();   // sc is read by the tile loads
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < L; k0 += GK) {
+        __syncthreads();
+        for (int e = tid; e < GK * GM; e += NT) {
+            const int k = e >> 6, m = e & 63;   // consecutive threads: consecutive columns
+            const int t = k0 + k;
+            As[k * GSTR + m] = (t < len && i0 + m < DK) ? to_f32(qb[(size_t)t * DK + i0 + m]) * scale * sc[t] : 0.f;
+            Bs[k * GSTR + m] = (t < len && j0 + m < DV) ? gtb[(size_t)t * DV + j0 + m] : 0.f;
+        }
+        __syncthreads();
+        tile_mma(As, Bs, acc);
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int i = i0 + 4 * tm + a;
+        if (i < DK) {
+#pragma unroll
+            for (int b2 = 0; b2 < 4; ++b2) {
+                const int j = j0 + 4 * tn + b2;
+                if (j < DV) GSc[(size_t)i * DV + j] = acc[a][b2];
+            }
         }
     }
 }
@@ -329,31 +470,27 @@ __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
     }
 }
 
-// ---------------------------------------------------------------- per chunk and column tile: dq, dk, dv
-// grid (BH, NC, NTK + NTV), NT threads.  Tiles z < NTK: 32 columns of DK (dq and dk); the rest:
-// 32 columns of DV (dv).  A thread owns column x of the tile for the rows ty + 8 r; the products
-// run with the reduction index outermost, so that a shared value read by the whole warp (a row of
-// the left factor) and one per lane (the lane's column of the right factor) feed the warp's rows,
-// four reduction steps per 16-byte load where the layout allows.
-constexpr int TS = 36;    // row stride of the 32-column tiles (16-byte aligned rows, no bank conflicts)
-
-template <typename T>
-__global__ void __launch_bounds__(NT) bwd_grad_kernel(Params p)
+// ---------------------------------------------------------------- per chunk and 64 columns: dq, dk, dv
+// grid (BH, NC, tiles): KIND 0 computes dq over ceil(DK / 64) tiles, KIND 1 dk over as many, KIND 2
+// dv over NJT tiles, each a product of 64 x 64 outputs with the chunk-local and the inter-chunk
+// terms stacked along the reduction:
+//   dqh = [dS | sc g] [K ; C_c^T] + sc dden n_c,          K = L + DV,
+//   dk  = [dS^T | w v] [qh ; G_end^T] + w dn_end,         K = L + DV,
+//   dv  = [A^T | w k] [g ; G_end],                        K = L + DK,
+// with w_s = exp(g_c - a_s + i~_s - m_{c+1}) the weight of token s in the state at the chunk's end.
+// The dq and dk tiles also leave the partial row sums q . dq and k . dk of their two 32-column
+// halves (QD, KD) for the gate gradients.
+template <typename T, int KIND>
+__global__ void __launch_bounds__(NT, 2) bwd_grad_kernel(Params p)
 {
     griddep_wait();
     griddep_launch_dependents();
-    extern __shared__ float sm[];
-    const int L = p.L, LP = L + 1, DK = p.DK, DV = p.DV;
-    float *Ms = sm;               // [L][LP]: dS (key tiles) or A (value tiles)
-    float *as_ = Ms + L * LP;     // [L][TS]
-    float *bs = as_ + L * TS;     // [L][TS]
-    float *cs = bs + L * TS;      // [32][TS]
-    float *cs2 = cs + 32 * TS;    // [32][TS]
-    float *xs_ = cs2 + 32 * TS, *mx = xs_ + L, *fl = mx + L, *sc = fl + L;
-
+    __shared__ __align__(16) float As[GK * GSTR], Bs[GK * GSTR];
+    __shared__ float xs_[128], mx[128], fl[128], sc[128], wt[128], dd[128];
+    const int L = p.L, DK = p.DK, DV = p.DV;
     const int bh = blockIdx.x, c = blockIdx.y, z = blockIdx.z;
     const int t0 = c * L, len = min(L, p.S - t0);
-    const int tid = threadIdx.x, x = tid & 31, ty = tid >> 5;
+    const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15;
     const float scale = rsqrtf((float)DK);
     const T *qb = static_cast<const T *>(p.q) + ((size_t)bh * p.S + t0) * DK;
     const T *kb = static_cast<const T *>(p.k) + ((size_t)bh * p.S + t0) * DK;
@@ -363,151 +500,107 @@ __global__ void __launch_bounds__(NT) bwd_grad_kernel(Params p)
     const float *nc = p.NS + ((size_t)bh * p.NC + c) * DK;
     const float *Ge = p.GS + ((size_t)bh * p.NC + c) * DK * DV;   // gradient of the state at the chunk's end
     const float *ge = p.GN + ((size_t)bh * p.NC + c) * DK;
-    const float *ddb = p.DD + (size_t)bh * p.S + t0;
-    const float gc = p.G[(size_t)bh * p.NC + c], mn = p.MC[(size_t)bh * (p.NC + 1) + c + 1];
-    const int RPT = L / 8;
+    const float *P2g = p.P2 + ((size_t)bh * p.NC + c) * L * L;
+    const float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
-    const float *Mg = (z < p.NTK ? p.P2 : p.AI) + ((size_t)bh * p.NC + c) * L * L;
-    for (int e = tid; e < L * L; e += NT) Ms[(e / L) * LP + e % L] = Mg[e];
-    __syncthreads();
-    // w_s = exp(g_c - a_s + i~_s - m_{c+1}): weight of token s in the state at the chunk's end
-    const float gm = gc - mn;
-    auto wtok = [&](int s) { return s < len ? expf(xs_[s] + gm) : 0.f; };
-
-    if (z < p.NTK) {
-        const int i0 = z * 32;
-        const int i = i0 + x;
-        for (int e = tid; e < L * 32; e += NT) {
-            const int t = e >> 5, xx = e & 31;
-            const bool ok = t < len && i0 + xx < DK;
-            as_[t * TS + xx] = ok ? to_f32(kb[(size_t)t * DK + i0 + xx]) : 0.f;
-            bs[t * TS + xx] = ok ? to_f32(qb[(size_t)t * DK + i0 + xx]) * scale : 0.f;
+    {
+        const float gm = p.G[(size_t)bh * p.NC + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1];
+        for (int t = tid; t < L; t += NT) {
+            wt[t] = t < len ? expf(xs_[t] + gm) : 0.f;
+            dd[t] = t < len ? p.DD[(size_t)bh * p.S + t0 + t] : 0.f;
         }
-        __syncthreads();
-        float aq[16], ak[16], iq[16], ik[16];
+    }
+    __syncthreads();   // sc, wt and dd are read by the tile loads
+    constexpr int kind = KIND;                 // dq, dk, dv
+    const int c0 = z * GM;                     // first output column
+    const int NC_ = kind == 2 ? DV : DK;       // output columns
+    const int nmt = (L + GM - 1) / GM;
+    for (int mt = 0; mt < nmt; ++mt) {
+        float acc[4][4] = {};
+        // the chunk-local term (reduction over the chunk's tokens), then the inter-chunk term
+        // (over DV for dq and dk, over DK for dv)
+        const int KI = kind == 2 ? DK : DV;
+        const int nloc = (L + GK - 1) / GK;
+        tile_gemm(nloc + (KI + GK - 1) / GK,
+                  [&](int st, int e, float &av, float &bv) {
+                      if (st < nloc) {
+                          const int k0 = st * GK;
+                          if (kind == 0) {          // As[u][t] = dS[t][u]
+                              const int m = e >> 5, k = e & 31, t = mt * GM + m;
+                              av = (t < L && k0 + k < L) ? P2g[(size_t)t * L + k0 + k] : 0.f;
+                          } else {                  // As[u][s] = dS[u][s] or A[u][s]
+                              const int k = e >> 6, m = e & 63, s2 = mt * GM + m;
+                              av = (s2 < L && k0 + k < L) ? (kind == 1 ? P2g : AIg)[(size_t)(k0 + k) * L + s2] : 0.f;
+                          }
+                          const int kk = e >> 6, n = e & 63, u = k0 + kk;   // Bs[u][col]: k, qh or g
+                          bv = 0.f;
+                          if (u < len && c0 + n < NC_) {
+                              if (kind == 0) bv = to_f32(kb[(size_t)u * DK + c0 + n]);
+                              else if (kind == 1) bv = to_f32(qb[(size_t)u * DK + c0 + n]) * scale;
+                              else bv = gtb[(size_t)u * DV + c0 + n];
+                          }
+                      } else {
+                          const int k0 = (st - nloc) * GK;
+                          const int m = e >> 5, k = e & 31, r = mt * GM + m;   // row r of the output tile
+                          av = 0.f;
+                          if (r < len && k0 + k < KI) {
+                              if (kind == 0) av = sc[r] * gtb[(size_t)r * DV + k0 + k];
+                              else if (kind == 1) av = wt[r] * to_f32(vb[(size_t)r * DV + k0 + k]);
+                              else av = wt[r] * to_f32(kb[(size_t)r * DK + k0 + k]);
+                          }
+                          if (kind == 2) {           // Bs[i][j] = G_end[i][j]
+                              const int kk = e >> 6, n = e & 63;
+                              bv = (k0 + kk < DK && c0 + n < DV) ? Ge[(size_t)(k0 + kk) * DV + c0 + n] : 0.f;
+                          } else {                   // Bs[j][i] = C_c[i][j] or G_end[i][j]
+                              const int n = e >> 5, kk = e & 31;
+                              bv = (c0 + n < DK && k0 + kk < DV) ? (kind == 0 ? Cc : Ge)[(size_t)(c0 + n) * DV + k0 + kk] : 0.f;
+                          }
+                      }
+                  },
+                  [&](int st, int e, float av, float bv) {
+                      if (st < nloc) {
+                          if (kind == 0) As[(e & 31) * GSTR + (e >> 5)] = av;
+                          else As[(e >> 6) * GSTR + (e & 63)] = av;
+                          Bs[(e >> 6) * GSTR + (e & 63)] = bv;
+                      } else {
+                          As[(e & 31) * GSTR + (e >> 5)] = av;
+                          if (kind == 2) Bs[(e >> 6) * GSTR + (e & 63)] = bv;
+                          else Bs[(e & 31) * GSTR + (e >> 5)] = bv;
+                      }
+                  },
+                  As, Bs, acc);
+        // epilogue
 #pragma unroll
-        for (int r = 0; r < 16; ++r) aq[r] = ak[r] = iq[r] = ik[r] = 0.f;
-        // dS K (row t: sum_s dS_ts k_s) and dS^T qh (row t: sum_u dS_ut qh_u); dS is zero above the
-        // diagonal and past the end of the sequence
-        for (int s = 0; s < L; ++s) {
-            const float ks = as_[s * TS + x], qs = bs[s * TS + x];
+        for (int a = 0; a < 4; ++a) {
+            const int r = mt * GM + 4 * tm + a;
+            float part = 0.f;
+            if (r < len) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                if (r < RPT) {
-                    const int t = ty + 8 * r;
-                    aq[r] = fmaf(Ms[t * LP + s], ks, aq[r]);
-                    ak[r] = fmaf(Ms[s * LP + t], qs, ak[r]);
-                }
-            }
-        }
-        // inter-chunk parts over slices of 32 of DV: g C_c^T (rows t) and V G_end^T (rows s)
-        for (int j0 = 0; j0 < DV; j0 += 32) {
-            __syncthreads();
-            for (int e = tid; e < L * 32; e += NT) {
-                const int t = e >> 5, xx = e & 31;
-                const bool ok = t < len && j0 + xx < DV;
-                as_[t * TS + xx] = ok ? gtb[(size_t)t * DV + j0 + xx] : 0.f;
-                bs[t * TS + xx] = ok ? to_f32(vb[(size_t)t * DV + j0 + xx]) : 0.f;
-            }
-            for (int e = tid; e < 32 * 32; e += NT) {
-                const int ii = e >> 5, xx = e & 31;
-                const bool ok = i0 + ii < DK && j0 + xx < DV;
-                cs[ii * TS + xx] = ok ? Cc[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
-                cs2[ii * TS + xx] = ok ? Ge[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
-            }
-            __syncthreads();
-#pragma unroll 2
-            for (int jj = 0; jj < 32; jj += 4) {
-                const float4 c4 = *reinterpret_cast<const float4 *>(cs + x * TS + jj);
-                const float4 e4 = *reinterpret_cast<const float4 *>(cs2 + x * TS + jj);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    if (r < RPT) {
-                        const int t = ty + 8 * r;
-                        const float4 g4 = *reinterpret_cast<const float4 *>(as_ + t * TS + jj);
-                        const float4 v4 = *reinterpret_cast<const float4 *>(bs + t * TS + jj);
-                        iq[r] = fmaf(g4.x, c4.x, fmaf(g4.y, c4.y, fmaf(g4.z, c4.z, fmaf(g4.w, c4.w, iq[r]))));
-                        ik[r] = fmaf(v4.x, e4.x, fmaf(v4.y, e4.y, fmaf(v4.z, e4.z, fmaf(v4.w, e4.w, ik[r]))));
+                for (int b2 = 0; b2 < 4; ++b2) {
+                    const int col = c0 + 4 * tn + b2;
+                    if (col < NC_) {
+                        if (kind == 0) {
+                            const float dqh = acc[a][b2] + sc[r] * dd[r] * nc[col];
+                            static_cast<T *>(p.dq)[((size_t)bh * p.S + t0 + r) * DK + col] = from_f32<T>(dqh * scale);
+                            part = fmaf(to_f32(qb[(size_t)r * DK + col]) * scale, dqh, part);
+                        } else if (kind == 1) {
+                            const float dkv = acc[a][b2] + wt[r] * ge[col];
+                            static_cast<T *>(p.dk)[((size_t)bh * p.S + t0 + r) * DK + col] = from_f32<T>(dkv);
+                            part = fmaf(to_f32(kb[(size_t)r * DK + col]), dkv, part);
+                        } else {
+                            static_cast<T *>(p.dv)[((size_t)bh * p.S + t0 + r) * DV + col] = from_f32<T>(acc[a][b2]);
+                        }
                     }
                 }
             }
-        }
-        const float ncx = i < DK ? nc[i] : 0.f, gex = i < DK ? ge[i] : 0.f;
-        T *dqb = static_cast<T *>(p.dq) + ((size_t)bh * p.S + t0) * DK;
-        T *dkb = static_cast<T *>(p.dk) + ((size_t)bh * p.S + t0) * DK;
+            if (kind < 2) {   // partial sums of the tile's two 32-column halves (8 threads each)
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int t = ty + 8 * r;
-            if (r < RPT) {
-                float qdq = 0.f, kdk = 0.f;
-                if (t < len && i < DK) {
-                    const float dqh = aq[r] + sc[t] * (iq[r] + ddb[t] * ncx);
-                    const float dkv = ak[r] + wtok(t) * (ik[r] + gex);
-                    const float qh = to_f32(qb[(size_t)t * DK + i]) * scale;
-                    const float kv = to_f32(kb[(size_t)t * DK + i]);
-                    dqb[(size_t)t * DK + i] = from_f32<T>(dqh * scale);
-                    dkb[(size_t)t * DK + i] = from_f32<T>(dkv);
-                    qdq = qh * dqh;
-                    kdk = kv * dkv;
-                }
-                qdq = warp_sum(qdq);
-                kdk = warp_sum(kdk);
-                if (x == 0 && t < len) {
-                    p.QD[((size_t)bh * p.S + t0 + t) * p.NTK + z] = qdq;
-                    p.KD[((size_t)bh * p.S + t0 + t) * p.NTK + z] = kdk;
-                }
+                for (int o = 4; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                const int half = (c0 >> 5) + (tn >> 3);
+                if ((tn & 7) == 0 && r < len && half * 32 < DK)
+                    (kind == 0 ? p.QD : p.KD)[((size_t)bh * p.S + t0 + r) * p.NTK + half] = part;
             }
-        }
-    } else {
-        const int j0 = (z - p.NTK) * 32;
-        const int j = j0 + x;
-        for (int e = tid; e < L * 32; e += NT) {
-            const int t = e >> 5, xx = e & 31;
-            as_[t * TS + xx] = (t < len && j0 + xx < DV) ? gtb[(size_t)t * DV + j0 + xx] : 0.f;
-        }
-        __syncthreads();
-        float av[16], iv[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) av[r] = iv[r] = 0.f;
-        // A^T g (row s: sum_u A_us g_u); A is zero above the diagonal and past the end
-        for (int u = 0; u < L; ++u) {
-            const float gu = as_[u * TS + x];
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r < RPT) av[r] = fmaf(Ms[u * LP + ty + 8 * r], gu, av[r]);
-        }
-        // K G_end over slices of 32 of DK; the slice of G_end transposed ([value column][DK]) so that
-        // a lane reads its column's four DK entries at once
-        float *gT = cs2;
-        for (int i0 = 0; i0 < DK; i0 += 32) {
-            __syncthreads();
-            for (int e = tid; e < L * 32; e += NT) {
-                const int t = e >> 5, xx = e & 31;
-                bs[t * TS + xx] = (t < len && i0 + xx < DK) ? to_f32(kb[(size_t)t * DK + i0 + xx]) : 0.f;
-            }
-            for (int e = tid; e < 32 * 32; e += NT) {
-                const int ii = e >> 5, xx = e & 31;
-                gT[xx * TS + ii] = (i0 + ii < DK && j0 + xx < DV) ? Ge[(size_t)(i0 + ii) * DV + j0 + xx] : 0.f;
-            }
-            __syncthreads();
-#pragma unroll 2
-            for (int ii = 0; ii < 32; ii += 4) {
-                const float4 e4 = *reinterpret_cast<const float4 *>(gT + x * TS + ii);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    if (r < RPT) {
-                        const float4 k4 = *reinterpret_cast<const float4 *>(bs + (ty + 8 * r) * TS + ii);
-                        iv[r] = fmaf(k4.x, e4.x, fmaf(k4.y, e4.y, fmaf(k4.z, e4.z, fmaf(k4.w, e4.w, iv[r]))));
-                    }
-                }
-            }
-        }
-        T *dvb = static_cast<T *>(p.dv) + ((size_t)bh * p.S + t0) * DV;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int s = ty + 8 * r;
-            if (r < RPT && s < len && j < DV) dvb[(size_t)s * DV + j] = from_f32<T>(av[r] + wtok(s) * iv[r]);
         }
     }
 }
@@ -562,18 +655,21 @@ __global__ void __launch_bounds__(GT) bwd_gate_kernel(Params p)
 template <typename T>
 cudaError_t launch_t(const Params &p, int BH, cudaStream_t st)
 {
-    const int ntv = (p.DV + TW - 1) / TW;
-    const size_t sm1 = sizeof(float) * chunk_smem_floats(p.L);
-    const size_t sm2 = sizeof(float) * grad_smem_floats(p.L);
     cudaError_t e;
-    if ((e = ensure_dynamic_smem((const void *)bwd_chunk_kernel<T>, (int)sm1)) != cudaSuccess) return e;
-    if ((e = ensure_dynamic_smem((const void *)bwd_grad_kernel<T>, (int)sm2)) != cudaSuccess) return e;
-    e = launch_kernel(bwd_chunk_kernel<T>, dim3(BH, p.NC), dim3(NT), sm1, st, 1, p);
+    e = launch_kernel(bwd_scores_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(bwd_num_kernel<T>, dim3(BH, p.NC, p.NJT), dim3(NT), 0, st, 1, p);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(bwd_ds_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
     e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV + 255) / 256, BH), dim3(256), 0, st, 1, p);
     if (e != cudaSuccess) return e;
-    e = launch_kernel(bwd_grad_kernel<T>, dim3(BH, p.NC, p.NTK + ntv), dim3(NT), sm2, st, 1, p);
-    if (e != cudaSuccess) return e;
+    const int nk = (p.DK + GM - 1) / GM;
+    if ((e = launch_kernel(bwd_grad_kernel<T, 0>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
+    if ((e = launch_kernel(bwd_grad_kernel<T, 1>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
+    if ((e = launch_kernel(bwd_grad_kernel<T, 2>, dim3(BH, p.NC, p.NJT), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
     return launch_kernel(bwd_gate_kernel, dim3(BH), dim3(GT), 0, st, 1, p);
 }
 
@@ -586,6 +682,7 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     p.q = a.q; p.k = a.k; p.v = a.v; p.o = a.ogate; p.dh = a.dh; p.ig = a.igate; p.fg = a.fgate;
     p.A = w.A; p.P = w.M; p.MC = w.MC; p.G = w.G; p.CS = w.CS; p.NS = w.NS;
     p.GS = w.GS; p.GN = w.GN; p.Gt = w.Gt; p.DD = w.DD; p.P2 = w.P2; p.AI = w.AI; p.QD = w.QD; p.KD = w.KD;
+    p.DEN = w.DEN; p.NRM = w.NRM; p.DOTP = w.DOTP; p.NJT = (a.DHV + 63) / 64;
     p.dq = a.dq; p.dk = a.dk; p.dv = a.dv; p.dog = a.ogate ? a.dogate : nullptr; p.dig = a.digate; p.dfg = a.dfgate;
     return a.bf16 ? bwd::launch_t<__nv_bfloat16>(p, a.BH, a.stream) : bwd::launch_t<float>(p, a.BH, a.stream);
 }

@@ -95,6 +95,9 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->AI = reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
     w->QD = reinterpret_cast<float *>(take(f * BH * S * NTK));
     w->KD = reinterpret_cast<float *>(take(f * BH * S * NTK));
+    w->DEN = reinterpret_cast<float *>(take(f * BH * S));
+    w->NRM = reinterpret_cast<float *>(take(f * BH * S));
+    w->DOTP = reinterpret_cast<float *>(take(f * BH * S * ((DHV + 63) / 64)));
     return off;
 }
 

@@ -78,6 +78,8 @@ struct BwdWorkspace {
     float *DD;                    // [BH][S] gradient of the denominator
     float *P2, *AI;               // [BH][NC][chunk][chunk] score gradients and scores
     float *QD, *KD;               // [BH][S][ceil(DHQK / 32)] partial q . dq, k . dk
+    float *DEN, *NRM;             // [BH][S] read-out denominator and its floored magnitude
+    float *DOTP;                  // [BH][S][ceil(DHV / 64)] partial row sums of g . hh
 };
 
 // Records the caller's phase events (mlstm_fwd_profiled); a no-op without events.
