@@ -51,7 +51,7 @@ struct Params {
     const void *q, *k, *v, *o, *dh;
     const float *ig, *fg;
     const float *A, *P, *MC, *G;     // gate preprocessing
-    const float *CS, *NS;            // chunk-start states [BH][NC][DK][DV], [BH][NC][DK]
+    float *CS, *NS;                  // chunk-start states [BH][NC][DK][DV], [BH][NC][DK]
     float *GS, *GN;                  // read-out state gradients, then chunk-end gradients (same layout)
     float *Gt;                       // g = o dh / N [BH][S][DV]
     float *DD;                       // dden [BH][S]
@@ -427,32 +427,43 @@ __global__ void __launch_bounds__(NT) bwd_dc_kernel(Params p)
 }
 
 // ---------------------------------------------------------------- reverse scan of the state gradients
-// grid (ceil(DK * DV / 256), BH): each thread one state element; G_c = dC_c + decay_c G_{c+1}, the
+// grid (ceil(DK * DV / 1024), BH): each thread four state elements; G_c = dC_c + decay_c G_{c+1}, the
 // slot of chunk c then holds G_{c+1} (the gradient of the state at the chunk's end).
 __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
 {
     griddep_wait();
     griddep_launch_dependents();
+    constexpr int SCAN_CHUNKS = 256;                   // decay factors staged per pass
+    __shared__ float decay[SCAN_CHUNKS];
     const int bh = blockIdx.y;
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
     const float *Gb = p.G + (size_t)bh * p.NC;
     const size_t nstate = (size_t)p.DK * p.DV;
-    if (e < p.DK * p.DV) {
-        float *slot = p.GS + (size_t)bh * p.NC * nstate + e;
-        float G = 0.f;
-        constexpr int BATCH = 8;
-        for (int c1 = p.NC; c1 > 0; c1 -= BATCH) {   // chunks c1 - 1 down to c1 - BATCH, loads first
-            float d[BATCH];
+    const size_t nq = nstate / 4;                      // DK DV is a multiple of 4 (DK % 8 == 0)
+    const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;   // a quad of state elements
+    float4 *slot = reinterpret_cast<float4 *>(p.GS + (size_t)bh * p.NC * nstate) + e;
+    float4 G = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = p.NC; c0 > 0; c0 -= SCAN_CHUNKS) {
+        // the decay factors of chunks cb .. c0 - 1, once per CTA
+        const int cb = max(0, c0 - SCAN_CHUNKS);
+        __syncthreads();
+        for (int c = cb + threadIdx.x; c < c0; c += blockDim.x) decay[c - cb] = expf(Gb[c] + MCb[c] - MCb[c + 1]);
+        __syncthreads();
+        if (e < nq) {
+            constexpr int BATCH = 8;
+            for (int c1 = c0; c1 > cb; c1 -= BATCH) {   // chunks c1 - 1 down to c1 - BATCH, loads first
+                float4 d[BATCH];
 #pragma unroll
-            for (int u = 0; u < BATCH; ++u)
-                if (c1 - 1 - u >= 0) d[u] = __ldcg(slot + (size_t)(c1 - 1 - u) * nstate);
+                for (int u = 0; u < BATCH; ++u)
+                    if (c1 - 1 - u >= cb) d[u] = __ldcg(slot + (size_t)(c1 - 1 - u) * nq);
 #pragma unroll
-            for (int u = 0; u < BATCH; ++u) {
-                const int c = c1 - 1 - u;
-                if (c >= 0) {
-                    slot[(size_t)c * nstate] = G;
-                    G = d[u] + expf(Gb[c] + MCb[c] - MCb[c + 1]) * G;
+                for (int u = 0; u < BATCH; ++u) {
+                    const int c = c1 - 1 - u;
+                    if (c >= cb) {
+                        slot[(size_t)c * nq] = G;
+                        const float f = decay[c - cb];
+                        G = make_float4(d[u].x + f * G.x, d[u].y + f * G.y, d[u].z + f * G.z, d[u].w + f * G.w);
+                    }
                 }
             }
         }
@@ -664,7 +675,7 @@ cudaError_t launch_t(const Params &p, int BH, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
-    e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV + 255) / 256, BH), dim3(256), 0, st, 1, p);
+    e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV / 4 + 255) / 256, BH), dim3(256), 0, st, 1, p);
     if (e != cudaSuccess) return e;
     const int nk = (p.DK + GM - 1) / GM;
     if ((e = launch_kernel(bwd_grad_kernel<T, 0>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
