@@ -32,6 +32,7 @@ def test_oversize_shape_is_rejected_before_any_launch():
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("B,NH,S,DK,DV,ch,dt", [(1, 4, 1024, 256, 256, 64, "bf16"),
+                                                 (1, 2, 700, 256, 512, 128, "bf16"),   # the paired walk
                                                  (1, 2, 100, 32, 32, 16, "f32")])
 def test_noalloc_matches_fwd_on_two_calls_in_a_row(cuda_lib, B, NH, S, DK, DV, ch, dt):
     need = binding.workspace_size(B, NH, S, DK, DV, ch, torch.bfloat16 if dt == "bf16" else torch.float32)
