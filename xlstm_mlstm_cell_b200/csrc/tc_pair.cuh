@@ -141,13 +141,5 @@ __device__ __forceinline__ void mma_commit_to(uint32_t bar_cluster)
                  : "memory");
 }
 
-// The same arrival on the barrier at this offset in both CTAs of the pair (two commits, no
-// multicast).
-__device__ __forceinline__ void mma_commit_pair(uint64_t *bar)
-{
-    mma_commit_to(map_to_rank(bar, 0));
-    mma_commit_to(map_to_rank(bar, 1));
-}
-
 }  // namespace tc
 }  // namespace mlstm
