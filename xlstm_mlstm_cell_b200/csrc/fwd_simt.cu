@@ -28,11 +28,51 @@ namespace mlstm {
 constexpr int ST = 32;   // state tile edge (rows of C and columns of C / h)
 
 // ---------------------------------------------------------------- carry
-// grid (BH, ceil(DHQK/32), ceil(DHV/32)), 256 threads; a thread owns 4 rows x 1 column
-// of a 32 x 32 tile of C.  Walks all chunks of its head in order, storing the
-// state at every chunk start (CS) and the final state.
+// grid (BH, ceil(DHQK/64), ceil(DHV/64)), 256 threads; thread (tx, ty) = (tid % 16, tid / 16)
+// owns rows 4 ty .. 4 ty + 3 and columns 4 tx .. 4 tx + 3 of a 64 x 64 tile of C, and in the tiles
+// of columns 0..63 threads 0..63 own n of their row.  Walks all chunks of its head in order,
+// storing the state at every chunk start (CS, NS) and the final state.  A chunk's k (fp32) and
+// w_s v_s are staged in shared memory, so that a step of the reduction over the chunk's tokens is
+// two 16-byte loads and 16 FMAs per thread; the next chunk's k, v and gates are loaded into
+// registers while the current chunk's steps run.  Every state element takes the operations of a
+// token-by-token fp32 update in their order: C <- decay C, then C += k_s (w_s v_s) for s
+// ascending (n <- decay n, then n += w_s k_s).
+constexpr int CT = 64;         // state tile edge of the carry
+constexpr int CKS = CT + 4;    // row stride (floats) of the staged tiles: rows 16 bytes apart in the banks
+
+// Eight consecutive elements of a k or v row as loaded (16-byte aligned), converted on staging.
+template <typename T> struct Seg8;
+template <> struct Seg8<float> {
+    float4 a, b;
+    MLSTM_DEVINL void load(const float *p)
+    {
+        a = *reinterpret_cast<const float4 *>(p);
+        b = *reinterpret_cast<const float4 *>(p + 4);
+    }
+    MLSTM_DEVINL void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    MLSTM_DEVINL void get(float (&f)[8]) const
+    {
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+};
+template <> struct Seg8<__nv_bfloat16> {
+    uint4 u;
+    MLSTM_DEVINL void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+    MLSTM_DEVINL void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+    MLSTM_DEVINL void get(float (&f)[8]) const
+    {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {   // bf16 -> fp32 is exact: the 16 bits are the high half
+            f[2 * z] = __uint_as_float(w[z] << 16);
+            f[2 * z + 1] = __uint_as_float(w[z] & 0xffff0000u);
+        }
+    }
+};
+
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ igate,
                   const float *__restrict__ A, const float *__restrict__ G, const float *__restrict__ MC,
                   int S, int L, int NC, int DHQK, int DHV,
@@ -42,73 +82,139 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
     griddep_wait();
     griddep_launch_dependents();
     extern __shared__ float sm[];
-    float *ks = sm;                    // [L][ST]
-    float *vs = ks + L * ST;           // [L][ST]
-    float *ws = vs + L * ST;           // [L]
-    const int bh = blockIdx.x, i0 = blockIdx.y * ST, j0 = blockIdx.z * ST;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // column, row group
-    const int j = j0 + tx;
-    const bool do_n = blockIdx.z == 0 && ty == 0;              // warp 0 of dv tile 0 keeps n
+    float *ks = sm;                    // [L][CKS] k_s, this tile's rows
+    float *wvs = ks + L * CKS;         // [L][CKS] w_s v_s, this tile's columns
+    float *wsb = wvs + L * CKS;        // [L] w_s
+    const int bh = blockIdx.x, i0 = blockIdx.y * CT, j0 = blockIdx.z * CT;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const bool n_warp = blockIdx.z == 0 && tid < CT;            // warps 0 and 1 of column tile 0
     const T *kb = k + (size_t)bh * S * DHQK;
     const T *vb = v + (size_t)bh * S * DHV;
     const float *igb = igate + (size_t)bh * S;
     const float *Ab = A + (size_t)bh * S;
-    // initial state (zero when C0 is NULL); C_final may alias C0: every element is read here,
-    // by the thread that writes it at the end
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
-    float nn = 0.f;
-    if (C0) {
+    const float *MCb = MC + (size_t)bh * (NC + 1);
+    const float *Gb = G + (size_t)bh * NC;
+    // the state elements of this thread: rows ri + r, columns cj .. cj + 3 (a group of four columns
+    // lies wholly inside or outside DHV, which is a multiple of 8)
+    const int ri = i0 + 4 * ty, cj = j0 + 4 * tx;
+    const bool cols_in = cj < DHV;
+
+    // initial state (zero when C0 is NULL); C_final may alias C0: every element is read here, by the
+    // thread that writes it at the end
+    float c[4][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = i0 + ty * 4 + r;
-            if (i < DHQK && j < DHV) c[r] = C0[((size_t)bh * DHQK + i) * DHV + j];
-        }
+    for (int r = 0; r < 4; ++r) {
+        float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (C0 && cols_in && ri + r < DHQK) x4 = *reinterpret_cast<const float4 *>(C0 + ((size_t)bh * DHQK + ri + r) * DHV + cj);
+        c[r][0] = x4.x; c[r][1] = x4.y; c[r][2] = x4.z; c[r][3] = x4.w;
     }
-    if (n0 && do_n && i0 + tx < DHQK) nn = n0[(size_t)bh * DHQK + i0 + tx];
+    float nn = 0.f;
+    if (n0 && n_warp && i0 + tid < DHQK) nn = n0[(size_t)bh * DHQK + i0 + tid];
+
+    // staging: thread tid takes row tid / 4 (and tid / 4 + 64 when L = 128) and the 16 columns
+    // 16 (tid % 4) .. of the k and v tiles, as two 8-element halves (each wholly inside or outside
+    // DHQK / DHV)
+    const int sl = tid >> 2, xp = (tid & 3) * 16;
+    Seg8<T> pk[2][2], pv[2][2];
+    float pa[2] = {0.f, 0.f}, pig[2] = {0.f, 0.f};
+    auto load_chunk = [&](int ch) {
+        const int t0 = ch * L, len = min(L, S - t0);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int s = sl + 64 * u;
+            const bool valid = s < len;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int xk = i0 + xp + 8 * h, xv = j0 + xp + 8 * h;
+                if (valid && xk < DHQK) pk[u][h].load(kb + (size_t)(t0 + s) * DHQK + xk);
+                else pk[u][h].zero();
+                if (valid && xv < DHV) pv[u][h].load(vb + (size_t)(t0 + s) * DHV + xv);
+                else pv[u][h].zero();
+            }
+            if (valid) {
+                pa[u] = Ab[t0 + s];
+                pig[u] = igb[t0 + s];
+            }
+        }
+    };
+    if (NC > 0) load_chunk(0);
 
     for (int ch = 0; ch < NC; ++ch) {
         const int t0 = ch * L, len = min(L, S - t0);
         // state at the chunk start
         float *cs = CS + ((size_t)bh * NC + ch) * DHQK * DHV;
+        if (cols_in) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = i0 + ty * 4 + r;
-            if (i < DHQK && j < DHV) cs[(size_t)i * DHV + j] = c[r];
+            for (int r = 0; r < 4; ++r)
+                if (ri + r < DHQK)
+                    *reinterpret_cast<float4 *>(cs + (size_t)(ri + r) * DHV + cj) = make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
         }
-        if (do_n && i0 + tx < DHQK) NS[((size_t)bh * NC + ch) * DHQK + i0 + tx] = nn;
+        if (n_warp && i0 + tid < DHQK) NS[((size_t)bh * NC + ch) * DHQK + i0 + tid] = nn;
 
-        const float mc = MC[(size_t)bh * (NC + 1) + ch], mn = MC[(size_t)bh * (NC + 1) + ch + 1];
-        const float g = G[(size_t)bh * NC + ch];
+        const float mc = MCb[ch], mn = MCb[ch + 1];
+        const float g = Gb[ch];
         const float decay = expf(g + mc - mn);
-        __syncthreads();
-        for (int e = threadIdx.x; e < len * ST; e += blockDim.x) {
-            const int s = e / ST, x = e % ST;
-            ks[e] = (i0 + x < DHQK) ? to_f32(kb[(size_t)(t0 + s) * DHQK + i0 + x]) : 0.f;
-            vs[e] = (j0 + x < DHV) ? to_f32(vb[(size_t)(t0 + s) * DHV + j0 + x]) : 0.f;
-        }
-        for (int s = threadIdx.x; s < len; s += blockDim.x)
-            ws[s] = expf(g - Ab[t0 + s] + igb[t0 + s] - mn);
-        __syncthreads();
+        __syncthreads();   // the previous chunk's steps have read the staged tiles
 #pragma unroll
-        for (int r = 0; r < 4; ++r) c[r] *= decay;
+        for (int u = 0; u < 2; ++u) {
+            const int s = sl + 64 * u;
+            if (s < L) {
+                const float w = s < len ? expf(g - pa[u] + pig[u] - mn) : 0.f;
+                if ((tid & 3) == 0) wsb[s] = w;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float f[8];
+                    pk[u][h].get(f);
+                    float *kd = ks + s * CKS + xp + 8 * h;
+                    *reinterpret_cast<float4 *>(kd) = make_float4(f[0], f[1], f[2], f[3]);
+                    *reinterpret_cast<float4 *>(kd + 4) = make_float4(f[4], f[5], f[6], f[7]);
+                    pv[u][h].get(f);
+                    float *vd = wvs + s * CKS + xp + 8 * h;
+                    *reinterpret_cast<float4 *>(vd) = make_float4(w * f[0], w * f[1], w * f[2], w * f[3]);
+                    *reinterpret_cast<float4 *>(vd + 4) = make_float4(w * f[4], w * f[5], w * f[6], w * f[7]);
+                }
+            }
+        }
+        __syncthreads();
+        if (ch + 1 < NC) load_chunk(ch + 1);   // lands while the steps below run
+
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) c[r][x] *= decay;
         nn *= decay;
-        for (int s = 0; s < len; ++s) {
-            const float wv = ws[s] * vs[s * ST + tx];
+        if (n_warp) {
+            for (int s = 0; s < len; ++s) {
+                const float4 kk = *reinterpret_cast<const float4 *>(ks + s * CKS + 4 * ty);
+                const float4 vv = *reinterpret_cast<const float4 *>(wvs + s * CKS + 4 * tx);
+                const float kr[4] = {kk.x, kk.y, kk.z, kk.w}, vr[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) c[r] = fmaf(ks[s * ST + ty * 4 + r], wv, c[r]);
-            if (do_n) nn = fmaf(ws[s], ks[s * ST + tx], nn);
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) c[r][x] = fmaf(kr[r], vr[x], c[r][x]);
+                nn = fmaf(wsb[s], ks[s * CKS + tid], nn);
+            }
+        } else {
+            for (int s = 0; s < len; ++s) {
+                const float4 kk = *reinterpret_cast<const float4 *>(ks + s * CKS + 4 * ty);
+                const float4 vv = *reinterpret_cast<const float4 *>(wvs + s * CKS + 4 * tx);
+                const float kr[4] = {kk.x, kk.y, kk.z, kk.w}, vr[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) c[r][x] = fmaf(kr[r], vr[x], c[r][x]);
+            }
         }
     }
-    if (C_final) {
+    if (C_final && cols_in) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int i = i0 + ty * 4 + r;
-            if (i < DHQK && j < DHV) C_final[((size_t)bh * DHQK + i) * DHV + j] = c[r];
-        }
+        for (int r = 0; r < 4; ++r)
+            if (ri + r < DHQK)
+                *reinterpret_cast<float4 *>(C_final + ((size_t)bh * DHQK + ri + r) * DHV + cj) =
+                    make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
     }
-    if (n_final && do_n && i0 + tx < DHQK) n_final[(size_t)bh * DHQK + i0 + tx] = nn;
-    if (m_final && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
-        m_final[bh] = MC[(size_t)bh * (NC + 1) + NC];
+    if (n_final && n_warp && i0 + tid < DHQK) n_final[(size_t)bh * DHQK + i0 + tid] = nn;
+    if (m_final && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) m_final[bh] = MCb[NC];
 }
 
 // ---------------------------------------------------------------- output
@@ -256,11 +362,14 @@ template <typename T>
 static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark)
 {
     const int L = a.chunk;
-    dim3 g1(a.BH, (a.DHQK + ST - 1) / ST, (a.DHV + ST - 1) / ST);
-    const size_t sm1 = sizeof(float) * (2 * (size_t)L * ST + L);
-    cudaError_t e = launch_kernel(carry_simt_kernel<T>, g1, dim3(256), sm1, a.stream, 1, (const T *)a.k,
-                                  (const T *)a.v, a.igate, w.A, w.G, w.MC, a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS,
-                                  a.C_final, a.n_final, a.m_final, a.C0, a.n0);
+    dim3 g1(a.BH, (a.DHQK + CT - 1) / CT, (a.DHV + CT - 1) / CT);
+    const size_t sm1 = sizeof(float) * (2 * (size_t)L * CKS + L);
+    cudaError_t e = cudaSuccess;
+    if (sm1 > 48 * 1024 && (e = ensure_dynamic_smem((const void *)carry_simt_kernel<T>, (int)sm1)) != cudaSuccess)
+        return e;
+    e = launch_kernel(carry_simt_kernel<T>, g1, dim3(256), sm1, a.stream, 1, (const T *)a.k, (const T *)a.v, a.igate,
+                      w.A, w.G, w.MC, a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS, a.C_final, a.n_final, a.m_final,
+                      a.C0, a.n0);
     if (e != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;   // the chunk scan is fused into the carry walk
     if ((e = mark(3)) != cudaSuccess) return e;
