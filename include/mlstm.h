@@ -231,10 +231,10 @@ int mlstm_fwd_paired_walk(int DHQK, int DHV, int chunk, mlstm_dtype dt);
 int mlstm_fwd_segments(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
 
 /*
- * Reports whether the last mlstm_fwd that used `workspace` ran to completion:
- * synchronizes `stream`, reads the status word kept in the workspace and
- * returns MLSTM_OK or MLSTM_ERR_TIMEOUT (a bounded device-side wait gave up;
- * the outputs of that call are then undefined).
+ * Reports whether the last mlstm_fwd (or mlstm_bwd) that used `workspace` ran
+ * to completion: synchronizes `stream`, reads the status word kept in the
+ * workspace and returns MLSTM_OK or MLSTM_ERR_TIMEOUT (a bounded device-side
+ * wait gave up; the outputs of that call are then undefined).
  */
 mlstm_status mlstm_fwd_status(const void *workspace, void *stream);
 
@@ -282,16 +282,32 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * then; ignored when ogate is NULL).  No gradient flows into or out of the
  * states: the sequence starts from the zero state and the final state is not
  * part of L.  The forward pass is recomputed inside (gate preprocessing and
- * the fp32 chunk-start states); every product is fp32 on the CUDA cores.
- * Shapes and chunk sizes as for mlstm_fwd.
+ * the fp32 chunk-start states).  The chunk's scores, read-out gradients and
+ * the state gradients are fp32 on the CUDA cores; the dq, dk and dv products
+ * run on the tensor cores (tcgen05, bf16 copies of the fp32 intermediates as
+ * operands, fp32 accumulation) when mlstm_bwd_tensor_path says so, else in
+ * fp32 on the CUDA cores.  Shapes and chunk sizes as for mlstm_fwd.
  *
  * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
  * (it holds the chunk-start states and their gradients and the chunk's scores:
  * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
- * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head, each
- * array 256-byte aligned).  Errors as for mlstm_fwd.
+ * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head, and on
+ * the tensor-core path also 4 DHQK DHV + 4 chunk^2 bytes per chunk and head
+ * and 2 DHV bytes per token and head, each array 256-byte aligned).  A bounded
+ * device-side wait of the tensor-core products that gives up records a
+ * timeout that mlstm_fwd_status reads from this workspace.  Errors as for
+ * mlstm_fwd.
  */
 size_t mlstm_bwd_workspace_size(int B, int NH, int S, int DHQK, int DHV, int chunk, mlstm_dtype dt);
+
+/*
+ * 1 when mlstm_bwd runs its dq, dk and dv products on the tensor cores for
+ * these head sizes, chunk and element type (bf16 inputs, chunk 64 or 128,
+ * DHQK and DHV multiples of 128), 0 when it runs them on the CUDA cores, -1
+ * when the combination is not supported at all.  No GPU work; a host-side
+ * query.
+ */
+int mlstm_bwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt);
 mlstm_status mlstm_bwd(const void *q, const void *k, const void *v,
                        const float *igate, const float *fgate, const void *ogate, const void *dh,
                        mlstm_dtype dt, int B, int NH, int S, int DHQK, int DHV, int chunk,

@@ -44,6 +44,25 @@ def test_status_strings(lib):
     assert lib.mlstm_status_string(0) == b"ok"
 
 
+def test_bwd_tensor_path_query(lib):
+    """Which backward products run on the tensor cores: bf16, chunk 64 or 128, head sizes % 128."""
+    bf, f32 = binding.MLSTM_BF16, binding.MLSTM_F32
+    assert lib.mlstm_bwd_tensor_path(256, 512, 64, bf) == 1
+    assert lib.mlstm_bwd_tensor_path(128, 128, 128, bf) == 1
+    assert lib.mlstm_bwd_tensor_path(256, 512, 32, bf) == 0     # chunk
+    assert lib.mlstm_bwd_tensor_path(64, 512, 64, bf) == 0      # DHQK % 128
+    assert lib.mlstm_bwd_tensor_path(256, 192, 64, bf) == 0     # DHV % 128
+    assert lib.mlstm_bwd_tensor_path(256, 512, 64, f32) == 0    # fp32 inputs stay on the CUDA cores
+    assert lib.mlstm_bwd_tensor_path(12, 512, 64, bf) == -1
+    assert lib.mlstm_bwd_tensor_path(256, 512, 48, bf) == -1
+    # the tensor-core path's workspace adds the bf16 copies: 4 DHQK DHV + 4 chunk^2 bytes per chunk
+    # and head and 2 DHV per token and head (each array rounded up to 256 bytes)
+    B, NH, S, DK, DV, ch = 1, 8, 8192, 256, 512, 64
+    extra = lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, bf) - lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, f32)
+    NC = S // ch
+    assert extra == B * NH * NC * (4 * DK * DV + 4 * ch * ch) + B * NH * S * 2 * DV
+
+
 def test_workspace_size(lib):
     ws = lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 512, 64, binding.MLSTM_BF16)
     assert ws > 0 and ws % 256 == 0

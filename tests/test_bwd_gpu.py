@@ -122,6 +122,7 @@ def test_bwd_full_workload_7b(cuda_lib):
     """The 7B-shaped prefill (B1 NH8 S8192 d256/512, chunk 64) at full size: every gradient of every
     head, whole-tensor rel-L2 (the oracle takes the heads in groups, a thread per head)."""
     w = WORKLOADS["fwd_bf16_7b"]
+    assert binding.bwd_tensor_path(w.DHQK, w.DHV, w.chunk, torch.bfloat16) == 1   # the tcgen05 products
     inputs = make_fwd_inputs(w)
     dh = make_dh(w.B, w.NH, w.S, w.DHV, w.dtype, seed=w.seed + 1)
     got = run_gpu(inputs, dh, w.chunk)

@@ -41,6 +41,7 @@ SIGNATURES = {
     "mlstm_fwd_kernel_launches": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_fwd_tensor_path": (_i, [_i, _i, _i, _i]),
     "mlstm_fwd_paired_walk": (_i, [_i, _i, _i, _i]),
+    "mlstm_bwd_tensor_path": (_i, [_i, _i, _i, _i]),
     "mlstm_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "mlstm_step": (_i, [_fp, _fp, _fp, _vp, _vp, _vp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "mlstm_status_string": (ctypes.c_char_p, [_i]),
@@ -184,6 +185,12 @@ def fwd(q, k, v, igate, fgate, ogate=None, chunk: int = 64, h_out=None, C_final=
         arr = (ctypes.c_void_p * (FWD_PHASES + 1))(*[None if e is None else e.cuda_event for e in events])
         _check("mlstm_fwd_profiled", lib.mlstm_fwd_profiled(*args, arr))
     return h_out, C_final, n_final, m_final
+
+
+def bwd_tensor_path(DHQK, DHV, chunk, dtype) -> int:
+    """mlstm_bwd_tensor_path: 1 for the tensor-core gradient products, 0 for the CUDA cores, -1 unsupported."""
+    dt = MLSTM_BF16 if dtype == torch.bfloat16 else MLSTM_F32
+    return int(load().mlstm_bwd_tensor_path(DHQK, DHV, chunk, dt))
 
 
 def bwd_workspace_size(B, NH, S, DHQK, DHV, chunk, dtype) -> int:

@@ -38,6 +38,7 @@
 // bwd_dc_kernel (dC of the read-out per 64 x 64 state tile), bwd_state_scan_kernel (the reverse scan
 // of the state gradients), bwd_grad_kernel (dq, dk, dv per chunk and 64 columns) and
 // bwd_gate_kernel.  The per-chunk products run as 64 x 64 output tiles on the CUDA cores in fp32.
+#include "bwd_tc.h"
 #include "common.cuh"
 #include "mlstm_internal.h"
 
@@ -59,6 +60,8 @@ struct Params {
     float *DOTP;                     // partial row sums of g . hh per 64 value columns [BH][S][NJT]
     int NJT;                         // ceil(DV / 64)
     float *P2, *AI;                  // dS and A per chunk [BH][NC][L][L]
+    // bf16 copies of GS (after the scan), Gt, P2 and AI for the tensor-core gradient products, or NULL
+    __nv_bfloat16 *GS16, *Gt16, *P216, *AI16;
     float *QD, *KD;                  // per dk tile partial q . dq and k . dk [BH][S][NTK]
     void *dq, *dk, *dv, *dog;
     float *dig, *dfg;
@@ -165,6 +168,7 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
     const T *kb = static_cast<const T *>(p.k) + ((size_t)bh * p.S + t0) * DK;
     const float *nc = p.NS + ((size_t)bh * p.NC + c) * DK;
     float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
+    __nv_bfloat16 *AI16 = p.AI16 ? p.AI16 + ((size_t)bh * p.NC + c) * L * L : nullptr;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
     for (int t = tid; t < L; t += NT) rsum[t] = 0.f;
@@ -192,7 +196,10 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
                     const int s2 = nt * GM + 4 * tn + b2;
                     float av = 0.f;
                     if (s2 <= t && t < len) av = acc[a][b2] * expf(xs_[s2] - mx[t]);
-                    if (t < L && s2 < L) AIg[(size_t)t * L + s2] = av;
+                    if (t < L && s2 < L) {
+                        AIg[(size_t)t * L + s2] = av;
+                        if (AI16) AI16[(size_t)t * L + s2] = __float2bfloat16_rn(av);
+                    }
                     part += av;
                 }
                 part = sum16(part);
@@ -202,7 +209,10 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
             if (nt < mt) {
                 for (int e = tid; e < GM * GM; e += NT) {
                     const int t = nt * GM + e / GM, s2 = mt * GM + e % GM;
-                    if (t < L && s2 < L) AIg[(size_t)t * L + s2] = 0.f;
+                    if (t < L && s2 < L) {
+                        AIg[(size_t)t * L + s2] = 0.f;
+                        if (AI16) AI16[(size_t)t * L + s2] = __float2bfloat16_rn(0.f);
+                    }
                 }
             }
         }
@@ -242,6 +252,7 @@ __global__ void __launch_bounds__(NT) bwd_num_kernel(Params p)
     const T *dhb = static_cast<const T *>(p.dh) + ((size_t)bh * p.S + t0) * DV;
     T *dob = p.dog ? static_cast<T *>(p.dog) + ((size_t)bh * p.S + t0) * DV : nullptr;
     float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
+    __nv_bfloat16 *gt16 = p.Gt16 ? p.Gt16 + ((size_t)bh * p.S + t0) * DV : nullptr;
     const float *Cc = p.CS + ((size_t)bh * p.NC + c) * DK * DV;
     const float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
     const float *nrm = p.NRM + (size_t)bh * p.S + t0;
@@ -292,6 +303,7 @@ __global__ void __launch_bounds__(NT) bwd_num_kernel(Params p)
                         if (dob) dob[off] = from_f32<T>(dhv * hh);
                         const float g = ov * dhv / N;
                         gtb[off] = g;
+                        if (gt16) gt16[off] = __float2bfloat16_rn(g);
                         part = fmaf(g, hh, part);
                     }
                 }
@@ -322,6 +334,7 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
     const T *vb = static_cast<const T *>(p.v) + ((size_t)bh * p.S + t0) * DV;
     const float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
     float *P2g = p.P2 + ((size_t)bh * p.NC + c) * L * L;
+    __nv_bfloat16 *P216 = p.P216 ? p.P216 + ((size_t)bh * p.NC + c) * L * L : nullptr;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
     for (int t = tid; t < L; t += NT) {
@@ -342,7 +355,10 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
             if (nt > mt) {   // above the diagonal: zeros
                 for (int e = tid; e < GM * GM; e += NT) {
                     const int t = mt * GM + e / GM, s2 = nt * GM + e % GM;
-                    if (t < L && s2 < L) P2g[(size_t)t * L + s2] = 0.f;
+                    if (t < L && s2 < L) {
+                        P2g[(size_t)t * L + s2] = 0.f;
+                        if (P216) P216[(size_t)t * L + s2] = __float2bfloat16_rn(0.f);
+                    }
                 }
                 continue;
             }
@@ -367,7 +383,10 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
                     const int s2 = nt * GM + 4 * tn + b2;
                     float pv = 0.f;
                     if (s2 <= t && t < len) pv = (acc[a][b2] + dd[t]) * expf(xs_[s2] - mx[t]);
-                    if (t < L && s2 < L) P2g[(size_t)t * L + s2] = pv;
+                    if (t < L && s2 < L) {
+                        P2g[(size_t)t * L + s2] = pv;
+                        if (P216) P216[(size_t)t * L + s2] = __float2bfloat16_rn(pv);
+                    }
                 }
             }
         }
@@ -461,6 +480,9 @@ __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
                     const int c = c1 - 1 - u;
                     if (c >= cb) {
                         slot[(size_t)c * nq] = G;
+                        if (p.GS16)   // the bf16 copy of the chunk-end gradient
+                            reinterpret_cast<uint2 *>(p.GS16 + (size_t)bh * p.NC * nstate)[(size_t)c * nq + e] =
+                                make_uint2(bf16x2_bits(G.x, G.y), bf16x2_bits(G.z, G.w));
                         const float f = decay[c - cb];
                         G = make_float4(d[u].x + f * G.x, d[u].y + f * G.y, d[u].z + f * G.z, d[u].w + f * G.w);
                     }
@@ -664,7 +686,7 @@ __global__ void __launch_bounds__(GT) bwd_gate_kernel(Params p)
 }
 
 template <typename T>
-cudaError_t launch_t(const Params &p, int BH, cudaStream_t st)
+cudaError_t launch_t(const Params &p, int BH, cudaStream_t st, const bwdtc::Args *tc)
 {
     cudaError_t e;
     e = launch_kernel(bwd_scores_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
@@ -677,6 +699,10 @@ cudaError_t launch_t(const Params &p, int BH, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV / 4 + 255) / 256, BH), dim3(256), 0, st, 1, p);
     if (e != cudaSuccess) return e;
+    if (tc) {   // dq, dk, dv on the tensor cores
+        if ((e = bwdtc::launch(*tc)) != cudaSuccess) return e;
+        return launch_kernel(bwd_gate_kernel, dim3(BH), dim3(GT), 0, st, 1, p);
+    }
     const int nk = (p.DK + GM - 1) / GM;
     if ((e = launch_kernel(bwd_grad_kernel<T, 0>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
     if ((e = launch_kernel(bwd_grad_kernel<T, 1>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
@@ -695,7 +721,25 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     p.GS = w.GS; p.GN = w.GN; p.Gt = w.Gt; p.DD = w.DD; p.P2 = w.P2; p.AI = w.AI; p.QD = w.QD; p.KD = w.KD;
     p.DEN = w.DEN; p.NRM = w.NRM; p.DOTP = w.DOTP; p.NJT = (a.DHV + 63) / 64;
     p.dq = a.dq; p.dk = a.dk; p.dv = a.dv; p.dog = a.ogate ? a.dogate : nullptr; p.dig = a.digate; p.dfg = a.dfgate;
-    return a.bf16 ? bwd::launch_t<__nv_bfloat16>(p, a.BH, a.stream) : bwd::launch_t<float>(p, a.BH, a.stream);
+    p.GS16 = w.GS16; p.Gt16 = w.Gt16; p.P216 = w.P216; p.AI16 = w.AI16;
+    if (!a.bf16) return bwd::launch_t<float>(p, a.BH, a.stream, nullptr);
+    if (!w.tc) return bwd::launch_t<__nv_bfloat16>(p, a.BH, a.stream, nullptr);
+    using bf = __nv_bfloat16;
+    bwdtc::Args t;
+    t.BH = a.BH; t.S = a.S; t.L = a.chunk; t.NC = w.NC; t.DK = a.DHQK; t.DV = a.DHV; t.NTK = p.NTK;
+    t.A = w.A; t.P = w.M; t.MC = w.MC; t.G = w.G; t.ig = a.igate; t.DD = w.DD; t.NS = w.NS; t.GN = w.GN;
+    t.q = static_cast<const bf *>(a.q); t.k = static_cast<const bf *>(a.k); t.v = static_cast<const bf *>(a.v);
+    t.C16 = w.CS16; t.G16 = w.GS16; t.g16 = w.Gt16; t.dS16 = w.P216; t.A16 = w.AI16;
+    t.dq = static_cast<bf *>(a.dq); t.dk = static_cast<bf *>(a.dk); t.dv = static_cast<bf *>(a.dv);
+    t.QD = w.QD; t.KD = w.KD; t.status = w.status; t.stream = a.stream;
+    return bwd::launch_t<bf>(p, a.BH, a.stream, &t);
+}
+
+bool bwd_tc_path(bool bf16, int BH, int S, int DHQK, int DHV, int chunk)
+{
+    // (the per-chunk state arrays are addressed as BH NC boxes of one tensor map dimension)
+    const long long NC = (S + (long long)chunk - 1) / chunk;
+    return bf16 && bwdtc::supported(DHQK, DHV, chunk) && (long long)BH * NC < (1LL << 31) && NC <= 65535;
 }
 
 }  // namespace mlstm

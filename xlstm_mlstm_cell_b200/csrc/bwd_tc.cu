@@ -1,0 +1,326 @@
+// bwd_tc.cu -- the dq, dk and dv products of the chunkwise backward pass on the 5th-generation
+// tensor cores (tcgen05, bf16 operands, fp32 accumulators in TMEM), for bf16 inputs.
+//
+// Per chunk c (L tokens) and head, the gradients of the read-out (the training form of the xLSTM
+// Guide's "The Dual Formulation: How mLSTM Enables Parallel GPU Training", taken chunkwise as in
+// "Exploit Chunkwise Hardware Kernels for Production Training") are each a chunk-local product
+// plus an inter-chunk product with the chunk's state or state gradient:
+//   dq^T = scale (K^T dS^T + sc (C_c g^T + n_c dden^T)),
+//   dk^T = scale Q^T dS + w (G_end V^T + dn_end 1^T),
+//   dv^T = g^T A + w (G_end^T K^T),
+// with sc_t = exp(m_c - max(m_c, p_t)), w_s = exp(g_c - a_s + i~_s - m_{c+1}), scale = 1/sqrt(DK)
+// and the per-token factors applied column-wise (columns = tokens) in the epilogue.  A CTA computes
+// 128 output columns (d or j: the MMA's M, one per TMEM lane) for all L tokens of one chunk (the
+// MMA's N) as two accumulators in TMEM, the chunk-local one (K = L tokens) and the inter-chunk one
+// (K = DV or DK).  Every operand is a [rows][64] bf16 tile loaded by TMA with the 128-byte swizzle
+// and read by the MMA as K-major (the reduction index runs along the row) or MN-major (along the
+// column), as it lies in memory: no operand is transposed.  The fp32 intermediates (dS, A, g and
+// the per-chunk states) reach this kernel as bf16 copies written by the kernels that compute them.
+//
+// Roles: warp 0 one TMA thread, warp 1 the MMA thread (and the TMEM allocation), warps 2..5 the
+// epilogue (TMEM lane quadrant = warp % 4).  Every wait is bounded; a timeout sets the call's
+// status word.
+#include "bwd_tc.h"
+#include "common.cuh"
+#include "tc_common.cuh"
+#include "tc_fwd.h"
+
+#include <cudaTypedefs.h>
+
+namespace mlstm {
+namespace bwdtc {
+
+using namespace tc;
+
+constexpr int TM = 128;                // output columns per CTA (M)
+constexpr int STAGES = 4;              // pipeline stages of 64 reduction elements
+constexpr int THREADS = 192;
+constexpr uint32_t SA = TM * 128;      // A tile of a stage: 128 rows of 64 bf16, or 64 rows x 2 blocks
+
+template <int L>
+struct Smem {
+    static constexpr uint32_t SB = L * 128;                   // B tile of a stage: L tokens x 64
+    static constexpr uint32_t STAGE = SA + SB;
+    static constexpr uint32_t F = STAGES * STAGE;             // floats: tokw [L], ddv [L]
+    static constexpr uint32_t BAR = F + 2 * L * 4;
+    static constexpr uint32_t NBAR = 2 * STAGES + 1;
+    static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 2 * L;              // the two accumulators
+};
+
+struct KParams {
+    int S, NC, DK, DV, NTK;
+    const float *A, *P, *MC, *G, *ig, *DD, *NS, *GN;
+    const __nv_bfloat16 *pq;               // q (KIND 0) or k (KIND 1): the partial row sums
+    __nv_bfloat16 *out;
+    float *part;
+    uint32_t *status;
+};
+
+// OR of a predicate over the `count` threads that meet at named barrier `id`: every thread gets the
+// same answer.
+__device__ __forceinline__ bool group_any(uint32_t id, uint32_t count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+// KIND 0: dq, 1: dk, 2: dv.  Operands of the chunk-local product (A1, B1) and of the inter-chunk
+// product (A2, B2), by tensor map:
+//   KIND 0: A1 = k [s][d] (MN-major), B1 = dS [t][s] (K-major), A2 = C_c [d][j] (K), B2 = g [t][j] (K)
+//   KIND 1: A1 = q [t][d] (MN),       B1 = dS [t][s] (MN),      A2 = G_end [d][j] (K), B2 = v [s][j] (K)
+//   KIND 2: A1 = g [t][j] (MN),       B1 = A [t][s] (MN),       A2 = G_end [d][j] (MN), B2 = k [s][d] (K)
+template <int KIND, int L>
+__global__ void __launch_bounds__(THREADS, 1)
+grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
+               const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_b2, KParams p)
+{
+    using SM = Smem<L>;
+    constexpr int A1_MN = 1, B1_MN = KIND == 0 ? 0 : 1, A2_MN = KIND == 2 ? 1 : 0, B2_MN = 0;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float *tokw = reinterpret_cast<float *>(smem + SM::F);   // sc_t (KIND 0) or w_s
+    float *ddv = tokw + L;                                    // dden_t (KIND 0)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
+    uint64_t *full = bars, *empty = bars + STAGES, *accf = bars + 2 * STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
+    uint32_t *abort_flag = tmem_slot + 1;
+
+    const int bh = blockIdx.x, c = blockIdx.y, m0 = blockIdx.z * TM;
+    const int t0 = c * L, len = min(L, p.S - t0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nloc = L / 64, ninter = (KIND == 2 ? p.DK : p.DV) / 64, nb = nloc + ninter;
+    WaitCtx wc{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_a1);
+        tma_prefetch(&tm_b1);
+        tma_prefetch(&tm_a2);
+        tma_prefetch(&tm_b2);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, SM::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    griddep_wait();   // every operand is written by the kernels before this one
+    griddep_launch_dependents();
+
+    if (warp == 0) {
+        if (lane == 0) {   // TMA producer
+            const int zc = bh * p.NC + c;   // (head, chunk) of the per-chunk arrays
+            int kb = 0;
+            for (; kb < nb; ++kb) {
+                const int st = kb % STAGES;
+                if (kb >= STAGES && !mbar_wait(&empty[st], (uint32_t)((kb / STAGES) - 1) & 1u, wc)) break;
+                mbar_arrive_expect_tx(&full[st], SM::STAGE);
+                uint8_t *a = smem + st * SM::STAGE, *b = a + SA;
+                if (kb < nloc) {
+                    const int k0 = kb * 64;   // first reduction token of the stage
+#pragma unroll
+                    for (int mb = 0; mb < 2; ++mb)   // A1 rows: the stage's 64 tokens, 2 x 64 output columns
+                        tma_load_3d(a + mb * 8192, &tm_a1, m0 + 64 * mb, t0 + k0, bh, &full[st]);
+#pragma unroll
+                    for (int n = 0; n < L / 64; ++n) {
+                        if (KIND == 0)   // dS rows t (N), columns s (K)
+                            tma_load_3d(b + n * 8192, &tm_b1, k0, t0 + 64 * n, bh, &full[st]);
+                        else             // dS or A rows t (K), columns s (N)
+                            tma_load_3d(b + n * 8192, &tm_b1, 64 * n, t0 + k0, bh, &full[st]);
+                    }
+                } else {
+                    const int k0 = (kb - nloc) * 64;
+#pragma unroll
+                    for (int mb = 0; mb < 2; ++mb) {
+                        if (KIND == 2)   // G_end rows d (K), columns j (M)
+                            tma_load_3d(a + mb * 8192, &tm_a2, m0 + 64 * mb, k0, zc, &full[st]);
+                        else             // C_c or G_end rows d (M), columns j (K)
+                            tma_load_3d(a + mb * 8192, &tm_a2, k0, m0 + 64 * mb, zc, &full[st]);
+                    }
+#pragma unroll
+                    for (int n = 0; n < L / 64; ++n)   // g, v or k rows (N), columns (K)
+                        tma_load_3d(b + n * 8192, &tm_b2, k0, t0 + 64 * n, bh, &full[st]);
+                }
+            }
+            // the last stages' copies have landed before the CTA may leave
+            for (int s = 0; s < STAGES && s < kb; ++s) {
+                const int last = kb - 1 - s;
+                mbar_wait_drain(&full[last % STAGES], (uint32_t)(last / STAGES) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // MMA issuer
+            constexpr uint32_t ID1 = idesc_bf16(TM, L, A1_MN, B1_MN), ID2 = idesc_bf16(TM, L, A2_MN, B2_MN);
+            bool ok = true;
+            for (int kb = 0; kb < nb; ++kb) {
+                const int st = kb % STAGES;
+                if (!mbar_wait(&full[st], (uint32_t)(kb / STAGES) & 1u, wc)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + st * SM::STAGE), b = a + SA;
+                const bool loc = kb < nloc;
+                const int amn = loc ? A1_MN : A2_MN, bmn = loc ? B1_MN : B2_MN;
+                const uint32_t d = tmem + (loc ? 0u : (uint32_t)L);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {   // 16 reduction elements per MMA
+                    // K-major: 32 bytes further along the 128-byte rows; MN-major: 16 rows further
+                    const uint64_t ad = amn ? smem_desc(a + kk * 2048, 8192, 1024) : smem_desc(a, 16, 1024) + (uint64_t)(kk * 2);
+                    const uint64_t bd = bmn ? smem_desc(b + kk * 2048, 8192, 1024) : smem_desc(b, 16, 1024) + (uint64_t)(kk * 2);
+                    const int first = loc ? kb : kb - nloc;
+                    mma_ss(d, ad, bd, loc ? ID1 : ID2, (first > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[st]);
+            }
+            if (ok) mma_commit(accf);
+        }
+    } else {
+        // ------------------------------------------------ epilogue: warps 2..5
+        const int et = threadIdx.x - 64;           // 0..127
+        const int q4 = warp & 3;                   // TMEM lane quadrant
+        const int col = m0 + q4 * 32 + lane;       // this thread's output column
+        const size_t g0 = (size_t)bh * p.S + t0;   // first token of the chunk
+        if (et < L) {
+            const int t = et;
+            const bool okt = t < len;
+            if (KIND == 0) {
+                const float mc = p.MC[(size_t)bh * (p.NC + 1) + c];
+                tokw[t] = okt ? expf(mc - fmaxf(mc, p.P[g0 + t])) : 0.f;
+                ddv[t] = okt ? p.DD[g0 + t] : 0.f;
+            } else {
+                const float gm = p.G[(size_t)bh * p.NC + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1];
+                tokw[t] = okt ? expf(p.ig[g0 + t] - p.A[g0 + t] + gm) : 0.f;
+                ddv[t] = 0.f;
+            }
+        }
+        float colv = 0.f;   // n_c (KIND 0) or dn_end (KIND 1) of this column
+        if (KIND == 0) colv = p.NS[((size_t)bh * p.NC + c) * p.DK + col];
+        if (KIND == 1) colv = p.GN[((size_t)bh * p.NC + c) * p.DK + col];
+        const float scale = rsqrtf((float)p.DK);
+        const int NCOL = KIND == 2 ? p.DV : p.DK;
+        named_sync(1, 128);   // tokw, ddv
+        // one thread waits for the accumulators; the four warps take its answer together (the TMEM
+        // loads below are warp-collective)
+        bool failed = false;
+        if (et == 0) failed = !mbar_wait(accf, 0, wc);
+        failed = group_any(2, 128, failed);
+        if (!failed) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int g = 0; g < L / 16; ++g) {
+                uint32_t r1[16], r2[16];
+                tmem_ld16(tmem_addr(tmem, q4 * 32, g * 16), r1);
+                tmem_ld16(tmem_addr(tmem, q4 * 32, L + g * 16), r2);
+                float pv[16];
+                if (KIND < 2) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int t = g * 16 + u;
+                        pv[u] = t < len ? __bfloat162float(p.pq[(g0 + t) * p.DK + col]) : 0.f;
+                    }
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int t = g * 16 + u;
+                    const float d1 = __uint_as_float(r1[u]), d2 = __uint_as_float(r2[u]);
+                    const float w = tokw[t];
+                    float o, pr = 0.f;
+                    if (KIND == 0) {
+                        const float dqh = d1 + w * (d2 + ddv[t] * colv);
+                        o = dqh * scale;
+                        pr = pv[u] * scale * dqh;
+                    } else if (KIND == 1) {
+                        o = scale * d1 + w * (d2 + colv);
+                        pr = pv[u] * o;
+                    } else {
+                        o = d1 + w * d2;
+                    }
+                    if (t < len) p.out[(g0 + t) * NCOL + col] = __float2bfloat16_rn(o);
+                    if (KIND < 2) {
+#pragma unroll
+                        for (int sh = 16; sh > 0; sh >>= 1) pr += __shfl_xor_sync(0xffffffffu, pr, sh);
+                        if (lane == 0 && t < len) p.part[(g0 + t) * p.NTK + (col >> 5)] = pr;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
+        // a wait gave up: let MMAs and copies this CTA may still have in flight finish (bounded)
+        const unsigned long long tb = global_timer();
+        while (global_timer() - tb < 100000ull) { }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, SM::TMEM_COLS);
+    }
+}
+
+// [BH][R][C] bf16 maps (boxes of 64 rows x 64 columns) over the arrays the products read.
+static bool map3(CUtensorMap *m, const void *base, int C, int R, int Z) { return tcfwd::make_map(m, base, C, R, Z, 64); }
+
+template <int KIND, int L>
+static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUtensorMap &b1, const CUtensorMap &a2,
+                               const CUtensorMap &b2)
+{
+    using SM = Smem<L>;
+    KParams p;
+    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV; p.NTK = a.NTK;
+    p.A = a.A; p.P = a.P; p.MC = a.MC; p.G = a.G; p.ig = a.ig; p.DD = a.DD; p.NS = a.NS; p.GN = a.GN;
+    p.pq = KIND == 0 ? a.q : a.k;
+    p.out = KIND == 0 ? a.dq : KIND == 1 ? a.dk : a.dv;
+    p.part = KIND == 0 ? a.QD : KIND == 1 ? a.KD : nullptr;
+    p.status = a.status;
+    cudaError_t e = ensure_dynamic_smem((const void *)grad_tc_kernel<KIND, L>, SM::TOTAL);
+    if (e != cudaSuccess) return e;
+    const int tiles = (KIND == 2 ? a.DV : a.DK) / TM;
+    return launch_kernel(grad_tc_kernel<KIND, L>, dim3(a.BH, a.NC, tiles), dim3(THREADS), SM::TOTAL, a.stream, 1, a1,
+                         b1, a2, b2, p);
+}
+
+template <int L>
+static cudaError_t launch_l(const Args &a)
+{
+    CUtensorMap mq, mk, mv, mg, mds, ma, mc, mG;
+    const int CL = a.NC * L;   // rows of the per-chunk score arrays
+    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&mk, a.k, a.DK, a.S, a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH) ||
+        !map3(&mg, a.g16, a.DV, a.S, a.BH) || !map3(&mds, a.dS16, L, CL, a.BH) || !map3(&ma, a.A16, L, CL, a.BH) ||
+        !map3(&mc, a.C16, a.DV, a.DK, a.BH * a.NC) || !map3(&mG, a.G16, a.DV, a.DK, a.BH * a.NC))
+        return cudaErrorInvalidValue;
+    cudaError_t e = launch_kind<0, L>(a, mk, mds, mc, mg);
+    if (e == cudaSuccess) e = launch_kind<1, L>(a, mq, mds, mG, mv);
+    if (e == cudaSuccess) e = launch_kind<2, L>(a, mg, ma, mG, mk);
+    return e;
+}
+
+bool supported(int DK, int DV, int L)
+{
+    return (L == 64 || L == 128) && DK % TM == 0 && DV % TM == 0 && DK <= 512 && DV <= 512;
+}
+
+cudaError_t launch(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_l<64>(a) : launch_l<128>(a);
+}
+
+}  // namespace bwdtc
+}  // namespace mlstm

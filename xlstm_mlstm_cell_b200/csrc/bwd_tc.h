@@ -1,0 +1,35 @@
+// bwd_tc.h -- the gradient products of the backward pass on the tensor cores (bwd_tc.cu): what the
+// CUDA-core backward (bwd_simt.cu) hands them.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mlstm {
+namespace bwdtc {
+
+struct Args {
+    int BH, S, L, NC, DK, DV, NTK;
+    // gate preprocessing [BH][S] (A: chunk-local cumulative log decay, P: chunk-local prefix maximum
+    // of i~ - A), chunk stabilizers MC [BH][NC + 1] and log decay sums G [BH][NC]; i~ [BH][S]
+    const float *A, *P, *MC, *G, *ig;
+    const float *DD;                        // gradient of the denominator [BH][S]
+    const float *NS, *GN;                   // n at the chunk starts, gradient of n at the chunk ends [BH][NC][DK]
+    const __nv_bfloat16 *q, *k, *v;         // inputs [BH][S][DK | DV]
+    // bf16 copies of the fp32 intermediates: chunk-start states and chunk-end state gradients
+    // [BH][NC][DK][DV], the read-out numerator's gradient g [BH][S][DV], dS and A [BH][NC][L][L]
+    const __nv_bfloat16 *C16, *G16, *g16, *dS16, *A16;
+    __nv_bfloat16 *dq, *dk, *dv;            // outputs [BH][S][DK | DV]
+    float *QD, *KD;                         // partial q . dq and k . dk per 32 columns [BH][S][NTK]
+    uint32_t *status;
+    cudaStream_t stream;
+};
+
+// bf16 inputs with chunk 64 or 128 and head sizes that are multiples of 128.
+bool supported(int DK, int DV, int L);
+// The dq, dk and dv products of every chunk (three launches on a.stream).
+cudaError_t launch(const Args &a);
+
+}  // namespace bwdtc
+}  // namespace mlstm

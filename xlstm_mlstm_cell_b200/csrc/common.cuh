@@ -19,6 +19,13 @@ template <typename T> MLSTM_DEVINL T from_f32(float x);
 template <> MLSTM_DEVINL float from_f32<float>(float x) { return x; }
 template <> MLSTM_DEVINL __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Two floats rounded to bf16 (nearest even) as one 32-bit word, the first in the low half.
+MLSTM_DEVINL uint32_t bf16x2_bits(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
 // Four consecutive elements as float (16-byte aligned for float, 8 for bf16).
 MLSTM_DEVINL float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 MLSTM_DEVINL float4 load4(const __nv_bfloat16 *p)

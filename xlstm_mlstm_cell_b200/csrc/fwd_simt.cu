@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256, 2)
 carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ igate,
                   const float *__restrict__ A, const float *__restrict__ G, const float *__restrict__ MC,
                   int S, int L, int NC, int DHQK, int DHV,
-                  float *__restrict__ CS, float *__restrict__ NS,
+                  float *__restrict__ CS, float *__restrict__ NS, __nv_bfloat16 *__restrict__ CS16,
                   float *C_final, float *n_final, float *__restrict__ m_final, const float *C0, const float *n0)
 {
     griddep_wait();
@@ -142,12 +142,16 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
     for (int ch = 0; ch < NC; ++ch) {
         const int t0 = ch * L, len = min(L, S - t0);
         // state at the chunk start
-        float *cs = CS + ((size_t)bh * NC + ch) * DHQK * DHV;
+        const size_t cso = ((size_t)bh * NC + ch) * DHQK * DHV;
         if (cols_in) {
 #pragma unroll
             for (int r = 0; r < 4; ++r)
-                if (ri + r < DHQK)
-                    *reinterpret_cast<float4 *>(cs + (size_t)(ri + r) * DHV + cj) = make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
+                if (ri + r < DHQK) {
+                    const size_t o = cso + (size_t)(ri + r) * DHV + cj;
+                    *reinterpret_cast<float4 *>(CS + o) = make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
+                    if (CS16)   // the bf16 copy the backward's tensor-core products read
+                        *reinterpret_cast<uint2 *>(CS16 + o) = make_uint2(bf16x2_bits(c[r][0], c[r][1]), bf16x2_bits(c[r][2], c[r][3]));
+                }
         }
         if (n_warp && i0 + tid < DHQK) NS[((size_t)bh * NC + ch) * DHQK + i0 + tid] = nn;
 
@@ -368,8 +372,8 @@ static cudaError_t launch_fwd_simt_t(const FwdArgs &a, const FwdWorkspace &w, co
     if (sm1 > 48 * 1024 && (e = ensure_dynamic_smem((const void *)carry_simt_kernel<T>, (int)sm1)) != cudaSuccess)
         return e;
     e = launch_kernel(carry_simt_kernel<T>, g1, dim3(256), sm1, a.stream, 1, (const T *)a.k, (const T *)a.v, a.igate,
-                      w.A, w.G, w.MC, a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS, a.C_final, a.n_final, a.m_final,
-                      a.C0, a.n0);
+                      w.A, w.G, w.MC, a.S, L, w.NC, a.DHQK, a.DHV, w.CS, w.NS, w.CS16, a.C_final, a.n_final,
+                      a.m_final, a.C0, a.n0);
     if (e != cudaSuccess) return e;
     if ((e = mark(2)) != cudaSuccess) return e;   // the chunk scan is fused into the carry walk
     if ((e = mark(3)) != cudaSuccess) return e;

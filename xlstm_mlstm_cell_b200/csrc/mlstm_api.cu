@@ -45,6 +45,7 @@ size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, b
     w->MC = reinterpret_cast<float *>(take(sizeof(float) * (size_t)BH * (NC + 1)));
     w->tc = tc_path_supported(bf16, DHQK, DHV, chunk) && S > 0;
     w->CS = w->NS = w->GP = w->SGb = w->DC = w->DN = nullptr;
+    w->CS16 = nullptr;
     w->NSEG = 0;
     w->R = 0;
     if (w->tc) {
@@ -65,7 +66,7 @@ size_t plan_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, b
 mlstm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA; }
 
 // Lays out the backward pass's workspace (base may be NULL to size it).  Returns the bytes used.
-size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, BwdWorkspace *w)
+size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chunk, bool tc, BwdWorkspace *w)
 {
     BwdWorkspace tmp;
     if (!w) w = &tmp;
@@ -98,6 +99,16 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->DEN = reinterpret_cast<float *>(take(f * BH * S));
     w->NRM = reinterpret_cast<float *>(take(f * BH * S));
     w->DOTP = reinterpret_cast<float *>(take(f * BH * S * ((DHV + 63) / 64)));
+    w->tc = tc;
+    w->CS16 = w->GS16 = w->Gt16 = w->P216 = w->AI16 = nullptr;
+    if (tc) {
+        const size_t h = sizeof(__nv_bfloat16);
+        w->CS16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * DHQK * DHV));
+        w->GS16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * DHQK * DHV));
+        w->Gt16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * S * DHV));
+        w->P216 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
+        w->AI16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
+    }
     return off;
 }
 
@@ -316,7 +327,14 @@ extern "C" size_t mlstm_bwd_workspace_size(int B, int NH, int S, int DHQK, int D
     if (B < 0 || NH < 0 || S < 0 || (dt != MLSTM_F32 && dt != MLSTM_BF16)) return 0;
     if (!dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return 0;
     if ((long long)B * NH > (1LL << 30) || (long long)S * DHV > (1LL << 40)) return 0;
-    return plan_bwd_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, nullptr);
+    return plan_bwd_workspace(nullptr, B * NH, S, DHQK, DHV, chunk, bwd_tc_path(dt == MLSTM_BF16, B * NH, S, DHQK, DHV, chunk),
+                              nullptr);
+}
+
+extern "C" int mlstm_bwd_tensor_path(int DHQK, int DHV, int chunk, mlstm_dtype dt)
+{
+    if ((dt != MLSTM_F32 && dt != MLSTM_BF16) || !dims_ok_fwd(DHQK, DHV) || !chunk_ok(chunk)) return -1;
+    return bwd_tc_path(dt == MLSTM_BF16, 1, chunk, DHQK, DHV, chunk) ? 1 : 0;
 }
 
 extern "C" mlstm_status mlstm_bwd(const void *q, const void *k, const void *v, const float *igate, const float *fgate,
@@ -334,14 +352,15 @@ extern "C" mlstm_status mlstm_bwd(const void *q, const void *k, const void *v, c
     for (const void *p : ins)
         if (!p || !aligned16(p)) return MLSTM_ERR_INVALID_ARG;
     if (ogate && (!dogate || !aligned16(ogate) || !aligned16(dogate))) return MLSTM_ERR_INVALID_ARG;
-    const size_t need = plan_bwd_workspace(nullptr, BH, S, DHQK, DHV, chunk, nullptr);
+    const bool bf16 = dt == MLSTM_BF16;
+    const bool tc = bwd_tc_path(bf16, BH, S, DHQK, DHV, chunk);
+    const size_t need = plan_bwd_workspace(nullptr, BH, S, DHQK, DHV, chunk, tc, nullptr);
     if (!workspace || workspace_bytes < need) return MLSTM_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLSTM_ERR_INVALID_ARG;
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     BwdWorkspace w;
-    plan_bwd_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, &w);
-    const bool bf16 = dt == MLSTM_BF16;
+    plan_bwd_workspace(static_cast<char *>(workspace), BH, S, DHQK, DHV, chunk, tc, &w);
     // gate preprocessing and the chunk-start states of the forward pass (its fp32 carry)
     GatePrepArgs gp{igate, fgate, BH, S, chunk, w.NC, w.A, w.M, w.G, w.Bc, w.MC, 0, 0, nullptr, nullptr, nullptr,
                     w.status, st};
@@ -350,7 +369,7 @@ extern "C" mlstm_status mlstm_bwd(const void *q, const void *k, const void *v, c
     fw.status = w.status;
     fw.NC = w.NC;
     fw.A = w.A; fw.M = w.M; fw.G = w.G; fw.Bc = w.Bc; fw.MC = w.MC;
-    fw.CS = w.CS; fw.NS = w.NS;
+    fw.CS = w.CS; fw.NS = w.NS; fw.CS16 = w.CS16;
     fw.tc = false;
     FwdArgs fa{q, k, v, nullptr, igate, fgate, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, BH, S, DHQK, DHV,
                chunk, bf16, st, false};

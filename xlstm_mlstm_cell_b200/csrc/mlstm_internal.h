@@ -1,6 +1,7 @@
 // mlstm_internal.h -- launch descriptors shared by the host side of libmlstm.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -48,6 +49,7 @@ struct FwdWorkspace {
     float *G, *Bc;         // [BH][NC] chunk log decay, chunk max-plus offset
     float *MC;             // [BH][NC+1] stabilizer at chunk starts (last = final m)
     float *CS, *NS;        // SIMT path: state at every chunk start
+    __nv_bfloat16 *CS16;   // optional bf16 copy of CS (the backward's tensor-core products), else NULL
     // tensor-core path
     bool tc;               // the tensor-core path is used
     int NSEG, R;           // segments per head and chunks per segment
@@ -80,6 +82,10 @@ struct BwdWorkspace {
     float *QD, *KD;               // [BH][S][ceil(DHQK / 32)] partial q . dq, k . dk
     float *DEN, *NRM;             // [BH][S] read-out denominator and its floored magnitude
     float *DOTP;                  // [BH][S][ceil(DHV / 64)] partial row sums of g . hh
+    // the tensor-core gradient products (bf16 inputs, bwd_tc_path): bf16 copies of CS, GS, Gt, P2
+    // and AI in the same layouts; NULL on the CUDA-core path
+    bool tc;
+    __nv_bfloat16 *CS16, *GS16, *Gt16, *P216, *AI16;
 };
 
 // Records the caller's phase events (mlstm_fwd_profiled); a no-op without events.
@@ -102,5 +108,7 @@ bool tc_path_supported(bool bf16, int DHQK, int DHV, int chunk);
 int tc_num_segments(int BH, int DHV, int NC);
 cudaError_t launch_fwd_tc(const FwdArgs &a, const FwdWorkspace &w, const PhaseMark &mark);
 cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w);
+// The backward's dq, dk and dv products run on the tensor cores for these arguments.
+bool bwd_tc_path(bool bf16, int BH, int S, int DHQK, int DHV, int chunk);
 
 }  // namespace mlstm
