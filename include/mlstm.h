@@ -284,15 +284,16 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * part of L.  The forward pass is recomputed inside (gate preprocessing and
  * the fp32 chunk-start states).  The chunk's scores, read-out gradients and
  * the state gradients are fp32 on the CUDA cores; the dq, dk and dv products
- * run on the tensor cores (tcgen05, bf16 copies of the fp32 intermediates as
- * operands, fp32 accumulation) when mlstm_bwd_tensor_path says so, else in
- * fp32 on the CUDA cores.  Shapes and chunk sizes as for mlstm_fwd.
+ * and the read-out numerator run on the tensor cores (tcgen05, bf16 copies of
+ * the fp32 intermediates as operands, the numerator's fp32 operands as two
+ * bf16 parts each, fp32 accumulation) when mlstm_bwd_tensor_path says so,
+ * else in fp32 on the CUDA cores.  Shapes and chunk sizes as for mlstm_fwd.
  *
  * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
  * (it holds the chunk-start states and their gradients and the chunk's scores:
  * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
  * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head, and on
- * the tensor-core path also 4 DHQK DHV + 4 chunk^2 bytes per chunk and head
+ * the tensor-core path also 6 DHQK DHV + 6 chunk^2 bytes per chunk and head
  * and 2 DHV bytes per token and head, each array 256-byte aligned).  A bounded
  * device-side wait of the tensor-core products that gives up records a
  * timeout that mlstm_fwd_status reads from this workspace.  Errors as for

@@ -55,12 +55,12 @@ def test_bwd_tensor_path_query(lib):
     assert lib.mlstm_bwd_tensor_path(256, 512, 64, f32) == 0    # fp32 inputs stay on the CUDA cores
     assert lib.mlstm_bwd_tensor_path(12, 512, 64, bf) == -1
     assert lib.mlstm_bwd_tensor_path(256, 512, 48, bf) == -1
-    # the tensor-core path's workspace adds the bf16 copies: 4 DHQK DHV + 4 chunk^2 bytes per chunk
+    # the tensor-core path's workspace adds the bf16 copies: 6 DHQK DHV + 6 chunk^2 bytes per chunk
     # and head and 2 DHV per token and head (each array rounded up to 256 bytes)
     B, NH, S, DK, DV, ch = 1, 8, 8192, 256, 512, 64
     extra = lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, bf) - lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, f32)
     NC = S // ch
-    assert extra == B * NH * NC * (4 * DK * DV + 4 * ch * ch) + B * NH * S * 2 * DV
+    assert extra == B * NH * NC * (6 * DK * DV + 6 * ch * ch) + B * NH * S * 2 * DV
 
 
 def test_workspace_size(lib):

@@ -60,7 +60,8 @@ struct Params {
     float *DOTP;                     // partial row sums of g . hh per 64 value columns [BH][S][NJT]
     int NJT;                         // ceil(DV / 64)
     float *P2, *AI;                  // dS and A per chunk [BH][NC][L][L]
-    // bf16 copies of GS (after the scan), Gt, P2 and AI for the tensor-core gradient products, or NULL
+    // bf16 copies of GS (after the scan), Gt and P2, and AI as two bf16 parts [BH][NC][2][L][L], for
+    // the tensor-core products, or NULL
     __nv_bfloat16 *GS16, *Gt16, *P216, *AI16;
     float *QD, *KD;                  // per dk tile partial q . dq and k . dk [BH][S][NTK]
     void *dq, *dk, *dv, *dog;
@@ -168,7 +169,8 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
     const T *kb = static_cast<const T *>(p.k) + ((size_t)bh * p.S + t0) * DK;
     const float *nc = p.NS + ((size_t)bh * p.NC + c) * DK;
     float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
-    __nv_bfloat16 *AI16 = p.AI16 ? p.AI16 + ((size_t)bh * p.NC + c) * L * L : nullptr;
+    // the two bf16 parts of A (value and residue) for the tensor-core read-out
+    __nv_bfloat16 *AI16 = p.AI16 ? p.AI16 + ((size_t)bh * p.NC + c) * 2 * L * L : nullptr;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
     for (int t = tid; t < L; t += NT) rsum[t] = 0.f;
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
                     if (s2 <= t && t < len) av = acc[a][b2] * expf(xs_[s2] - mx[t]);
                     if (t < L && s2 < L) {
                         AIg[(size_t)t * L + s2] = av;
-                        if (AI16) AI16[(size_t)t * L + s2] = __float2bfloat16_rn(av);
+                        if (AI16) bf16_parts(av, AI16[(size_t)t * L + s2], AI16[(size_t)L * L + t * L + s2]);
                     }
                     part += av;
                 }
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
                     const int t = nt * GM + e / GM, s2 = mt * GM + e % GM;
                     if (t < L && s2 < L) {
                         AIg[(size_t)t * L + s2] = 0.f;
-                        if (AI16) AI16[(size_t)t * L + s2] = __float2bfloat16_rn(0.f);
+                        if (AI16) bf16_parts(0.f, AI16[(size_t)t * L + s2], AI16[(size_t)L * L + t * L + s2]);
                     }
                 }
             }
@@ -691,7 +693,7 @@ cudaError_t launch_t(const Params &p, int BH, cudaStream_t st, const bwdtc::Args
     cudaError_t e;
     e = launch_kernel(bwd_scores_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
-    e = launch_kernel(bwd_num_kernel<T>, dim3(BH, p.NC, p.NJT), dim3(NT), 0, st, 1, p);
+    e = tc ? bwdtc::launch_num(*tc) : launch_kernel(bwd_num_kernel<T>, dim3(BH, p.NC, p.NJT), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
     e = launch_kernel(bwd_ds_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
@@ -732,6 +734,9 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     t.C16 = w.CS16; t.G16 = w.GS16; t.g16 = w.Gt16; t.dS16 = w.P216; t.A16 = w.AI16;
     t.dq = static_cast<bf *>(a.dq); t.dk = static_cast<bf *>(a.dk); t.dv = static_cast<bf *>(a.dv);
     t.QD = w.QD; t.KD = w.KD; t.status = w.status; t.stream = a.stream;
+    t.dh = static_cast<const bf *>(a.dh); t.o = static_cast<const bf *>(a.ogate); t.NRM = w.NRM;
+    t.Gt = w.Gt; t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
+    t.NJT = p.NJT;
     return bwd::launch_t<bf>(p, a.BH, a.stream, &t);
 }
 

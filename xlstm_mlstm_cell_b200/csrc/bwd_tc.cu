@@ -41,19 +41,24 @@ template <int L>
 struct Smem {
     static constexpr uint32_t SB = L * 128;                   // B tile of a stage: L tokens x 64
     static constexpr uint32_t STAGE = SA + SB;
-    static constexpr uint32_t F = STAGES * STAGE;             // floats: tokw [L], ddv [L]
-    static constexpr uint32_t BAR = F + 2 * L * 4;
+    static constexpr uint32_t F = STAGES * STAGE;             // floats: tokw [L], ddv [L], red [4][L]
+    static constexpr uint32_t BAR = F + 6 * L * 4;
     static constexpr uint32_t NBAR = 2 * STAGES + 1;
     static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 2 * L;              // the two accumulators
 };
 
 struct KParams {
-    int S, NC, DK, DV, NTK;
+    int S, NC, DK, DV, NTK, NJT;
     const float *A, *P, *MC, *G, *ig, *DD, *NS, *GN;
     const __nv_bfloat16 *pq;               // q (KIND 0) or k (KIND 1): the partial row sums
     __nv_bfloat16 *out;
     float *part;
+    // KIND 3 (the read-out numerator)
+    const __nv_bfloat16 *dh, *o;
+    const float *NRM;
+    float *Gt, *DOTP;
+    __nv_bfloat16 *g16w, *dog;
     uint32_t *status;
 };
 
@@ -73,22 +78,62 @@ __device__ __forceinline__ bool group_any(uint32_t id, uint32_t count, bool pred
     return r != 0;
 }
 
-// KIND 0: dq, 1: dk, 2: dv.  Operands of the chunk-local product (A1, B1) and of the inter-chunk
-// product (A2, B2), by tensor map:
+// The read-out numerator's epilogue for 16 tokens g * 16 .. of a thread's value column:
+// num = A V + sc scale q C_c (r1, r2: the two accumulators' columns), hh = num / N, do = dh hh,
+// g = o dh / N; the warp's row sums of g . hh go to red[t].
+__device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&r1)[16], const uint32_t (&r2)[16],
+                                             const float *tokw, const float *nrm, float *red, int grp, int len,
+                                             size_t g0, int col, float scale, int lane)
+{
+    float dhv[16], ov[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int t = grp * 16 + u;
+        const size_t off = (g0 + t) * p.DV + col;
+        dhv[u] = t < len ? __bfloat162float(p.dh[off]) : 0.f;
+        ov[u] = (t < len && p.o) ? __bfloat162float(p.o[off]) : 1.f;
+    }
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int t = grp * 16 + u;
+        const size_t off = (g0 + t) * p.DV + col;
+        const float num = __uint_as_float(r1[u]) + tokw[t] * scale * __uint_as_float(r2[u]);
+        const float N = nrm[t];
+        const float hh = num / N;
+        const float g = ov[u] * dhv[u] / N;
+        float pr = 0.f;
+        if (t < len) {
+            if (p.dog) p.dog[off] = __float2bfloat16_rn(dhv[u] * hh);
+            p.Gt[off] = g;
+            p.g16w[off] = __float2bfloat16_rn(g);
+            pr = g * hh;
+        }
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) pr += __shfl_xor_sync(0xffffffffu, pr, sh);
+        if (lane == 0) red[t] = pr;
+    }
+}
+
+// KIND 0: dq, 1: dk, 2: dv, 3: the read-out numerator num^T = V^T A^T + sc scale C_c^T Q^T.
+// Operands of the chunk-local product (A1, B1) and of the inter-chunk product (A2, B2), by tensor map:
 //   KIND 0: A1 = k [s][d] (MN-major), B1 = dS [t][s] (K-major), A2 = C_c [d][j] (K), B2 = g [t][j] (K)
 //   KIND 1: A1 = q [t][d] (MN),       B1 = dS [t][s] (MN),      A2 = G_end [d][j] (K), B2 = v [s][j] (K)
 //   KIND 2: A1 = g [t][j] (MN),       B1 = A [t][s] (MN),       A2 = G_end [d][j] (MN), B2 = k [s][d] (K)
+//   KIND 3: A1 = v [s][j] (MN),       B1 = A [t][s] (K),        A2 = C_c [d][j] (MN),   B2 = q [t][d] (K)
 template <int KIND, int L>
 __global__ void __launch_bounds__(THREADS, 1)
 grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_b2, KParams p)
 {
     using SM = Smem<L>;
-    constexpr int A1_MN = 1, B1_MN = KIND == 0 ? 0 : 1, A2_MN = KIND == 2 ? 1 : 0, B2_MN = 0;
+    constexpr int A1_MN = 1, B1_MN = (KIND == 0 || KIND == 3) ? 0 : 1, A2_MN = (KIND == 2 || KIND == 3) ? 1 : 0;
+    constexpr int B2_MN = 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *tokw = reinterpret_cast<float *>(smem + SM::F);   // sc_t (KIND 0) or w_s
-    float *ddv = tokw + L;                                    // dden_t (KIND 0)
+    float *ddv = tokw + L;                                    // dden_t (KIND 0), N_t (KIND 3)
+    float *red = ddv + L;                                     // [4][L] per-warp row sums (KIND 3)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
     uint64_t *full = bars, *empty = bars + STAGES, *accf = bars + 2 * STAGES;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
@@ -97,7 +142,11 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
     const int bh = blockIdx.x, c = blockIdx.y, m0 = blockIdx.z * TM;
     const int t0 = c * L, len = min(L, p.S - t0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nloc = L / 64, ninter = (KIND == 2 ? p.DK : p.DV) / 64, nb = nloc + ninter;
+    // KIND 3 takes its fp32 operands (A and C_c) as two bf16 parts, the value and the rounding
+    // residue, and sums both products in the accumulator
+    constexpr int NPART = KIND == 3 ? 2 : 1;
+    const int nloc = L / 64, ninter = (KIND >= 2 ? p.DK : p.DV) / 64;
+    const int nl = NPART * nloc, nb = nl + NPART * ninter;
     WaitCtx wc{abort_flag, p.status};
 
     if (threadIdx.x == 0) {
@@ -133,29 +182,34 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 if (kb >= STAGES && !mbar_wait(&empty[st], (uint32_t)((kb / STAGES) - 1) & 1u, wc)) break;
                 mbar_arrive_expect_tx(&full[st], SM::STAGE);
                 uint8_t *a = smem + st * SM::STAGE, *b = a + SA;
-                if (kb < nloc) {
-                    const int k0 = kb * 64;   // first reduction token of the stage
+                const bool loc = kb < nl;
+                const int idx = loc ? kb : kb - nl, nper = loc ? nloc : ninter;
+                const int part = idx / nper, k0 = 64 * (idx % nper);   // bf16 part, first reduction index
+                if (loc) {
 #pragma unroll
                     for (int mb = 0; mb < 2; ++mb)   // A1 rows: the stage's 64 tokens, 2 x 64 output columns
                         tma_load_3d(a + mb * 8192, &tm_a1, m0 + 64 * mb, t0 + k0, bh, &full[st]);
+                    // the chunk's first row in the score arrays: A holds two parts per chunk
+                    const int rb = KIND >= 2 ? 2 * t0 + part * L : t0;
 #pragma unroll
                     for (int n = 0; n < L / 64; ++n) {
-                        if (KIND == 0)   // dS rows t (N), columns s (K)
-                            tma_load_3d(b + n * 8192, &tm_b1, k0, t0 + 64 * n, bh, &full[st]);
+                        if (!B1_MN)      // dS or A rows t (N), columns s (K)
+                            tma_load_3d(b + n * 8192, &tm_b1, k0, rb + 64 * n, bh, &full[st]);
                         else             // dS or A rows t (K), columns s (N)
-                            tma_load_3d(b + n * 8192, &tm_b1, 64 * n, t0 + k0, bh, &full[st]);
+                            tma_load_3d(b + n * 8192, &tm_b1, 64 * n, rb + k0, bh, &full[st]);
                     }
                 } else {
-                    const int k0 = (kb - nloc) * 64;
+                    // C_c holds two parts per chunk, G_end one
+                    const int za = (KIND == 0 || KIND == 3) ? 2 * zc + part : zc;
 #pragma unroll
                     for (int mb = 0; mb < 2; ++mb) {
-                        if (KIND == 2)   // G_end rows d (K), columns j (M)
-                            tma_load_3d(a + mb * 8192, &tm_a2, m0 + 64 * mb, k0, zc, &full[st]);
+                        if (A2_MN)       // G_end or C_c rows d (K), columns j (M)
+                            tma_load_3d(a + mb * 8192, &tm_a2, m0 + 64 * mb, k0, za, &full[st]);
                         else             // C_c or G_end rows d (M), columns j (K)
-                            tma_load_3d(a + mb * 8192, &tm_a2, k0, m0 + 64 * mb, zc, &full[st]);
+                            tma_load_3d(a + mb * 8192, &tm_a2, k0, m0 + 64 * mb, za, &full[st]);
                     }
 #pragma unroll
-                    for (int n = 0; n < L / 64; ++n)   // g, v or k rows (N), columns (K)
+                    for (int n = 0; n < L / 64; ++n)   // g, v, k or q rows (N), columns (K)
                         tma_load_3d(b + n * 8192, &tm_b2, k0, t0 + 64 * n, bh, &full[st]);
                 }
             }
@@ -174,7 +228,8 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 if (!mbar_wait(&full[st], (uint32_t)(kb / STAGES) & 1u, wc)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a = smem_u32(smem + st * SM::STAGE), b = a + SA;
-                const bool loc = kb < nloc;
+                const bool loc = kb < nl;
+                const int first = loc ? kb : kb - nl;   // blocks of this accumulator before this one
                 const int amn = loc ? A1_MN : A2_MN, bmn = loc ? B1_MN : B2_MN;
                 const uint32_t d = tmem + (loc ? 0u : (uint32_t)L);
 #pragma unroll
@@ -182,7 +237,6 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                     // K-major: 32 bytes further along the 128-byte rows; MN-major: 16 rows further
                     const uint64_t ad = amn ? smem_desc(a + kk * 2048, 8192, 1024) : smem_desc(a, 16, 1024) + (uint64_t)(kk * 2);
                     const uint64_t bd = bmn ? smem_desc(b + kk * 2048, 8192, 1024) : smem_desc(b, 16, 1024) + (uint64_t)(kk * 2);
-                    const int first = loc ? kb : kb - nloc;
                     mma_ss(d, ad, bd, loc ? ID1 : ID2, (first > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&empty[st]);
@@ -198,10 +252,11 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
         if (et < L) {
             const int t = et;
             const bool okt = t < len;
-            if (KIND == 0) {
+            if (KIND == 0 || KIND == 3) {
                 const float mc = p.MC[(size_t)bh * (p.NC + 1) + c];
                 tokw[t] = okt ? expf(mc - fmaxf(mc, p.P[g0 + t])) : 0.f;
-                ddv[t] = okt ? p.DD[g0 + t] : 0.f;
+                if (KIND == 0) ddv[t] = okt ? p.DD[g0 + t] : 0.f;
+                else ddv[t] = okt ? p.NRM[g0 + t] : 1.f;
             } else {
                 const float gm = p.G[(size_t)bh * p.NC + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1];
                 tokw[t] = okt ? expf(p.ig[g0 + t] - p.A[g0 + t] + gm) : 0.f;
@@ -212,7 +267,7 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
         if (KIND == 0) colv = p.NS[((size_t)bh * p.NC + c) * p.DK + col];
         if (KIND == 1) colv = p.GN[((size_t)bh * p.NC + c) * p.DK + col];
         const float scale = rsqrtf((float)p.DK);
-        const int NCOL = KIND == 2 ? p.DV : p.DK;
+        const int NCOL = KIND >= 2 ? p.DV : p.DK;
         named_sync(1, 128);   // tokw, ddv
         // one thread waits for the accumulators; the four warps take its answer together (the TMEM
         // loads below are warp-collective)
@@ -227,6 +282,10 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 tmem_ld16(tmem_addr(tmem, q4 * 32, g * 16), r1);
                 tmem_ld16(tmem_addr(tmem, q4 * 32, L + g * 16), r2);
                 float pv[16];
+                if (KIND == 3) {
+                    epilogue_num(p, r1, r2, tokw, ddv, red + q4 * L, g, len, g0, col, scale, lane);
+                    continue;
+                }
                 if (KIND < 2) {
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
@@ -261,6 +320,16 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
             }
         }
     }
+    if (KIND == 3 && warp >= 2) {
+        // the row sums of g . hh over each 64 value columns: the two warps of a 64-column half
+        named_sync(1, 128);
+        const int et = threadIdx.x - 64;
+        for (int e = et; e < 2 * L; e += 128) {
+            const int h2 = e / L, t = e % L;
+            if (t < len && !*reinterpret_cast<volatile uint32_t *>(abort_flag))
+                p.DOTP[((size_t)bh * p.S + t0 + t) * p.NJT + (m0 >> 6) + h2] = red[(2 * h2) * L + t] + red[(2 * h2 + 1) * L + t];
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
@@ -283,7 +352,8 @@ static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUten
 {
     using SM = Smem<L>;
     KParams p;
-    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV; p.NTK = a.NTK;
+    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV; p.NTK = a.NTK; p.NJT = a.NJT;
+    p.dh = a.dh; p.o = a.o; p.NRM = a.NRM; p.Gt = a.Gt; p.DOTP = a.DOTP; p.g16w = a.g16w; p.dog = a.dog;
     p.A = a.A; p.P = a.P; p.MC = a.MC; p.G = a.G; p.ig = a.ig; p.DD = a.DD; p.NS = a.NS; p.GN = a.GN;
     p.pq = KIND == 0 ? a.q : a.k;
     p.out = KIND == 0 ? a.dq : KIND == 1 ? a.dk : a.dv;
@@ -291,7 +361,7 @@ static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUten
     p.status = a.status;
     cudaError_t e = ensure_dynamic_smem((const void *)grad_tc_kernel<KIND, L>, SM::TOTAL);
     if (e != cudaSuccess) return e;
-    const int tiles = (KIND == 2 ? a.DV : a.DK) / TM;
+    const int tiles = (KIND >= 2 ? a.DV : a.DK) / TM;
     return launch_kernel(grad_tc_kernel<KIND, L>, dim3(a.BH, a.NC, tiles), dim3(THREADS), SM::TOTAL, a.stream, 1, a1,
                          b1, a2, b2, p);
 }
@@ -300,15 +370,31 @@ template <int L>
 static cudaError_t launch_l(const Args &a)
 {
     CUtensorMap mq, mk, mv, mg, mds, ma, mc, mG;
-    const int CL = a.NC * L;   // rows of the per-chunk score arrays
+    const int CL = a.NC * L;   // rows of the per-chunk score arrays (A and C_c: two parts each)
     if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&mk, a.k, a.DK, a.S, a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH) ||
-        !map3(&mg, a.g16, a.DV, a.S, a.BH) || !map3(&mds, a.dS16, L, CL, a.BH) || !map3(&ma, a.A16, L, CL, a.BH) ||
-        !map3(&mc, a.C16, a.DV, a.DK, a.BH * a.NC) || !map3(&mG, a.G16, a.DV, a.DK, a.BH * a.NC))
+        !map3(&mg, a.g16, a.DV, a.S, a.BH) || !map3(&mds, a.dS16, L, CL, a.BH) || !map3(&ma, a.A16, L, 2 * CL, a.BH) ||
+        !map3(&mc, a.C16, a.DV, a.DK, 2 * a.BH * a.NC) || !map3(&mG, a.G16, a.DV, a.DK, a.BH * a.NC))
         return cudaErrorInvalidValue;
     cudaError_t e = launch_kind<0, L>(a, mk, mds, mc, mg);
     if (e == cudaSuccess) e = launch_kind<1, L>(a, mq, mds, mG, mv);
     if (e == cudaSuccess) e = launch_kind<2, L>(a, mg, ma, mG, mk);
     return e;
+}
+
+template <int L>
+static cudaError_t launch_num_l(const Args &a)
+{
+    CUtensorMap mq, mv, ma, mc;
+    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH) ||
+        !map3(&ma, a.A16, L, 2 * a.NC * L, a.BH) || !map3(&mc, a.C16, a.DV, a.DK, 2 * a.BH * a.NC))
+        return cudaErrorInvalidValue;
+    return launch_kind<3, L>(a, mv, ma, mc, mq);
+}
+
+cudaError_t launch_num(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_num_l<64>(a) : launch_num_l<128>(a);
 }
 
 bool supported(int DK, int DV, int L)

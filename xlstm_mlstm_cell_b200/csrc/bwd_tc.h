@@ -17,11 +17,21 @@ struct Args {
     const float *DD;                        // gradient of the denominator [BH][S]
     const float *NS, *GN;                   // n at the chunk starts, gradient of n at the chunk ends [BH][NC][DK]
     const __nv_bfloat16 *q, *k, *v;         // inputs [BH][S][DK | DV]
-    // bf16 copies of the fp32 intermediates: chunk-start states and chunk-end state gradients
-    // [BH][NC][DK][DV], the read-out numerator's gradient g [BH][S][DV], dS and A [BH][NC][L][L]
+    // bf16 copies of the fp32 intermediates: chunk-start states C16 [BH][NC][2][DK][DV] and scores
+    // A16 [BH][NC][2][L][L] as two parts each (the bf16 value and the bf16 of its rounding
+    // residue: together about 16 significant bits), chunk-end state gradients G16 [BH][NC][DK][DV],
+    // the read-out numerator's gradient g16 [BH][S][DV] and dS16 [BH][NC][L][L]
     const __nv_bfloat16 *C16, *G16, *g16, *dS16, *A16;
     __nv_bfloat16 *dq, *dk, *dv;            // outputs [BH][S][DK | DV]
     float *QD, *KD;                         // partial q . dq and k . dk per 32 columns [BH][S][NTK]
+    // the read-out numerator: dh, o (NULL without an output gate) [BH][S][DV], N = max(|den|,
+    // exp(-m)) [BH][S]; writes g (fp32 and its bf16 copy g16), do (when o is given) and the partial
+    // row sums of g . hh per 64 value columns DOTP [BH][S][NJT]
+    const __nv_bfloat16 *dh, *o;
+    const float *NRM;
+    float *Gt, *DOTP;
+    __nv_bfloat16 *g16w, *dog;
+    int NJT;
     uint32_t *status;
     cudaStream_t stream;
 };
@@ -30,6 +40,8 @@ struct Args {
 bool supported(int DK, int DV, int L);
 // The dq, dk and dv products of every chunk (three launches on a.stream).
 cudaError_t launch(const Args &a);
+// The read-out numerator of every chunk, num = sc qh C_c + A V, and what follows from it (one launch).
+cudaError_t launch_num(const Args &a);
 
 }  // namespace bwdtc
 }  // namespace mlstm

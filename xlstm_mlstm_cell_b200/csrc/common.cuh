@@ -26,6 +26,13 @@ MLSTM_DEVINL uint32_t bf16x2_bits(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// A float as two bf16: its rounding and the rounding of the residue (about 16 significant bits).
+MLSTM_DEVINL void bf16_parts(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
+{
+    hi = __float2bfloat16_rn(x);
+    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
 // Four consecutive elements as float (16-byte aligned for float, 8 for bf16).
 MLSTM_DEVINL float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 MLSTM_DEVINL float4 load4(const __nv_bfloat16 *p)

@@ -149,8 +149,14 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
                 if (ri + r < DHQK) {
                     const size_t o = cso + (size_t)(ri + r) * DHV + cj;
                     *reinterpret_cast<float4 *>(CS + o) = make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
-                    if (CS16)   // the bf16 copy the backward's tensor-core products read
-                        *reinterpret_cast<uint2 *>(CS16 + o) = make_uint2(bf16x2_bits(c[r][0], c[r][1]), bf16x2_bits(c[r][2], c[r][3]));
+                    if (CS16) {   // the two bf16 parts the backward's tensor-core products read
+                        __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) bf16_parts(c[r][x], hi[x], lo[x]);
+                        const size_t o16 = 2 * cso + (size_t)(ri + r) * DHV + cj;
+                        *reinterpret_cast<uint2 *>(CS16 + o16) = *reinterpret_cast<const uint2 *>(hi);
+                        *reinterpret_cast<uint2 *>(CS16 + o16 + (size_t)DHQK * DHV) = *reinterpret_cast<const uint2 *>(lo);
+                    }
                 }
         }
         if (n_warp && i0 + tid < DHQK) NS[((size_t)bh * NC + ch) * DHQK + i0 + tid] = nn;

@@ -103,11 +103,11 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->CS16 = w->GS16 = w->Gt16 = w->P216 = w->AI16 = nullptr;
     if (tc) {
         const size_t h = sizeof(__nv_bfloat16);
-        w->CS16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * DHQK * DHV));
+        w->CS16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * DHQK * DHV));   // two parts
         w->GS16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * DHQK * DHV));
         w->Gt16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * S * DHV));
         w->P216 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
-        w->AI16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
+        w->AI16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * chunk * chunk));   // two parts
     }
     return off;
 }

@@ -49,7 +49,7 @@ struct FwdWorkspace {
     float *G, *Bc;         // [BH][NC] chunk log decay, chunk max-plus offset
     float *MC;             // [BH][NC+1] stabilizer at chunk starts (last = final m)
     float *CS, *NS;        // SIMT path: state at every chunk start
-    __nv_bfloat16 *CS16;   // optional bf16 copy of CS (the backward's tensor-core products), else NULL
+    __nv_bfloat16 *CS16;   // optional bf16 parts of CS [BH][NC][2][DHQK][DHV] (the backward), else NULL
     // tensor-core path
     bool tc;               // the tensor-core path is used
     int NSEG, R;           // segments per head and chunks per segment
@@ -82,8 +82,9 @@ struct BwdWorkspace {
     float *QD, *KD;               // [BH][S][ceil(DHQK / 32)] partial q . dq, k . dk
     float *DEN, *NRM;             // [BH][S] read-out denominator and its floored magnitude
     float *DOTP;                  // [BH][S][ceil(DHV / 64)] partial row sums of g . hh
-    // the tensor-core gradient products (bf16 inputs, bwd_tc_path): bf16 copies of CS, GS, Gt, P2
-    // and AI in the same layouts; NULL on the CUDA-core path
+    // the tensor-core products (bf16 inputs, bwd_tc_path): bf16 copies of GS, Gt and P2 in the same
+    // layouts, and of CS and AI as two parts each (value and rounding residue: [BH][NC][2][...]);
+    // NULL on the CUDA-core path
     bool tc;
     __nv_bfloat16 *CS16, *GS16, *Gt16, *P216, *AI16;
 };
