@@ -292,9 +292,10 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
  * (it holds the chunk-start states and their gradients and the chunk's scores:
  * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
- * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head, and on
- * the tensor-core path also 6 DHQK DHV + 6 chunk^2 bytes per chunk and head
- * and 2 DHV bytes per token and head, each array 256-byte aligned).  A bounded
+ * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head; on the
+ * tensor-core path the chunk-start states are kept as bf16 parts instead of
+ * fp32 and bf16 copies are added, 2 DHQK DHV + 6 chunk^2 more bytes per chunk
+ * and head and 6 DHV more per token and head; each array 256-byte aligned).  A bounded
  * device-side wait of the tensor-core products that gives up records a
  * timeout that mlstm_fwd_status reads from this workspace.  Errors as for
  * mlstm_fwd.

@@ -697,7 +697,8 @@ cudaError_t launch_t(const Params &p, int BH, cudaStream_t st, const bwdtc::Args
     if (e != cudaSuccess) return e;
     e = launch_kernel(bwd_ds_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
-    e = launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
+    e = tc ? bwdtc::launch_dc(*tc)
+           : launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
     e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV / 4 + 255) / 256, BH), dim3(256), 0, st, 1, p);
     if (e != cudaSuccess) return e;
@@ -736,7 +737,7 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     t.QD = w.QD; t.KD = w.KD; t.status = w.status; t.stream = a.stream;
     t.dh = static_cast<const bf *>(a.dh); t.o = static_cast<const bf *>(a.ogate); t.NRM = w.NRM;
     t.Gt = w.Gt; t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
-    t.NJT = p.NJT;
+    t.NJT = p.NJT; t.sg16 = w.SG16; t.GS = w.GS;
     return bwd::launch_t<bf>(p, a.BH, a.stream, &t);
 }
 

@@ -58,7 +58,7 @@ struct KParams {
     const __nv_bfloat16 *dh, *o;
     const float *NRM;
     float *Gt, *DOTP;
-    __nv_bfloat16 *g16w, *dog;
+    __nv_bfloat16 *g16w, *dog, *sg16;
     uint32_t *status;
 };
 
@@ -83,7 +83,7 @@ __device__ __forceinline__ bool group_any(uint32_t id, uint32_t count, bool pred
 // g = o dh / N; the warp's row sums of g . hh go to red[t].
 __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&r1)[16], const uint32_t (&r2)[16],
                                              const float *tokw, const float *nrm, float *red, int grp, int len,
-                                             size_t g0, int col, float scale, int lane)
+                                             size_t g0, int col, float scale, int lane, __nv_bfloat16 *sg_hi)
 {
     float dhv[16], ov[16];
 #pragma unroll
@@ -107,6 +107,9 @@ __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&
             if (p.dog) p.dog[off] = __float2bfloat16_rn(dhv[u] * hh);
             p.Gt[off] = g;
             p.g16w[off] = __float2bfloat16_rn(g);
+            // sc_t g_t as two bf16 parts, [BH][2][S][DV]: the operand of the state gradient
+            const size_t o2 = (size_t)t * p.DV + col;
+            bf16_parts(tokw[t] * g, sg_hi[o2], sg_hi[o2 + (size_t)p.S * p.DV]);
             pr = g * hh;
         }
 #pragma unroll
@@ -283,7 +286,8 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 tmem_ld16(tmem_addr(tmem, q4 * 32, L + g * 16), r2);
                 float pv[16];
                 if (KIND == 3) {
-                    epilogue_num(p, r1, r2, tokw, ddv, red + q4 * L, g, len, g0, col, scale, lane);
+                    epilogue_num(p, r1, r2, tokw, ddv, red + q4 * L, g, len, g0, col, scale, lane,
+                                 p.sg16 + ((size_t)2 * bh * p.S + t0) * p.DV);
                     continue;
                 }
                 if (KIND < 2) {
@@ -354,6 +358,7 @@ static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUten
     KParams p;
     p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV; p.NTK = a.NTK; p.NJT = a.NJT;
     p.dh = a.dh; p.o = a.o; p.NRM = a.NRM; p.Gt = a.Gt; p.DOTP = a.DOTP; p.g16w = a.g16w; p.dog = a.dog;
+    p.sg16 = a.sg16;
     p.A = a.A; p.P = a.P; p.MC = a.MC; p.G = a.G; p.ig = a.ig; p.DD = a.DD; p.NS = a.NS; p.GN = a.GN;
     p.pq = KIND == 0 ? a.q : a.k;
     p.out = KIND == 0 ? a.dq : KIND == 1 ? a.dk : a.dv;
@@ -395,6 +400,136 @@ cudaError_t launch_num(const Args &a)
 {
     if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
     return a.L == 64 ? launch_num_l<64>(a) : launch_num_l<128>(a);
+}
+
+// ---------------------------------------------------------------- the read-out's state gradient
+// dC_c[d][j] = scale sum_t q_t[d] (sc_t g_t[j]) over the chunk's tokens, one 128 x 128 state tile
+// per CTA: A = q [t][d] (MN-major), B = sc g [t][j] as two bf16 parts (MN-major), K = L tokens per
+// part, one TMEM accumulator of 128 columns, the tile written to dC in fp32.
+template <int L>
+struct DcSmem {
+    static constexpr int NB = 2 * (L / 64);                   // stages: 64 tokens of one part
+    static constexpr uint32_t STAGE = 2 * 8192 + 2 * 8192;    // q: 64 x 128, sc g: 64 x 128
+    static constexpr uint32_t BAR = NB * STAGE;
+    static constexpr uint32_t TOTAL = BAR + (NB + 1) * 8 + 16 + 1024;
+};
+
+template <int L>
+__global__ void __launch_bounds__(THREADS, 1)
+dc_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sg, KParams p,
+             float *__restrict__ GS)
+{
+    using SM = DcSmem<L>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::BAR), *accf = full + SM::NB;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
+    uint32_t *abort_flag = tmem_slot + 1;
+    const int bh = blockIdx.x, c = blockIdx.y;
+    const int ntj = p.DV / 128, i0 = (blockIdx.z / ntj) * 128, j0 = (blockIdx.z % ntj) * 128;
+    const int t0 = c * L;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    WaitCtx wc{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s <= SM::NB; ++s) mbar_init(&full[s], 1);   // (full[NB] is accf)
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_q);
+        tma_prefetch(&tm_sg);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    griddep_wait();
+    griddep_launch_dependents();
+
+    if (warp == 0) {
+        if (lane == 0) {   // every stage has its own buffer: all loads at once
+            for (int kb = 0; kb < SM::NB; ++kb) {
+                const int part = kb / (L / 64), k0 = 64 * (kb % (L / 64));
+                uint8_t *a = smem + kb * SM::STAGE, *b = a + 16384;
+                mbar_arrive_expect_tx(&full[kb], SM::STAGE);
+                for (int mb = 0; mb < 2; ++mb) tma_load_3d(a + mb * 8192, &tm_q, i0 + 64 * mb, t0 + k0, bh, &full[kb]);
+                for (int nb = 0; nb < 2; ++nb)
+                    tma_load_3d(b + nb * 8192, &tm_sg, j0 + 64 * nb, t0 + k0, 2 * bh + part, &full[kb]);
+            }
+            for (int kb = 0; kb < SM::NB; ++kb) mbar_wait_drain(&full[kb], 0);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t ID = idesc_bf16(128, 128, 1, 1);
+            bool ok = true;
+            for (int kb = 0; kb < SM::NB && ok; ++kb) {
+                if (!mbar_wait(&full[kb], 0, wc)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + kb * SM::STAGE), b = a + 16384;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem, smem_desc(a + kk * 2048, 8192, 1024), smem_desc(b + kk * 2048, 8192, 1024), ID,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            if (ok) mma_commit(accf);
+        }
+    } else {
+        const int et = threadIdx.x - 64, q4 = warp & 3;
+        const int i = i0 + q4 * 32 + lane;   // this thread's state row
+        bool failed = false;
+        if (et == 0) failed = !mbar_wait(accf, 0, wc);
+        failed = group_any(2, 128, failed);
+        if (!failed) {
+            tc_fence_after();
+            const float scale = rsqrtf((float)p.DK);
+            float *row = GS + (((size_t)bh * p.NC + c) * p.DK + i) * p.DV + j0;
+#pragma unroll 1
+            for (int g = 0; g < 128 / 16; ++g) {
+                uint32_t r[16];
+                tmem_ld16(tmem_addr(tmem, q4 * 32, g * 16), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; u += 4)
+                    *reinterpret_cast<float4 *>(row + g * 16 + u) =
+                        make_float4(scale * __uint_as_float(r[u]), scale * __uint_as_float(r[u + 1]),
+                                    scale * __uint_as_float(r[u + 2]), scale * __uint_as_float(r[u + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
+        const unsigned long long tb = global_timer();
+        while (global_timer() - tb < 100000ull) { }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+template <int L>
+static cudaError_t launch_dc_l(const Args &a)
+{
+    using SM = DcSmem<L>;
+    CUtensorMap mq, msg;
+    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&msg, a.sg16, a.DV, a.S, 2 * a.BH)) return cudaErrorInvalidValue;
+    KParams p{};
+    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
+    p.status = a.status;
+    cudaError_t e = ensure_dynamic_smem((const void *)dc_tc_kernel<L>, SM::TOTAL);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(dc_tc_kernel<L>, dim3(a.BH, a.NC, (a.DK / 128) * (a.DV / 128)), dim3(THREADS), SM::TOTAL,
+                         a.stream, 1, mq, msg, p, a.GS);
+}
+
+cudaError_t launch_dc(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_dc_l<64>(a) : launch_dc_l<128>(a);
 }
 
 bool supported(int DK, int DV, int L)

@@ -32,6 +32,10 @@ struct Args {
     float *Gt, *DOTP;
     __nv_bfloat16 *g16w, *dog;
     int NJT;
+    // sc_t g_t as two bf16 parts [BH][2][S][DV] (written by the numerator's epilogue, read by the
+    // read-out's state gradient), and that gradient dC_c = scale (sc Q)^T g, fp32 [BH][NC][DK][DV]
+    __nv_bfloat16 *sg16;
+    float *GS;
     uint32_t *status;
     cudaStream_t stream;
 };
@@ -42,6 +46,8 @@ bool supported(int DK, int DV, int L);
 cudaError_t launch(const Args &a);
 // The read-out numerator of every chunk, num = sc qh C_c + A V, and what follows from it (one launch).
 cudaError_t launch_num(const Args &a);
+// The read-out's state gradient of every chunk, dC_c = (sc qh)^T g (one launch).
+cudaError_t launch_dc(const Args &a);
 
 }  // namespace bwdtc
 }  // namespace mlstm

@@ -31,7 +31,8 @@ constexpr int ST = 32;   // state tile edge (rows of C and columns of C / h)
 // grid (BH, ceil(DHQK/64), ceil(DHV/64)), 256 threads; thread (tx, ty) = (tid % 16, tid / 16)
 // owns rows 4 ty .. 4 ty + 3 and columns 4 tx .. 4 tx + 3 of a 64 x 64 tile of C, and in the tiles
 // of columns 0..63 threads 0..63 own n of their row.  Walks all chunks of its head in order,
-// storing the state at every chunk start (CS, NS) and the final state.  A chunk's k (fp32) and
+// storing the state at every chunk start (CS, or its two bf16 parts CS16 when given; NS) and the
+// final state.  A chunk's k (fp32) and
 // w_s v_s are staged in shared memory, so that a step of the reduction over the chunk's tokens is
 // two 16-byte loads and 16 FMAs per thread; the next chunk's k, v and gates are loaded into
 // registers while the current chunk's steps run.  Every state element takes the operations of a
@@ -148,8 +149,9 @@ carry_simt_kernel(const T *__restrict__ k, const T *__restrict__ v, const float 
             for (int r = 0; r < 4; ++r)
                 if (ri + r < DHQK) {
                     const size_t o = cso + (size_t)(ri + r) * DHV + cj;
-                    *reinterpret_cast<float4 *>(CS + o) = make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
-                    if (CS16) {   // the two bf16 parts the backward's tensor-core products read
+                    if (!CS16) {
+                        *reinterpret_cast<float4 *>(CS + o) = make_float4(c[r][0], c[r][1], c[r][2], c[r][3]);
+                    } else {   // only the two bf16 parts, which the backward's tensor-core products read
                         __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
                         for (int x = 0; x < 4; ++x) bf16_parts(c[r][x], hi[x], lo[x]);

@@ -86,7 +86,8 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->G = reinterpret_cast<float *>(take(f * BH * NC));
     w->Bc = reinterpret_cast<float *>(take(f * BH * NC));
     w->MC = reinterpret_cast<float *>(take(f * BH * (NC + 1)));
-    w->CS = reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
+    // (the tensor-core path keeps the chunk-start states only as their bf16 parts, below)
+    w->CS = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
     w->NS = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
     w->GS = reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
     w->GN = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
@@ -100,7 +101,7 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->NRM = reinterpret_cast<float *>(take(f * BH * S));
     w->DOTP = reinterpret_cast<float *>(take(f * BH * S * ((DHV + 63) / 64)));
     w->tc = tc;
-    w->CS16 = w->GS16 = w->Gt16 = w->P216 = w->AI16 = nullptr;
+    w->CS16 = w->GS16 = w->Gt16 = w->P216 = w->AI16 = w->SG16 = nullptr;
     if (tc) {
         const size_t h = sizeof(__nv_bfloat16);
         w->CS16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * DHQK * DHV));   // two parts
@@ -108,6 +109,7 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
         w->Gt16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * S * DHV));
         w->P216 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
         w->AI16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * chunk * chunk));   // two parts
+        w->SG16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * S * DHV));             // two parts
     }
     return off;
 }

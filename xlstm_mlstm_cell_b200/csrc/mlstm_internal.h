@@ -87,6 +87,7 @@ struct BwdWorkspace {
     // NULL on the CUDA-core path
     bool tc;
     __nv_bfloat16 *CS16, *GS16, *Gt16, *P216, *AI16;
+    __nv_bfloat16 *SG16;          // sc_t g_t as two bf16 parts [BH][2][S][DHV]
 };
 
 // Records the caller's phase events (mlstm_fwd_profiled); a no-op without events.
