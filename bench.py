@@ -674,14 +674,19 @@ def bwd_extra(w: Workload, device, peaks, reps: int = 5):
     torch.cuda.synchronize()
     t = e0.elapsed_time(e1) / reps / 1e3
     bw = bwd_work(w)
-    roof = roofline(bw, t, peaks, False)
+    tensor = binding.bwd_tensor_path(w.DHQK, w.DHV, w.chunk, w.torch_dtype) == 1
+    roof = roofline(bw, t, peaks, tensor)
     roof["kernel"] = "mlstm_bwd (all kernels of the call)"
     del s, dh, ws, out
     torch.cuda.empty_cache()
     return {"workload": "%s shape (B%d NH%d S%d d%d/%d chunk %d, %s)" % (w.name, w.B, w.NH, w.S, w.DHQK, w.DHV, w.chunk,
                                                                         w.dtype),
             "ms": t * 1e3, "tokens_per_s": w.B * w.S / t, "tflops": bw["flops"] / t / 1e12,
-            "kernel_launches": "gate preprocessing, chunk-start states, 4 backward kernels", "roofline": roof}
+            "products": ("read-out numerator, its state gradient and dq, dk, dv on tcgen05 (bf16 operands, fp32 "
+                         "accumulation); scores, dS and the scans on the CUDA cores") if tensor else
+                        "every product on the CUDA cores (fp32)",
+            "kernel_launches": "gate preprocessing, chunk-start states, scores, numerator, dS, state gradient, "
+                               "state-gradient scan, dq, dk, dv, gate gradients", "roofline": roof}
 
 
 def extras(device, peaks, skip=None):

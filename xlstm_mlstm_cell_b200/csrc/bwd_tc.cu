@@ -78,6 +78,27 @@ __device__ __forceinline__ bool group_any(uint32_t id, uint32_t count, bool pred
     return r != 0;
 }
 
+// Sums v[u] (u < 16) over the 32 lanes of the warp for every u at once: each step hands half of the
+// remaining values to the lane partner and keeps the other half.  Lane l ends with the sum of value
+// sum16_index(l) (both lanes of a pair hold it).
+__device__ __forceinline__ float warp_sum16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int o = 16, nv = 16; o >= 2; o >>= 1, nv >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int z = 0; z < nv / 2; ++z) {
+            const float send = up ? v[z] : v[z + nv / 2], keep = up ? v[z + nv / 2] : v[z];
+            v[z] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+__device__ __forceinline__ int sum16_index(int lane)
+{
+    return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
+
 // The read-out numerator's epilogue for 16 tokens g * 16 .. of a thread's value column:
 // num = A V + sc scale q C_c (r1, r2: the two accumulators' columns), hh = num / N, do = dh hh,
 // g = o dh / N; the warp's row sums of g . hh go to red[t].
@@ -94,15 +115,16 @@ __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&
         ov[u] = (t < len && p.o) ? __bfloat162float(p.o[off]) : 1.f;
     }
     tmem_wait_ld();
+    float pr[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
         const int t = grp * 16 + u;
         const size_t off = (g0 + t) * p.DV + col;
         const float num = __uint_as_float(r1[u]) + tokw[t] * scale * __uint_as_float(r2[u]);
-        const float N = nrm[t];
-        const float hh = num / N;
-        const float g = ov[u] * dhv[u] / N;
-        float pr = 0.f;
+        const float rN = nrm[t];   // 1 / N
+        const float hh = num * rN;
+        const float g = ov[u] * dhv[u] * rN;
+        pr[u] = 0.f;
         if (t < len) {
             if (p.dog) p.dog[off] = __float2bfloat16_rn(dhv[u] * hh);
             p.Gt[off] = g;
@@ -110,12 +132,11 @@ __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&
             // sc_t g_t as two bf16 parts, [BH][2][S][DV]: the operand of the state gradient
             const size_t o2 = (size_t)t * p.DV + col;
             bf16_parts(tokw[t] * g, sg_hi[o2], sg_hi[o2 + (size_t)p.S * p.DV]);
-            pr = g * hh;
+            pr[u] = g * hh;
         }
-#pragma unroll
-        for (int sh = 16; sh > 0; sh >>= 1) pr += __shfl_xor_sync(0xffffffffu, pr, sh);
-        if (lane == 0) red[t] = pr;
     }
+    const float sum = warp_sum16(pr, lane);
+    if ((lane & 1) == 0) red[grp * 16 + sum16_index(lane)] = sum;
 }
 
 // KIND 0: dq, 1: dk, 2: dv, 3: the read-out numerator num^T = V^T A^T + sc scale C_c^T Q^T.
@@ -125,7 +146,7 @@ __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&
 //   KIND 2: A1 = g [t][j] (MN),       B1 = A [t][s] (MN),       A2 = G_end [d][j] (MN), B2 = k [s][d] (K)
 //   KIND 3: A1 = v [s][j] (MN),       B1 = A [t][s] (K),        A2 = C_c [d][j] (MN),   B2 = q [t][d] (K)
 template <int KIND, int L>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)   // two CTAs per SM: one's epilogue beside the other's loads
 grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_b2, KParams p)
 {
@@ -135,7 +156,7 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *tokw = reinterpret_cast<float *>(smem + SM::F);   // sc_t (KIND 0) or w_s
-    float *ddv = tokw + L;                                    // dden_t (KIND 0), N_t (KIND 3)
+    float *ddv = tokw + L;                                    // dden_t (KIND 0), 1 / N_t (KIND 3)
     float *red = ddv + L;                                     // [4][L] per-warp row sums (KIND 3)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
     uint64_t *full = bars, *empty = bars + STAGES, *accf = bars + 2 * STAGES;
@@ -259,7 +280,7 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 const float mc = p.MC[(size_t)bh * (p.NC + 1) + c];
                 tokw[t] = okt ? expf(mc - fmaxf(mc, p.P[g0 + t])) : 0.f;
                 if (KIND == 0) ddv[t] = okt ? p.DD[g0 + t] : 0.f;
-                else ddv[t] = okt ? p.NRM[g0 + t] : 1.f;
+                else ddv[t] = okt ? 1.f / p.NRM[g0 + t] : 1.f;
             } else {
                 const float gm = p.G[(size_t)bh * p.NC + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1];
                 tokw[t] = okt ? expf(p.ig[g0 + t] - p.A[g0 + t] + gm) : 0.f;
@@ -298,6 +319,7 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                     }
                 }
                 tmem_wait_ld();
+                float prs[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int t = g * 16 + u;
@@ -315,11 +337,12 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                         o = d1 + w * d2;
                     }
                     if (t < len) p.out[(g0 + t) * NCOL + col] = __float2bfloat16_rn(o);
-                    if (KIND < 2) {
-#pragma unroll
-                        for (int sh = 16; sh > 0; sh >>= 1) pr += __shfl_xor_sync(0xffffffffu, pr, sh);
-                        if (lane == 0 && t < len) p.part[(g0 + t) * p.NTK + (col >> 5)] = pr;
-                    }
+                    prs[u] = pr;
+                }
+                if (KIND < 2) {   // q . dq or k . dk over the warp's 32 columns, per token
+                    const float sum = warp_sum16(prs, lane);
+                    const int t = g * 16 + sum16_index(lane);
+                    if ((lane & 1) == 0 && t < len) p.part[(g0 + t) * p.NTK + (col >> 5)] = sum;
                 }
             }
         }
