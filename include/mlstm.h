@@ -282,12 +282,14 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * then; ignored when ogate is NULL).  No gradient flows into or out of the
  * states: the sequence starts from the zero state and the final state is not
  * part of L.  The forward pass is recomputed inside (gate preprocessing and
- * the fp32 chunk-start states).  The chunk's scores, read-out gradients and
- * the state gradients are fp32 on the CUDA cores; the dq, dk and dv products
- * and the read-out numerator run on the tensor cores (tcgen05, bf16 copies of
- * the fp32 intermediates as operands, the numerator's fp32 operands as two
- * bf16 parts each, fp32 accumulation) when mlstm_bwd_tensor_path says so,
- * else in fp32 on the CUDA cores.  Shapes and chunk sizes as for mlstm_fwd.
+ * the chunk-start states).  When mlstm_bwd_tensor_path says so, the products
+ * (the chunk-start states' contributions, the read-out numerator and its state
+ * gradient, dq, dk and dv) run on the tensor cores (tcgen05, fp32
+ * accumulation; bf16 operands, where an operand is an fp32 intermediate that
+ * the result is sensitive to, as two bf16 parts, value and rounding residue)
+ * and the scores, dS and the scans in fp32 on the CUDA cores; otherwise every
+ * step runs in fp32 on the CUDA cores.  Shapes and chunk sizes as for
+ * mlstm_fwd.
  *
  * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
  * (it holds the chunk-start states and their gradients and the chunk's scores:
@@ -295,7 +297,8 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head; on the
  * tensor-core path the chunk-start states are kept as bf16 parts instead of
  * fp32 and bf16 copies are added, 2 DHQK DHV + 6 chunk^2 more bytes per chunk
- * and head and 6 DHV more per token and head; each array 256-byte aligned).  A bounded
+ * and head and 4 DHQK + 6 DHV more per token and head; each array 256-byte
+ * aligned).  A bounded
  * device-side wait of the tensor-core products that gives up records a
  * timeout that mlstm_fwd_status reads from this workspace.  Errors as for
  * mlstm_fwd.

@@ -738,6 +738,9 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     t.dh = static_cast<const bf *>(a.dh); t.o = static_cast<const bf *>(a.ogate); t.NRM = w.NRM;
     t.Gt = w.Gt; t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
     t.NJT = p.NJT; t.sg16 = w.SG16; t.GS = w.GS;
+    t.wk16 = w.WK16; t.C16w = w.CS16; t.NSw = w.NS;
+    cudaError_t e = bwdtc::launch_carry(t);   // the chunk-start states
+    if (e != cudaSuccess) return e;
     return bwd::launch_t<bf>(p, a.BH, a.stream, &t);
 }
 

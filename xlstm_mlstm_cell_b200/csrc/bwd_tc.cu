@@ -27,6 +27,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 namespace mlstm {
 namespace bwdtc {
 
@@ -553,6 +555,233 @@ cudaError_t launch_dc(const Args &a)
 {
     if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
     return a.L == 64 ? launch_dc_l<64>(a) : launch_dc_l<128>(a);
+}
+
+// ---------------------------------------------------------------- the forward carry
+// w_s k_s[d] as two bf16 parts, w_s = exp(g_c - a_s + i~_s - m_{c+1}) (c the chunk of token s): the
+// weight of token s in the state at its chunk's end, in that state's stabilized frame (<= 1).
+__global__ void __launch_bounds__(256) wk_parts_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ A,
+                                                       const float *__restrict__ ig, const float *__restrict__ G,
+                                                       const float *__restrict__ MC, int BH, int S, int L, int NC,
+                                                       int DK, __nv_bfloat16 *__restrict__ wk)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    const int n8 = DK / 8;
+    const size_t items = (size_t)BH * S * n8;
+    for (size_t it = (size_t)blockIdx.x * blockDim.x + threadIdx.x; it < items; it += (size_t)gridDim.x * blockDim.x) {
+        const size_t tok = it / n8;                // bh * S + s
+        const int d0 = (int)(it % n8) * 8;
+        const int bh = (int)(tok / S), s = (int)(tok % S), c = s / L;
+        const float w = expf(G[(size_t)bh * NC + c] - A[tok] + ig[tok] - MC[(size_t)bh * (NC + 1) + c + 1]);
+        const uint4 u = *reinterpret_cast<const uint4 *>(k + tok * DK + d0);
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+        __nv_bfloat16 hi[8], lo[8];
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+            bf16_parts(w * __uint_as_float(wd[z] << 16), hi[2 * z], lo[2 * z]);
+            bf16_parts(w * __uint_as_float(wd[z] & 0xffff0000u), hi[2 * z + 1], lo[2 * z + 1]);
+        }
+        __nv_bfloat16 *dst = wk + ((size_t)(2 * bh) * S + s) * DK + d0;
+        *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(hi);
+        *reinterpret_cast<uint4 *>(dst + (size_t)S * DK) = *reinterpret_cast<const uint4 *>(lo);
+    }
+}
+
+// The walk over the chunks of one 128 x 64 tile of the state (rows d, columns j): per chunk the
+// contribution U_c = sum_s (w_s k_s) v_s^T as MMAs (A = w k, two parts, MN-major; B = v, MN-major)
+// into one of two TMEM buffers, and in the tiles of columns 0..63 also sum_s w_s k_s (B = a tile of
+// ones), while the epilogue warps, which hold the fp32 state in registers (a TMEM lane = a row d,
+// 64 columns per thread), write the state at the chunk's start as two bf16 parts and n, then
+// C <- exp(g_c + m_c - m_{c+1}) C + U_c.
+constexpr int CSTAGES = 4;
+struct CarrySmem {
+    static constexpr uint32_t STAGE = 2 * 16384 + 8192;      // w k: 2 parts x 64 tokens x 128 rows; v: 64 x 64
+    static constexpr uint32_t ONES = CSTAGES * STAGE;        // 16 rows x 64 bf16 ones (K-major B of n)
+    static constexpr uint32_t BAR = ONES + 2048;
+    static constexpr uint32_t NBAR = 2 * CSTAGES + 4;
+    static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
+};
+
+template <int L>
+__global__ void __launch_bounds__(THREADS, 1)
+carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_v, KParams p,
+                __nv_bfloat16 *__restrict__ C16, float *__restrict__ NSo)
+{
+    using SM = CarrySmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
+    uint64_t *full = bars, *empty = bars + CSTAGES, *ufull = bars + 2 * CSTAGES, *ufree = ufull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
+    uint32_t *abort_flag = tmem_slot + 1;
+    const int bh = blockIdx.x, d0 = blockIdx.y * 128, j0 = blockIdx.z * 64;
+    const bool with_n = blockIdx.z == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int KB = L / 64;                 // 64-token blocks per chunk
+    const int nblk = (p.NC - 1) * KB;          // (the last chunk's contribution is not needed)
+    WaitCtx wc{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < CSTAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ufull[b], 1);
+            mbar_init(&ufree[b], 4);   // one arrival per epilogue warp
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_wk);
+        tma_prefetch(&tm_v);
+    }
+    // the ones tile (every element 1.0, so its layout needs no swizzle care)
+    for (int e = threadIdx.x; e < 2048 / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(smem + SM::ONES)[e] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+    fence_proxy_async();
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;   // U buffers at columns 0 and 64, n buffers at 128 and 144
+    griddep_wait();
+    griddep_launch_dependents();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int kb = 0;
+            for (; kb < nblk; ++kb) {
+                const int st = kb % CSTAGES;
+                if (kb >= CSTAGES && !mbar_wait(&empty[st], (uint32_t)((kb / CSTAGES) - 1) & 1u, wc)) break;
+                mbar_arrive_expect_tx(&full[st], SM::STAGE);
+                uint8_t *a = smem + st * SM::STAGE, *b = a + 32768;
+                const int t = kb * 64;   // first token of the block
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int mb = 0; mb < 2; ++mb)
+                        tma_load_3d(a + part * 16384 + mb * 8192, &tm_wk, d0 + 64 * mb, t, 2 * bh + part, &full[st]);
+                tma_load_3d(b, &tm_v, j0, t, bh, &full[st]);
+            }
+            for (int s = 0; s < CSTAGES && s < kb; ++s) {
+                const int last = kb - 1 - s;
+                mbar_wait_drain(&full[last % CSTAGES], (uint32_t)(last / CSTAGES) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t IDU = idesc_bf16(128, 64, 1, 1), IDN = idesc_bf16(128, 16, 1, 0);
+            const uint64_t ones = smem_desc(smem_u32(smem + SM::ONES), 16, 1024);
+            bool ok = true;
+            for (int c = 0; c < p.NC - 1 && ok; ++c) {
+                const int ub = c & 1;
+                if (c >= 2 && !mbar_wait(&ufree[ub], (uint32_t)((c >> 1) - 1) & 1u, wc)) { ok = false; break; }
+                for (int q = 0; q < KB; ++q) {
+                    const int kb = c * KB + q, st = kb % CSTAGES;
+                    if (!mbar_wait(&full[st], (uint32_t)(kb / CSTAGES) & 1u, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(smem + st * SM::STAGE), b = a + 32768;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = smem_desc(a + part * 16384 + kk * 2048, 8192, 1024);
+                            const uint32_t acc = (q > 0 || part > 0 || kk > 0) ? 1u : 0u;
+                            mma_ss(tmem + ub * 64, ad, smem_desc(b + kk * 2048, 8192, 1024), IDU, acc);
+                            if (with_n) mma_ss(tmem + 128 + ub * 16, ad, ones + (uint64_t)(kk * 2), IDN, acc);
+                        }
+                    mma_commit(&empty[st]);
+                }
+                if (ok) mma_commit(&ufull[ub]);
+            }
+        }
+    } else {
+        const int q4 = warp & 3;
+        const int d = d0 + q4 * 32 + lane;   // this thread's state row
+        const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
+        const float *Gb = p.G + (size_t)bh * p.NC;
+        float C[64];
+#pragma unroll
+        for (int x = 0; x < 64; ++x) C[x] = 0.f;
+        float n = 0.f;
+        for (int c = 0; c < p.NC; ++c) {
+            // the state at the chunk's start: its two bf16 parts, and n
+            __nv_bfloat16 *dst = C16 + (((size_t)bh * p.NC + c) * 2 * p.DK + d) * p.DV + j0;
+#pragma unroll
+            for (int x = 0; x < 64; x += 8) {
+                __nv_bfloat16 hi[8], lo[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) bf16_parts(C[x + z], hi[z], lo[z]);
+                *reinterpret_cast<uint4 *>(dst + x) = *reinterpret_cast<const uint4 *>(hi);
+                *reinterpret_cast<uint4 *>(dst + (size_t)p.DK * p.DV + x) = *reinterpret_cast<const uint4 *>(lo);
+            }
+            if (with_n) NSo[((size_t)bh * p.NC + c) * p.DK + d] = n;
+            if (c == p.NC - 1) break;   // (the final state is not needed)
+            const float decay = expf(Gb[c] + MCb[c] - MCb[c + 1]);
+            const int ub = c & 1;
+            bool failed = false;
+            if (lane == 0) failed = !mbar_wait(&ufull[ub], (uint32_t)(c >> 1) & 1u, wc);
+            if (__shfl_sync(0xffffffffu, failed ? 1 : 0, 0)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint32_t r[16];
+                tmem_ld16(tmem_addr(tmem, q4 * 32, ub * 64 + g * 16), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int z = 0; z < 16; ++z) C[g * 16 + z] = fmaf(decay, C[g * 16 + z], __uint_as_float(r[z]));
+            }
+            if (with_n) {
+                uint32_t r4[4];
+                tmem_ld4(tmem_addr(tmem, q4 * 32, 128 + ub * 16), r4);
+                tmem_wait_ld();
+                n = fmaf(decay, n, __uint_as_float(r4[0]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ufree[ub]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
+        const unsigned long long tb = global_timer();
+        while (global_timer() - tb < 100000ull) { }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+template <int L>
+static cudaError_t launch_carry_l(const Args &a)
+{
+    using SM = CarrySmem;
+    const size_t items = (size_t)a.BH * a.S * (a.DK / 8);
+    const unsigned nblk = (unsigned)std::min<size_t>((items + 255) / 256, 148 * 16);
+    cudaError_t e = launch_kernel(wk_parts_kernel, dim3(nblk), dim3(256), 0, a.stream, 1, a.k, a.A, a.ig, a.G, a.MC,
+                                  a.BH, a.S, L, a.NC, a.DK, a.wk16);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mwk, mv;
+    if (!map3(&mwk, a.wk16, a.DK, a.S, 2 * a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH)) return cudaErrorInvalidValue;
+    KParams p{};
+    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
+    p.MC = a.MC; p.G = a.G;
+    p.status = a.status;
+    if ((e = ensure_dynamic_smem((const void *)carry_tc_kernel<L>, SM::TOTAL)) != cudaSuccess) return e;
+    return launch_kernel(carry_tc_kernel<L>, dim3(a.BH, a.DK / 128, a.DV / 64), dim3(THREADS), SM::TOTAL, a.stream, 1,
+                         mwk, mv, p, a.C16w, a.NSw);
+}
+
+cudaError_t launch_carry(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_carry_l<64>(a) : launch_carry_l<128>(a);
 }
 
 bool supported(int DK, int DV, int L)

@@ -36,6 +36,10 @@ struct Args {
     // read-out's state gradient), and that gradient dC_c = scale (sc Q)^T g, fp32 [BH][NC][DK][DV]
     __nv_bfloat16 *sg16;
     float *GS;
+    // the forward carry (launch_carry): w_s k_s as two bf16 parts [BH][2][S][DK] (written, then
+    // read), and its outputs, the chunk-start states as two bf16 parts (the array C16 above) and n
+    __nv_bfloat16 *wk16, *C16w;
+    float *NSw;
     uint32_t *status;
     cudaStream_t stream;
 };
@@ -48,6 +52,10 @@ cudaError_t launch(const Args &a);
 cudaError_t launch_num(const Args &a);
 // The read-out's state gradient of every chunk, dC_c = (sc qh)^T g (one launch).
 cudaError_t launch_dc(const Args &a);
+// The forward pass's chunk-start states C_c (as two bf16 parts) and n_c from the zero state: w_s k_s
+// as two bf16 parts, then a walk over the chunks per state tile with each chunk's contribution
+// sum_s (w_s k_s) v_s^T on tcgen05 and the fp32 state in registers (two launches).
+cudaError_t launch_carry(const Args &a);
 
 }  // namespace bwdtc
 }  // namespace mlstm

@@ -101,7 +101,7 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->NRM = reinterpret_cast<float *>(take(f * BH * S));
     w->DOTP = reinterpret_cast<float *>(take(f * BH * S * ((DHV + 63) / 64)));
     w->tc = tc;
-    w->CS16 = w->GS16 = w->Gt16 = w->P216 = w->AI16 = w->SG16 = nullptr;
+    w->CS16 = w->GS16 = w->Gt16 = w->P216 = w->AI16 = w->SG16 = w->WK16 = nullptr;
     if (tc) {
         const size_t h = sizeof(__nv_bfloat16);
         w->CS16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * DHQK * DHV));   // two parts
@@ -110,6 +110,7 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
         w->P216 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
         w->AI16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * chunk * chunk));   // two parts
         w->SG16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * S * DHV));             // two parts
+        w->WK16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * S * DHQK));            // two parts
     }
     return off;
 }
@@ -375,7 +376,8 @@ extern "C" mlstm_status mlstm_bwd(const void *q, const void *k, const void *v, c
     fw.tc = false;
     FwdArgs fa{q, k, v, nullptr, igate, fgate, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, BH, S, DHQK, DHV,
                chunk, bf16, st, false};
-    if (launch_fwd_simt(fa, fw, PhaseMark{}) != cudaSuccess) return MLSTM_ERR_CUDA;
+    // (on the tensor-core path the backward's own carry walk computes the chunk-start states)
+    if (!w.tc && launch_fwd_simt(fa, fw, PhaseMark{}) != cudaSuccess) return MLSTM_ERR_CUDA;
     BwdArgs ba{q, k, v, ogate, dh, igate, fgate, dq, dk, dv, dogate, digate, dfgate, BH, S, DHQK, DHV, chunk, bf16,
                st};
     return cuda_status(launch_bwd(ba, w));

@@ -88,6 +88,7 @@ struct BwdWorkspace {
     bool tc;
     __nv_bfloat16 *CS16, *GS16, *Gt16, *P216, *AI16;
     __nv_bfloat16 *SG16;          // sc_t g_t as two bf16 parts [BH][2][S][DHV]
+    __nv_bfloat16 *WK16;          // w_s k_s as two bf16 parts [BH][2][S][DHQK] (the carry walk)
 };
 
 // Records the caller's phase events (mlstm_fwd_profiled); a no-op without events.
