@@ -295,9 +295,10 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * (it holds the chunk-start states and their gradients and the chunk's scores:
  * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
  * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head; on the
- * tensor-core path the chunk-start states are kept as bf16 parts instead of
- * fp32 and bf16 copies are added, 2 DHQK DHV + 6 chunk^2 more bytes per chunk
- * and head and 4 DHQK + 6 DHV more per token and head; each array 256-byte
+ * tensor-core path, where the chunk-start states, the scores and g are kept
+ * as bf16 parts instead of fp32, 10 DHQK DHV + 8 DHQK + 6 chunk^2 + 12 bytes
+ * per chunk and head, plus 4 DHQK + 8 DHV + 8 ceil(DHQK / 32) +
+ * 4 ceil(DHV / 64) + 20 bytes per token and head; each array 256-byte
  * aligned).  A bounded
  * device-side wait of the tensor-core products that gives up records a
  * timeout that mlstm_fwd_status reads from this workspace.  Errors as for

@@ -481,10 +481,11 @@ __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
                 for (int u = 0; u < BATCH; ++u) {
                     const int c = c1 - 1 - u;
                     if (c >= cb) {
-                        slot[(size_t)c * nq] = G;
-                        if (p.GS16)   // the bf16 copy of the chunk-end gradient
+                        if (p.GS16)   // only the bf16 copy of the chunk-end gradient: all its readers take that
                             reinterpret_cast<uint2 *>(p.GS16 + (size_t)bh * p.NC * nstate)[(size_t)c * nq + e] =
                                 make_uint2(bf16x2_bits(G.x, G.y), bf16x2_bits(G.z, G.w));
+                        else
+                            slot[(size_t)c * nq] = G;
                         const float f = decay[c - cb];
                         G = make_float4(d[u].x + f * G.x, d[u].y + f * G.y, d[u].z + f * G.z, d[u].w + f * G.w);
                     }
@@ -691,11 +692,11 @@ template <typename T>
 cudaError_t launch_t(const Params &p, int BH, cudaStream_t st, const bwdtc::Args *tc)
 {
     cudaError_t e;
-    e = launch_kernel(bwd_scores_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
+    e = tc ? bwdtc::launch_scores(*tc) : launch_kernel(bwd_scores_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
     e = tc ? bwdtc::launch_num(*tc) : launch_kernel(bwd_num_kernel<T>, dim3(BH, p.NC, p.NJT), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
-    e = launch_kernel(bwd_ds_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
+    e = tc ? bwdtc::launch_ds(*tc) : launch_kernel(bwd_ds_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
     e = tc ? bwdtc::launch_dc(*tc)
            : launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
@@ -736,9 +737,10 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     t.dq = static_cast<bf *>(a.dq); t.dk = static_cast<bf *>(a.dk); t.dv = static_cast<bf *>(a.dv);
     t.QD = w.QD; t.KD = w.KD; t.status = w.status; t.stream = a.stream;
     t.dh = static_cast<const bf *>(a.dh); t.o = static_cast<const bf *>(a.ogate); t.NRM = w.NRM;
-    t.Gt = w.Gt; t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
+    t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
     t.NJT = p.NJT; t.sg16 = w.SG16; t.GS = w.GS;
     t.wk16 = w.WK16; t.C16w = w.CS16; t.NSw = w.NS;
+    t.DENw = w.DEN; t.NRMw = w.NRM; t.DDw = w.DD; t.GNw = w.GN; t.A16w = w.AI16; t.dS16w = w.P216;
     cudaError_t e = bwdtc::launch_carry(t);   // the chunk-start states
     if (e != cudaSuccess) return e;
     return bwd::launch_t<bf>(p, a.BH, a.stream, &t);

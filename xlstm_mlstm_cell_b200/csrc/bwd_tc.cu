@@ -59,7 +59,7 @@ struct KParams {
     // KIND 3 (the read-out numerator)
     const __nv_bfloat16 *dh, *o;
     const float *NRM;
-    float *Gt, *DOTP;
+    float *DOTP;
     __nv_bfloat16 *g16w, *dog, *sg16;
     uint32_t *status;
 };
@@ -106,7 +106,8 @@ __device__ __forceinline__ int sum16_index(int lane)
 // g = o dh / N; the warp's row sums of g . hh go to red[t].
 __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&r1)[16], const uint32_t (&r2)[16],
                                              const float *tokw, const float *nrm, float *red, int grp, int len,
-                                             size_t g0, int col, float scale, int lane, __nv_bfloat16 *sg_hi)
+                                             size_t g0, int col, float scale, int lane, __nv_bfloat16 *sg_hi,
+                                             __nv_bfloat16 *g_hi)
 {
     float dhv[16], ov[16];
 #pragma unroll
@@ -129,10 +130,10 @@ __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&
         pr[u] = 0.f;
         if (t < len) {
             if (p.dog) p.dog[off] = __float2bfloat16_rn(dhv[u] * hh);
-            p.Gt[off] = g;
-            p.g16w[off] = __float2bfloat16_rn(g);
-            // sc_t g_t as two bf16 parts, [BH][2][S][DV]: the operand of the state gradient
+            // g and sc_t g_t as two bf16 parts each, [BH][2][S][DV]: the operands of dS, dq, dv and
+            // of the state gradient
             const size_t o2 = (size_t)t * p.DV + col;
+            bf16_parts(g, g_hi[o2], g_hi[o2 + (size_t)p.S * p.DV]);
             bf16_parts(tokw[t] * g, sg_hi[o2], sg_hi[o2 + (size_t)p.S * p.DV]);
             pr[u] = g * hh;
         }
@@ -214,7 +215,7 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 if (loc) {
 #pragma unroll
                     for (int mb = 0; mb < 2; ++mb)   // A1 rows: the stage's 64 tokens, 2 x 64 output columns
-                        tma_load_3d(a + mb * 8192, &tm_a1, m0 + 64 * mb, t0 + k0, bh, &full[st]);
+                        tma_load_3d(a + mb * 8192, &tm_a1, m0 + 64 * mb, t0 + k0, KIND == 2 ? 2 * bh : bh, &full[st]);
                     // the chunk's first row in the score arrays: A holds two parts per chunk
                     const int rb = KIND >= 2 ? 2 * t0 + part * L : t0;
 #pragma unroll
@@ -236,7 +237,7 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                     }
 #pragma unroll
                     for (int n = 0; n < L / 64; ++n)   // g, v, k or q rows (N), columns (K)
-                        tma_load_3d(b + n * 8192, &tm_b2, k0, t0 + 64 * n, bh, &full[st]);
+                        tma_load_3d(b + n * 8192, &tm_b2, k0, t0 + 64 * n, KIND == 0 ? 2 * bh : bh, &full[st]);
                 }
             }
             // the last stages' copies have landed before the CTA may leave
@@ -310,7 +311,8 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                 float pv[16];
                 if (KIND == 3) {
                     epilogue_num(p, r1, r2, tokw, ddv, red + q4 * L, g, len, g0, col, scale, lane,
-                                 p.sg16 + ((size_t)2 * bh * p.S + t0) * p.DV);
+                                 p.sg16 + ((size_t)2 * bh * p.S + t0) * p.DV,
+                                 p.g16w + ((size_t)2 * bh * p.S + t0) * p.DV);
                     continue;
                 }
                 if (KIND < 2) {
@@ -382,7 +384,7 @@ static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUten
     using SM = Smem<L>;
     KParams p;
     p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV; p.NTK = a.NTK; p.NJT = a.NJT;
-    p.dh = a.dh; p.o = a.o; p.NRM = a.NRM; p.Gt = a.Gt; p.DOTP = a.DOTP; p.g16w = a.g16w; p.dog = a.dog;
+    p.dh = a.dh; p.o = a.o; p.NRM = a.NRM; p.DOTP = a.DOTP; p.g16w = a.g16w; p.dog = a.dog;
     p.sg16 = a.sg16;
     p.A = a.A; p.P = a.P; p.MC = a.MC; p.G = a.G; p.ig = a.ig; p.DD = a.DD; p.NS = a.NS; p.GN = a.GN;
     p.pq = KIND == 0 ? a.q : a.k;
@@ -402,7 +404,7 @@ static cudaError_t launch_l(const Args &a)
     CUtensorMap mq, mk, mv, mg, mds, ma, mc, mG;
     const int CL = a.NC * L;   // rows of the per-chunk score arrays (A and C_c: two parts each)
     if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&mk, a.k, a.DK, a.S, a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH) ||
-        !map3(&mg, a.g16, a.DV, a.S, a.BH) || !map3(&mds, a.dS16, L, CL, a.BH) || !map3(&ma, a.A16, L, 2 * CL, a.BH) ||
+        !map3(&mg, a.g16, a.DV, a.S, 2 * a.BH) || !map3(&mds, a.dS16, L, CL, a.BH) || !map3(&ma, a.A16, L, 2 * CL, a.BH) ||
         !map3(&mc, a.C16, a.DV, a.DK, 2 * a.BH * a.NC) || !map3(&mG, a.G16, a.DV, a.DK, a.BH * a.NC))
         return cudaErrorInvalidValue;
     cudaError_t e = launch_kind<0, L>(a, mk, mds, mc, mg);
@@ -782,6 +784,252 @@ cudaError_t launch_carry(const Args &a)
 {
     if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
     return a.L == 64 ? launch_carry_l<64>(a) : launch_carry_l<128>(a);
+}
+
+// ---------------------------------------------------------------- the chunk's scores and dS
+// One CTA per 128 consecutive tokens of a head (128 / L chunks): D = X Y^T over those tokens
+// (M = N = 128, both operands K-major), of which only the blocks of each chunk with itself (on
+// the diagonal) are used.  KIND 0: X = q, Y = k (bf16 inputs: the products are exact in the fp32
+// accumulator), K = DK; A = D * scale * exp(x_s - mx_t) on the causal triangle (two bf16 parts),
+// den_t = rowsum(A)_t + sc_t scale n_c . q_t and N_t.  KIND 1: X = g (two bf16 parts), Y = v,
+// K = DV; dden_t, dS = (D + dden_t) exp(x_s - mx_t) on the causal triangle (bf16) and
+// dn_c = sum_t sc_t dden_t scale q_t.  A TMEM lane is a token t (row), a column a token s.
+constexpr int XSTAGES = 4;
+struct ChunkSmem {
+    static constexpr uint32_t STAGE = 2 * 16384;              // X and Y: 128 rows x 64 each
+    static constexpr uint32_t F = XSTAGES * STAGE;            // floats: xs, mx, fl, sc, dd [128]; ns [2][512]
+    static constexpr uint32_t BAR = F + (5 * 128 + 2 * 512) * 4;
+    static constexpr uint32_t NBAR = 2 * XSTAGES + 1;
+    static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
+};
+
+template <int KIND, int L>
+__global__ void __launch_bounds__(THREADS, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y, Args a)
+{
+    using SM = ChunkSmem;
+    constexpr int NPART = KIND == 1 ? 2 : 1;
+    constexpr int CPB = 128 / L;                 // chunks per block
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float *xs = reinterpret_cast<float *>(smem + SM::F), *mx = xs + 128, *fl = mx + 128, *sc = fl + 128;
+    float *dd = sc + 128, *ns = dd + 128;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
+    uint64_t *full = bars, *empty = bars + XSTAGES, *accf = bars + 2 * XSTAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
+    uint32_t *abort_flag = tmem_slot + 1;
+    const int bh = blockIdx.x, tb = blockIdx.y * 128;   // first token of the block
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nkb = NPART * (KIND == 0 ? a.DK : a.DV) / 64;
+    WaitCtx wc{abort_flag, a.status};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < XSTAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_x);
+        tma_prefetch(&tm_y);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    griddep_wait();
+    griddep_launch_dependents();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int st = kb % XSTAGES;
+                if (kb >= XSTAGES && !mbar_wait(&empty[st], (uint32_t)((kb / XSTAGES) - 1) & 1u, wc)) break;
+                mbar_arrive_expect_tx(&full[st], SM::STAGE);
+                uint8_t *x = smem + st * SM::STAGE, *y = x + 16384;
+                const int per = nkb / NPART, part = kb / per, k0 = 64 * (kb % per);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {   // rows tb .. tb + 127 in two boxes of 64
+                    tma_load_3d(x + h * 8192, &tm_x, k0, tb + 64 * h, NPART * bh + part, &full[st]);
+                    tma_load_3d(y + h * 8192, &tm_y, k0, tb + 64 * h, bh, &full[st]);
+                }
+            }
+            for (int s = 0; s < XSTAGES && s < kb; ++s) {
+                const int last = kb - 1 - s;
+                mbar_wait_drain(&full[last % XSTAGES], (uint32_t)(last / XSTAGES) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t ID = idesc_bf16(128, 128, 0, 0);
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int st = kb % XSTAGES;
+                if (!mbar_wait(&full[st], (uint32_t)(kb / XSTAGES) & 1u, wc)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t x = smem_u32(smem + st * SM::STAGE), y = x + 16384;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem, smem_desc(x, 16, 1024) + (uint64_t)(kk * 2), smem_desc(y, 16, 1024) + (uint64_t)(kk * 2),
+                           ID, (kb > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&empty[st]);
+            }
+            if (ok) mma_commit(accf);
+        }
+    } else {
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;          // this thread's token row in the block (TMEM lane: a
+        const int r = row;                       // warp reaches its lane quadrant only)
+        const int t = tb + row;                  // token within the head
+        const int c = t / L, tl = t % L;         // its chunk and place in the chunk
+        const int cb = (row / L) * L;            // the chunk's first column in the block
+        const bool chunk_ok = c < a.NC;
+        const int len = chunk_ok ? min(L, a.S - c * L) : 0;
+        const bool ok_t = tl < len;
+        const size_t gt = (size_t)bh * a.S + t;
+        const float scale = rsqrtf((float)a.DK);
+        // per-token gate terms (forms in which the chunk-local cumulative log decay cancels)
+        {
+            const float mc = chunk_ok ? a.MC[(size_t)bh * (a.NC + 1) + c] : 0.f;
+            const float av = ok_t ? a.A[gt] : 0.f;
+            const float m = ok_t ? fmaxf(mc, a.P[gt]) : 0.f;
+            xs[r] = ok_t ? a.ig[gt] - av : -INFINITY;
+            mx[r] = m;
+            fl[r] = ok_t ? expf(-(av + m)) : 1.f;
+            sc[r] = ok_t ? expf(mc - m) : 0.f;
+        }
+        float ddv = 0.f;
+        if (KIND == 0) {   // n of the block's chunks
+            for (int e = r; e < CPB * a.DK; e += 128) {
+                const int cc = tb / L + e / a.DK;
+                ns[e] = cc < a.NC ? a.NS[((size_t)bh * a.NC + cc) * a.DK + e % a.DK] : 0.f;
+            }
+        } else if (ok_t) {   // dden_t
+            float dot = 0.f;
+            for (int u = 0; u < a.NJT; ++u) dot += a.DOTP[gt * a.NJT + u];
+            const float den = a.DENw[gt];   // (written by the scores kernel)
+            if (fabsf(den) > fl[r]) ddv = -dot * copysignf(1.f, den);
+            a.DDw[gt] = ddv;
+        }
+        dd[r] = ddv;
+        named_sync(1, 128);
+        bool failed = false;
+        if (r == 0) failed = !mbar_wait(accf, 0, wc);
+        failed = group_any(2, 128, failed);
+        if (!failed) {
+            tc_fence_after();
+            const float mxr = mx[r];
+            float rsum = 0.f;
+            // this row of the chunk's L x L block: A16 (two parts) or dS16 (one), zeros off the triangle
+            __nv_bfloat16 *dst = KIND == 0 ? a.A16w + ((size_t)bh * a.NC + c) * 2 * L * L + (size_t)tl * L
+                                           : a.dS16w + ((size_t)bh * a.NC + c) * L * L + (size_t)tl * L;
+#pragma unroll 1
+            for (int g = 0; g < L / 16; ++g) {
+                uint32_t rr[16];
+                tmem_ld16(tmem_addr(tmem, q4 * 32, cb + g * 16), rr);
+                tmem_wait_ld();
+                __nv_bfloat16 hi[16], lo[16];
+#pragma unroll
+                for (int z = 0; z < 16; ++z) {
+                    const int sl = g * 16 + z;
+                    float v = 0.f;
+                    if (sl <= tl && ok_t) {
+                        const float dcy = expf(xs[cb + sl] - mxr);
+                        v = KIND == 0 ? __uint_as_float(rr[z]) * scale * dcy : (__uint_as_float(rr[z]) + ddv) * dcy;
+                    }
+                    rsum += v;
+                    if (KIND == 0) bf16_parts(v, hi[z], lo[z]);
+                    else hi[z] = __float2bfloat16_rn(v);
+                }
+                if (chunk_ok) {
+                    *reinterpret_cast<uint4 *>(dst + g * 16) = *reinterpret_cast<const uint4 *>(hi);
+                    *reinterpret_cast<uint4 *>(dst + g * 16 + 8) = *reinterpret_cast<const uint4 *>(hi + 8);
+                    if (KIND == 0) {
+                        *reinterpret_cast<uint4 *>(dst + (size_t)L * L + g * 16) = *reinterpret_cast<const uint4 *>(lo);
+                        *reinterpret_cast<uint4 *>(dst + (size_t)L * L + g * 16 + 8) = *reinterpret_cast<const uint4 *>(lo + 8);
+                    }
+                }
+            }
+            if (KIND == 0 && ok_t) {   // den and N
+                const float *nc = ns + (row / L) * a.DK;
+                const __nv_bfloat16 *qr = a.q + gt * a.DK;
+                float qn = 0.f;
+                for (int d = 0; d < a.DK; d += 8) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(qr + d);
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) {
+                        qn = fmaf(nc[d + 2 * z], __uint_as_float(w4[z] << 16), qn);
+                        qn = fmaf(nc[d + 2 * z + 1], __uint_as_float(w4[z] & 0xffff0000u), qn);
+                    }
+                }
+                const float den = rsum + qn * scale * sc[r];
+                a.DENw[gt] = den;
+                a.NRMw[gt] = fmaxf(fabsf(den), fl[r]);
+            }
+        }
+        if (KIND == 1) {   // dn_c = sum_t sc_t dden_t scale q_t of each chunk of the block
+            named_sync(1, 128);
+            if (!failed) {
+                for (int cc = 0; cc < CPB; ++cc) {
+                    const int ch = tb / L + cc;
+                    if (ch >= a.NC) break;
+                    const int clen = min(L, a.S - ch * L);
+                    const __nv_bfloat16 *qb = a.q + ((size_t)bh * a.S + ch * L) * a.DK;
+                    for (int i = r; i < a.DK; i += 128) {
+                        float a2 = 0.f;
+                        for (int u = 0; u < clen; ++u)
+                            a2 = fmaf(sc[cc * L + u] * dd[cc * L + u], __bfloat162float(qb[(size_t)u * a.DK + i]) * scale, a2);
+                        a.GNw[((size_t)bh * a.NC + ch) * a.DK + i] = a2;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
+        const unsigned long long tq = global_timer();
+        while (global_timer() - tq < 100000ull) { }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+template <int KIND, int L>
+static cudaError_t launch_chunk_l(const Args &a)
+{
+    using SM = ChunkSmem;
+    CUtensorMap mx, my;
+    if (KIND == 0) {
+        if (!map3(&mx, a.q, a.DK, a.S, a.BH) || !map3(&my, a.k, a.DK, a.S, a.BH)) return cudaErrorInvalidValue;
+    } else {
+        if (!map3(&mx, a.g16, a.DV, a.S, 2 * a.BH) || !map3(&my, a.v, a.DV, a.S, a.BH)) return cudaErrorInvalidValue;
+    }
+    cudaError_t e = ensure_dynamic_smem((const void *)chunk_tc_kernel<KIND, L>, SM::TOTAL);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(chunk_tc_kernel<KIND, L>, dim3(a.BH, (a.S + 127) / 128), dim3(THREADS), SM::TOTAL, a.stream, 1,
+                         mx, my, a);
+}
+
+cudaError_t launch_scores(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_chunk_l<0, 64>(a) : launch_chunk_l<0, 128>(a);
+}
+
+cudaError_t launch_ds(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_chunk_l<1, 64>(a) : launch_chunk_l<1, 128>(a);
 }
 
 bool supported(int DK, int DV, int L)

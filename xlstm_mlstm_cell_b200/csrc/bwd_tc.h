@@ -17,19 +17,20 @@ struct Args {
     const float *DD;                        // gradient of the denominator [BH][S]
     const float *NS, *GN;                   // n at the chunk starts, gradient of n at the chunk ends [BH][NC][DK]
     const __nv_bfloat16 *q, *k, *v;         // inputs [BH][S][DK | DV]
-    // bf16 copies of the fp32 intermediates: chunk-start states C16 [BH][NC][2][DK][DV] and scores
-    // A16 [BH][NC][2][L][L] as two parts each (the bf16 value and the bf16 of its rounding
-    // residue: together about 16 significant bits), chunk-end state gradients G16 [BH][NC][DK][DV],
-    // the read-out numerator's gradient g16 [BH][S][DV] and dS16 [BH][NC][L][L]
+    // bf16 copies of the fp32 intermediates: chunk-start states C16 [BH][NC][2][DK][DV], scores
+    // A16 [BH][NC][2][L][L] and the read-out numerator's gradient g16 [BH][2][S][DV] as two parts
+    // each (the bf16 value and the bf16 of its rounding residue: together about 16 significant
+    // bits; products that need only the value read part 0), chunk-end state gradients G16
+    // [BH][NC][DK][DV] and dS16 [BH][NC][L][L]
     const __nv_bfloat16 *C16, *G16, *g16, *dS16, *A16;
     __nv_bfloat16 *dq, *dk, *dv;            // outputs [BH][S][DK | DV]
     float *QD, *KD;                         // partial q . dq and k . dk per 32 columns [BH][S][NTK]
     // the read-out numerator: dh, o (NULL without an output gate) [BH][S][DV], N = max(|den|,
-    // exp(-m)) [BH][S]; writes g (fp32 and its bf16 copy g16), do (when o is given) and the partial
+    // exp(-m)) [BH][S]; writes g (its two bf16 parts, g16w), do (when o is given) and the partial
     // row sums of g . hh per 64 value columns DOTP [BH][S][NJT]
     const __nv_bfloat16 *dh, *o;
     const float *NRM;
-    float *Gt, *DOTP;
+    float *DOTP;
     __nv_bfloat16 *g16w, *dog;
     int NJT;
     // sc_t g_t as two bf16 parts [BH][2][S][DV] (written by the numerator's epilogue, read by the
@@ -40,6 +41,10 @@ struct Args {
     // read), and its outputs, the chunk-start states as two bf16 parts (the array C16 above) and n
     __nv_bfloat16 *wk16, *C16w;
     float *NSw;
+    // the scores and dS (launch_scores, launch_ds): write DEN, NRM [BH][S] and A16 (two parts);
+    // DD [BH][S], dS16 and the read-out's dn_c GNw [BH][NC][DK]
+    float *DENw, *NRMw, *DDw, *GNw;
+    __nv_bfloat16 *A16w, *dS16w;
     uint32_t *status;
     cudaStream_t stream;
 };
@@ -52,6 +57,10 @@ cudaError_t launch(const Args &a);
 cudaError_t launch_num(const Args &a);
 // The read-out's state gradient of every chunk, dC_c = (sc qh)^T g (one launch).
 cudaError_t launch_dc(const Args &a);
+// The chunk's scores A = D * (qh K^T) (two bf16 parts), den and N (one launch).
+cudaError_t launch_scores(const Args &a);
+// dden, dS = (g V^T + dden) * D (bf16) and the read-out's dn_c (one launch; after the numerator).
+cudaError_t launch_ds(const Args &a);
 // The forward pass's chunk-start states C_c (as two bf16 parts) and n_c from the zero state: w_s k_s
 // as two bf16 parts, then a walk over the chunks per state tile with each chunk's contribution
 // sum_s (w_s k_s) v_s^T on tcgen05 and the fp32 state in registers (two launches).

@@ -91,10 +91,11 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->NS = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
     w->GS = reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
     w->GN = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
-    w->Gt = reinterpret_cast<float *>(take(f * BH * S * DHV));
+    // (the tensor-core path keeps g, dS and A only as bf16 parts or copies, below)
+    w->Gt = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * S * DHV));
     w->DD = reinterpret_cast<float *>(take(f * BH * S));
-    w->P2 = reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
-    w->AI = reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
+    w->P2 = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
+    w->AI = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
     w->QD = reinterpret_cast<float *>(take(f * BH * S * NTK));
     w->KD = reinterpret_cast<float *>(take(f * BH * S * NTK));
     w->DEN = reinterpret_cast<float *>(take(f * BH * S));
@@ -106,7 +107,7 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
         const size_t h = sizeof(__nv_bfloat16);
         w->CS16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * DHQK * DHV));   // two parts
         w->GS16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * DHQK * DHV));
-        w->Gt16 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * S * DHV));
+        w->Gt16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * S * DHV));             // two parts
         w->P216 = reinterpret_cast<__nv_bfloat16 *>(take(h * BH * NC * chunk * chunk));
         w->AI16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * NC * chunk * chunk));   // two parts
         w->SG16 = reinterpret_cast<__nv_bfloat16 *>(take(2 * h * BH * S * DHV));             // two parts
