@@ -296,7 +296,7 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
  * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head; on the
  * tensor-core path, where the chunk-start states, the scores and g are kept
- * as bf16 parts instead of fp32, 10 DHQK DHV + 8 DHQK + 6 chunk^2 + 12 bytes
+ * as bf16 parts instead of fp32, 6 DHQK DHV + 8 DHQK + 6 chunk^2 + 12 bytes
  * per chunk and head, plus 4 DHQK + 8 DHV + 8 ceil(DHQK / 32) +
  * 4 ceil(DHV / 64) + 20 bytes per token and head; each array 256-byte
  * aligned).  A bounded

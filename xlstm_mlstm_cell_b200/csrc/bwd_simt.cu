@@ -60,9 +60,6 @@ struct Params {
     float *DOTP;                     // partial row sums of g . hh per 64 value columns [BH][S][NJT]
     int NJT;                         // ceil(DV / 64)
     float *P2, *AI;                  // dS and A per chunk [BH][NC][L][L]
-    // bf16 copies of GS (after the scan), Gt and P2, and AI as two bf16 parts [BH][NC][2][L][L], for
-    // the tensor-core products, or NULL
-    __nv_bfloat16 *GS16, *Gt16, *P216, *AI16;
     float *QD, *KD;                  // per dk tile partial q . dq and k . dk [BH][S][NTK]
     void *dq, *dk, *dv, *dog;
     float *dig, *dfg;
@@ -169,8 +166,6 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
     const T *kb = static_cast<const T *>(p.k) + ((size_t)bh * p.S + t0) * DK;
     const float *nc = p.NS + ((size_t)bh * p.NC + c) * DK;
     float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
-    // the two bf16 parts of A (value and residue) for the tensor-core read-out
-    __nv_bfloat16 *AI16 = p.AI16 ? p.AI16 + ((size_t)bh * p.NC + c) * 2 * L * L : nullptr;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
     for (int t = tid; t < L; t += NT) rsum[t] = 0.f;
@@ -198,10 +193,7 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
                     const int s2 = nt * GM + 4 * tn + b2;
                     float av = 0.f;
                     if (s2 <= t && t < len) av = acc[a][b2] * expf(xs_[s2] - mx[t]);
-                    if (t < L && s2 < L) {
-                        AIg[(size_t)t * L + s2] = av;
-                        if (AI16) bf16_parts(av, AI16[(size_t)t * L + s2], AI16[(size_t)L * L + t * L + s2]);
-                    }
+                    if (t < L && s2 < L) AIg[(size_t)t * L + s2] = av;
                     part += av;
                 }
                 part = sum16(part);
@@ -211,10 +203,7 @@ __global__ void __launch_bounds__(NT) bwd_scores_kernel(Params p)
             if (nt < mt) {
                 for (int e = tid; e < GM * GM; e += NT) {
                     const int t = nt * GM + e / GM, s2 = mt * GM + e % GM;
-                    if (t < L && s2 < L) {
-                        AIg[(size_t)t * L + s2] = 0.f;
-                        if (AI16) bf16_parts(0.f, AI16[(size_t)t * L + s2], AI16[(size_t)L * L + t * L + s2]);
-                    }
+                    if (t < L && s2 < L) AIg[(size_t)t * L + s2] = 0.f;
                 }
             }
         }
@@ -254,7 +243,6 @@ __global__ void __launch_bounds__(NT) bwd_num_kernel(Params p)
     const T *dhb = static_cast<const T *>(p.dh) + ((size_t)bh * p.S + t0) * DV;
     T *dob = p.dog ? static_cast<T *>(p.dog) + ((size_t)bh * p.S + t0) * DV : nullptr;
     float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
-    __nv_bfloat16 *gt16 = p.Gt16 ? p.Gt16 + ((size_t)bh * p.S + t0) * DV : nullptr;
     const float *Cc = p.CS + ((size_t)bh * p.NC + c) * DK * DV;
     const float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
     const float *nrm = p.NRM + (size_t)bh * p.S + t0;
@@ -305,7 +293,6 @@ __global__ void __launch_bounds__(NT) bwd_num_kernel(Params p)
                         if (dob) dob[off] = from_f32<T>(dhv * hh);
                         const float g = ov * dhv / N;
                         gtb[off] = g;
-                        if (gt16) gt16[off] = __float2bfloat16_rn(g);
                         part = fmaf(g, hh, part);
                     }
                 }
@@ -336,7 +323,6 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
     const T *vb = static_cast<const T *>(p.v) + ((size_t)bh * p.S + t0) * DV;
     const float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
     float *P2g = p.P2 + ((size_t)bh * p.NC + c) * L * L;
-    __nv_bfloat16 *P216 = p.P216 ? p.P216 + ((size_t)bh * p.NC + c) * L * L : nullptr;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
     for (int t = tid; t < L; t += NT) {
@@ -357,10 +343,7 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
             if (nt > mt) {   // above the diagonal: zeros
                 for (int e = tid; e < GM * GM; e += NT) {
                     const int t = mt * GM + e / GM, s2 = nt * GM + e % GM;
-                    if (t < L && s2 < L) {
-                        P2g[(size_t)t * L + s2] = 0.f;
-                        if (P216) P216[(size_t)t * L + s2] = __float2bfloat16_rn(0.f);
-                    }
+                    if (t < L && s2 < L) P2g[(size_t)t * L + s2] = 0.f;
                 }
                 continue;
             }
@@ -385,10 +368,7 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
                     const int s2 = nt * GM + 4 * tn + b2;
                     float pv = 0.f;
                     if (s2 <= t && t < len) pv = (acc[a][b2] + dd[t]) * expf(xs_[s2] - mx[t]);
-                    if (t < L && s2 < L) {
-                        P2g[(size_t)t * L + s2] = pv;
-                        if (P216) P216[(size_t)t * L + s2] = __float2bfloat16_rn(pv);
-                    }
+                    if (t < L && s2 < L) P2g[(size_t)t * L + s2] = pv;
                 }
             }
         }
@@ -481,11 +461,7 @@ __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
                 for (int u = 0; u < BATCH; ++u) {
                     const int c = c1 - 1 - u;
                     if (c >= cb) {
-                        if (p.GS16)   // only the bf16 copy of the chunk-end gradient: all its readers take that
-                            reinterpret_cast<uint2 *>(p.GS16 + (size_t)bh * p.NC * nstate)[(size_t)c * nq + e] =
-                                make_uint2(bf16x2_bits(G.x, G.y), bf16x2_bits(G.z, G.w));
-                        else
-                            slot[(size_t)c * nq] = G;
+                        slot[(size_t)c * nq] = G;
                         const float f = decay[c - cb];
                         G = make_float4(d[u].x + f * G.x, d[u].y + f * G.y, d[u].z + f * G.z, d[u].w + f * G.w);
                     }
@@ -698,10 +674,13 @@ cudaError_t launch_t(const Params &p, int BH, cudaStream_t st, const bwdtc::Args
     if (e != cudaSuccess) return e;
     e = tc ? bwdtc::launch_ds(*tc) : launch_kernel(bwd_ds_kernel<T>, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     if (e != cudaSuccess) return e;
-    e = tc ? bwdtc::launch_dc(*tc)
-           : launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
-    if (e != cudaSuccess) return e;
-    e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV / 4 + 255) / 256, BH), dim3(256), 0, st, 1, p);
+    if (tc) {   // the read-out's state gradients and their reverse scan in one walk
+        e = bwdtc::launch_gstate(*tc);
+    } else {
+        e = launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
+        if (e != cudaSuccess) return e;
+        e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV / 4 + 255) / 256, BH), dim3(256), 0, st, 1, p);
+    }
     if (e != cudaSuccess) return e;
     if (tc) {   // dq, dk, dv on the tensor cores
         if ((e = bwdtc::launch(*tc)) != cudaSuccess) return e;
@@ -725,7 +704,6 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     p.GS = w.GS; p.GN = w.GN; p.Gt = w.Gt; p.DD = w.DD; p.P2 = w.P2; p.AI = w.AI; p.QD = w.QD; p.KD = w.KD;
     p.DEN = w.DEN; p.NRM = w.NRM; p.DOTP = w.DOTP; p.NJT = (a.DHV + 63) / 64;
     p.dq = a.dq; p.dk = a.dk; p.dv = a.dv; p.dog = a.ogate ? a.dogate : nullptr; p.dig = a.digate; p.dfg = a.dfgate;
-    p.GS16 = w.GS16; p.Gt16 = w.Gt16; p.P216 = w.P216; p.AI16 = w.AI16;
     if (!a.bf16) return bwd::launch_t<float>(p, a.BH, a.stream, nullptr);
     if (!w.tc) return bwd::launch_t<__nv_bfloat16>(p, a.BH, a.stream, nullptr);
     using bf = __nv_bfloat16;
@@ -738,7 +716,7 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     t.QD = w.QD; t.KD = w.KD; t.status = w.status; t.stream = a.stream;
     t.dh = static_cast<const bf *>(a.dh); t.o = static_cast<const bf *>(a.ogate); t.NRM = w.NRM;
     t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
-    t.NJT = p.NJT; t.sg16 = w.SG16; t.GS = w.GS;
+    t.NJT = p.NJT; t.sg16 = w.SG16; t.G16w = w.GS16;
     t.wk16 = w.WK16; t.C16w = w.CS16; t.NSw = w.NS;
     t.DENw = w.DEN; t.NRMw = w.NRM; t.DDw = w.DD; t.GNw = w.GN; t.A16w = w.AI16; t.dS16w = w.P216;
     cudaError_t e = bwdtc::launch_carry(t);   // the chunk-start states

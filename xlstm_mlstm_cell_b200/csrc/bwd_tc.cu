@@ -429,136 +429,6 @@ cudaError_t launch_num(const Args &a)
     return a.L == 64 ? launch_num_l<64>(a) : launch_num_l<128>(a);
 }
 
-// ---------------------------------------------------------------- the read-out's state gradient
-// dC_c[d][j] = scale sum_t q_t[d] (sc_t g_t[j]) over the chunk's tokens, one 128 x 128 state tile
-// per CTA: A = q [t][d] (MN-major), B = sc g [t][j] as two bf16 parts (MN-major), K = L tokens per
-// part, one TMEM accumulator of 128 columns, the tile written to dC in fp32.
-template <int L>
-struct DcSmem {
-    static constexpr int NB = 2 * (L / 64);                   // stages: 64 tokens of one part
-    static constexpr uint32_t STAGE = 2 * 8192 + 2 * 8192;    // q: 64 x 128, sc g: 64 x 128
-    static constexpr uint32_t BAR = NB * STAGE;
-    static constexpr uint32_t TOTAL = BAR + (NB + 1) * 8 + 16 + 1024;
-};
-
-template <int L>
-__global__ void __launch_bounds__(THREADS, 1)
-dc_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sg, KParams p,
-             float *__restrict__ GS)
-{
-    using SM = DcSmem<L>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::BAR), *accf = full + SM::NB;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
-    uint32_t *abort_flag = tmem_slot + 1;
-    const int bh = blockIdx.x, c = blockIdx.y;
-    const int ntj = p.DV / 128, i0 = (blockIdx.z / ntj) * 128, j0 = (blockIdx.z % ntj) * 128;
-    const int t0 = c * L;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WaitCtx wc{abort_flag, p.status};
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s <= SM::NB; ++s) mbar_init(&full[s], 1);   // (full[NB] is accf)
-        *abort_flag = 0u;
-        fence_barrier_init();
-        tma_prefetch(&tm_q);
-        tma_prefetch(&tm_sg);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 128);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    griddep_wait();
-    griddep_launch_dependents();
-
-    if (warp == 0) {
-        if (lane == 0) {   // every stage has its own buffer: all loads at once
-            for (int kb = 0; kb < SM::NB; ++kb) {
-                const int part = kb / (L / 64), k0 = 64 * (kb % (L / 64));
-                uint8_t *a = smem + kb * SM::STAGE, *b = a + 16384;
-                mbar_arrive_expect_tx(&full[kb], SM::STAGE);
-                for (int mb = 0; mb < 2; ++mb) tma_load_3d(a + mb * 8192, &tm_q, i0 + 64 * mb, t0 + k0, bh, &full[kb]);
-                for (int nb = 0; nb < 2; ++nb)
-                    tma_load_3d(b + nb * 8192, &tm_sg, j0 + 64 * nb, t0 + k0, 2 * bh + part, &full[kb]);
-            }
-            for (int kb = 0; kb < SM::NB; ++kb) mbar_wait_drain(&full[kb], 0);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t ID = idesc_bf16(128, 128, 1, 1);
-            bool ok = true;
-            for (int kb = 0; kb < SM::NB && ok; ++kb) {
-                if (!mbar_wait(&full[kb], 0, wc)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t a = smem_u32(smem + kb * SM::STAGE), b = a + 16384;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tmem, smem_desc(a + kk * 2048, 8192, 1024), smem_desc(b + kk * 2048, 8192, 1024), ID,
-                           (kb > 0 || kk > 0) ? 1u : 0u);
-            }
-            if (ok) mma_commit(accf);
-        }
-    } else {
-        const int et = threadIdx.x - 64, q4 = warp & 3;
-        const int i = i0 + q4 * 32 + lane;   // this thread's state row
-        bool failed = false;
-        if (et == 0) failed = !mbar_wait(accf, 0, wc);
-        failed = group_any(2, 128, failed);
-        if (!failed) {
-            tc_fence_after();
-            const float scale = rsqrtf((float)p.DK);
-            float *row = GS + (((size_t)bh * p.NC + c) * p.DK + i) * p.DV + j0;
-#pragma unroll 1
-            for (int g = 0; g < 128 / 16; ++g) {
-                uint32_t r[16];
-                tmem_ld16(tmem_addr(tmem, q4 * 32, g * 16), r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 16; u += 4)
-                    *reinterpret_cast<float4 *>(row + g * 16 + u) =
-                        make_float4(scale * __uint_as_float(r[u]), scale * __uint_as_float(r[u + 1]),
-                                    scale * __uint_as_float(r[u + 2]), scale * __uint_as_float(r[u + 3]));
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
-        const unsigned long long tb = global_timer();
-        while (global_timer() - tb < 100000ull) { }
-    }
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 128);
-    }
-}
-
-template <int L>
-static cudaError_t launch_dc_l(const Args &a)
-{
-    using SM = DcSmem<L>;
-    CUtensorMap mq, msg;
-    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&msg, a.sg16, a.DV, a.S, 2 * a.BH)) return cudaErrorInvalidValue;
-    KParams p{};
-    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
-    p.status = a.status;
-    cudaError_t e = ensure_dynamic_smem((const void *)dc_tc_kernel<L>, SM::TOTAL);
-    if (e != cudaSuccess) return e;
-    return launch_kernel(dc_tc_kernel<L>, dim3(a.BH, a.NC, (a.DK / 128) * (a.DV / 128)), dim3(THREADS), SM::TOTAL,
-                         a.stream, 1, mq, msg, p, a.GS);
-}
-
-cudaError_t launch_dc(const Args &a)
-{
-    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
-    return a.L == 64 ? launch_dc_l<64>(a) : launch_dc_l<128>(a);
-}
-
 // ---------------------------------------------------------------- the forward carry
 // w_s k_s[d] as two bf16 parts, w_s = exp(g_c - a_s + i~_s - m_{c+1}) (c the chunk of token s): the
 // weight of token s in the state at its chunk's end, in that state's stabilized frame (<= 1).
@@ -710,7 +580,15 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
 #pragma unroll
         for (int x = 0; x < 64; ++x) C[x] = 0.f;
         float n = 0.f;
+        // the chunk's decay terms, loaded one chunk ahead (off the chain of chunk steps)
+        float g_c = Gb[0], mc_c = MCb[0], mn_c = MCb[p.NC > 1 ? 1 : 0];
         for (int c = 0; c < p.NC; ++c) {
+            const float decay = expf(g_c + mc_c - mn_c);
+            if (c + 2 <= p.NC - 1) {
+                g_c = Gb[c + 1];
+                mc_c = mn_c;
+                mn_c = MCb[c + 2];
+            }
             // the state at the chunk's start: its two bf16 parts, and n
             __nv_bfloat16 *dst = C16 + (((size_t)bh * p.NC + c) * 2 * p.DK + d) * p.DV + j0;
 #pragma unroll
@@ -723,7 +601,6 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
             }
             if (with_n) NSo[((size_t)bh * p.NC + c) * p.DK + d] = n;
             if (c == p.NC - 1) break;   // (the final state is not needed)
-            const float decay = expf(Gb[c] + MCb[c] - MCb[c + 1]);
             const int ub = c & 1;
             bool failed = false;
             if (lane == 0) failed = !mbar_wait(&ufull[ub], (uint32_t)(c >> 1) & 1u, wc);
@@ -758,6 +635,189 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
+}
+
+// The reverse walk of the state gradients over the chunks of one 128 x 64 tile (rows d, columns j):
+// per chunk the read-out's dC_c = scale sum_t q_t (sc_t g_t)^T as MMAs (A = q, MN-major; B = sc g,
+// two parts, MN-major) into one of two TMEM buffers, while the epilogue warps, which hold the fp32
+// gradient in registers, write the gradient of the state at the chunk's end (bf16) and then
+// G <- dC_c + exp(g_c + m_c - m_{c+1}) G; the tiles of columns 0..63 run the normalizer's gradient
+// through GN the same way, in place (dn_c in, the chunk-end gradient out).
+template <int L>
+__global__ void __launch_bounds__(THREADS, 1)
+gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sg, KParams p,
+                 __nv_bfloat16 *__restrict__ G16, float *__restrict__ GN)
+{
+    using SM = CarrySmem;   // (a stage: q 64 tokens x 128 rows, then sc g 2 parts x 64 tokens x 64)
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
+    uint64_t *full = bars, *empty = bars + CSTAGES, *ufull = bars + 2 * CSTAGES, *ufree = ufull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
+    uint32_t *abort_flag = tmem_slot + 1;
+    const int bh = blockIdx.x, d0 = blockIdx.y * 128, j0 = blockIdx.z * 64;
+    const bool with_n = blockIdx.z == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int KB = L / 64;
+    const int nblk = (p.NC - 1) * KB;          // chunks NC - 1 .. 1 (the gradient of the start state is not needed)
+    WaitCtx wc{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < CSTAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ufull[b], 1);
+            mbar_init(&ufree[b], 4);
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch(&tm_q);
+        tma_prefetch(&tm_sg);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;   // dC buffers at columns 0 and 64
+    griddep_wait();
+    griddep_launch_dependents();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int kb = 0;
+            for (; kb < nblk; ++kb) {
+                const int st = kb % CSTAGES;
+                if (kb >= CSTAGES && !mbar_wait(&empty[st], (uint32_t)((kb / CSTAGES) - 1) & 1u, wc)) break;
+                mbar_arrive_expect_tx(&full[st], 2 * 16384);
+                uint8_t *a = smem + st * SM::STAGE, *b = a + 16384;
+                const int c = p.NC - 1 - kb / KB, t = c * L + 64 * (kb % KB);
+#pragma unroll
+                for (int mb = 0; mb < 2; ++mb) tma_load_3d(a + mb * 8192, &tm_q, d0 + 64 * mb, t, bh, &full[st]);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) tma_load_3d(b + part * 8192, &tm_sg, j0, t, 2 * bh + part, &full[st]);
+            }
+            for (int s = 0; s < CSTAGES && s < kb; ++s) {
+                const int last = kb - 1 - s;
+                mbar_wait_drain(&full[last % CSTAGES], (uint32_t)(last / CSTAGES) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t IDU = idesc_bf16(128, 64, 1, 1);
+            bool ok = true;
+            for (int i = 0; i < p.NC - 1 && ok; ++i) {   // i-th chunk from the end
+                const int ub = i & 1;
+                if (i >= 2 && !mbar_wait(&ufree[ub], (uint32_t)((i >> 1) - 1) & 1u, wc)) { ok = false; break; }
+                for (int q = 0; q < KB; ++q) {
+                    const int kb = i * KB + q, st = kb % CSTAGES;
+                    if (!mbar_wait(&full[st], (uint32_t)(kb / CSTAGES) & 1u, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(smem + st * SM::STAGE), b = a + 16384;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem + ub * 64, smem_desc(a + kk * 2048, 8192, 1024),
+                                   smem_desc(b + part * 8192 + kk * 2048, 8192, 1024), IDU,
+                                   (q > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&empty[st]);
+                }
+                if (ok) mma_commit(&ufull[ub]);
+            }
+        }
+    } else {
+        const int q4 = warp & 3;
+        const int d = d0 + q4 * 32 + lane;   // this thread's state row
+        const float *MCb = p.MC + (size_t)bh * (p.NC + 1);
+        const float *Gb = p.G + (size_t)bh * p.NC;
+        const float scale = rsqrtf((float)p.DK);
+        float Gs[64];
+#pragma unroll
+        for (int x = 0; x < 64; ++x) Gs[x] = 0.f;
+        float gn = 0.f;
+        int c = p.NC - 1;
+        float g_c = Gb[c], mc_c = MCb[c], mn_c = MCb[c + 1];
+        for (int i = 0; i < p.NC; ++i, --c) {
+            const float decay = expf(g_c + mc_c - mn_c);
+            if (c >= 1) {   // the next chunk's terms, one step ahead
+                mn_c = mc_c;
+                g_c = Gb[c - 1];
+                mc_c = MCb[c - 1];
+            }
+            // the gradient of the state at this chunk's end
+            __nv_bfloat16 *dst = G16 + (((size_t)bh * p.NC + c) * p.DK + d) * p.DV + j0;
+#pragma unroll
+            for (int x = 0; x < 64; x += 8) {
+                uint4 w;
+                w.x = bf16x2_bits(Gs[x], Gs[x + 1]);
+                w.y = bf16x2_bits(Gs[x + 2], Gs[x + 3]);
+                w.z = bf16x2_bits(Gs[x + 4], Gs[x + 5]);
+                w.w = bf16x2_bits(Gs[x + 6], Gs[x + 7]);
+                *reinterpret_cast<uint4 *>(dst + x) = w;
+            }
+            float dn = 0.f;
+            if (with_n) {
+                float *slot = GN + ((size_t)bh * p.NC + c) * p.DK + d;
+                dn = *slot;
+                *slot = gn;
+            }
+            if (c == 0) break;   // (the gradient of the start state is not needed)
+            if (with_n) gn = fmaf(decay, gn, dn);
+            const int ub = i & 1;
+            bool failed = false;
+            if (lane == 0) failed = !mbar_wait(&ufull[ub], (uint32_t)(i >> 1) & 1u, wc);
+            if (__shfl_sync(0xffffffffu, failed ? 1 : 0, 0)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint32_t r[16];
+                tmem_ld16(tmem_addr(tmem, q4 * 32, ub * 64 + g * 16), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int z = 0; z < 16; ++z) Gs[g * 16 + z] = fmaf(decay, Gs[g * 16 + z], scale * __uint_as_float(r[z]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ufree[ub]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*reinterpret_cast<volatile uint32_t *>(abort_flag)) {
+        const unsigned long long tb = global_timer();
+        while (global_timer() - tb < 100000ull) { }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+template <int L>
+static cudaError_t launch_gstate_l(const Args &a)
+{
+    using SM = CarrySmem;
+    CUtensorMap mq, msg;
+    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&msg, a.sg16, a.DV, a.S, 2 * a.BH)) return cudaErrorInvalidValue;
+    KParams p{};
+    p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
+    p.MC = a.MC; p.G = a.G;
+    p.status = a.status;
+    cudaError_t e = ensure_dynamic_smem((const void *)gstate_tc_kernel<L>, SM::TOTAL);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(gstate_tc_kernel<L>, dim3(a.BH, a.DK / 128, a.DV / 64), dim3(THREADS), SM::TOTAL, a.stream, 1,
+                         mq, msg, p, a.G16w, a.GNw);
+}
+
+cudaError_t launch_gstate(const Args &a)
+{
+    if (!supported(a.DK, a.DV, a.L)) return cudaErrorInvalidValue;
+    return a.L == 64 ? launch_gstate_l<64>(a) : launch_gstate_l<128>(a);
 }
 
 template <int L>

@@ -34,9 +34,8 @@ struct Args {
     __nv_bfloat16 *g16w, *dog;
     int NJT;
     // sc_t g_t as two bf16 parts [BH][2][S][DV] (written by the numerator's epilogue, read by the
-    // read-out's state gradient), and that gradient dC_c = scale (sc Q)^T g, fp32 [BH][NC][DK][DV]
-    __nv_bfloat16 *sg16;
-    float *GS;
+    // state-gradient walk), and that walk's output, the chunk-end state gradients (the array G16)
+    __nv_bfloat16 *sg16, *G16w;
     // the forward carry (launch_carry): w_s k_s as two bf16 parts [BH][2][S][DK] (written, then
     // read), and its outputs, the chunk-start states as two bf16 parts (the array C16 above) and n
     __nv_bfloat16 *wk16, *C16w;
@@ -55,8 +54,10 @@ bool supported(int DK, int DV, int L);
 cudaError_t launch(const Args &a);
 // The read-out numerator of every chunk, num = sc qh C_c + A V, and what follows from it (one launch).
 cudaError_t launch_num(const Args &a);
-// The read-out's state gradient of every chunk, dC_c = (sc qh)^T g (one launch).
-cudaError_t launch_dc(const Args &a);
+// The state gradients at the chunk ends, G_end (bf16), from the read-out's dC_c = (sc qh)^T g of every
+// chunk, and the normalizer's in GN (in place: dn_c in, the chunk-end gradient out), by a reverse walk
+// over the chunks per state tile with dC_c on tcgen05 (one launch).
+cudaError_t launch_gstate(const Args &a);
 // The chunk's scores A = D * (qh K^T) (two bf16 parts), den and N (one launch).
 cudaError_t launch_scores(const Args &a);
 // dden, dS = (g V^T + dden) * D (bf16) and the read-out's dn_c (one launch; after the numerator).

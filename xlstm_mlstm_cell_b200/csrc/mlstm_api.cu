@@ -89,7 +89,7 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     // (the tensor-core path keeps the chunk-start states only as their bf16 parts, below)
     w->CS = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
     w->NS = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
-    w->GS = reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
+    w->GS = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * NC * DHQK * DHV));
     w->GN = reinterpret_cast<float *>(take(f * BH * NC * DHQK));
     // (the tensor-core path keeps g, dS and A only as bf16 parts or copies, below)
     w->Gt = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * S * DHV));

@@ -82,9 +82,10 @@ struct BwdWorkspace {
     float *QD, *KD;               // [BH][S][ceil(DHQK / 32)] partial q . dq, k . dk
     float *DEN, *NRM;             // [BH][S] read-out denominator and its floored magnitude
     float *DOTP;                  // [BH][S][ceil(DHV / 64)] partial row sums of g . hh
-    // the tensor-core path (bf16 inputs, bwd_tc_path; there CS, Gt, P2 and AI are NULL): bf16 copies
-    // of GS and P2 in the same layouts, and of CS, AI ([BH][NC][2][...]) and Gt ([BH][2][S][DHV]) as
-    // two parts each (value and rounding residue); NULL on the CUDA-core path
+    // the tensor-core path (bf16 inputs, bwd_tc_path; there CS, GS, Gt, P2 and AI are NULL): the
+    // chunk-end state gradients and dS as bf16 (layouts of GS, P2), the chunk-start states, the
+    // scores ([BH][NC][2][...]) and g ([BH][2][S][DHV]) as two bf16 parts each (value and rounding
+    // residue); NULL on the CUDA-core path
     bool tc;
     __nv_bfloat16 *CS16, *GS16, *Gt16, *P216, *AI16;
     __nv_bfloat16 *SG16;          // sc_t g_t as two bf16 parts [BH][2][S][DHV]
