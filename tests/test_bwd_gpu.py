@@ -118,6 +118,26 @@ def test_bwd_every_chunk_size(cuda_lib, dt, DHQK, DHV, chunk):
     check(inputs, make_dh(1, 2, 300, DHV, dt, seed=4), chunk, BWD_TOL[dt])
 
 
+# Shapes of the tensor-core path (bf16, chunk 64 or 128, head sizes multiples of 128) at its edges:
+# one token; one whole chunk; a last chunk of one token; three key or value tiles (384); the
+# largest head sizes; several sequences.
+TC_EDGE = [
+    # B, NH, S, DHQK, DHV, chunk
+    (1, 1, 1, 128, 128, 64),
+    (1, 2, 64, 256, 384, 64),
+    (3, 1, 129, 384, 128, 128),
+    (1, 1, 520, 512, 512, 128),
+    (2, 2, 200, 128, 256, 64),
+]
+
+
+@pytest.mark.parametrize("B,NH,S,DHQK,DHV,chunk", TC_EDGE)
+def test_bwd_tensor_core_edge_shapes(cuda_lib, B, NH, S, DHQK, DHV, chunk):
+    assert binding.bwd_tensor_path(DHQK, DHV, chunk, torch.bfloat16) == 1
+    inputs = make_custom(B, NH, S, DHQK, DHV, "bf16", seed=11, ig=(-1.0, 2.0), fg=(3.0, 1.5))
+    check(inputs, make_dh(B, NH, S, DHV, "bf16", seed=12), chunk, BWD_TOL["bf16"])
+
+
 def test_bwd_full_workload_7b(cuda_lib):
     """The 7B-shaped prefill (B1 NH8 S8192 d256/512, chunk 64) at full size: every gradient of every
     head, whole-tensor rel-L2 (the oracle takes the heads in groups, a thread per head)."""
