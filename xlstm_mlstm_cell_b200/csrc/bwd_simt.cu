@@ -726,9 +726,11 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
 
 bool bwd_tc_path(bool bf16, int BH, int S, int DHQK, int DHV, int chunk)
 {
-    // (the per-chunk state arrays are addressed as BH NC boxes of one tensor map dimension)
+    // (tensor-map extents are 32-bit: the chunk-start states' two parts span 2 BH NC boxes, the
+    // scores' two parts 2 NC chunk rows; the grids take NC chunks in y)
     const long long NC = (S + (long long)chunk - 1) / chunk;
-    return bf16 && bwdtc::supported(DHQK, DHV, chunk) && (long long)BH * NC < (1LL << 31) && NC <= 65535;
+    return bf16 && bwdtc::supported(DHQK, DHV, chunk) && 2LL * BH * NC < (1LL << 31) &&
+           2LL * NC * chunk < (1LL << 31) && NC <= 65535;
 }
 
 }  // namespace mlstm
