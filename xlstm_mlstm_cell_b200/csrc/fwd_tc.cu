@@ -44,7 +44,9 @@
 //    X = Cbar exp(-rho) (Cbar the unstabilized state), the chunk decay is folded
 //    into rho instead of rescaling TMEM, and new tokens enter with weight
 //    W_s = exp(i~_s - a_s - rho) <= exp(THRESH).  TMEM is rescaled only when that
-//    bound would be exceeded.  Cb is always the stabilized C_c = X exp(rho - m_c).
+//    bound would be exceeded, between the chunk's read-out and its state update, so
+//    that the read-out always sees the chunk's starting frame (rho >= m_c - THRESH).
+//    Cb is always the stabilized C_c = X exp(rho - m_c).
 #include "common.cuh"
 #include "mlstm_internal.h"
 #include "tc_common.cuh"
@@ -734,8 +736,9 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float rho_new = rescale ? (mn - g) : rho;
             const float alpha = expf(rho - mc);
             const float beta = expf(rho - rho_new);
-            // scale of the TMEM state (after this chunk's rescale) as the tf32 inter product reads it
-            const float ahc = SM::TF ? expf(rho_new - mc) : 1.f;
+            // scale of the TMEM state as the tf32 inter product reads it: the chunk's starting frame rho
+            // (the frame moves only after that product, see the K pass)
+            const float ahc = SM::TF ? alpha : 1.f;
 
             if (p.o) {   // bring this thread's output-gate rows of the epilogue into L2 early
 #pragma unroll
@@ -786,29 +789,17 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
 
             // (b) Cb = fp16(C_c 2^-kc) into TMEM, kc from max |C_c| over the tile; rescale the
-            //     fp32 state when the frame moves
+            //     fp32 state when the frame moves (at chunk 64 the state is read in place, and the
+            //     frame moves in the K pass)
             if (ct == 0) WALK_TRACE(11);
             // the previous chunk's state update must be complete before the state is read or
-            // rescaled here; at chunk 64 without a rescale nothing here touches it (the inter-chunk
-            // MMA is ordered after the update in the MMA pipe, and Q', P are free since h_full)
-            if (i > 0 && (!SM::TF || rescale) && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
+            // rescaled here; at chunk 64 nothing here touches it (the inter-chunk MMA is ordered
+            // after the update in the MMA pipe, and Q', P are free since h_full)
+            if (i > 0 && !SM::TF && !mbar_wait(c_upd, ph ^ 1u, wc)) { ok = false; break; }
             if (ct == 0) WALK_TRACE(12);
             tc_fence_after();
             int kc = 0;
-            if constexpr (SM::TF) {   // tf32 inter product: only the frame move touches the state here
-                if (rescale) {
-#pragma unroll
-                    for (int uc = 0; uc < CQ / 16; ++uc) {
-                        const int c0 = hq * CQ + uc * 16;
-                        uint32_t r[16];
-                        tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
-                        tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
-                    }
-                    tmem_wait_st();
-                }
+            if constexpr (SM::TF) {
                 named_sync(1, 512);                   // the per-row arrays are complete
             } else {
             float cmax = 0.f;
@@ -1011,6 +1002,31 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             //     K' = W k in bf16 in place, the operand of the state update.  A warp owns CPW 16-byte
             //     chunks of every row (lane = row), so that its n sums reduce inside the warp and go
             //     straight into nX
+            // The frame move of the tf32 path, per warp on its part of the state before its K' arrival:
+            // the output MMA reads the state in the chunk's starting frame, so the state is rescaled
+            // only once that MMA has completed, and before the update adds the chunk's tokens in the new
+            // frame.  (One fp32 frame cannot serve both ends of a chunk whose log decay is in the
+            // hundreds: exp(rho_new - m_c) overflows while exp(rho - rho_new) underflows.)
+            auto move_frame = [&]() {
+                if constexpr (SM::TF) {
+                    uint32_t done = 1u;
+                    if (lane == 0) done = mbar_wait(h_full, ph, wc) ? 1u : 0u;
+                    if (!__shfl_sync(0xffffffffu, done, 0)) return;   // aborted: (g) leaves the loop
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int uc = 0; uc < CQ / 16; ++uc) {
+                        const int c0 = hq * CQ + uc * 16;
+                        uint32_t r[16];
+                        tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
+                        tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                }
+            };
             if (!last) {
                 constexpr int NCH = DK / 8;                   // chunks per row
                 constexpr int CPW = NCH >= 16 ? NCH / 16 : 1; // chunks per warp
@@ -1053,6 +1069,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                     fence_proxy_async();
                     __syncwarp();
+                    if (beta < 1.f) move_frame();            // (beta < exp(-THRESH) exactly when the frame moves)
                     if (lane == 0) mbar_arrive(kready);      // K' is ready: the state update can start
                     // transposed reduction over the 32 lanes: each exchange halves the values a lane
                     // holds, so that lane l ends with the sum of value l / (32 / NV)
@@ -1081,6 +1098,7 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                 } else {
                     __syncwarp();
+                    if (beta < 1.f) move_frame();
                     if (lane == 0) mbar_arrive(kready);
                 }
             }

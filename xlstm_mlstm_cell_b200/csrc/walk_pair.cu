@@ -327,7 +327,7 @@ walk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool run = nck > 0 && issue_s(0);
             for (int i = 0; i < nck && run; ++i) {
                 const uint32_t ph = (uint32_t)i & 1u;
-                // both CTAs: Q' and a frame move of the state are ready, the previous outputs are read
+                // both CTAs: Q' is ready, the previous outputs are read
                 if (!mbar_wait(&bars[B_EPQ], ph, wc)) break;
                 if (i > 0 && !mbar_wait(&bars[B_HSFREE], ph ^ 1u, wc)) break;
                 PAIR_TRACE(3, i);
@@ -463,7 +463,7 @@ walk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             alpha = expf(rho - mc);
             beta = expf(rho - rho_new);
             rho_next = rho_new + g;
-            const float ahc = expf(rho_new - mc);   // scale of the TMEM state as the tf32 product reads it
+            const float ahc = alpha;   // scale of the TMEM state as the tf32 product reads it (frame rho)
             if (ct < L) {
                 if (ct < len) {
                     const float mt = ca + fmaxf(mc, cm);
@@ -512,22 +512,6 @@ walk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (!last) mbar_arrive_expect_tx(&bars[B_NREADY0 + ((i + 1) & 1)], (DK / 2) * 4);
                 mbar_arrive_expect_tx(&bars[B_INVREADY0 + b], HL * 4);
             }
-            // (a) a frame move rescales this CTA's state after the previous update
-            if (rescale) {
-                if (i > 0 && !group_wait(&bars[B_CUPD], ph ^ 1u, wc, ct == 0, true, 1, GA)) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int c0 = hq * (DK / 4); c0 < (hq + 1) * (DK / 4); c0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
-                    tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
-                }
-                tmem_wait_st();
-            }
-
             // (b) S of this chunk is done (so q has landed) and the other CTA's half of n has arrived;
             //     the previous chunk's h store has read the upper half of the Q' buffer.  The group's
             //     barrier also orders the gate arrays written at the end of the previous chunk.
@@ -579,11 +563,11 @@ walk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int u = CPT / 2; u < CPT; ++u) put(u);
             }
             fence_proxy_async();
-            tc_fence_before();   // (the frame move's TMEM stores)
+            tc_fence_before();   // (the segment's start state in TMEM)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bars[B_QEMPTY]);   // this warp has read q
-                mbar_arrive(&bars[B_EPQ]);      // this warp's Q' (and state) are ready
+                mbar_arrive(&bars[B_EPQ]);      // this warp's Q' is ready
             }
             if (ct == 0) PAIR_TRACE(13, i);
 
@@ -676,6 +660,29 @@ walk_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 fence_proxy_async();
                 __syncwarp();
+                // A frame move rescales this warp's part of the state once the output MMA, which reads
+                // the state in the chunk's starting frame, has completed, and before the update adds
+                // the chunk's tokens in the new frame.  (One fp32 frame cannot serve both ends of a
+                // chunk whose log decay is in the hundreds: exp(rho_new - m_c) overflows while
+                // exp(rho - rho_new) underflows.)
+                if (rescale) {
+                    uint32_t done = 1u;
+                    if (lane == 0) done = mbar_wait(&bars[B_HFULL], ph, wc) ? 1u : 0u;
+                    if (__shfl_sync(0xffffffffu, done, 0)) {   // (aborted: (g) leaves the loop)
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c0 = hq * (DK / 4); c0 < (hq + 1) * (DK / 4); c0 += 16) {
+                            uint32_t r[16];
+                            tmem_ld16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * beta);
+                            tmem_st16(tmem_addr(tmem, q * 32, SM::C_COL + c0), r);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                    }
+                }
                 if (lane == 0) mbar_arrive(&bars[B_KREADY]);   // this warp's K' is ready
                 float nacc[8];
 #pragma unroll
