@@ -289,16 +289,20 @@ mlstm_status mlstm_step(float *C, float *n, float *m,
  * the result is sensitive to, as two bf16 parts, value and rounding residue)
  * and the scores, dS and the scans in fp32 on the CUDA cores; otherwise every
  * step runs in fp32 on the CUDA cores.  Shapes and chunk sizes as for
- * mlstm_fwd.
+ * mlstm_fwd.  The forget-gate gradient of token j sums the terms of the token
+ * pairs s < j <= t (those whose decay includes f_j) themselves, in four
+ * disjoint groups (pairs inside j's chunk, pairs with one token in it, pairs
+ * that skip it), rather than as a difference of cumulative sums in which all
+ * other pairs cancel: strongly forgetting gates keep its accuracy.
  *
  * workspace: at least mlstm_bwd_workspace_size() bytes, 256-byte aligned
  * (it holds the chunk-start states and their gradients and the chunk's scores:
- * 8 DHQK (DHV + 1) + 8 chunk^2 + 12 bytes per chunk and head, plus 4 DHV +
- * 8 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 20 bytes per token and head; on the
+ * 8 DHQK (DHV + 1) + 8 chunk^2 + 16 bytes per chunk and head, plus 4 DHV +
+ * 12 ceil(DHQK / 32) + 4 ceil(DHV / 64) + 24 bytes per token and head; on the
  * tensor-core path, where the chunk-start states, the scores and g are kept
- * as bf16 parts instead of fp32, 6 DHQK DHV + 8 DHQK + 6 chunk^2 + 12 bytes
- * per chunk and head, plus 4 DHQK + 8 DHV + 8 ceil(DHQK / 32) +
- * 4 ceil(DHV / 64) + 20 bytes per token and head; each array 256-byte
+ * as bf16 parts instead of fp32, 6 DHQK DHV + DHQK DHV / 512 + 8 DHQK +
+ * 6 chunk^2 + 12 bytes per chunk and head, plus 4 DHQK + 8 DHV + 12 ceil(DHQK / 32) +
+ * 4 ceil(DHV / 64) + 24 bytes per token and head; each array 256-byte
  * aligned).  A bounded
  * device-side wait of the tensor-core products that gives up records a
  * timeout that mlstm_fwd_status reads from this workspace.  Errors as for

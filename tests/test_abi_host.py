@@ -57,12 +57,14 @@ def test_bwd_tensor_path_query(lib):
     assert lib.mlstm_bwd_tensor_path(256, 512, 48, bf) == -1
     # the tensor-core path's workspace keeps the chunk-start states, the scores and g as bf16 parts
     # instead of fp32, the state gradients only as bf16 and adds bf16 copies: 2 DHQK DHV + 2 chunk^2
-    # bytes less per chunk and head and 4 DHQK + 4 DHV more per token and head (here every array is a
+    # bytes less per chunk and head and 4 DHQK + 4 DHV more per token and head; its walk leaves
+    # DHQK DHV / 2048 partial sums of E_c per chunk and head instead of one (here every array is a
     # multiple of 256 bytes)
     B, NH, S, DK, DV, ch = 1, 8, 8192, 256, 512, 64
     extra = lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, bf) - lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, f32)
     NC = S // ch
-    assert extra == -B * NH * NC * (2 * DK * DV + 2 * ch * ch) + B * NH * S * (4 * DK + 4 * DV)
+    assert extra == (-B * NH * NC * (2 * DK * DV + 2 * ch * ch) + B * NH * S * (4 * DK + 4 * DV)
+                     + B * NH * NC * 4 * (DK * DV // 2048 - 1))
 
 
 def test_workspace_size(lib):

@@ -38,9 +38,40 @@ def run_gpu(inputs, dh, chunk):
     return tuple(None if x is None else x.cpu() for x in out)
 
 
-def check(inputs, dh, chunk, tol):
+def ulp_sensitivity(inputs, dh, ref, draws=2):
+    """Per gradient, the largest rel-L2 change of the oracle's result when every fp32 input moves by
+    -1, 0 or +1 ulp at random: the scale of error that rounding the inputs alone causes, so the least
+    any fp32 evaluation can promise on these inputs."""
+    rng = np.random.default_rng(0)
+
+    def nudge(x):
+        if x is None:
+            return None
+        a = x.float().numpy()
+        step = rng.integers(-1, 2, size=a.shape)
+        b = np.where(step > 0, np.nextafter(a, np.float32(np.inf)),
+                     np.where(step < 0, np.nextafter(a, np.float32(-np.inf)), a))
+        return torch.from_numpy(b.astype(np.float32))
+
+    sens = {}
+    for _ in range(draws):
+        got = oracle.mlstm_adjoint(*[nudge(x) for x in inputs], nudge(dh))
+        for name, x, r in zip(NAMES, got, ref):
+            if r is not None:
+                sens[name] = max(sens.get(name, 0.0), rel_l2(x, r))
+    return sens
+
+
+def check(inputs, dh, chunk, tol, cond_factor=None):
+    """Rel-L2 of every gradient against the oracle within `tol`; with cond_factor, within
+    max(tol, cond_factor x the gradient's one-ulp input sensitivity) (fp32 inputs whose gradients
+    are ill-conditioned)."""
     got = run_gpu(inputs, dh, chunk)
     ref = oracle.mlstm_adjoint(*inputs, dh)
+    tols = {n: tol for n in NAMES}
+    if cond_factor is not None:
+        for n, v in ulp_sensitivity(inputs, dh, ref).items():
+            tols[n] = max(tol, cond_factor * v)
     errs = {}
     for name, x, r in zip(NAMES, got, ref):
         if r is None:
@@ -49,8 +80,8 @@ def check(inputs, dh, chunk, tol):
         xx = x.double().numpy()
         assert np.all(np.isfinite(xx)), name
         errs[name] = rel_l2(xx, r)
-    bad = {n: e for n, e in errs.items() if not e <= tol}
-    assert not bad, "rel-L2 above %.0e: %s (all: %s)" % (tol, bad, errs)
+    bad = {n: (e, tols[n]) for n, e in errs.items() if not e <= tols[n]}
+    assert not bad, "rel-L2 above the bound (error, bound): %s (all: %s)" % (bad, errs)
     return errs
 
 
@@ -80,6 +111,20 @@ def test_bwd_small_shapes(cuda_lib, B, NH, S, DHQK, DHV, chunk, dt):
 def test_bwd_adversarial_gates(cuda_lib, ig, fg, dt, DHQK, DHV, chunk):
     inputs = make_custom(1, 2, 3 * chunk + 5, DHQK, DHV, dt, seed=13, ig=ig, fg=fg)
     check(inputs, make_dh(1, 2, 3 * chunk + 5, DHV, dt, seed=14), chunk, BWD_TOL[dt])
+
+
+@pytest.mark.parametrize("ig,fg", [((0.0, 8.0), (-4.0, 1.0)), ((0.0, 1.0), (-4.0, 1.0)), ((0.0, 4.0), (1.0, 2.0))])
+@pytest.mark.parametrize("dt,DHQK,DHV,chunk", [("f32", 64, 64, 32), ("bf16", 256, 512, 64), ("bf16", 256, 512, 128)])
+def test_bwd_strong_forgetting_many_chunks(cuda_lib, ig, fg, dt, DHQK, DHV, chunk):
+    """Gates whose log decay per chunk is in the hundreds (forget pre-activations around -4) or whose
+    input gates reach e^8, over many chunks: every chunk-start state is nearly forgotten by the next
+    one, and the stabilizer moves at every chunk.  With fp32 inputs these gradients are
+    ill-conditioned (one ulp of the inputs moves dq by up to 3.5e-5 here), so each is held to four
+    times its measured one-ulp sensitivity where that exceeds the fixed bound; bf16 inputs keep 1e-2."""
+    S = 1024 + 7
+    inputs = make_custom(1, 2, S, DHQK, DHV, dt, seed=chunk + 21, ig=ig, fg=fg)
+    check(inputs, make_dh(1, 2, S, DHV, dt, seed=chunk + 22), chunk, BWD_TOL[dt],
+          cond_factor=4.0 if dt == "f32" else None)
 
 
 def test_bwd_floor_binds(cuda_lib):

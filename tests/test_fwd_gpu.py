@@ -83,17 +83,18 @@ def test_fwd_adversarial_gates(cuda_lib, ig, fg, dt, DHQK, DHV, chunk):
     check_against_oracle(inputs, chunk, TOL[dt])
 
 
+@pytest.mark.parametrize("DHQK,DHV", [(256, 512), (128, 256)])
 @pytest.mark.parametrize("chunk", [64, 128])
 @pytest.mark.parametrize("ig,fg", [((0.0, 8.0), (-4.0, 1.0)), ((0.0, 1.0), (-4.0, 1.0)), ((0.0, 4.0), (1.0, 2.0))])
-def test_fwd_frame_moves_within_segments(cuda_lib, chunk, ig, fg):
-    """Gates that move the stabilizer frame of the walk's state at (nearly) every chunk, on a shape
+def test_fwd_frame_moves_within_segments(cuda_lib, DHQK, DHV, chunk, ig, fg):
+    """Gates that move the stabilizer frame of the walk's state at (nearly) every chunk, on shapes
     whose segments hold several chunks (at small sizes every segment is one chunk and the walk never
-    moves its frame): B1 NH8 S4096 d256/512, the paired walk at chunk 128 and the one-CTA walk at
-    chunk 64."""
+    moves its frame): B1 NH8 S4096, d256/512 (the paired walk at chunk 128, the one-CTA tf32 walk at
+    chunk 64) and d128/256 (the one-CTA walk: fp16 state copy at chunk 128, tf32 at chunk 64)."""
     S = 4096
-    nseg = binding.fwd_segments(1, 8, S, 256, 512, chunk, torch.bfloat16)
+    nseg = binding.fwd_segments(1, 8, S, DHQK, DHV, chunk, torch.bfloat16)
     assert 0 < nseg < S // chunk, nseg   # several chunks per segment
-    inputs = make_custom(1, 8, S, 256, 512, "bf16", seed=chunk + 5, ig=ig, fg=fg)
+    inputs = make_custom(1, 8, S, DHQK, DHV, "bf16", seed=chunk + DHQK + 5, ig=ig, fg=fg)
     check_against_oracle(inputs, chunk, TOL["bf16"], nthreads=oracle.default_threads())
 
 

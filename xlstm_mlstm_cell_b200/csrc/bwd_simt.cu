@@ -26,18 +26,28 @@
 //   dqh_t = sum_s dS_ts k_s + sc_t (C_c g_t + dden_t n_c),
 //   dk_s  = sum_t dS_ts qh_t + w_s (G_{c+1} v_s + dn_{c+1}),
 //   dv_s  = sum_t A_ts g_t + w_s G_{c+1}^T k_s,          dq = dqh / sqrt(DHQK).
-// Gate gradients: h depends on the global cumulative log decay A_t only through exp(A_t) qh_t
-// and exp(i~_s - A_s) k_s (the unstabilized read-out), so
-//   dL/di~_t = k_t . dk_t,  dL/dA_t = q_t . dq_t - k_t . dk_t,
-//   dL/dlog f_j = sum_{t >= j} dL/dA_t,  dL/df~_j = dL/dlog f_j * sigmoid(-f~_j),
-// a reverse cumulative sum over the sequence (accumulated in fp64).
+// Gate gradients.  h depends on the gates through the weights D_ts of the pairs s <= t (the
+// unstabilized read-out weighs v_s for query t by exp(i~_s + sum_{s < u <= t} log f_u)); with
+// R_ts = dL/dD_ts D_ts (inside a chunk dA_ts A_ts; for tokens of different chunks the same quantity,
+// reached through the chunk's state) the gradients are
+//   dL/di~_s = sum_{t >= s} R_ts = k_s . dk_s,
+//   dL/dlog f_j = sum_{s < j <= t} R_ts,  dL/df~_j = dL/dlog f_j * sigmoid(-f~_j).
+// For j in chunk c the pairs that straddle j fall into four disjoint groups, each summed on its own:
+//   F_j = E_c + sum_{t in c, t >= j} q_t . dq^inter_t + sum_{s in c, s < j} k_s . dk^inter_s + RECT_j,
+// E_c = exp(g_c + m_c - m_{c+1}) (<G_{c+1}, C_c> + <dn_{c+1}, n_c>) the pairs that skip chunk c (the
+// gradient of the state at its end against the decayed state at its start), dq^inter and dk^inter the
+// inter-chunk terms alone (q_t . dq^inter_t sums R_ts over the s before t's chunk, k_s . dk^inter_s over
+// the t after s's chunk) and RECT_j the pairs inside the chunk, summed from R in the dS kernel.  The
+// shorter form sum_{t >= j} (q_t . dq_t - k_t . dk_t) equals F_j, but every pair at or after j cancels
+// there, the pairs s = t (the largest terms) among them, and with strongly forgetting gates the
+// result was lost to fp32 rounding.
 //
 // Kernels, in launch order (after the gate preprocessing and the forward's fp32 carry that stores
 // the chunk-start states): bwd_scores_kernel (A, den, N per chunk), bwd_num_kernel (the read-out
-// numerator, g and do per chunk and 64 value columns), bwd_ds_kernel (dden, dS, dn of the read-out),
+// numerator, g and do per chunk and 64 value columns), bwd_ds_kernel (dden, dS, dn of the read-out, RECT),
 // bwd_dc_kernel (dC of the read-out per 64 x 64 state tile), bwd_state_scan_kernel (the reverse scan
-// of the state gradients), bwd_grad_kernel (dq, dk, dv per chunk and 64 columns) and
-// bwd_gate_kernel.  The per-chunk products run as 64 x 64 output tiles on the CUDA cores in fp32.
+// of the state gradients), bwd_skip_kernel (E_c), bwd_grad_kernel (dq, dk, dv per chunk and 64
+// columns) and bwd_gate_kernel.  The per-chunk products run as 64 x 64 output tiles on the CUDA cores in fp32.
 #include "bwd_tc.h"
 #include "common.cuh"
 #include "mlstm_internal.h"
@@ -60,7 +70,12 @@ struct Params {
     float *DOTP;                     // partial row sums of g . hh per 64 value columns [BH][S][NJT]
     int NJT;                         // ceil(DV / 64)
     float *P2, *AI;                  // dS and A per chunk [BH][NC][L][L]
-    float *QD, *KD;                  // per dk tile partial q . dq and k . dk [BH][S][NTK]
+    // per 32 columns of dk: partial q . dq^inter, k . dk and k . dk^inter [BH][S][NTK] (^inter: the
+    // inter-chunk term alone), and RECT [BH][S], the sum of dA_ts A_ts over the pairs s < j <= t of
+    // token j's chunk (written by the dS kernels)
+    float *QD, *KD, *KI, *RECT;
+    float *EP;                       // partial sums of E_c [BH][NC][NEP] (the pairs that skip chunk c)
+    int NEP;
     void *dq, *dk, *dv, *dog;
     float *dig, *dfg;
 };
@@ -314,6 +329,7 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
     griddep_launch_dependents();
     __shared__ __align__(16) float As[GK * GSTR], Bs[GK * GSTR];
     __shared__ float xs_[128], mx[128], fl[128], sc[128], dd[128];
+    __shared__ float rowl[128], colb[128], cpart[NT / 32][GM];   // sums of R by row and column
     const int L = p.L, DK = p.DK, DV = p.DV;
     const int bh = blockIdx.x, c = blockIdx.y;
     const int t0 = c * L, len = min(L, p.S - t0);
@@ -323,8 +339,10 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
     const T *vb = static_cast<const T *>(p.v) + ((size_t)bh * p.S + t0) * DV;
     const float *gtb = p.Gt + ((size_t)bh * p.S + t0) * DV;
     float *P2g = p.P2 + ((size_t)bh * p.NC + c) * L * L;
+    const float *AIg = p.AI + ((size_t)bh * p.NC + c) * L * L;
 
     chunk_rows(p, bh, c, t0, len, xs_, mx, fl, sc);
+    for (int t = tid; t < 128; t += NT) rowl[t] = colb[t] = 0.f;
     for (int t = tid; t < L; t += NT) {
         float v = 0.f;
         if (t < len) {
@@ -360,19 +378,60 @@ __global__ void __launch_bounds__(NT) bwd_ds_kernel(Params p)
                           Bs[(e & 31) * GSTR + (e >> 5)] = bv;
                       },
                       As, Bs, acc);
+            // dS, and R_ts = dA_ts A_ts of the pairs s < t (the derivative of the loss by the log decay
+            // between them): its sums along the rows (left of the diagonal) and columns (below it)
+            float cp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
                 const int t = mt * GM + 4 * tm + a;
+                float rp = 0.f;
 #pragma unroll
                 for (int b2 = 0; b2 < 4; ++b2) {
                     const int s2 = nt * GM + 4 * tn + b2;
                     float pv = 0.f;
-                    if (s2 <= t && t < len) pv = (acc[a][b2] + dd[t]) * expf(xs_[s2] - mx[t]);
+                    if (s2 <= t && t < len) {
+                        const float da = acc[a][b2] + dd[t];
+                        pv = da * expf(xs_[s2] - mx[t]);
+                        if (s2 < t) {
+                            const float rv = da * AIg[(size_t)t * L + s2];
+                            rp += rv;
+                            cp[b2] += rv;
+                        }
+                    }
                     if (t < L && s2 < L) P2g[(size_t)t * L + s2] = pv;
                 }
+                rp = sum16(rp);
+                if (tn == 0 && t < L) rowl[t] += rp;   // one thread per row: tiles in order
+            }
+#pragma unroll
+            for (int b2 = 0; b2 < 4; ++b2) {
+                cp[b2] += __shfl_xor_sync(0xffffffffu, cp[b2], 16);
+                if (tm % 2 == 0) cpart[tid >> 5][4 * tn + b2] = cp[b2];
+            }
+            __syncthreads();
+            if (tid < GM && nt * GM + tid < L) {
+                float v = 0.f;
+                for (int w2 = 0; w2 < NT / 32; ++w2) v += cpart[w2][tid];
+                colb[nt * GM + tid] += v;
             }
         }
     __syncthreads();
+    if (tid < 32) {   // RECT_j = sum_{s < j} (colb_s - rowl_s) over the chunk (a warp scan in fp64)
+        const int per = (L + 31) / 32, sb = tid * per;
+        double loc = 0.0;
+        for (int u = sb; u < min(sb + per, len); ++u) loc += (double)colb[u] - (double)rowl[u];
+        double inc = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (tid >= o) inc += y;
+        }
+        double run = inc - loc;
+        for (int u = sb; u < min(sb + per, len); ++u) {
+            p.RECT[(size_t)bh * p.S + t0 + u] = (float)run;
+            run += (double)colb[u] - (double)rowl[u];
+        }
+    }
     float *GNc = p.GN + ((size_t)bh * p.NC + c) * DK;
     for (int i = tid; i < DK; i += NT) {
         float a2 = 0.f;
@@ -490,8 +549,8 @@ __global__ void __launch_bounds__(256) bwd_state_scan_kernel(Params p)
 //   dk  = [dS^T | w v] [qh ; G_end^T] + w dn_end,         K = L + DV,
 //   dv  = [A^T | w k] [g ; G_end],                        K = L + DK,
 // with w_s = exp(g_c - a_s + i~_s - m_{c+1}) the weight of token s in the state at the chunk's end.
-// The dq and dk tiles also leave the partial row sums q . dq and k . dk of their two 32-column
-// halves (QD, KD) for the gate gradients.
+// The dq and dk tiles also leave, for the gate gradients, the partial row sums of their two 32-column
+// halves: q . dq^inter (QD), k . dk^inter (KI) of the inter-chunk term alone, and k . dk (KD).
 template <typename T, int KIND>
 __global__ void __launch_bounds__(NT, 2) bwd_grad_kernel(Params p)
 {
@@ -530,58 +589,86 @@ __global__ void __launch_bounds__(NT, 2) bwd_grad_kernel(Params p)
     const int nmt = (L + GM - 1) / GM;
     for (int mt = 0; mt < nmt; ++mt) {
         float acc[4][4] = {};
-        // the chunk-local term (reduction over the chunk's tokens), then the inter-chunk term
-        // (over DV for dq and dk, over DK for dv)
+        // steps 0 .. nloc - 1: the chunk-local term (reduction over the chunk's tokens); from nloc: the
+        // inter-chunk term (over DV for dq and dk, over DK for dv)
         const int KI = kind == 2 ? DK : DV;
-        const int nloc = (L + GK - 1) / GK;
-        tile_gemm(nloc + (KI + GK - 1) / GK,
-                  [&](int st, int e, float &av, float &bv) {
-                      if (st < nloc) {
-                          const int k0 = st * GK;
-                          if (kind == 0) {          // As[u][t] = dS[t][u]
-                              const int m = e >> 5, k = e & 31, t = mt * GM + m;
-                              av = (t < L && k0 + k < L) ? P2g[(size_t)t * L + k0 + k] : 0.f;
-                          } else {                  // As[u][s] = dS[u][s] or A[u][s]
-                              const int k = e >> 6, m = e & 63, s2 = mt * GM + m;
-                              av = (s2 < L && k0 + k < L) ? (kind == 1 ? P2g : AIg)[(size_t)(k0 + k) * L + s2] : 0.f;
-                          }
-                          const int kk = e >> 6, n = e & 63, u = k0 + kk;   // Bs[u][col]: k, qh or g
-                          bv = 0.f;
-                          if (u < len && c0 + n < NC_) {
-                              if (kind == 0) bv = to_f32(kb[(size_t)u * DK + c0 + n]);
-                              else if (kind == 1) bv = to_f32(qb[(size_t)u * DK + c0 + n]) * scale;
-                              else bv = gtb[(size_t)u * DV + c0 + n];
-                          }
-                      } else {
-                          const int k0 = (st - nloc) * GK;
-                          const int m = e >> 5, k = e & 31, r = mt * GM + m;   // row r of the output tile
-                          av = 0.f;
-                          if (r < len && k0 + k < KI) {
-                              if (kind == 0) av = sc[r] * gtb[(size_t)r * DV + k0 + k];
-                              else if (kind == 1) av = wt[r] * to_f32(vb[(size_t)r * DV + k0 + k]);
-                              else av = wt[r] * to_f32(kb[(size_t)r * DK + k0 + k]);
-                          }
-                          if (kind == 2) {           // Bs[i][j] = G_end[i][j]
-                              const int kk = e >> 6, n = e & 63;
-                              bv = (k0 + kk < DK && c0 + n < DV) ? Ge[(size_t)(k0 + kk) * DV + c0 + n] : 0.f;
-                          } else {                   // Bs[j][i] = C_c[i][j] or G_end[i][j]
-                              const int n = e >> 5, kk = e & 31;
-                              bv = (c0 + n < DK && k0 + kk < DV) ? (kind == 0 ? Cc : Ge)[(size_t)(c0 + n) * DV + k0 + kk] : 0.f;
-                          }
-                      }
-                  },
-                  [&](int st, int e, float av, float bv) {
-                      if (st < nloc) {
-                          if (kind == 0) As[(e & 31) * GSTR + (e >> 5)] = av;
-                          else As[(e >> 6) * GSTR + (e & 63)] = av;
-                          Bs[(e >> 6) * GSTR + (e & 63)] = bv;
-                      } else {
-                          As[(e & 31) * GSTR + (e >> 5)] = av;
-                          if (kind == 2) Bs[(e >> 6) * GSTR + (e & 63)] = bv;
-                          else Bs[(e & 31) * GSTR + (e >> 5)] = bv;
-                      }
-                  },
-                  As, Bs, acc);
+        const int nloc = (L + GK - 1) / GK, ninter = (KI + GK - 1) / GK;
+        auto get = [&](int st, int e, float &av, float &bv) {
+            if (st < nloc) {
+                const int k0 = st * GK;
+                if (kind == 0) {          // As[u][t] = dS[t][u]
+                    const int m = e >> 5, k = e & 31, t = mt * GM + m;
+                    av = (t < L && k0 + k < L) ? P2g[(size_t)t * L + k0 + k] : 0.f;
+                } else {                  // As[u][s] = dS[u][s] or A[u][s]
+                    const int k = e >> 6, m = e & 63, s2 = mt * GM + m;
+                    av = (s2 < L && k0 + k < L) ? (kind == 1 ? P2g : AIg)[(size_t)(k0 + k) * L + s2] : 0.f;
+                }
+                const int kk = e >> 6, n = e & 63, u = k0 + kk;   // Bs[u][col]: k, qh or g
+                bv = 0.f;
+                if (u < len && c0 + n < NC_) {
+                    if (kind == 0) bv = to_f32(kb[(size_t)u * DK + c0 + n]);
+                    else if (kind == 1) bv = to_f32(qb[(size_t)u * DK + c0 + n]) * scale;
+                    else bv = gtb[(size_t)u * DV + c0 + n];
+                }
+            } else {
+                const int k0 = (st - nloc) * GK;
+                const int m = e >> 5, k = e & 31, r = mt * GM + m;   // row r of the output tile
+                av = 0.f;
+                if (r < len && k0 + k < KI) {
+                    if (kind == 0) av = sc[r] * gtb[(size_t)r * DV + k0 + k];
+                    else if (kind == 1) av = wt[r] * to_f32(vb[(size_t)r * DV + k0 + k]);
+                    else av = wt[r] * to_f32(kb[(size_t)r * DK + k0 + k]);
+                }
+                if (kind == 2) {           // Bs[i][j] = G_end[i][j]
+                    const int kk = e >> 6, n = e & 63;
+                    bv = (k0 + kk < DK && c0 + n < DV) ? Ge[(size_t)(k0 + kk) * DV + c0 + n] : 0.f;
+                } else {                   // Bs[j][i] = C_c[i][j] or G_end[i][j]
+                    const int n = e >> 5, kk = e & 31;
+                    bv = (c0 + n < DK && k0 + kk < DV) ? (kind == 0 ? Cc : Ge)[(size_t)(c0 + n) * DV + k0 + kk] : 0.f;
+                }
+            }
+        };
+        auto put = [&](int st, int e, float av, float bv) {
+            if (st < nloc) {
+                if (kind == 0) As[(e & 31) * GSTR + (e >> 5)] = av;
+                else As[(e >> 6) * GSTR + (e & 63)] = av;
+                Bs[(e >> 6) * GSTR + (e & 63)] = bv;
+            } else {
+                As[(e & 31) * GSTR + (e >> 5)] = av;
+                if (kind == 2) Bs[(e >> 6) * GSTR + (e & 63)] = bv;
+                else Bs[(e & 31) * GSTR + (e >> 5)] = bv;
+            }
+        };
+        // the inter-chunk term first: for dq and dk its own row sums q . dq^inter, k . dk^inter (the
+        // pairs of tokens in different chunks, for the forget-gate gradients) are taken before the
+        // chunk-local term joins the accumulator
+        tile_gemm(ninter, [&](int st, int e, float &av, float &bv) { get(nloc + st, e, av, bv); },
+                  [&](int st, int e, float av, float bv) { put(nloc + st, e, av, bv); }, As, Bs, acc);
+        auto row_parts = [&](int a, float part, float *dst) {   // the tile's two 32-column halves
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            const int r = mt * GM + 4 * tm + a, half = (c0 >> 5) + (tn >> 3);
+            if ((tn & 7) == 0 && r < len && half * 32 < DK) dst[((size_t)bh * p.S + t0 + r) * p.NTK + half] = part;
+        };
+        if (kind < 2) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = mt * GM + 4 * tm + a;
+                float part = 0.f;
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2) {
+                    const int col = c0 + 4 * tn + b2;
+                    if (r < len && col < NC_) {
+                        if (kind == 0)
+                            part = fmaf(to_f32(qb[(size_t)r * DK + col]) * scale, acc[a][b2] + sc[r] * dd[r] * nc[col], part);
+                        else
+                            part = fmaf(to_f32(kb[(size_t)r * DK + col]), acc[a][b2] + wt[r] * ge[col], part);
+                    }
+                }
+                row_parts(a, part, kind == 0 ? p.QD : p.KI);
+            }
+        }
+        tile_gemm(nloc, get, put, As, Bs, acc);
         // epilogue
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
@@ -595,7 +682,6 @@ __global__ void __launch_bounds__(NT, 2) bwd_grad_kernel(Params p)
                         if (kind == 0) {
                             const float dqh = acc[a][b2] + sc[r] * dd[r] * nc[col];
                             static_cast<T *>(p.dq)[((size_t)bh * p.S + t0 + r) * DK + col] = from_f32<T>(dqh * scale);
-                            part = fmaf(to_f32(qb[(size_t)r * DK + col]) * scale, dqh, part);
                         } else if (kind == 1) {
                             const float dkv = acc[a][b2] + wt[r] * ge[col];
                             static_cast<T *>(p.dk)[((size_t)bh * p.S + t0 + r) * DK + col] = from_f32<T>(dkv);
@@ -606,61 +692,108 @@ __global__ void __launch_bounds__(NT, 2) bwd_grad_kernel(Params p)
                     }
                 }
             }
-            if (kind < 2) {   // partial sums of the tile's two 32-column halves (8 threads each)
-#pragma unroll
-                for (int o = 4; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                const int half = (c0 >> 5) + (tn >> 3);
-                if ((tn & 7) == 0 && r < len && half * 32 < DK)
-                    (kind == 0 ? p.QD : p.KD)[((size_t)bh * p.S + t0 + r) * p.NTK + half] = part;
-            }
+            if (kind == 1) row_parts(a, part, p.KD);   // k . dk (the input-gate gradient)
         }
     }
 }
 
 // ---------------------------------------------------------------- gate gradients
-// grid (BH), 1024 threads: dL/di~_t = k_t . dk_t; dL/df~_j = sigmoid(-f~_j) sum_{t >= j} (q_t . dq_t - k_t . dk_t).
-constexpr int GT = 1024;
+// grid (BH, ceil(NC / 8)), 256 threads, a warp per chunk (a lane takes L / 32 consecutive tokens):
+// dL/di~_t = k_t . dk_t and dL/df~_j = sigmoid(-f~_j) F_j with, for j in chunk c,
+//   F_j = E_c + sum_{t in c, t >= j} q_t . dq^inter_t + sum_{s in c, s < j} k_s . dk^inter_s + RECT_j,
+// the four disjoint sets of the pairs s < j <= t, summed in fp64 (E_c from its NEP partial sums).
+constexpr int GT = 256;
+
+__device__ __forceinline__ double warp_scan_incl(double v, int lane)   // sum over lanes <= lane
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    return v;
+}
 
 __global__ void __launch_bounds__(GT) bwd_gate_kernel(Params p)
 {
     griddep_wait();
     griddep_launch_dependents();
-    __shared__ double wsum[GT / 32];
-    const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (p.S + GT - 1) / GT;
-    const int tb = min(tid * per, p.S), te = min(tb + per, p.S);
-    const float *qd = p.QD + (size_t)bh * p.S * p.NTK;
-    const float *kd = p.KD + (size_t)bh * p.S * p.NTK;
-    auto da = [&](int t, double *kdk) {
-        double a = 0.0, b = 0.0;
-        for (int z = 0; z < p.NTK; ++z) {
-            a += (double)qd[(size_t)t * p.NTK + z];
-            b += (double)kd[(size_t)t * p.NTK + z];
-        }
-        *kdk = b;
-        return a - b;
-    };
-    double loc = 0.0, kk;
-    for (int t = tb; t < te; ++t) loc += da(t, &kk);
-    // exclusive suffix sum over the threads after this one (the tokens after this thread's range)
-    double inc = loc;
+    const int bh = blockIdx.x, lane = threadIdx.x & 31;
+    const int c = blockIdx.y * (GT / 32) + (threadIdx.x >> 5);
+    if (c >= p.NC) return;                       // (whole warps)
+    const int t0 = c * p.L, len = min(p.L, p.S - t0);
+    constexpr int MAXPER = 4;                    // chunk <= 128
+    const int per = (p.L + 31) / 32;
+    double e = 0.0;                              // E_c: the pairs that skip the chunk
+    for (int z = lane; z < p.NEP; z += 32) e += (double)p.EP[((size_t)bh * p.NC + c) * p.NEP + z];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const double y = __shfl_down_sync(0xffffffffu, inc, o);
-        if (lane + o < 32) inc += y;
+    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    double ki[MAXPER], qi[MAXPER], kd[MAXPER];
+    double lk = 0.0, lq = 0.0;
+#pragma unroll
+    for (int u = 0; u < MAXPER; ++u) {
+        ki[u] = qi[u] = kd[u] = 0.0;
+        const int tl = lane * per + u;
+        if (u < per && tl < len) {
+            const size_t r = ((size_t)bh * p.S + t0 + tl) * p.NTK;
+            for (int z = 0; z < p.NTK; ++z) {
+                ki[u] += (double)p.KI[r + z];
+                qi[u] += (double)p.QD[r + z];
+                kd[u] += (double)p.KD[r + z];
+            }
+        }
+        lk += ki[u];
+        lq += qi[u];
     }
-    if (lane == 0) wsum[warp] = inc;   // the warp's total
+    // k . dk^inter over the chunk's tokens before this lane's, q . dq^inter over those from it on
+    double kpre = warp_scan_incl(lk, lane) - lk;
+    double qtot = lq;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qtot += __shfl_xor_sync(0xffffffffu, qtot, o);
+    double qsuf = qtot - (warp_scan_incl(lq, lane) - lq);
+#pragma unroll
+    for (int u = 0; u < MAXPER; ++u) {
+        const int tl = lane * per + u;
+        if (u < per && tl < len) {
+            const size_t g = (size_t)bh * p.S + t0 + tl;
+            p.dig[g] = (float)kd[u];
+            const float f = p.fg[g];
+            const float sgm = f >= 0.f ? expf(-f) / (1.f + expf(-f)) : 1.f / (1.f + expf(f));   // sigmoid(-f)
+            p.dfg[g] = (float)(e + qsuf + kpre + (double)p.RECT[g]) * sgm;
+        }
+        kpre += ki[u];
+        qsuf -= qi[u];
+    }
+}
+
+// ---------------------------------------------------------------- the pairs that skip a chunk
+// grid (BH, NC), 256 threads: EP[c] = E_c = exp(g_c + m_c - m_{c+1}) (<G_end, C_c> + <dn_end, n_c>), the
+// gradient of the state at chunk c's end against the decayed state at its start (fp32 arrays).
+__global__ void __launch_bounds__(NT) bwd_skip_kernel(Params p)
+{
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ double wsum[NT / 32];
+    const int bh = blockIdx.x, c = blockIdx.y, tid = threadIdx.x;
+    const size_t nstate = (size_t)p.DK * p.DV, zc = (size_t)bh * p.NC + c;
+    const float4 *ge = reinterpret_cast<const float4 *>(p.GS + zc * nstate);
+    const float4 *cs = reinterpret_cast<const float4 *>(p.CS + zc * nstate);
+    float acc = 0.f;
+    for (size_t e = tid; e < nstate / 4; e += NT) {
+        const float4 a = ge[e], b = cs[e];
+        acc = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+    }
+    for (int d = tid; d < p.DK; d += NT) acc = fmaf(p.GN[zc * p.DK + d], p.NS[zc * p.DK + d], acc);
+    double v = acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) wsum[tid >> 5] = v;
     __syncthreads();
-    double after = inc - loc;           // later lanes of this warp
-    for (int w2 = warp + 1; w2 < GT / 32; ++w2) after += wsum[w2];
-    double run = after;
-    for (int t = te - 1; t >= tb; --t) {
-        run += da(t, &kk);
-        const size_t g = (size_t)bh * p.S + t;
-        p.dig[g] = (float)kk;
-        const float f = p.fg[g];
-        const float sgm = f >= 0.f ? expf(-f) / (1.f + expf(-f)) : 1.f / (1.f + expf(f));   // sigmoid(-f)
-        p.dfg[g] = (float)run * sgm;
+    if (tid == 0) {
+        double t = 0.0;
+        for (int w = 0; w < NT / 32; ++w) t += wsum[w];
+        const float decay = expf(p.G[zc] + p.MC[(size_t)bh * (p.NC + 1) + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1]);
+        p.EP[zc] = (float)t * decay;
     }
 }
 
@@ -680,17 +813,18 @@ cudaError_t launch_t(const Params &p, int BH, cudaStream_t st, const bwdtc::Args
         e = launch_kernel(bwd_dc_kernel<T>, dim3(BH * p.NC, (p.DK + GM - 1) / GM, p.NJT), dim3(NT), 0, st, 1, p);
         if (e != cudaSuccess) return e;
         e = launch_kernel(bwd_state_scan_kernel, dim3((p.DK * p.DV / 4 + 255) / 256, BH), dim3(256), 0, st, 1, p);
+        if (e == cudaSuccess) e = launch_kernel(bwd_skip_kernel, dim3(BH, p.NC), dim3(NT), 0, st, 1, p);
     }
     if (e != cudaSuccess) return e;
     if (tc) {   // dq, dk, dv on the tensor cores
         if ((e = bwdtc::launch(*tc)) != cudaSuccess) return e;
-        return launch_kernel(bwd_gate_kernel, dim3(BH), dim3(GT), 0, st, 1, p);
+        return launch_kernel(bwd_gate_kernel, dim3(BH, (p.NC + GT / 32 - 1) / (GT / 32)), dim3(GT), 0, st, 1, p);
     }
     const int nk = (p.DK + GM - 1) / GM;
     if ((e = launch_kernel(bwd_grad_kernel<T, 0>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
     if ((e = launch_kernel(bwd_grad_kernel<T, 1>, dim3(BH, p.NC, nk), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
     if ((e = launch_kernel(bwd_grad_kernel<T, 2>, dim3(BH, p.NC, p.NJT), dim3(NT), 0, st, 1, p)) != cudaSuccess) return e;
-    return launch_kernel(bwd_gate_kernel, dim3(BH), dim3(GT), 0, st, 1, p);
+    return launch_kernel(bwd_gate_kernel, dim3(BH, (p.NC + GT / 32 - 1) / (GT / 32)), dim3(GT), 0, st, 1, p);
 }
 
 }  // namespace bwd
@@ -702,7 +836,7 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     p.q = a.q; p.k = a.k; p.v = a.v; p.o = a.ogate; p.dh = a.dh; p.ig = a.igate; p.fg = a.fgate;
     p.A = w.A; p.P = w.M; p.MC = w.MC; p.G = w.G; p.CS = w.CS; p.NS = w.NS;
     p.GS = w.GS; p.GN = w.GN; p.Gt = w.Gt; p.DD = w.DD; p.P2 = w.P2; p.AI = w.AI; p.QD = w.QD; p.KD = w.KD;
-    p.DEN = w.DEN; p.NRM = w.NRM; p.DOTP = w.DOTP; p.NJT = (a.DHV + 63) / 64;
+    p.KI = w.KI; p.RECT = w.RECT; p.EP = w.EP; p.NEP = w.NEP; p.DEN = w.DEN; p.NRM = w.NRM; p.DOTP = w.DOTP; p.NJT = (a.DHV + 63) / 64;
     p.dq = a.dq; p.dk = a.dk; p.dv = a.dv; p.dog = a.ogate ? a.dogate : nullptr; p.dig = a.digate; p.dfg = a.dfgate;
     if (!a.bf16) return bwd::launch_t<float>(p, a.BH, a.stream, nullptr);
     if (!w.tc) return bwd::launch_t<__nv_bfloat16>(p, a.BH, a.stream, nullptr);
@@ -713,7 +847,7 @@ cudaError_t launch_bwd(const BwdArgs &a, const BwdWorkspace &w)
     t.q = static_cast<const bf *>(a.q); t.k = static_cast<const bf *>(a.k); t.v = static_cast<const bf *>(a.v);
     t.C16 = w.CS16; t.G16 = w.GS16; t.g16 = w.Gt16; t.dS16 = w.P216; t.A16 = w.AI16;
     t.dq = static_cast<bf *>(a.dq); t.dk = static_cast<bf *>(a.dk); t.dv = static_cast<bf *>(a.dv);
-    t.QD = w.QD; t.KD = w.KD; t.status = w.status; t.stream = a.stream;
+    t.QD = w.QD; t.KD = w.KD; t.KI = w.KI; t.RECTw = w.RECT; t.EPw = w.EP; t.NEP = w.NEP; t.status = w.status; t.stream = a.stream;
     t.dh = static_cast<const bf *>(a.dh); t.o = static_cast<const bf *>(a.ogate); t.NRM = w.NRM;
     t.DOTP = w.DOTP; t.g16w = w.Gt16; t.dog = a.ogate ? static_cast<bf *>(a.dogate) : nullptr;
     t.NJT = p.NJT; t.sg16 = w.SG16; t.G16w = w.GS16;

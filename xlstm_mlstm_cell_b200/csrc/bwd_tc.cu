@@ -55,7 +55,8 @@ struct KParams {
     const float *A, *P, *MC, *G, *ig, *DD, *NS, *GN;
     const __nv_bfloat16 *pq;               // q (KIND 0) or k (KIND 1): the partial row sums
     __nv_bfloat16 *out;
-    float *part;
+    float *part;                           // q . dq^inter (KIND 0: the inter-chunk term alone) or k . dk
+    float *part2;                          // k . dk^inter (KIND 1)
     // KIND 3 (the read-out numerator)
     const __nv_bfloat16 *dh, *o;
     const float *NRM;
@@ -323,30 +324,39 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                     }
                 }
                 tmem_wait_ld();
-                float prs[16];
+                float prs[16], prs2[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int t = g * 16 + u;
                     const float d1 = __uint_as_float(r1[u]), d2 = __uint_as_float(r2[u]);
                     const float w = tokw[t];
-                    float o, pr = 0.f;
+                    float o, pr = 0.f, pr2 = 0.f;
                     if (KIND == 0) {
-                        const float dqh = d1 + w * (d2 + ddv[t] * colv);
-                        o = dqh * scale;
-                        pr = pv[u] * scale * dqh;
+                        const float dqi = w * (d2 + ddv[t] * colv);   // the inter-chunk term
+                        o = (d1 + dqi) * scale;
+                        pr = pv[u] * scale * dqi;
                     } else if (KIND == 1) {
-                        o = scale * d1 + w * (d2 + colv);
+                        const float dki = w * (d2 + colv);
+                        o = scale * d1 + dki;
                         pr = pv[u] * o;
+                        pr2 = pv[u] * dki;
                     } else {
                         o = d1 + w * d2;
                     }
                     if (t < len) p.out[(g0 + t) * NCOL + col] = __float2bfloat16_rn(o);
                     prs[u] = pr;
+                    prs2[u] = pr2;
                 }
-                if (KIND < 2) {   // q . dq or k . dk over the warp's 32 columns, per token
+                // per token over the warp's 32 columns: q . dq^inter (KIND 0), k . dk and k . dk^inter
+                if (KIND < 2) {
                     const float sum = warp_sum16(prs, lane);
                     const int t = g * 16 + sum16_index(lane);
                     if ((lane & 1) == 0 && t < len) p.part[(g0 + t) * p.NTK + (col >> 5)] = sum;
+                }
+                if (KIND == 1) {
+                    const float sum = warp_sum16(prs2, lane);
+                    const int t = g * 16 + sum16_index(lane);
+                    if ((lane & 1) == 0 && t < len) p.part2[(g0 + t) * p.NTK + (col >> 5)] = sum;
                 }
             }
         }
@@ -390,6 +400,7 @@ static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUten
     p.pq = KIND == 0 ? a.q : a.k;
     p.out = KIND == 0 ? a.dq : KIND == 1 ? a.dk : a.dv;
     p.part = KIND == 0 ? a.QD : KIND == 1 ? a.KD : nullptr;
+    p.part2 = KIND == 1 ? a.KI : nullptr;
     p.status = a.status;
     cudaError_t e = ensure_dynamic_smem((const void *)grad_tc_kernel<KIND, L>, SM::TOTAL);
     if (e != cudaSuccess) return e;
@@ -637,7 +648,8 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
     }
 }
 
-// The reverse walk of the state gradients over the chunks of one 128 x 64 tile (rows d, columns j):
+// The reverse walk of the state gradients over the chunks of one 128 x 64 tile (rows d, columns j); it
+// also leaves, per warp and chunk, the tile's share of E_c (the pairs of tokens that skip chunk c):
 // per chunk the read-out's dC_c = scale sum_t q_t (sc_t g_t)^T as MMAs (A = q, MN-major; B = sc g,
 // two parts, MN-major) into one of two TMEM buffers, while the epilogue warps, which hold the fp32
 // gradient in registers, write the gradient of the state at the chunk's end (bf16) and then
@@ -646,7 +658,8 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
 template <int L>
 __global__ void __launch_bounds__(THREADS, 1)
 gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sg, KParams p,
-                 __nv_bfloat16 *__restrict__ G16, float *__restrict__ GN)
+                 __nv_bfloat16 *__restrict__ G16, float *__restrict__ GN, const __nv_bfloat16 *__restrict__ C16,
+                 float *__restrict__ EP, int NEP)
 {
     using SM = CarrySmem;   // (a stage: q 64 tokens x 128 rows, then sc g 2 parts x 64 tokens x 64)
     extern __shared__ uint8_t smem_raw[];
@@ -742,12 +755,39 @@ gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float gn = 0.f;
         int c = p.NC - 1;
         float g_c = Gb[c], mc_c = MCb[c], mn_c = MCb[c + 1];
+        // this row of the chunk-start state C_c (its bf16 value part), loaded a chunk ahead: the partial
+        // sums of E_c = exp(g_c + m_c - m_{c+1}) (<G_end, C_c> + <dn_end, n_c>), the pairs of tokens
+        // that skip chunk c, per warp (the forget-gate gradients)
+        auto crow = [&](int cc) { return C16 + (((size_t)bh * p.NC + cc) * 2 * p.DK + d) * p.DV + j0; };
+        uint4 cr[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) cr[x] = *reinterpret_cast<const uint4 *>(crow(c) + 8 * x);
+        const int ep0 = ((int)blockIdx.y * (p.DV / 64) + (int)blockIdx.z) * 4 + q4;
         for (int i = 0; i < p.NC; ++i, --c) {
             const float decay = expf(g_c + mc_c - mn_c);
             if (c >= 1) {   // the next chunk's terms, one step ahead
                 mn_c = mc_c;
                 g_c = Gb[c - 1];
                 mc_c = MCb[c - 1];
+            }
+            {
+                float e = with_n ? gn * p.NS[((size_t)bh * p.NC + c) * p.DK + d] : 0.f;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const uint32_t w4[4] = {cr[x].x, cr[x].y, cr[x].z, cr[x].w};
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) {
+                        e = fmaf(Gs[8 * x + 2 * z], __uint_as_float(w4[z] << 16), e);
+                        e = fmaf(Gs[8 * x + 2 * z + 1], __uint_as_float(w4[z] & 0xffff0000u), e);
+                    }
+                }
+                if (c >= 1) {
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) cr[x] = *reinterpret_cast<const uint4 *>(crow(c - 1) + 8 * x);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+                if (lane == 0) EP[((size_t)bh * p.NC + c) * NEP + ep0] = e * decay;
             }
             // the gradient of the state at this chunk's end
             __nv_bfloat16 *dst = G16 + (((size_t)bh * p.NC + c) * p.DK + d) * p.DV + j0;
@@ -806,12 +846,12 @@ static cudaError_t launch_gstate_l(const Args &a)
     if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&msg, a.sg16, a.DV, a.S, 2 * a.BH)) return cudaErrorInvalidValue;
     KParams p{};
     p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
-    p.MC = a.MC; p.G = a.G;
+    p.MC = a.MC; p.G = a.G; p.NS = a.NS;
     p.status = a.status;
     cudaError_t e = ensure_dynamic_smem((const void *)gstate_tc_kernel<L>, SM::TOTAL);
     if (e != cudaSuccess) return e;
     return launch_kernel(gstate_tc_kernel<L>, dim3(a.BH, a.DK / 128, a.DV / 64), dim3(THREADS), SM::TOTAL, a.stream, 1,
-                         mq, msg, p, a.G16w, a.GNw);
+                         mq, msg, p, a.G16w, a.GNw, a.C16, a.EPw, a.NEP);
 }
 
 cudaError_t launch_gstate(const Args &a)
@@ -852,8 +892,10 @@ cudaError_t launch_carry(const Args &a)
 // the diagonal) are used.  KIND 0: X = q, Y = k (bf16 inputs: the products are exact in the fp32
 // accumulator), K = DK; A = D * scale * exp(x_s - mx_t) on the causal triangle (two bf16 parts),
 // den_t = rowsum(A)_t + sc_t scale n_c . q_t and N_t.  KIND 1: X = g (two bf16 parts), Y = v,
-// K = DV; dden_t, dS = (D + dden_t) exp(x_s - mx_t) on the causal triangle (bf16) and
-// dn_c = sum_t sc_t dden_t scale q_t.  A TMEM lane is a token t (row), a column a token s.
+// K = DV; dden_t, dS = (D + dden_t) exp(x_s - mx_t) on the causal triangle (bf16),
+// dn_c = sum_t sc_t dden_t scale q_t and, for the forget-gate gradients, RECT_j = the sum of
+// R_ts = dA_ts A_ts (dA = D + dden_t, A read back as its two parts) over the pairs s < j <= t of the
+// chunk.  A TMEM lane is a token t (row), a column a token s.
 constexpr int XSTAGES = 4;
 struct ChunkSmem {
     static constexpr uint32_t STAGE = 2 * 16384;              // X and Y: 128 rows x 64 each
@@ -982,6 +1024,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         bool failed = false;
         if (r == 0) failed = !mbar_wait(accf, 0, wc);
         failed = group_any(2, 128, failed);
+        // KIND 1: R_ts = dA_ts A_ts over the pairs s < t of the chunk (the derivative of the loss by
+        // the log decay between s and t), summed along this row (rowl) and, per warp, down the columns
+        // (cpart [4][128], in the n array's place)
+        float rowl = 0.f;
+        float *cpart = ns;
         if (!failed) {
             tc_fence_after();
             const float mxr = mx[r];
@@ -989,23 +1036,49 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // this row of the chunk's L x L block: A16 (two parts) or dS16 (one), zeros off the triangle
             __nv_bfloat16 *dst = KIND == 0 ? a.A16w + ((size_t)bh * a.NC + c) * 2 * L * L + (size_t)tl * L
                                            : a.dS16w + ((size_t)bh * a.NC + c) * L * L + (size_t)tl * L;
+            const __nv_bfloat16 *arow = a.A16 + ((size_t)bh * a.NC + c) * 2 * L * L + (size_t)tl * L;
 #pragma unroll 1
             for (int g = 0; g < L / 16; ++g) {
                 uint32_t rr[16];
                 tmem_ld16(tmem_addr(tmem, q4 * 32, cb + g * 16), rr);
+                uint4 ah[2] = {}, al[2] = {};
+                if (KIND == 1 && chunk_ok) {   // this row of A (two parts: value and residue)
+                    ah[0] = *reinterpret_cast<const uint4 *>(arow + g * 16);
+                    ah[1] = *reinterpret_cast<const uint4 *>(arow + g * 16 + 8);
+                    al[0] = *reinterpret_cast<const uint4 *>(arow + (size_t)L * L + g * 16);
+                    al[1] = *reinterpret_cast<const uint4 *>(arow + (size_t)L * L + g * 16 + 8);
+                }
                 tmem_wait_ld();
                 __nv_bfloat16 hi[16], lo[16];
+                float rv[16];
 #pragma unroll
                 for (int z = 0; z < 16; ++z) {
                     const int sl = g * 16 + z;
                     float v = 0.f;
+                    rv[z] = 0.f;
                     if (sl <= tl && ok_t) {
                         const float dcy = expf(xs[cb + sl] - mxr);
-                        v = KIND == 0 ? __uint_as_float(rr[z]) * scale * dcy : (__uint_as_float(rr[z]) + ddv) * dcy;
+                        if (KIND == 0) {
+                            v = __uint_as_float(rr[z]) * scale * dcy;
+                        } else {
+                            const float da = __uint_as_float(rr[z]) + ddv;
+                            v = da * dcy;
+                            const uint32_t wh = reinterpret_cast<const uint32_t *>(ah)[z >> 1];
+                            const uint32_t wl = reinterpret_cast<const uint32_t *>(al)[z >> 1];
+                            const float av = (z & 1) ? __uint_as_float(wh & 0xffff0000u) + __uint_as_float(wl & 0xffff0000u)
+                                                     : __uint_as_float(wh << 16) + __uint_as_float(wl << 16);
+                            if (sl < tl) rv[z] = da * av;
+                        }
                     }
                     rsum += v;
                     if (KIND == 0) bf16_parts(v, hi[z], lo[z]);
                     else hi[z] = __float2bfloat16_rn(v);
+                }
+                if (KIND == 1) {
+#pragma unroll
+                    for (int z = 0; z < 16; ++z) rowl += rv[z];
+                    const float cs = warp_sum16(rv, lane);   // the warp's 32 rows, column sum16_index(lane)
+                    if ((lane & 1) == 0) cpart[q4 * 128 + cb + g * 16 + sum16_index(lane)] = cs;
                 }
                 if (chunk_ok) {
                     *reinterpret_cast<uint4 *>(dst + g * 16) = *reinterpret_cast<const uint4 *>(hi);
@@ -1036,6 +1109,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
         if (KIND == 1) {   // dn_c = sum_t sc_t dden_t scale q_t of each chunk of the block
             named_sync(1, 128);
+            float *drow = ns + 512;   // [128] colb_t - rowl_t
             if (!failed) {
                 for (int cc = 0; cc < CPB; ++cc) {
                     const int ch = tb / L + cc;
@@ -1047,6 +1121,38 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         for (int u = 0; u < clen; ++u)
                             a2 = fmaf(sc[cc * L + u] * dd[cc * L + u], __bfloat162float(qb[(size_t)u * a.DK + i]) * scale, a2);
                         a.GNw[((size_t)bh * a.NC + ch) * a.DK + i] = a2;
+                    }
+                }
+                // colb_t: the column sum of R below the diagonal, over the warps of this row's chunk
+                const int w0 = (r / L) * (L / 32);
+                float colb = 0.f;
+                for (int w2 = w0; w2 < w0 + L / 32; ++w2) colb += cpart[w2 * 128 + r];
+                drow[r] = colb - rowl;
+            }
+            named_sync(1, 128);
+            // RECT_j = sum_{s < j} drow_s over the chunk: the pairs s < j <= t inside it (a warp per
+            // chunk, a scan in fp64)
+            if (!failed && q4 < CPB) {
+                const int ch = tb / L + q4;
+                if (ch < a.NC) {
+                    constexpr int PER = L / 32;
+                    const int clen = min(L, a.S - ch * L);
+                    const float *dv = drow + q4 * L + lane * PER;
+                    double loc = 0.0;
+#pragma unroll
+                    for (int u = 0; u < PER; ++u) loc += (double)dv[u];
+                    double inc = loc;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const double y = __shfl_up_sync(0xffffffffu, inc, o);
+                        if (lane >= o) inc += y;
+                    }
+                    double run = inc - loc;
+#pragma unroll
+                    for (int u = 0; u < PER; ++u) {
+                        const int tl2 = lane * PER + u;
+                        if (tl2 < clen) a.RECTw[(size_t)bh * a.S + (size_t)ch * L + tl2] = (float)run;
+                        run += (double)dv[u];
                     }
                 }
             }

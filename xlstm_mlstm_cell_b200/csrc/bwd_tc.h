@@ -24,7 +24,9 @@ struct Args {
     // [BH][NC][DK][DV] and dS16 [BH][NC][L][L]
     const __nv_bfloat16 *C16, *G16, *g16, *dS16, *A16;
     __nv_bfloat16 *dq, *dk, *dv;            // outputs [BH][S][DK | DV]
-    float *QD, *KD;                         // partial q . dq and k . dk per 32 columns [BH][S][NTK]
+    // partial q . dq^inter (the inter-chunk term alone), k . dk and k . dk^inter per 32 columns
+    // [BH][S][NTK], for the gate gradients
+    float *QD, *KD, *KI;
     // the read-out numerator: dh, o (NULL without an output gate) [BH][S][DV], N = max(|den|,
     // exp(-m)) [BH][S]; writes g (its two bf16 parts, g16w), do (when o is given) and the partial
     // row sums of g . hh per 64 value columns DOTP [BH][S][NJT]
@@ -43,6 +45,11 @@ struct Args {
     // the scores and dS (launch_scores, launch_ds): write DEN, NRM [BH][S] and A16 (two parts);
     // DD [BH][S], dS16 and the read-out's dn_c GNw [BH][NC][DK]
     float *DENw, *NRMw, *DDw, *GNw;
+    // dS also writes RECT [BH][S]: sum of dA_ts A_ts over the pairs s < j <= t of token j's chunk;
+    // the state-gradient walk writes the partial sums of E_c = exp(g_c + m_c - m_{c+1})
+    // (<G_end, C_c> + <dn_end, n_c>) [BH][NC][NEP], NEP = 4 (DK / 128) (DV / 64) (a warp of each tile)
+    float *RECTw, *EPw;
+    int NEP;
     __nv_bfloat16 *A16w, *dS16w;
     uint32_t *status;
     cudaStream_t stream;

@@ -98,6 +98,10 @@ size_t plan_bwd_workspace(char *base, int BH, int S, int DHQK, int DHV, int chun
     w->AI = tc ? nullptr : reinterpret_cast<float *>(take(f * BH * NC * chunk * chunk));
     w->QD = reinterpret_cast<float *>(take(f * BH * S * NTK));
     w->KD = reinterpret_cast<float *>(take(f * BH * S * NTK));
+    w->KI = reinterpret_cast<float *>(take(f * BH * S * NTK));
+    w->RECT = reinterpret_cast<float *>(take(f * BH * S));
+    w->NEP = tc ? 4 * (DHQK / 128) * (DHV / 64) : 1;
+    w->EP = reinterpret_cast<float *>(take(f * BH * NC * w->NEP));
     w->DEN = reinterpret_cast<float *>(take(f * BH * S));
     w->NRM = reinterpret_cast<float *>(take(f * BH * S));
     w->DOTP = reinterpret_cast<float *>(take(f * BH * S * ((DHV + 63) / 64)));

@@ -79,7 +79,12 @@ struct BwdWorkspace {
     float *Gt;                    // [BH][S][DHV] gradient of the read-out numerator
     float *DD;                    // [BH][S] gradient of the denominator
     float *P2, *AI;               // [BH][NC][chunk][chunk] score gradients and scores
-    float *QD, *KD;               // [BH][S][ceil(DHQK / 32)] partial q . dq, k . dk
+    // [BH][S][ceil(DHQK / 32)] partial q . dq^inter, k . dk and k . dk^inter (^inter: the term of the
+    // tokens of other chunks, through the chunk's state or state gradient)
+    float *QD, *KD, *KI;
+    float *RECT;                  // [BH][S] sum of dA_ts A_ts over the pairs s < j <= t of j's chunk
+    float *EP;                    // [BH][NC][NEP] partial sums of E_c, the pairs that skip chunk c
+    int NEP;                      // 1 on the CUDA-core path, 4 (DHQK / 128) (DHV / 64) on the tensor-core path
     float *DEN, *NRM;             // [BH][S] read-out denominator and its floored magnitude
     float *DOTP;                  // [BH][S][ceil(DHV / 64)] partial row sums of g . hh
     // the tensor-core path (bf16 inputs, bwd_tc_path; there CS, GS, Gt, P2 and AI are NULL): the
