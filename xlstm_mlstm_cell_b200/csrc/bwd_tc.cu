@@ -481,15 +481,24 @@ constexpr int CSTAGES = 4;
 struct CarrySmem {
     static constexpr uint32_t STAGE = 2 * 16384 + 8192;      // w k: 2 parts x 64 tokens x 128 rows; v: 64 x 64
     static constexpr uint32_t ONES = CSTAGES * STAGE;        // 16 rows x 64 bf16 ones (K-major B of n)
-    static constexpr uint32_t BAR = ONES + 2048;
-    static constexpr uint32_t NBAR = 2 * CSTAGES + 4;
+    // per epilogue warp, tiles of its 32 state rows x 64 columns (bf16, 128-byte swizzle, 4 KB each)
+    // that TMA moves: the carry's chunk-start state (two parts) out; the state-gradient walk's
+    // chunk-end gradient out (one) and C_c in (two buffers)
+    static constexpr uint32_t STG = ONES + 2048;
+    static constexpr uint32_t STG_BYTES = 4 * 3 * 4096;
+    static constexpr uint32_t BAR = STG + STG_BYTES;
+    static constexpr uint32_t NBAR = 2 * CSTAGES + 4 + 8;   // (+ the C_c tiles' barriers, two per warp)
     static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
+    static_assert(STG % 1024 == 0 && TOTAL <= 232448, "carry smem");
 };
+
+// Byte offset of 16-byte chunk x (0..7) of row r in a [rows][64] bf16 tile under the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_tile(int r, int x) { return (uint32_t)(r * 128 + ((x ^ (r & 7)) << 4)); }
 
 template <int L>
 __global__ void __launch_bounds__(THREADS, 1)
-carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_v, KParams p,
-                __nv_bfloat16 *__restrict__ C16, float *__restrict__ NSo)
+carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ CUtensorMap tm_cs, KParams p, float *__restrict__ NSo)
 {
     using SM = CarrySmem;
     extern __shared__ uint8_t smem_raw[];
@@ -518,6 +527,7 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
         fence_barrier_init();
         tma_prefetch(&tm_wk);
         tma_prefetch(&tm_v);
+        tma_prefetch(&tm_cs);
     }
     // the ones tile (every element 1.0, so its layout needs no swizzle care)
     for (int e = threadIdx.x; e < 2048 / 16; e += blockDim.x)
@@ -600,15 +610,29 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
                 mc_c = mn_c;
                 mn_c = MCb[c + 2];
             }
-            // the state at the chunk's start: its two bf16 parts, and n
-            __nv_bfloat16 *dst = C16 + (((size_t)bh * p.NC + c) * 2 * p.DK + d) * p.DV + j0;
+            // the state at the chunk's start: its two bf16 parts (this warp's 32 rows through a swizzled
+            // tile per part and a TMA store each, once the previous chunk's stores have read the tiles),
+            // and n
+            {
+                uint8_t *stg = smem + SM::STG + q4 * 8192;
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
 #pragma unroll
-            for (int x = 0; x < 64; x += 8) {
-                __nv_bfloat16 hi[8], lo[8];
+                for (int x = 0; x < 8; ++x) {
+                    __nv_bfloat16 hi[8], lo[8];
 #pragma unroll
-                for (int z = 0; z < 8; ++z) bf16_parts(C[x + z], hi[z], lo[z]);
-                *reinterpret_cast<uint4 *>(dst + x) = *reinterpret_cast<const uint4 *>(hi);
-                *reinterpret_cast<uint4 *>(dst + (size_t)p.DK * p.DV + x) = *reinterpret_cast<const uint4 *>(lo);
+                    for (int z = 0; z < 8; ++z) bf16_parts(C[8 * x + z], hi[z], lo[z]);
+                    *reinterpret_cast<uint4 *>(stg + sw_tile(lane, x)) = *reinterpret_cast<const uint4 *>(hi);
+                    *reinterpret_cast<uint4 *>(stg + 4096 + sw_tile(lane, x)) = *reinterpret_cast<const uint4 *>(lo);
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) {
+                    const int z0 = 2 * (bh * p.NC + c);
+                    tma_store_3d(&tm_cs, stg, j0, d0 + q4 * 32, z0);
+                    tma_store_3d(&tm_cs, stg + 4096, j0, d0 + q4 * 32, z0 + 1);
+                    bulk_commit();
+                }
             }
             if (with_n) NSo[((size_t)bh * p.NC + c) * p.DK + d] = n;
             if (c == p.NC - 1) break;   // (the final state is not needed)
@@ -635,6 +659,7 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&ufree[ub]);
         }
+        if (lane == 0) bulk_wait0();   // this warp's state stores are complete
     }
     tc_fence_before();
     __syncthreads();
@@ -657,9 +682,9 @@ carry_tc_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant
 // through GN the same way, in place (dn_c in, the chunk-end gradient out).
 template <int L>
 __global__ void __launch_bounds__(THREADS, 1)
-gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sg, KParams p,
-                 __nv_bfloat16 *__restrict__ G16, float *__restrict__ GN, const __nv_bfloat16 *__restrict__ C16,
-                 float *__restrict__ EP, int NEP)
+gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sg,
+                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_c, KParams p,
+                 float *__restrict__ GN, float *__restrict__ EP, int NEP)
 {
     using SM = CarrySmem;   // (a stage: q 64 tokens x 128 rows, then sc g 2 parts x 64 tokens x 64)
     extern __shared__ uint8_t smem_raw[];
@@ -684,10 +709,13 @@ gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(&ufull[b], 1);
             mbar_init(&ufree[b], 4);
         }
+        for (int b = 0; b < 8; ++b) mbar_init(&ufree[2 + b], 1);   // the C_c tiles, two per epilogue warp
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch(&tm_q);
         tma_prefetch(&tm_sg);
+        tma_prefetch(&tm_g);
+        tma_prefetch(&tm_c);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 128);
@@ -755,13 +783,22 @@ gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float gn = 0.f;
         int c = p.NC - 1;
         float g_c = Gb[c], mc_c = MCb[c], mn_c = MCb[c + 1];
-        // this row of the chunk-start state C_c (its bf16 value part), loaded a chunk ahead: the partial
-        // sums of E_c = exp(g_c + m_c - m_{c+1}) (<G_end, C_c> + <dn_end, n_c>), the pairs of tokens
-        // that skip chunk c, per warp (the forget-gate gradients)
-        auto crow = [&](int cc) { return C16 + (((size_t)bh * p.NC + cc) * 2 * p.DK + d) * p.DV + j0; };
-        uint4 cr[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) cr[x] = *reinterpret_cast<const uint4 *>(crow(c) + 8 * x);
+        // E_c = exp(g_c + m_c - m_{c+1}) (<G_end, C_c> + <dn_end, n_c>), the pairs of tokens that skip
+        // chunk c (the forget-gate gradients): per warp its 32 rows of the tile, from C_c's bf16 value
+        // part, which TMA brings into a swizzled tile two chunks ahead
+        uint64_t *cfull = ufree + 2 + q4 * 2;
+        uint8_t *cbuf = smem + SM::STG + 16384 + q4 * 8192;   // two 4 KB tiles
+        uint8_t *gstg = smem + SM::STG + q4 * 4096;           // the chunk-end gradient out
+        auto load_c = [&](int cc, int b) {
+            mbar_arrive_expect_tx(&cfull[b], 4096);
+            tma_load_3d(cbuf + b * 4096, &tm_c, j0, d0 + q4 * 32, 2 * (bh * p.NC + cc), &cfull[b]);
+        };
+        if (lane == 0) {
+            load_c(c, 0);
+            if (c >= 1) load_c(c - 1, 1);
+        }
+        auto nval = [&](int cc) { return with_n ? p.NS[((size_t)bh * p.NC + cc) * p.DK + d] : 0.f; };
+        float nsv = nval(c);
         const int ep0 = ((int)blockIdx.y * (p.DV / 64) + (int)blockIdx.z) * 4 + q4;
         for (int i = 0; i < p.NC; ++i, --c) {
             const float decay = expf(g_c + mc_c - mn_c);
@@ -770,35 +807,60 @@ gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 g_c = Gb[c - 1];
                 mc_c = MCb[c - 1];
             }
+            // this thread's share (8 independent sums); the warp's sum is taken and stored once the
+            // chunk's step is handed back to the MMA warp
+            const int b = i & 1;
+            const bool cok = mbar_wait(&cfull[b], (uint32_t)(i >> 1) & 1u, wc);
+            if (!__all_sync(0xffffffffu, cok)) break;
+            float epart;
             {
-                float e = with_n ? gn * p.NS[((size_t)bh * p.NC + c) * p.DK + d] : 0.f;
+                const uint8_t *crow = cbuf + b * 4096;
+                float e8[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
-                    const uint32_t w4[4] = {cr[x].x, cr[x].y, cr[x].z, cr[x].w};
+                    const uint4 cr = *reinterpret_cast<const uint4 *>(crow + sw_tile(lane, x));
+                    const uint32_t w4[4] = {cr.x, cr.y, cr.z, cr.w};
+                    float e = 0.f;
 #pragma unroll
                     for (int z = 0; z < 4; ++z) {
                         e = fmaf(Gs[8 * x + 2 * z], __uint_as_float(w4[z] << 16), e);
                         e = fmaf(Gs[8 * x + 2 * z + 1], __uint_as_float(w4[z] & 0xffff0000u), e);
                     }
+                    e8[x] = e;
                 }
-                if (c >= 1) {
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) cr[x] = *reinterpret_cast<const uint4 *>(crow(c - 1) + 8 * x);
+                epart = (((e8[0] + e8[1]) + (e8[2] + e8[3])) + ((e8[4] + e8[5]) + (e8[6] + e8[7]))) + gn * nsv;
+                epart *= decay;   // (nsv is 0 outside the tiles of columns 0..63)
+                __syncwarp();     // the tile has been read: it takes chunk c - 2
+                if (lane == 0 && c >= 2) {
+                    fence_proxy_async();
+                    load_c(c - 2, b);
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-                if (lane == 0) EP[((size_t)bh * p.NC + c) * NEP + ep0] = e * decay;
+                if (c >= 1) nsv = nval(c - 1);
             }
-            // the gradient of the state at this chunk's end
-            __nv_bfloat16 *dst = G16 + (((size_t)bh * p.NC + c) * p.DK + d) * p.DV + j0;
+            const int c_ep = c;
+            auto store_ep = [&]() {
 #pragma unroll
-            for (int x = 0; x < 64; x += 8) {
+                for (int o = 16; o > 0; o >>= 1) epart += __shfl_xor_sync(0xffffffffu, epart, o);
+                if (lane == 0) EP[((size_t)bh * p.NC + c_ep) * NEP + ep0] = epart;
+            };
+            // the gradient of the state at this chunk's end: this warp's 32 rows through a swizzled
+            // tile and a TMA store, once the previous chunk's store has read the tile
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
                 uint4 w;
-                w.x = bf16x2_bits(Gs[x], Gs[x + 1]);
-                w.y = bf16x2_bits(Gs[x + 2], Gs[x + 3]);
-                w.z = bf16x2_bits(Gs[x + 4], Gs[x + 5]);
-                w.w = bf16x2_bits(Gs[x + 6], Gs[x + 7]);
-                *reinterpret_cast<uint4 *>(dst + x) = w;
+                w.x = bf16x2_bits(Gs[8 * x], Gs[8 * x + 1]);
+                w.y = bf16x2_bits(Gs[8 * x + 2], Gs[8 * x + 3]);
+                w.z = bf16x2_bits(Gs[8 * x + 4], Gs[8 * x + 5]);
+                w.w = bf16x2_bits(Gs[8 * x + 6], Gs[8 * x + 7]);
+                *reinterpret_cast<uint4 *>(gstg + sw_tile(lane, x)) = w;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(&tm_g, gstg, j0, d0 + q4 * 32, bh * p.NC + c);
+                bulk_commit();
             }
             float dn = 0.f;
             if (with_n) {
@@ -806,7 +868,10 @@ gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 dn = *slot;
                 *slot = gn;
             }
-            if (c == 0) break;   // (the gradient of the start state is not needed)
+            if (c == 0) {        // (the gradient of the start state is not needed)
+                store_ep();
+                break;
+            }
             if (with_n) gn = fmaf(decay, gn, dn);
             const int ub = i & 1;
             bool failed = false;
@@ -824,7 +889,9 @@ gstate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ufree[ub]);
+            store_ep();
         }
+        if (lane == 0) bulk_wait0();   // this warp's gradient stores are complete
     }
     tc_fence_before();
     __syncthreads();
@@ -842,8 +909,11 @@ template <int L>
 static cudaError_t launch_gstate_l(const Args &a)
 {
     using SM = CarrySmem;
-    CUtensorMap mq, msg;
-    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&msg, a.sg16, a.DV, a.S, 2 * a.BH)) return cudaErrorInvalidValue;
+    CUtensorMap mq, msg, mg, mc;
+    if (!map3(&mq, a.q, a.DK, a.S, a.BH) || !map3(&msg, a.sg16, a.DV, a.S, 2 * a.BH) ||
+        !tcfwd::make_map(&mg, a.G16w, a.DV, a.DK, a.BH * a.NC, 32) ||
+        !tcfwd::make_map(&mc, a.C16, a.DV, a.DK, 2 * a.BH * a.NC, 32))
+        return cudaErrorInvalidValue;
     KParams p{};
     p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
     p.MC = a.MC; p.G = a.G; p.NS = a.NS;
@@ -851,7 +921,7 @@ static cudaError_t launch_gstate_l(const Args &a)
     cudaError_t e = ensure_dynamic_smem((const void *)gstate_tc_kernel<L>, SM::TOTAL);
     if (e != cudaSuccess) return e;
     return launch_kernel(gstate_tc_kernel<L>, dim3(a.BH, a.DK / 128, a.DV / 64), dim3(THREADS), SM::TOTAL, a.stream, 1,
-                         mq, msg, p, a.G16w, a.GNw, a.C16, a.EPw, a.NEP);
+                         mq, msg, mg, mc, p, a.GNw, a.EPw, a.NEP);
 }
 
 cudaError_t launch_gstate(const Args &a)
@@ -869,15 +939,17 @@ static cudaError_t launch_carry_l(const Args &a)
     cudaError_t e = launch_kernel(wk_parts_kernel, dim3(nblk), dim3(256), 0, a.stream, 1, a.k, a.A, a.ig, a.G, a.MC,
                                   a.BH, a.S, L, a.NC, a.DK, a.wk16);
     if (e != cudaSuccess) return e;
-    CUtensorMap mwk, mv;
-    if (!map3(&mwk, a.wk16, a.DK, a.S, 2 * a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH)) return cudaErrorInvalidValue;
+    CUtensorMap mwk, mv, mcs;
+    if (!map3(&mwk, a.wk16, a.DK, a.S, 2 * a.BH) || !map3(&mv, a.v, a.DV, a.S, a.BH) ||
+        !tcfwd::make_map(&mcs, a.C16w, a.DV, a.DK, 2 * a.BH * a.NC, 32))
+        return cudaErrorInvalidValue;
     KParams p{};
     p.S = a.S; p.NC = a.NC; p.DK = a.DK; p.DV = a.DV;
     p.MC = a.MC; p.G = a.G;
     p.status = a.status;
     if ((e = ensure_dynamic_smem((const void *)carry_tc_kernel<L>, SM::TOTAL)) != cudaSuccess) return e;
     return launch_kernel(carry_tc_kernel<L>, dim3(a.BH, a.DK / 128, a.DV / 64), dim3(THREADS), SM::TOTAL, a.stream, 1,
-                         mwk, mv, p, a.C16w, a.NSw);
+                         mwk, mv, mcs, p, a.NSw);
 }
 
 cudaError_t launch_carry(const Args &a)
