@@ -45,13 +45,15 @@ struct Smem {
     static constexpr uint32_t STAGE = SA + SB;
     static constexpr uint32_t F = STAGES * STAGE;             // floats: tokw [L], ddv [L], red [4][L]
     static constexpr uint32_t BAR = F + 6 * L * 4;
-    static constexpr uint32_t NBAR = 2 * STAGES + 1;
+    static constexpr uint32_t NBAR = 2 * STAGES + 4;          // full, empty, accf [2], tfree [2]
     static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
-    static constexpr uint32_t TMEM_COLS = 2 * L;              // the two accumulators
+    // the two accumulators of a tile, twice: the MMAs of the next tile run while the epilogue reads one
+    static constexpr uint32_t TMEM_COLS = 4 * L;
+    static constexpr int CTAS_PER_SM = L == 64 ? 2 : 1;       // (TMEM: 512 columns per SM)
 };
 
 struct KParams {
-    int S, NC, DK, DV, NTK, NJT;
+    int S, NC, DK, DV, NTK, NJT, BH;
     const float *A, *P, *MC, *G, *ig, *DD, *NS, *GN;
     const __nv_bfloat16 *pq;               // q (KIND 0) or k (KIND 1): the partial row sums
     __nv_bfloat16 *out;
@@ -150,7 +152,7 @@ __device__ __forceinline__ void epilogue_num(const KParams &p, const uint32_t (&
 //   KIND 2: A1 = g [t][j] (MN),       B1 = A [t][s] (MN),       A2 = G_end [d][j] (MN), B2 = k [s][d] (K)
 //   KIND 3: A1 = v [s][j] (MN),       B1 = A [t][s] (K),        A2 = C_c [d][j] (MN),   B2 = q [t][d] (K)
 template <int KIND, int L>
-__global__ void __launch_bounds__(THREADS, 2)   // two CTAs per SM: one's epilogue beside the other's loads
+__global__ void __launch_bounds__(THREADS, Smem<L>::CTAS_PER_SM)
 grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                const __grid_constant__ CUtensorMap tm_a2, const __grid_constant__ CUtensorMap tm_b2, KParams p)
 {
@@ -163,12 +165,14 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
     float *ddv = tokw + L;                                    // dden_t (KIND 0), 1 / N_t (KIND 3)
     float *red = ddv + L;                                     // [4][L] per-warp row sums (KIND 3)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
-    uint64_t *full = bars, *empty = bars + STAGES, *accf = bars + 2 * STAGES;
+    uint64_t *full = bars, *empty = bars + STAGES, *accf = bars + 2 * STAGES, *tfree = accf + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
     uint32_t *abort_flag = tmem_slot + 1;
 
-    const int bh = blockIdx.x, c = blockIdx.y, m0 = blockIdx.z * TM;
-    const int t0 = c * L, len = min(L, p.S - t0);
+    // persistent: this CTA takes tiles blockIdx.x, + gridDim.x, ...; a tile is (head, chunk, 128 output
+    // columns), the output-column tiles of a chunk consecutive (they share the chunk's B operands)
+    const int MT = (KIND >= 2 ? p.DV : p.DK) / TM;
+    const long long ntiles = (long long)p.BH * p.NC * MT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // KIND 3 takes its fp32 operands (A and C_c) as two bf16 parts, the value and the rounding
     // residue, and sums both products in the accumulator
@@ -176,13 +180,25 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
     const int nloc = L / 64, ninter = (KIND >= 2 ? p.DK : p.DV) / 64;
     const int nl = NPART * nloc, nb = nl + NPART * ninter;
     WaitCtx wc{abort_flag, p.status};
+    struct Tile { int bh, c, m0; };
+    auto tile_of = [&](long long t) {
+        Tile r;
+        r.m0 = (int)(t % MT) * TM;
+        const long long bc = t / MT;
+        r.c = (int)(bc % p.NC);
+        r.bh = (int)(bc / p.NC);
+        return r;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&tfree[b], 4);   // one arrival per epilogue warp
+        }
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch(&tm_a1);
@@ -202,113 +218,132 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
     griddep_launch_dependents();
 
     if (warp == 0) {
-        if (lane == 0) {   // TMA producer
-            const int zc = bh * p.NC + c;   // (head, chunk) of the per-chunk arrays
-            int kb = 0;
-            for (; kb < nb; ++kb) {
-                const int st = kb % STAGES;
-                if (kb >= STAGES && !mbar_wait(&empty[st], (uint32_t)((kb / STAGES) - 1) & 1u, wc)) break;
-                mbar_arrive_expect_tx(&full[st], SM::STAGE);
-                uint8_t *a = smem + st * SM::STAGE, *b = a + SA;
-                const bool loc = kb < nl;
-                const int idx = loc ? kb : kb - nl, nper = loc ? nloc : ninter;
-                const int part = idx / nper, k0 = 64 * (idx % nper);   // bf16 part, first reduction index
-                if (loc) {
+        if (lane == 0) {   // TMA producer: one ring of stages across this CTA's tiles
+            long long kg = 0;
+            bool ok = true;
+            for (long long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const Tile T = tile_of(tile);
+                const int bh = T.bh, t0 = T.c * L, m0 = T.m0;
+                const int zc = bh * p.NC + T.c;   // (head, chunk) of the per-chunk arrays
+                for (int kb = 0; kb < nb; ++kb, ++kg) {
+                    const int st = (int)(kg % STAGES);
+                    if (kg >= STAGES && !mbar_wait(&empty[st], (uint32_t)((kg / STAGES) - 1) & 1u, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[st], SM::STAGE);
+                    uint8_t *a = smem + st * SM::STAGE, *b = a + SA;
+                    const bool loc = kb < nl;
+                    const int idx = loc ? kb : kb - nl, nper = loc ? nloc : ninter;
+                    const int part = idx / nper, k0 = 64 * (idx % nper);   // bf16 part, first reduction index
+                    if (loc) {
 #pragma unroll
-                    for (int mb = 0; mb < 2; ++mb)   // A1 rows: the stage's 64 tokens, 2 x 64 output columns
-                        tma_load_3d(a + mb * 8192, &tm_a1, m0 + 64 * mb, t0 + k0, KIND == 2 ? 2 * bh : bh, &full[st]);
-                    // the chunk's first row in the score arrays: A holds two parts per chunk
-                    const int rb = KIND >= 2 ? 2 * t0 + part * L : t0;
+                        for (int mb = 0; mb < 2; ++mb)   // A1 rows: the stage's 64 tokens, 2 x 64 output columns
+                            tma_load_3d(a + mb * 8192, &tm_a1, m0 + 64 * mb, t0 + k0, KIND == 2 ? 2 * bh : bh, &full[st]);
+                        // the chunk's first row in the score arrays: A holds two parts per chunk
+                        const int rb = KIND >= 2 ? 2 * t0 + part * L : t0;
 #pragma unroll
-                    for (int n = 0; n < L / 64; ++n) {
-                        if (!B1_MN)      // dS or A rows t (N), columns s (K)
-                            tma_load_3d(b + n * 8192, &tm_b1, k0, rb + 64 * n, bh, &full[st]);
-                        else             // dS or A rows t (K), columns s (N)
-                            tma_load_3d(b + n * 8192, &tm_b1, 64 * n, rb + k0, bh, &full[st]);
+                        for (int n = 0; n < L / 64; ++n) {
+                            if (!B1_MN)      // dS or A rows t (N), columns s (K)
+                                tma_load_3d(b + n * 8192, &tm_b1, k0, rb + 64 * n, bh, &full[st]);
+                            else             // dS or A rows t (K), columns s (N)
+                                tma_load_3d(b + n * 8192, &tm_b1, 64 * n, rb + k0, bh, &full[st]);
+                        }
+                    } else {
+                        // C_c holds two parts per chunk, G_end one
+                        const int za = (KIND == 0 || KIND == 3) ? 2 * zc + part : zc;
+#pragma unroll
+                        for (int mb = 0; mb < 2; ++mb) {
+                            if (A2_MN)       // G_end or C_c rows d (K), columns j (M)
+                                tma_load_3d(a + mb * 8192, &tm_a2, m0 + 64 * mb, k0, za, &full[st]);
+                            else             // C_c or G_end rows d (M), columns j (K)
+                                tma_load_3d(a + mb * 8192, &tm_a2, k0, m0 + 64 * mb, za, &full[st]);
+                        }
+#pragma unroll
+                        for (int n = 0; n < L / 64; ++n)   // g, v, k or q rows (N), columns (K)
+                            tma_load_3d(b + n * 8192, &tm_b2, k0, t0 + 64 * n, KIND == 0 ? 2 * bh : bh, &full[st]);
                     }
-                } else {
-                    // C_c holds two parts per chunk, G_end one
-                    const int za = (KIND == 0 || KIND == 3) ? 2 * zc + part : zc;
-#pragma unroll
-                    for (int mb = 0; mb < 2; ++mb) {
-                        if (A2_MN)       // G_end or C_c rows d (K), columns j (M)
-                            tma_load_3d(a + mb * 8192, &tm_a2, m0 + 64 * mb, k0, za, &full[st]);
-                        else             // C_c or G_end rows d (M), columns j (K)
-                            tma_load_3d(a + mb * 8192, &tm_a2, k0, m0 + 64 * mb, za, &full[st]);
-                    }
-#pragma unroll
-                    for (int n = 0; n < L / 64; ++n)   // g, v, k or q rows (N), columns (K)
-                        tma_load_3d(b + n * 8192, &tm_b2, k0, t0 + 64 * n, KIND == 0 ? 2 * bh : bh, &full[st]);
                 }
             }
             // the last stages' copies have landed before the CTA may leave
-            for (int s = 0; s < STAGES && s < kb; ++s) {
-                const int last = kb - 1 - s;
+            for (int s = 0; s < STAGES && s < kg; ++s) {
+                const long long last = kg - 1 - s;
                 mbar_wait_drain(&full[last % STAGES], (uint32_t)(last / STAGES) & 1u);
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {   // MMA issuer
+        if (lane == 0) {   // MMA issuer: tile it into TMEM buffer it & 1 once the epilogue has read it
             constexpr uint32_t ID1 = idesc_bf16(TM, L, A1_MN, B1_MN), ID2 = idesc_bf16(TM, L, A2_MN, B2_MN);
+            long long kg = 0;
+            int it = 0;
             bool ok = true;
-            for (int kb = 0; kb < nb; ++kb) {
-                const int st = kb % STAGES;
-                if (!mbar_wait(&full[st], (uint32_t)(kb / STAGES) & 1u, wc)) { ok = false; break; }
+            for (long long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+                const int buf = it & 1;
+                if (it >= 2 && !mbar_wait(&tfree[buf], (uint32_t)((it >> 1) - 1) & 1u, wc)) break;
                 tc_fence_after();
-                const uint32_t a = smem_u32(smem + st * SM::STAGE), b = a + SA;
-                const bool loc = kb < nl;
-                const int first = loc ? kb : kb - nl;   // blocks of this accumulator before this one
-                const int amn = loc ? A1_MN : A2_MN, bmn = loc ? B1_MN : B2_MN;
-                const uint32_t d = tmem + (loc ? 0u : (uint32_t)L);
+                for (int kb = 0; kb < nb; ++kb, ++kg) {
+                    const int st = (int)(kg % STAGES);
+                    if (!mbar_wait(&full[st], (uint32_t)(kg / STAGES) & 1u, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a = smem_u32(smem + st * SM::STAGE), b = a + SA;
+                    const bool loc = kb < nl;
+                    const int first = loc ? kb : kb - nl;   // blocks of this accumulator before this one
+                    const int amn = loc ? A1_MN : A2_MN, bmn = loc ? B1_MN : B2_MN;
+                    const uint32_t d = tmem + (uint32_t)(buf * 2 * L) + (loc ? 0u : (uint32_t)L);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {   // 16 reduction elements per MMA
-                    // K-major: 32 bytes further along the 128-byte rows; MN-major: 16 rows further
-                    const uint64_t ad = amn ? smem_desc(a + kk * 2048, 8192, 1024) : smem_desc(a, 16, 1024) + (uint64_t)(kk * 2);
-                    const uint64_t bd = bmn ? smem_desc(b + kk * 2048, 8192, 1024) : smem_desc(b, 16, 1024) + (uint64_t)(kk * 2);
-                    mma_ss(d, ad, bd, loc ? ID1 : ID2, (first > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {   // 16 reduction elements per MMA
+                        // K-major: 32 bytes further along the 128-byte rows; MN-major: 16 rows further
+                        const uint64_t ad = amn ? smem_desc(a + kk * 2048, 8192, 1024) : smem_desc(a, 16, 1024) + (uint64_t)(kk * 2);
+                        const uint64_t bd = bmn ? smem_desc(b + kk * 2048, 8192, 1024) : smem_desc(b, 16, 1024) + (uint64_t)(kk * 2);
+                        mma_ss(d, ad, bd, loc ? ID1 : ID2, (first > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[st]);
                 }
-                mma_commit(&empty[st]);
+                if (ok) mma_commit(&accf[buf]);
             }
-            if (ok) mma_commit(accf);
         }
     } else {
         // ------------------------------------------------ epilogue: warps 2..5
         const int et = threadIdx.x - 64;           // 0..127
         const int q4 = warp & 3;                   // TMEM lane quadrant
-        const int col = m0 + q4 * 32 + lane;       // this thread's output column
-        const size_t g0 = (size_t)bh * p.S + t0;   // first token of the chunk
-        if (et < L) {
-            const int t = et;
-            const bool okt = t < len;
-            if (KIND == 0 || KIND == 3) {
-                const float mc = p.MC[(size_t)bh * (p.NC + 1) + c];
-                tokw[t] = okt ? expf(mc - fmaxf(mc, p.P[g0 + t])) : 0.f;
-                if (KIND == 0) ddv[t] = okt ? p.DD[g0 + t] : 0.f;
-                else ddv[t] = okt ? 1.f / p.NRM[g0 + t] : 1.f;
-            } else {
-                const float gm = p.G[(size_t)bh * p.NC + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1];
-                tokw[t] = okt ? expf(p.ig[g0 + t] - p.A[g0 + t] + gm) : 0.f;
-                ddv[t] = 0.f;
-            }
-        }
-        float colv = 0.f;   // n_c (KIND 0) or dn_end (KIND 1) of this column
-        if (KIND == 0) colv = p.NS[((size_t)bh * p.NC + c) * p.DK + col];
-        if (KIND == 1) colv = p.GN[((size_t)bh * p.NC + c) * p.DK + col];
         const float scale = rsqrtf((float)p.DK);
         const int NCOL = KIND >= 2 ? p.DV : p.DK;
-        named_sync(1, 128);   // tokw, ddv
-        // one thread waits for the accumulators; the four warps take its answer together (the TMEM
-        // loads below are warp-collective)
-        bool failed = false;
-        if (et == 0) failed = !mbar_wait(accf, 0, wc);
-        failed = group_any(2, 128, failed);
-        if (!failed) {
+        int it = 0;
+        for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const Tile T = tile_of(tile);
+            const int bh = T.bh, c = T.c, m0 = T.m0, buf = it & 1;
+            const int t0 = c * L, len = min(L, p.S - t0);
+            const int col = m0 + q4 * 32 + lane;       // this thread's output column
+            const size_t g0 = (size_t)bh * p.S + t0;   // first token of the chunk
+            named_sync(1, 128);   // the previous tile's readers of tokw, ddv and red are done
+            if (et < L) {
+                const int t = et;
+                const bool okt = t < len;
+                if (KIND == 0 || KIND == 3) {
+                    const float mc = p.MC[(size_t)bh * (p.NC + 1) + c];
+                    tokw[t] = okt ? expf(mc - fmaxf(mc, p.P[g0 + t])) : 0.f;
+                    if (KIND == 0) ddv[t] = okt ? p.DD[g0 + t] : 0.f;
+                    else ddv[t] = okt ? 1.f / p.NRM[g0 + t] : 1.f;
+                } else {
+                    const float gm = p.G[(size_t)bh * p.NC + c] - p.MC[(size_t)bh * (p.NC + 1) + c + 1];
+                    tokw[t] = okt ? expf(p.ig[g0 + t] - p.A[g0 + t] + gm) : 0.f;
+                    ddv[t] = 0.f;
+                }
+            }
+            float colv = 0.f;   // n_c (KIND 0) or dn_end (KIND 1) of this column
+            if (KIND == 0) colv = p.NS[((size_t)bh * p.NC + c) * p.DK + col];
+            if (KIND == 1) colv = p.GN[((size_t)bh * p.NC + c) * p.DK + col];
+            named_sync(1, 128);   // tokw, ddv
+            // one thread waits for the accumulators; the four warps take its answer together (the TMEM
+            // loads below are warp-collective)
+            bool failed = false;
+            if (et == 0) failed = !mbar_wait(&accf[buf], (uint32_t)(it >> 1) & 1u, wc);
+            failed = group_any(2, 128, failed);
+            if (failed) break;
             tc_fence_after();
+            const uint32_t tb = (uint32_t)(buf * 2 * L);
 #pragma unroll 1
             for (int g = 0; g < L / 16; ++g) {
                 uint32_t r1[16], r2[16];
-                tmem_ld16(tmem_addr(tmem, q4 * 32, g * 16), r1);
-                tmem_ld16(tmem_addr(tmem, q4 * 32, L + g * 16), r2);
+                tmem_ld16(tmem_addr(tmem, q4 * 32, tb + g * 16), r1);
+                tmem_ld16(tmem_addr(tmem, q4 * 32, tb + L + g * 16), r2);
                 float pv[16];
                 if (KIND == 3) {
                     epilogue_num(p, r1, r2, tokw, ddv, red + q4 * L, g, len, g0, col, scale, lane,
@@ -359,16 +394,19 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
                     if ((lane & 1) == 0 && t < len) p.part2[(g0 + t) * p.NTK + (col >> 5)] = sum;
                 }
             }
-        }
-    }
-    if (KIND == 3 && warp >= 2) {
-        // the row sums of g . hh over each 64 value columns: the two warps of a 64-column half
-        named_sync(1, 128);
-        const int et = threadIdx.x - 64;
-        for (int e = et; e < 2 * L; e += 128) {
-            const int h2 = e / L, t = e % L;
-            if (t < len && !*reinterpret_cast<volatile uint32_t *>(abort_flag))
-                p.DOTP[((size_t)bh * p.S + t0 + t) * p.NJT + (m0 >> 6) + h2] = red[(2 * h2) * L + t] + red[(2 * h2 + 1) * L + t];
+            // the accumulators of this buffer have been read: the MMAs of tile it + 2 may take them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tfree[buf]);
+            if (KIND == 3) {
+                // the row sums of g . hh over each 64 value columns: the two warps of a 64-column half
+                named_sync(1, 128);
+                for (int e = et; e < 2 * L; e += 128) {
+                    const int h2 = e / L, t = e % L;
+                    if (t < len)
+                        p.DOTP[((size_t)bh * p.S + t0 + t) * p.NJT + (m0 >> 6) + h2] = red[(2 * h2) * L + t] + red[(2 * h2 + 1) * L + t];
+                }
+            }
         }
     }
     tc_fence_before();
@@ -402,10 +440,15 @@ static cudaError_t launch_kind(const Args &a, const CUtensorMap &a1, const CUten
     p.part = KIND == 0 ? a.QD : KIND == 1 ? a.KD : nullptr;
     p.part2 = KIND == 1 ? a.KI : nullptr;
     p.status = a.status;
+    p.BH = a.BH;
     cudaError_t e = ensure_dynamic_smem((const void *)grad_tc_kernel<KIND, L>, SM::TOTAL);
     if (e != cudaSuccess) return e;
-    const int tiles = (KIND >= 2 ? a.DV : a.DK) / TM;
-    return launch_kernel(grad_tc_kernel<KIND, L>, dim3(a.BH, a.NC, tiles), dim3(THREADS), SM::TOTAL, a.stream, 1, a1,
+    int sms = 0;
+    if ((e = sm_count(&sms)) != cudaSuccess) return e;
+    // persistent CTAs, SM::CTAS_PER_SM on every SM (fewer when there are fewer tiles)
+    const long long tiles = (long long)a.BH * a.NC * ((KIND >= 2 ? a.DV : a.DK) / TM);
+    const int grid = (int)std::min<long long>(tiles, (long long)sms * SM::CTAS_PER_SM);
+    return launch_kernel(grad_tc_kernel<KIND, L>, dim3(grid), dim3(THREADS), SM::TOTAL, a.stream, 1, a1,
                          b1, a2, b2, p);
 }
 

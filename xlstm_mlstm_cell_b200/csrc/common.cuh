@@ -132,4 +132,21 @@ inline cudaError_t ensure_dynamic_smem(const void *kernel, int bytes)
     return cudaSuccess;
 }
 
+// The SM count of the current device, looked up once per device.  Thread-safe.
+inline cudaError_t sm_count(int *n)
+{
+    static int cached[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> guard(host_cache_mutex());
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+        *n = cached[dev];
+        return cudaSuccess;
+    }
+    if ((e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) cached[dev] = *n;
+    return cudaSuccess;
+}
+
 }  // namespace mlstm
