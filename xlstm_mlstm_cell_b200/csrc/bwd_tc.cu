@@ -1231,11 +1231,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     if (ch >= a.NC) break;
                     const int clen = min(L, a.S - ch * L);
                     const __nv_bfloat16 *qb = a.q + ((size_t)bh * a.S + ch * L) * a.DK;
-                    for (int i = r; i < a.DK; i += 128) {
-                        float a2 = 0.f;
-                        for (int u = 0; u < clen; ++u)
-                            a2 = fmaf(sc[cc * L + u] * dd[cc * L + u], __bfloat162float(qb[(size_t)u * a.DK + i]) * scale, a2);
-                        a.GNw[((size_t)bh * a.NC + ch) * a.DK + i] = a2;
+                    // a thread per column pair; four independent sums, so that the loads of q overlap
+                    for (int i = 2 * r; i < a.DK; i += 256) {
+                        float ax[4] = {0.f, 0.f, 0.f, 0.f}, ay[4] = {0.f, 0.f, 0.f, 0.f};
+                        int u = 0;
+                        for (; u + 4 <= clen; u += 4) {
+#pragma unroll
+                            for (int z = 0; z < 4; ++z) {
+                                const float w = sc[cc * L + u + z] * dd[cc * L + u + z];
+                                const uint32_t qq = *reinterpret_cast<const uint32_t *>(qb + (size_t)(u + z) * a.DK + i);
+                                ax[z] = fmaf(w, __uint_as_float(qq << 16), ax[z]);
+                                ay[z] = fmaf(w, __uint_as_float(qq & 0xffff0000u), ay[z]);
+                            }
+                        }
+                        for (; u < clen; ++u) {
+                            const float w = sc[cc * L + u] * dd[cc * L + u];
+                            const uint32_t qq = *reinterpret_cast<const uint32_t *>(qb + (size_t)u * a.DK + i);
+                            ax[0] = fmaf(w, __uint_as_float(qq << 16), ax[0]);
+                            ay[0] = fmaf(w, __uint_as_float(qq & 0xffff0000u), ay[0]);
+                        }
+                        float *gd = a.GNw + ((size_t)bh * a.NC + ch) * a.DK + i;
+                        gd[0] = ((ax[0] + ax[1]) + (ax[2] + ax[3])) * scale;
+                        gd[1] = ((ay[0] + ay[1]) + (ay[2] + ay[3])) * scale;
                     }
                 }
                 // colb_t: the column sum of R below the diagonal, over the warps of this row's chunk
