@@ -330,6 +330,22 @@ grad_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant_
             float colv = 0.f;   // n_c (KIND 0) or dn_end (KIND 1) of this column
             if (KIND == 0) colv = p.NS[((size_t)bh * p.NC + c) * p.DK + col];
             if (KIND == 1) colv = p.GN[((size_t)bh * p.NC + c) * p.DK + col];
+            // the rows the epilogue reads (dh and o, or q or k: L tokens x 128 columns) into L2 while
+            // the tile's MMAs run, a 128-byte line per thread and array
+            if (KIND != 2) {
+                for (int e = et; e < 2 * L; e += 128) {
+                    const int t = e >> 1;
+                    if (t < len) {
+                        const size_t off = (g0 + t) * (size_t)(KIND == 3 ? p.DV : p.DK) + m0 + (e & 1) * 64;
+                        if (KIND == 3) {
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.dh + off));
+                            if (p.o) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + off));
+                        } else {
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.pq + off));
+                        }
+                    }
+                }
+            }
             named_sync(1, 128);   // tokw, ddv
             // one thread waits for the accumulators; the four warps take its answer together (the TMEM
             // loads below are warp-collective)
