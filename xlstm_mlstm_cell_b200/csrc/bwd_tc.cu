@@ -1030,15 +1030,20 @@ cudaError_t launch_carry(const Args &a)
 constexpr int XSTAGES = 4;
 struct ChunkSmem {
     static constexpr uint32_t STAGE = 2 * 16384;              // X and Y: 128 rows x 64 each
-    static constexpr uint32_t F = XSTAGES * STAGE;            // floats: xs, mx, fl, sc, dd [128]; ns [2][512]
+    // (once the MMAs are done, the stages take the epilogue's output tiles: per warp its 32 rows of A's
+    // two parts or of dS, in [32][64] bf16 tiles under the 128-byte swizzle, stored by TMA)
+    static constexpr uint32_t ATILE = XSTAGES * STAGE;        // the dS kernel's A rows, loaded by TMA
+    static constexpr uint32_t F = ATILE + 4 * 2 * 2 * 4096;   // floats: xs, mx, fl, sc, dd [128]; ns [2][512]
     static constexpr uint32_t BAR = F + (5 * 128 + 2 * 512) * 4;
-    static constexpr uint32_t NBAR = 2 * XSTAGES + 1;
+    static constexpr uint32_t NBAR = 2 * XSTAGES + 2;         // full, empty, accf, the A rows
     static constexpr uint32_t TOTAL = BAR + NBAR * 8 + 16 + 1024;
+    static_assert(TOTAL <= 232448, "chunk smem");
 };
 
 template <int KIND, int L>
 __global__ void __launch_bounds__(THREADS, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y, Args a)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
+                const __grid_constant__ CUtensorMap tm_st, const __grid_constant__ CUtensorMap tm_a, Args a)
 {
     using SM = ChunkSmem;
     constexpr int NPART = KIND == 1 ? 2 : 1;
@@ -1048,8 +1053,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     float *xs = reinterpret_cast<float *>(smem + SM::F), *mx = xs + 128, *fl = mx + 128, *sc = fl + 128;
     float *dd = sc + 128, *ns = dd + 128;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::BAR);
-    uint64_t *full = bars, *empty = bars + XSTAGES, *accf = bars + 2 * XSTAGES;
+    uint64_t *full = bars, *empty = bars + XSTAGES, *accf = bars + 2 * XSTAGES, *abar = accf + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + SM::NBAR);
+    constexpr int NB = L / 64;                   // 64-column boxes per row of the chunk's block
+    constexpr int NPS = KIND == 0 ? 2 : 1;       // parts of the stored array (A: two, dS: one)
     uint32_t *abort_flag = tmem_slot + 1;
     const int bh = blockIdx.x, tb = blockIdx.y * 128;   // first token of the block
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1062,10 +1069,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
+        mbar_init(abar, 1);
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch(&tm_x);
         tma_prefetch(&tm_y);
+        tma_prefetch(&tm_st);
+        if (KIND == 1) tma_prefetch(&tm_a);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 128);
@@ -1080,6 +1090,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     if (warp == 0) {
         if (lane == 0) {
+            if (KIND == 1) {   // the rows of A (two parts) that the epilogue reads, first
+                uint32_t bytes = 0;
+                for (int w = 0; w < 4; ++w)
+                    if ((tb + 32 * w) / L < a.NC) bytes += 2 * NB * 4096;
+                mbar_arrive_expect_tx(abar, bytes);
+                for (int w = 0; w < 4; ++w) {
+                    const int t0w = tb + 32 * w, cw = t0w / L;
+                    if (cw >= a.NC) continue;
+                    for (int part = 0; part < 2; ++part)
+                        for (int h = 0; h < NB; ++h)
+                            tma_load_3d(smem + SM::ATILE + ((w * 2 + part) * NB + h) * 4096, &tm_a, 64 * h,
+                                        (cw * 2 + part) * L + t0w % L, bh, abar);
+                }
+            }
             int kb = 0;
             for (; kb < nkb; ++kb) {
                 const int st = kb % XSTAGES;
@@ -1153,7 +1177,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         dd[r] = ddv;
         named_sync(1, 128);
         bool failed = false;
-        if (r == 0) failed = !mbar_wait(accf, 0, wc);
+        if (r == 0) failed = !mbar_wait(accf, 0, wc) || (KIND == 1 && !mbar_wait(abar, 0, wc));
         failed = group_any(2, 128, failed);
         // KIND 1: R_ts = dA_ts A_ts over the pairs s < t of the chunk (the derivative of the loss by
         // the log decay between s and t), summed along this row (rowl) and, per warp, down the columns
@@ -1164,20 +1188,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             tc_fence_after();
             const float mxr = mx[r];
             float rsum = 0.f;
-            // this row of the chunk's L x L block: A16 (two parts) or dS16 (one), zeros off the triangle
-            __nv_bfloat16 *dst = KIND == 0 ? a.A16w + ((size_t)bh * a.NC + c) * 2 * L * L + (size_t)tl * L
-                                           : a.dS16w + ((size_t)bh * a.NC + c) * L * L + (size_t)tl * L;
-            const __nv_bfloat16 *arow = a.A16 + ((size_t)bh * a.NC + c) * 2 * L * L + (size_t)tl * L;
+            // this row of the chunk's L x L block, A (two parts) or dS (one) with zeros off the triangle,
+            // into the warp's output tiles (the stages, free now), then out by TMA
+            uint8_t *stg = smem + q4 * (2 * NB * 4096);
+            const uint8_t *atl = smem + SM::ATILE + q4 * (2 * NB * 4096);   // this warp's rows of A
 #pragma unroll 1
             for (int g = 0; g < L / 16; ++g) {
                 uint32_t rr[16];
                 tmem_ld16(tmem_addr(tmem, q4 * 32, cb + g * 16), rr);
+                const int hb = g >> 2, x0 = 2 * (g & 3);   // box and 16-byte chunk of columns 16 g ..
                 uint4 ah[2] = {}, al[2] = {};
-                if (KIND == 1 && chunk_ok) {   // this row of A (two parts: value and residue)
-                    ah[0] = *reinterpret_cast<const uint4 *>(arow + g * 16);
-                    ah[1] = *reinterpret_cast<const uint4 *>(arow + g * 16 + 8);
-                    al[0] = *reinterpret_cast<const uint4 *>(arow + (size_t)L * L + g * 16);
-                    al[1] = *reinterpret_cast<const uint4 *>(arow + (size_t)L * L + g * 16 + 8);
+                if (KIND == 1) {   // this row of A (two parts: value and residue)
+                    ah[0] = *reinterpret_cast<const uint4 *>(atl + hb * 4096 + sw_tile(lane, x0));
+                    ah[1] = *reinterpret_cast<const uint4 *>(atl + hb * 4096 + sw_tile(lane, x0 + 1));
+                    al[0] = *reinterpret_cast<const uint4 *>(atl + (NB + hb) * 4096 + sw_tile(lane, x0));
+                    al[1] = *reinterpret_cast<const uint4 *>(atl + (NB + hb) * 4096 + sw_tile(lane, x0 + 1));
                 }
                 tmem_wait_ld();
                 __nv_bfloat16 hi[16], lo[16];
@@ -1211,14 +1236,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     const float cs = warp_sum16(rv, lane);   // the warp's 32 rows, column sum16_index(lane)
                     if ((lane & 1) == 0) cpart[q4 * 128 + cb + g * 16 + sum16_index(lane)] = cs;
                 }
-                if (chunk_ok) {
-                    *reinterpret_cast<uint4 *>(dst + g * 16) = *reinterpret_cast<const uint4 *>(hi);
-                    *reinterpret_cast<uint4 *>(dst + g * 16 + 8) = *reinterpret_cast<const uint4 *>(hi + 8);
-                    if (KIND == 0) {
-                        *reinterpret_cast<uint4 *>(dst + (size_t)L * L + g * 16) = *reinterpret_cast<const uint4 *>(lo);
-                        *reinterpret_cast<uint4 *>(dst + (size_t)L * L + g * 16 + 8) = *reinterpret_cast<const uint4 *>(lo + 8);
-                    }
+                *reinterpret_cast<uint4 *>(stg + hb * 4096 + sw_tile(lane, x0)) = *reinterpret_cast<const uint4 *>(hi);
+                *reinterpret_cast<uint4 *>(stg + hb * 4096 + sw_tile(lane, x0 + 1)) = *reinterpret_cast<const uint4 *>(hi + 8);
+                if (KIND == 0) {
+                    *reinterpret_cast<uint4 *>(stg + (NB + hb) * 4096 + sw_tile(lane, x0)) = *reinterpret_cast<const uint4 *>(lo);
+                    *reinterpret_cast<uint4 *>(stg + (NB + hb) * 4096 + sw_tile(lane, x0 + 1)) = *reinterpret_cast<const uint4 *>(lo + 8);
                 }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0 && chunk_ok) {   // (a warp's 32 rows lie in one chunk)
+                for (int part = 0; part < NPS; ++part)
+                    for (int h = 0; h < NB; ++h)
+                        tma_store_3d(&tm_st, stg + (part * NB + h) * 4096, 64 * h, (c * NPS + part) * L + (tl - lane), bh);
+                bulk_commit();
             }
             if (KIND == 0 && ok_t) {   // den and N
                 const float *nc = ns + (row / L) * a.DK;
@@ -1305,6 +1336,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
         }
+        if (lane == 0) bulk_wait0();   // this warp's output tiles are stored
     }
     tc_fence_before();
     __syncthreads();
@@ -1322,7 +1354,13 @@ template <int KIND, int L>
 static cudaError_t launch_chunk_l(const Args &a)
 {
     using SM = ChunkSmem;
-    CUtensorMap mx, my;
+    CUtensorMap mx, my, mst, ma;
+    // the stored array's rows: A [NC][2][L][L] or dS [NC][L][L] per head, in [32][64] boxes; the dS
+    // kernel also reads A's rows
+    if (!tcfwd::make_map(&mst, KIND == 0 ? (const void *)a.A16w : (const void *)a.dS16w, L,
+                         (KIND == 0 ? 2 : 1) * a.NC * L, a.BH, 32) ||
+        !tcfwd::make_map(&ma, a.A16, L, 2 * a.NC * L, a.BH, 32))
+        return cudaErrorInvalidValue;
     if (KIND == 0) {
         if (!map3(&mx, a.q, a.DK, a.S, a.BH) || !map3(&my, a.k, a.DK, a.S, a.BH)) return cudaErrorInvalidValue;
     } else {
@@ -1331,7 +1369,7 @@ static cudaError_t launch_chunk_l(const Args &a)
     cudaError_t e = ensure_dynamic_smem((const void *)chunk_tc_kernel<KIND, L>, SM::TOTAL);
     if (e != cudaSuccess) return e;
     return launch_kernel(chunk_tc_kernel<KIND, L>, dim3(a.BH, (a.S + 127) / 128), dim3(THREADS), SM::TOTAL, a.stream, 1,
-                         mx, my, a);
+                         mx, my, mst, ma, a);
 }
 
 cudaError_t launch_scores(const Args &a)
