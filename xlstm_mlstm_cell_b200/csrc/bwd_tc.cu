@@ -1,5 +1,8 @@
-// bwd_tc.cu -- the dq, dk and dv products of the chunkwise backward pass on the 5th-generation
-// tensor cores (tcgen05, bf16 operands, fp32 accumulators in TMEM), for bf16 inputs.
+// bwd_tc.cu -- the chunkwise backward pass's products on the 5th-generation tensor cores (tcgen05,
+// bf16 operands, fp32 accumulators in TMEM), for bf16 inputs: dq, dk, dv and the read-out
+// numerator (grad_tc_kernel), the chunk's scores and dS (chunk_tc_kernel), and the two walks over
+// the chunks per state tile, the forward carry (carry_tc_kernel) and the state gradients
+// (gstate_tc_kernel).
 //
 // Per chunk c (L tokens) and head, the gradients of the read-out (the training form of the xLSTM
 // Guide's "The Dual Formulation: How mLSTM Enables Parallel GPU Training", taken chunkwise as in
@@ -9,10 +12,12 @@
 //   dk^T = scale Q^T dS + w (G_end V^T + dn_end 1^T),
 //   dv^T = g^T A + w (G_end^T K^T),
 // with sc_t = exp(m_c - max(m_c, p_t)), w_s = exp(g_c - a_s + i~_s - m_{c+1}), scale = 1/sqrt(DK)
-// and the per-token factors applied column-wise (columns = tokens) in the epilogue.  A CTA computes
+// and the per-token factors applied column-wise (columns = tokens) in the epilogue.  A tile is
 // 128 output columns (d or j: the MMA's M, one per TMEM lane) for all L tokens of one chunk (the
-// MMA's N) as two accumulators in TMEM, the chunk-local one (K = L tokens) and the inter-chunk one
-// (K = DV or DK).  Every operand is a [rows][64] bf16 tile loaded by TMA with the 128-byte swizzle
+// MMA's N), computed as two accumulators in TMEM, the chunk-local one (K = L tokens) and the
+// inter-chunk one (K = DV or DK).  The CTAs are persistent and keep a tile's two accumulators twice
+// in TMEM, so that one tile's epilogue runs while the next tile's loads and MMAs do.  Every operand
+// is a [rows][64] bf16 tile loaded by TMA with the 128-byte swizzle
 // and read by the MMA as K-major (the reduction index runs along the row) or MN-major (along the
 // column), as it lies in memory: no operand is transposed.  The fp32 intermediates (dS, A, g and
 // the per-chunk states) reach this kernel as bf16 copies written by the kernels that compute them.
