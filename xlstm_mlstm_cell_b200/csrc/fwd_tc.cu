@@ -1171,8 +1171,8 @@ walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (tau < len) {
                         const size_t off = ((size_t)bh * p.S + t0 + tau) * p.DV + j0 + q * 32 + jh * 16;
                         const float iv = inv[tau];
-#pragma unroll
                         const uint64_t iv2 = f2_pack(iv, iv);
+#pragma unroll
                         for (int c8 = 0; c8 < 2; ++c8) {
                             // o h / den in packed pairs (bf16 1.0 = 0x3F80 when there is no output gate)
                             const float *hh = hv + c8 * 8;
