@@ -67,6 +67,28 @@ def test_bwd_tensor_path_query(lib):
                      + B * NH * NC * 4 * (DK * DV // 2048 - 1))
 
 
+@pytest.mark.parametrize("DK,DV,ch,dt", [(64, 128, 64, "f32"), (96, 40, 32, "f32"), (128, 256, 64, "bf16"),
+                                          (256, 512, 128, "bf16")])
+def test_bwd_workspace_formula(lib, DK, DV, ch, dt):
+    """mlstm_bwd_workspace_size equals the byte counts include/mlstm.h documents: a 256-byte status
+    word, 4 bytes per head for the last chunk stabilizer, and per chunk and head and per token and
+    head (with 64 heads every array is a multiple of 256 bytes, so no alignment padding enters)."""
+    B, NH, S = 1, 64, 1000
+    NC, BH = -(-S // ch), B * NH
+    ntk, njt = -(-DK // 32), -(-DV // 64)
+    code = binding.MLSTM_BF16 if dt == "bf16" else binding.MLSTM_F32
+    tc = lib.mlstm_bwd_tensor_path(DK, DV, ch, code) == 1
+    assert tc == (dt == "bf16")
+    if tc:
+        per_chunk = 6 * DK * DV + DK * DV // 512 + 8 * DK + 6 * ch * ch + 12
+        per_token = 4 * DK + 8 * DV + 12 * ntk + 4 * njt + 24
+    else:
+        per_chunk = 8 * DK * (DV + 1) + 8 * ch * ch + 16
+        per_token = 4 * DV + 12 * ntk + 4 * njt + 24
+    expected = 256 + 4 * BH + BH * NC * per_chunk + BH * S * per_token
+    assert lib.mlstm_bwd_workspace_size(B, NH, S, DK, DV, ch, code) == expected
+
+
 def test_workspace_size(lib):
     ws = lib.mlstm_fwd_workspace_size(1, 8, 8192, 256, 512, 64, binding.MLSTM_BF16)
     assert ws > 0 and ws % 256 == 0
